@@ -1,0 +1,449 @@
+/*
+ * lowbit_oracle.c -- the oracle for the low-bit-weight linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This is a plain, slow, scalar CPU statement of
+ * what the GPU path computes: quantise -> pack -> unpack -> integer dot ->
+ * rescale.  Only tests/, __graft_entry__.smoke() and bench.py's cpu_baseline
+ * leg may load or call it.  It shares no code, header, table or constant with
+ * the CUDA library; the two are written independently from the same pages:
+ *
+ *   [M8.8]   "M8.8 - Native Binary and Ternary Transformers"
+ *            (transformer-system.numinens.com), sections 0x02C-0x02E, 0x05A-0x05D,
+ *            0x06E, 0x09A-0x09C.
+ *   [Atomic] "Atomic-1Bit" README, opening section (add/sub/skip rule) and the
+ *            "Config presets" text (four ternary codes per byte).
+ *   [T4NT]   "T4NT-0.5B" model card, "What is T4NT?" and the Architecture table
+ *            (15 symmetric levels, tanh(w/3)*3 clipping).
+ *   [Impeto] "Extreme DQT with an FP4 Optimizer", abstract and "Attention"
+ *            (INT1 weights with INT8 activations).
+ *
+ * Floating point: built with -O2 -ffp-contract=off (no FMA contraction, no
+ * fast-math).  Every float operation below is one IEEE-754 operation in the
+ * stated precision, round-to-nearest-even, in the stated order.
+ *
+ * Parity status of each function (the pins live in tests/test_oracle_pins.py):
+ *   orc_ternary_codes, orc_binary_codes, orc_int4_codes, orc_tanh,
+ *   orc_act_quant_*, orc_int_dot, orc_rescale_*, orc_pack/unpack (binary):
+ *     pinned (closed forms, worked cases, library routines, brute force).
+ *   orc_pack/orc_unpack for TERNARY2 and INT4: the pages fix "four codes per
+ *     byte" and "two's complement" but not the bit assignment inside a byte, so
+ *     the bit layout itself is "parity unpinned" (only round-trip, alphabet and
+ *     reserved-pattern invariants pin it).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Status values.  The numbers are part of the library's documented contract
+ * (include/lowbit.h states the same numbers); they are restated here, not
+ * shared. */
+enum {
+    ORC_OK = 0,
+    ORC_EINVAL = 1,
+    ORC_EOVERFLOW = 4,
+    ORC_ENONFINITE = 5,
+    ORC_ERESERVED = 6,
+};
+
+enum { ORC_TERNARY2 = 0, ORC_BINARY1 = 1, ORC_INT4 = 2 };
+
+/* ------------------------------------------------------------------------ */
+/* Small helpers                                                             */
+/* ------------------------------------------------------------------------ */
+
+static float f32_from_bits(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+static uint32_t bits_from_f32(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+
+/* bf16 is the high half of an fp32 bit pattern; widening is exact. */
+float orc_bf16_to_f32(uint16_t h) { return f32_from_bits((uint32_t)h << 16); }
+
+/* fp32 -> bf16, round to nearest even, from the IEEE bit definition: keep the
+ * top 16 bits, add half of the dropped range, and break exact ties toward the
+ * kept value whose lowest bit is 0.  NaN stays a quiet NaN with its sign. */
+uint16_t orc_f32_to_bf16(float f)
+{
+    uint32_t u = bits_from_f32(f);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu) != 0)
+        return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t keep_lsb = (u >> 16) & 1u;
+    u += 0x7fffu + keep_lsb;
+    return (uint16_t)(u >> 16);
+}
+
+static int finite_f32(float f) { return (bits_from_f32(f) & 0x7f800000u) != 0x7f800000u; }
+
+/* ------------------------------------------------------------------------ */
+/* tanh, written out for the 4-bit clipping 3*tanh(w/3) [T4NT]               */
+/* ------------------------------------------------------------------------ */
+/* The pages fix the clipping function but not how tanh is evaluated; a
+ * last-bit difference in tanh can move a weight across a rounding boundary.
+ * So the oracle evaluates tanh with its own fixed sequence of fp64 operations:
+ *
+ *   tanh(a) = e / (e + 2),  e = expm1(2a),  a >= 0, sign restored after;
+ *   expm1(u): if u <= ln2/2, Taylor series sum_{n>=1} u^n/n! to n = 16,
+ *             evaluated by Horner as u*(1 + u/2*(1 + u/3*(...)));
+ *             else Cody-Waite reduction u = k*ln2 + r with ln2 split into a
+ *             high part (21 trailing zero bits, so k*hi is exact) and a low
+ *             part, expm1(u) = 2^k*(1 + expm1(r)) - 1;
+ *   tanh(a) = 1 for a > 20 (1 - tanh(20) < 2^-55).
+ *
+ * Truncation after u^16/16! at |u| <= ln2/2 leaves < 2^-60 relative error. */
+static const double ORC_LN2_HI = 0x1.62e42fee00000p-1;
+static const double ORC_LN2_LO = 0x1.a39ef35793c76p-33;
+static const double ORC_HALF_LN2 = 0x1.62e42fefa39efp-2; /* RN(ln 2) / 2 */
+
+static double orc_expm1_series(double r)
+{
+    double p = 1.0;
+    for (int n = 16; n >= 2; --n)
+        p = 1.0 + (r * p) / (double)n;
+    return r * p;
+}
+
+static double orc_expm1_nonneg(double u)
+{
+    if (u <= ORC_HALF_LN2)
+        return orc_expm1_series(u);
+    double k = rint(u / (ORC_LN2_HI + ORC_LN2_LO));
+    double r = (u - k * ORC_LN2_HI) - k * ORC_LN2_LO;
+    double p = orc_expm1_series(r);
+    return ldexp(1.0 + p, (int)k) - 1.0;
+}
+
+double orc_tanh(double z)
+{
+    if (z != z) return z;
+    double a = fabs(z);
+    double t;
+    if (a > 20.0) {
+        t = 1.0;
+    } else {
+        double e = orc_expm1_nonneg(2.0 * a);
+        t = e / (e + 2.0);
+    }
+    return z < 0 ? -t : t;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Weight quantisers                                                          */
+/* ------------------------------------------------------------------------ */
+
+/* Ternary absmean codes [M8.8 §0x05A, §0x05B]: gamma = mean|W| over the whole
+ * tensor; Q = clip(round(W / (gamma + eps)), -1, 1), round = nearest-even; the
+ * decode scale is gamma itself (scaled_ternary, §0x05B).
+ * The sum is fp64, k ascending within a row, then rows ascending.  gamma is
+ * the fp64 mean rounded once to fp32; the divide and round are fp32.
+ * A zero denominator (all-zero tensor with eps = 0) gives all-zero codes. */
+int orc_ternary_codes(const float *w, long N, long K, long ldw, float eps,
+                      int8_t *codes, float *gamma_out)
+{
+    if (N <= 0 || K <= 0 || ldw < K || !(eps >= 0.0f) || !finite_f32(eps)) return ORC_EINVAL;
+    double S = 0.0;
+    for (long n = 0; n < N; ++n) {
+        double r = 0.0;
+        for (long k = 0; k < K; ++k) {
+            float v = w[n * ldw + k];
+            if (!finite_f32(v)) return ORC_ENONFINITE;
+            r += fabs((double)v);
+        }
+        S += r;
+    }
+    float gamma = (float)(S / (double)(N * K));
+    float d = gamma + eps;
+    for (long n = 0; n < N; ++n)
+        for (long k = 0; k < K; ++k) {
+            int8_t c = 0;
+            if (d != 0.0f) {
+                float t = rintf(w[n * ldw + k] / d);
+                c = (int8_t)(t > 1.0f ? 1 : (t < -1.0f ? -1 : (int)t));
+            }
+            codes[n * K + k] = c;
+        }
+    *gamma_out = gamma;
+    return ORC_OK;
+}
+
+/* Binary sign codes with the total rule "+1 if w >= 0 else -1", so both signed
+ * zeros give +1 [M8.8 §0x06E]; one scale per output row, s_w[n] = mean_k |W|
+ * (the mean-absolute binary scale of §0x02B, taken per row).  fp64 sum, k
+ * ascending, divided by K in fp64, rounded once to fp32. */
+int orc_binary_codes(const float *w, long N, long K, long ldw, int8_t *codes, float *s_w)
+{
+    if (N <= 0 || K <= 0 || ldw < K) return ORC_EINVAL;
+    for (long n = 0; n < N; ++n) {
+        double r = 0.0;
+        for (long k = 0; k < K; ++k) {
+            float v = w[n * ldw + k];
+            if (!finite_f32(v)) return ORC_ENONFINITE;
+            r += fabs((double)v);
+            codes[n * K + k] = (int8_t)(v >= 0.0f ? 1 : -1);
+        }
+        s_w[n] = (float)(r / (double)K);
+    }
+    return ORC_OK;
+}
+
+/* 4-bit symmetric codes [T4NT]: clip w_c = 3*tanh(w/3) (fp64, rounded once to
+ * fp32), per row s_w[n] = max_k |w_c| / 7 (fp32), q = clip(round(w_c / s_w),
+ * -7, 7) (fp32 divide, nearest-even), 15 levels.  A row whose scale is zero
+ * gets zero codes. */
+int orc_int4_codes(const float *w, long N, long K, long ldw, int8_t *codes, float *s_w)
+{
+    if (N <= 0 || K <= 0 || ldw < K) return ORC_EINVAL;
+    float *wc = (float *)malloc(sizeof(float) * (size_t)K);
+    if (!wc) return ORC_EINVAL;
+    for (long n = 0; n < N; ++n) {
+        float m = 0.0f;
+        for (long k = 0; k < K; ++k) {
+            float v = w[n * ldw + k];
+            if (!finite_f32(v)) { free(wc); return ORC_ENONFINITE; }
+            double z = (double)v / 3.0;
+            wc[k] = (float)(3.0 * orc_tanh(z));
+            float a = fabsf(wc[k]);
+            if (a > m) m = a;
+        }
+        float s = m / 7.0f;
+        s_w[n] = s;
+        for (long k = 0; k < K; ++k) {
+            int8_t c = 0;
+            if (s != 0.0f) {
+                float t = rintf(wc[k] / s);
+                c = (int8_t)(t > 7.0f ? 7 : (t < -7.0f ? -7 : (int)t));
+            }
+            codes[n * K + k] = c;
+        }
+    }
+    free(wc);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Packing                                                                    */
+/* ------------------------------------------------------------------------ */
+/* Row n of the artifact starts at byte n*ldp; bytes past the logical extent
+ * of a row are zero.
+ *   TERNARY2: four codes per byte [Atomic]; code k sits in bits
+ *             2*(k%4)+1 .. 2*(k%4) of byte k/4 as a 2-bit two's-complement
+ *             field: 00 = 0, 01 = +1, 11 = -1, 10 reserved.
+ *   BINARY1:  bit (k%8) of byte k/8 is (1 - c)/2, little-bit-first, i.e.
+ *             bit 1 means -1 [M8.8 §0x06E].
+ *   INT4:     code 2j in the low nibble and 2j+1 in the high nibble of byte
+ *             j, 4-bit two's complement; 1000 (-8) is reserved (15 levels). */
+long orc_row_bytes(int fmt, long K)
+{
+    switch (fmt) {
+    case ORC_TERNARY2: return (K + 3) / 4;
+    case ORC_BINARY1: return (K + 7) / 8;
+    case ORC_INT4: return (K + 1) / 2;
+    default: return -1;
+    }
+}
+
+int orc_pack(const int8_t *codes, long N, long K, int fmt, uint8_t *packed, long ldp)
+{
+    long rb = orc_row_bytes(fmt, K);
+    if (N <= 0 || K <= 0 || rb < 0 || ldp < rb) return ORC_EINVAL;
+    for (long n = 0; n < N; ++n) {
+        uint8_t *row = packed + n * ldp;
+        memset(row, 0, (size_t)ldp);
+        for (long k = 0; k < K; ++k) {
+            int c = codes[n * K + k];
+            uint32_t field;
+            switch (fmt) {
+            case ORC_TERNARY2:
+                if (c < -1 || c > 1) return ORC_EINVAL;
+                field = (uint32_t)c & 3u;
+                row[k / 4] |= (uint8_t)(field << (2 * (k % 4)));
+                break;
+            case ORC_BINARY1:
+                if (c != 1 && c != -1) return ORC_EINVAL;
+                field = (uint32_t)((1 - c) / 2);
+                row[k / 8] |= (uint8_t)(field << (k % 8));
+                break;
+            default: /* INT4 */
+                if (c < -7 || c > 7) return ORC_EINVAL;
+                field = (uint32_t)c & 15u;
+                row[k / 2] |= (uint8_t)(field << (4 * (k % 2)));
+                break;
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+/* Inverse of orc_pack.  Rejects a reserved pattern inside the logical extent
+ * and any non-zero bit outside it [M8.8 §0x06E, §0x0BB "reserved patterns
+ * reject"]. */
+int orc_unpack(const uint8_t *packed, long ldp, long N, long K, int fmt, int8_t *codes)
+{
+    long rb = orc_row_bytes(fmt, K);
+    if (N <= 0 || K <= 0 || rb < 0 || ldp < rb) return ORC_EINVAL;
+    int status = ORC_OK;
+    for (long n = 0; n < N; ++n) {
+        const uint8_t *row = packed + n * ldp;
+        for (long k = 0; k < K; ++k) {
+            int c;
+            if (fmt == ORC_TERNARY2) {
+                uint32_t f = (row[k / 4] >> (2 * (k % 4))) & 3u;
+                if (f == 2u) { status = ORC_ERESERVED; c = 0; }
+                else c = (f == 3u) ? -1 : (int)f;
+            } else if (fmt == ORC_BINARY1) {
+                uint32_t b = (row[k / 8] >> (k % 8)) & 1u;
+                c = b ? -1 : 1;
+            } else {
+                uint32_t f = (row[k / 2] >> (4 * (k % 2))) & 15u;
+                if (f == 8u) { status = ORC_ERESERVED; c = 0; }
+                else c = (f >= 8u) ? (int)f - 16 : (int)f;
+            }
+            codes[n * K + k] = (int8_t)c;
+        }
+        /* padding: bits past code K-1 in the last used byte, then whole bytes */
+        long used_bits = K * (fmt == ORC_TERNARY2 ? 2 : (fmt == ORC_BINARY1 ? 1 : 4));
+        for (long bit = used_bits; bit < ldp * 8; ++bit)
+            if ((row[bit / 8] >> (bit % 8)) & 1u) status = ORC_ERESERVED;
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Activation quantiser, per token absmax to int8 [M8.8 §0x05C]               */
+/* ------------------------------------------------------------------------ */
+/* gamma_t = max_k |x[t,k]| (fp32, exact in any order);
+ * gamma_t == 0: q = 0, s_x = 0 (a zero row gives zero codes and scale);
+ * else q = clip(round((x * 127) / (gamma_t + eps)), -128, 127) with an fp32
+ * multiply, an fp32 divide and nearest-even rounding, and
+ * s_x = gamma_t / 127 (the reconstruction scale leaves eps out, §0x05C).
+ * A non-finite x, or an x*127 that overflows, returns ORC_ENONFINITE. */
+static int act_quant_row(const float *x, long K, float eps, int8_t *q, float *s_x)
+{
+    float g = 0.0f;
+    for (long k = 0; k < K; ++k) {
+        if (!finite_f32(x[k]) || !finite_f32(x[k] * 127.0f)) return ORC_ENONFINITE;
+        float a = fabsf(x[k]);
+        if (a > g) g = a;
+    }
+    if (g == 0.0f) {
+        for (long k = 0; k < K; ++k) q[k] = 0;
+        *s_x = 0.0f;
+        return ORC_OK;
+    }
+    float d = g + eps;
+    for (long k = 0; k < K; ++k) {
+        float t = rintf((x[k] * 127.0f) / d);
+        q[k] = (int8_t)(t > 127.0f ? 127 : (t < -128.0f ? -128 : (int)t));
+    }
+    *s_x = g / 127.0f;
+    return ORC_OK;
+}
+
+int orc_act_quant_f32(const float *x, long M, long K, long ldx, float eps,
+                      int8_t *q, long ldq, float *s_x)
+{
+    if (M <= 0 || K <= 0 || ldx < K || ldq < K || !(eps >= 0.0f) || !finite_f32(eps))
+        return ORC_EINVAL;
+    int status = ORC_OK;
+    for (long t = 0; t < M; ++t) {
+        int st = act_quant_row(x + t * ldx, K, eps, q + t * ldq, s_x + t);
+        if (st != ORC_OK) status = st;
+    }
+    return status;
+}
+
+int orc_act_quant_bf16(const uint16_t *x, long M, long K, long ldx, float eps,
+                       int8_t *q, long ldq, float *s_x)
+{
+    if (M <= 0 || K <= 0 || ldx < K || ldq < K || !(eps >= 0.0f) || !finite_f32(eps))
+        return ORC_EINVAL;
+    float *row = (float *)malloc(sizeof(float) * (size_t)K);
+    if (!row) return ORC_EINVAL;
+    int status = ORC_OK;
+    for (long t = 0; t < M; ++t) {
+        for (long k = 0; k < K; ++k) row[k] = orc_bf16_to_f32(x[t * ldx + k]);
+        int st = act_quant_row(row, K, eps, q + t * ldq, s_x + t);
+        if (st != ORC_OK) status = st;
+    }
+    free(row);
+    return status;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Integer dot and rescale                                                    */
+/* ------------------------------------------------------------------------ */
+/* acc[t,n] = sum_k q[t,k] * c[n,k], in int64.  For ternary and binary codes it
+ * is written as the add / subtract / skip rule [Atomic; M8.8 §0x05D]: c = +1
+ * adds the activation, c = -1 subtracts it, c = 0 skips it.  4-bit codes
+ * multiply.  The worst case |acc| <= 128 * cmax * K must fit int32
+ * [M8.8 §0x09C]: K > INT32_MAX / (128 * cmax) returns ORC_EOVERFLOW.
+ * Rows t are independent; nthreads > 1 splits them across OpenMP threads
+ * without changing any result. */
+int orc_int_dot(const int8_t *q, long ldq, const int8_t *codes, long M, long N, long K,
+                int fmt, int64_t *acc, int nthreads)
+{
+    if (M <= 0 || N <= 0 || K <= 0 || ldq < K) return ORC_EINVAL;
+    long cmax = (fmt == ORC_INT4) ? 7 : 1;
+    if (K > 2147483647L / (128L * cmax)) return ORC_EOVERFLOW;
+#ifdef _OPENMP
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#endif
+    for (long t = 0; t < M; ++t) {
+        const int8_t *qt = q + t * ldq;
+        for (long n = 0; n < N; ++n) {
+            const int8_t *cn = codes + n * K;
+            int64_t a = 0;
+            if (fmt == ORC_INT4) {
+                for (long k = 0; k < K; ++k) a += (int64_t)cn[k] * (int64_t)qt[k];
+            } else {
+                for (long k = 0; k < K; ++k) {
+                    if (cn[k] == 1) a += qt[k];
+                    else if (cn[k] == -1) a -= qt[k];
+                }
+            }
+            acc[t * N + n] = a;
+        }
+    }
+    return ORC_OK;
+}
+
+/* Rescale [M8.8 §0x02D, §0x09C]: y[t,n] = float(acc) * (s_w * s_x[t]), the two
+ * scales multiplied first in fp32, then one fp32 multiply.  s_w has one entry
+ * (sw_count == 1, per-tensor ternary scale) or one per output row. */
+int orc_rescale_f32(const int64_t *acc, long M, long N, const float *s_w, long sw_count,
+                    const float *s_x, float *y, long ldy)
+{
+    if (M <= 0 || N <= 0 || ldy < N || (sw_count != 1 && sw_count != N)) return ORC_EINVAL;
+    for (long t = 0; t < M; ++t)
+        for (long n = 0; n < N; ++n) {
+            float sw = s_w[sw_count == 1 ? 0 : n];
+            float sc = sw * s_x[t];
+            y[t * ldy + n] = (float)acc[t * N + n] * sc;
+        }
+    return ORC_OK;
+}
+
+int orc_rescale_bf16(const int64_t *acc, long M, long N, const float *s_w, long sw_count,
+                     const float *s_x, uint16_t *y, long ldy)
+{
+    if (M <= 0 || N <= 0 || ldy < N || (sw_count != 1 && sw_count != N)) return ORC_EINVAL;
+    for (long t = 0; t < M; ++t)
+        for (long n = 0; n < N; ++n) {
+            float sw = s_w[sw_count == 1 ? 0 : n];
+            float sc = sw * s_x[t];
+            y[t * ldy + n] = orc_f32_to_bf16((float)acc[t * N + n] * sc);
+        }
+    return ORC_OK;
+}
+
+/* Number of threads OpenMP would use by default (reported beside timings). */
+int orc_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
