@@ -26,9 +26,9 @@
  *   orc_act_quant_*, orc_int_dot, orc_rescale_*, orc_pack/unpack (binary):
  *     pinned (closed forms, worked cases, library routines, brute force).
  *   orc_pack/orc_unpack for TERNARY2 and INT4: the pages fix "four codes per
- *     byte" and "two's complement" but not the bit assignment inside a byte, so
- *     the bit layout itself is "parity unpinned" (only round-trip, alphabet and
- *     reserved-pattern invariants pin it).
+ *     byte" and "two's complement" but not the order of codes inside a byte, so
+ *     that order is "parity unpinned" (round-trip, alphabet, field encoding and
+ *     reserved-pattern invariants pin the rest).
  */
 #include <math.h>
 #include <stdint.h>
@@ -224,21 +224,37 @@ int orc_int4_codes(const float *w, long N, long K, long ldw, int8_t *codes, floa
 /* ------------------------------------------------------------------------ */
 /* Packing                                                                    */
 /* ------------------------------------------------------------------------ */
-/* Row n of the artifact starts at byte n*ldp; bytes past the logical extent
- * of a row are zero.
- *   TERNARY2: four codes per byte [Atomic]; code k sits in bits
- *             2*(k%4)+1 .. 2*(k%4) of byte k/4 as a 2-bit two's-complement
- *             field: 00 = 0, 01 = +1, 11 = -1, 10 reserved.
- *   BINARY1:  bit (k%8) of byte k/8 is (1 - c)/2, little-bit-first, i.e.
- *             bit 1 means -1 [M8.8 §0x06E].
- *   INT4:     code 2j in the low nibble and 2j+1 in the high nibble of byte
- *             j, 4-bit two's complement; 1000 (-8) is reserved (15 levels). */
+/* Row n of the artifact starts at byte n*ldp; bits past the logical extent of
+ * a row are zero.
+ *   BINARY1:  bit (k%8) of byte k/8 is (1 - c)/2, little-bit-first, i.e. bit 1
+ *             means -1 [M8.8 §0x06E]; a row takes ceil(K/8) bytes.
+ *   TERNARY2: four codes per byte [Atomic], as 2-bit two's-complement fields
+ *             00 = 0, 01 = +1, 11 = -1, 10 reserved.  The pages do not fix the
+ *             order of codes inside a byte; this build stores them plane by
+ *             plane within each little-endian 32-bit word of 16 codes: code k
+ *             lives in word k/16, byte (k%16)%4, field (k%16)/4, i.e. bits
+ *             8*((k%16)%4) + 2*((k%16)/4) and the bit above.  A row takes
+ *             4*ceil(K/16) bytes.
+ *   INT4:     4-bit two's-complement fields, 1000 (-8) reserved (15 levels
+ *             [T4NT]).  Same plane order: code k lives in word k/8, byte
+ *             (k%8)%4, nibble (k%8)/4.  A row takes 4*ceil(K/8) bytes. */
+static long code_bits(int fmt) { return fmt == ORC_TERNARY2 ? 2 : (fmt == ORC_BINARY1 ? 1 : 4); }
+
+/* Bit position of code k inside its row. */
+static long code_bit_pos(int fmt, long k)
+{
+    if (fmt == ORC_BINARY1) return k;
+    long per_word = 32 / code_bits(fmt);
+    long word = k / per_word, kk = k % per_word;
+    return 32 * word + 8 * (kk % 4) + code_bits(fmt) * (kk / 4);
+}
+
 long orc_row_bytes(int fmt, long K)
 {
     switch (fmt) {
-    case ORC_TERNARY2: return (K + 3) / 4;
+    case ORC_TERNARY2: return 4 * ((K + 15) / 16);
     case ORC_BINARY1: return (K + 7) / 8;
-    case ORC_INT4: return (K + 1) / 2;
+    case ORC_INT4: return 4 * ((K + 7) / 8);
     default: return -1;
     }
 }
@@ -247,65 +263,56 @@ int orc_pack(const int8_t *codes, long N, long K, int fmt, uint8_t *packed, long
 {
     long rb = orc_row_bytes(fmt, K);
     if (N <= 0 || K <= 0 || rb < 0 || ldp < rb) return ORC_EINVAL;
+    long cmax = (fmt == ORC_INT4) ? 7 : 1;
+    uint32_t mask = (1u << code_bits(fmt)) - 1u;
     for (long n = 0; n < N; ++n) {
         uint8_t *row = packed + n * ldp;
         memset(row, 0, (size_t)ldp);
         for (long k = 0; k < K; ++k) {
             int c = codes[n * K + k];
-            uint32_t field;
-            switch (fmt) {
-            case ORC_TERNARY2:
-                if (c < -1 || c > 1) return ORC_EINVAL;
-                field = (uint32_t)c & 3u;
-                row[k / 4] |= (uint8_t)(field << (2 * (k % 4)));
-                break;
-            case ORC_BINARY1:
-                if (c != 1 && c != -1) return ORC_EINVAL;
-                field = (uint32_t)((1 - c) / 2);
-                row[k / 8] |= (uint8_t)(field << (k % 8));
-                break;
-            default: /* INT4 */
-                if (c < -7 || c > 7) return ORC_EINVAL;
-                field = (uint32_t)c & 15u;
-                row[k / 2] |= (uint8_t)(field << (4 * (k % 2)));
-                break;
-            }
+            if (c < -cmax || c > cmax || (fmt == ORC_BINARY1 && c == 0)) return ORC_EINVAL;
+            uint32_t field = (fmt == ORC_BINARY1) ? (uint32_t)((1 - c) / 2) : ((uint32_t)c & mask);
+            long pos = code_bit_pos(fmt, k);
+            row[pos / 8] |= (uint8_t)(field << (pos % 8));
         }
     }
     return ORC_OK;
 }
 
 /* Inverse of orc_pack.  Rejects a reserved pattern inside the logical extent
- * and any non-zero bit outside it [M8.8 §0x06E, §0x0BB "reserved patterns
- * reject"]. */
+ * and any non-zero bit that no code owns [M8.8 §0x06E, §0x0BB "reserved
+ * patterns reject"]. */
 int orc_unpack(const uint8_t *packed, long ldp, long N, long K, int fmt, int8_t *codes)
 {
     long rb = orc_row_bytes(fmt, K);
     if (N <= 0 || K <= 0 || rb < 0 || ldp < rb) return ORC_EINVAL;
+    long b = code_bits(fmt);
+    uint32_t mask = (1u << b) - 1u;
+    uint8_t *owned = (uint8_t *)calloc((size_t)ldp * 8, 1);
+    if (!owned) return ORC_EINVAL;
     int status = ORC_OK;
     for (long n = 0; n < N; ++n) {
         const uint8_t *row = packed + n * ldp;
+        memset(owned, 0, (size_t)ldp * 8);
         for (long k = 0; k < K; ++k) {
+            long pos = code_bit_pos(fmt, k);
+            for (long j = 0; j < b; ++j) owned[pos + j] = 1;
+            uint32_t f = (uint32_t)(row[pos / 8] >> (pos % 8)) & mask;
             int c;
-            if (fmt == ORC_TERNARY2) {
-                uint32_t f = (row[k / 4] >> (2 * (k % 4))) & 3u;
-                if (f == 2u) { status = ORC_ERESERVED; c = 0; }
-                else c = (f == 3u) ? -1 : (int)f;
-            } else if (fmt == ORC_BINARY1) {
-                uint32_t b = (row[k / 8] >> (k % 8)) & 1u;
-                c = b ? -1 : 1;
+            if (fmt == ORC_BINARY1) {
+                c = f ? -1 : 1;
+            } else if (f == (1u << (b - 1))) { /* 10 or 1000: reserved */
+                status = ORC_ERESERVED;
+                c = 0;
             } else {
-                uint32_t f = (row[k / 2] >> (4 * (k % 2))) & 15u;
-                if (f == 8u) { status = ORC_ERESERVED; c = 0; }
-                else c = (f >= 8u) ? (int)f - 16 : (int)f;
+                c = (f >= (1u << (b - 1))) ? (int)f - (int)(1u << b) : (int)f;
             }
             codes[n * K + k] = (int8_t)c;
         }
-        /* padding: bits past code K-1 in the last used byte, then whole bytes */
-        long used_bits = K * (fmt == ORC_TERNARY2 ? 2 : (fmt == ORC_BINARY1 ? 1 : 4));
-        for (long bit = used_bits; bit < ldp * 8; ++bit)
-            if ((row[bit / 8] >> (bit % 8)) & 1u) status = ORC_ERESERVED;
+        for (long bit = 0; bit < ldp * 8; ++bit)
+            if (!owned[bit] && ((row[bit / 8] >> (bit % 8)) & 1u)) status = ORC_ERESERVED;
     }
+    free(owned);
     return status;
 }
 

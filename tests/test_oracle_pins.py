@@ -248,45 +248,65 @@ def test_pack_roundtrip(fmt, alphabet, K):
         assert not packed[:, rb:].any()
 
 
+def test_ternary_four_codes_per_byte():
+    # Atomic-1Bit README: ternary weights are packed four per byte.
+    for K in (16, 64, 2560):
+        assert oracle.row_bytes(oracle.TERNARY2, K) == K // 4
+        assert oracle.row_bytes(oracle.INT4, K) == K // 2
+        assert oracle.row_bytes(oracle.BINARY1, K) == K // 8
+
+
 def test_ternary_byte_table_exhaustive():
-    # Every byte value decodes to 4 valid codes, or is rejected exactly when
-    # one of its 2-bit fields is the reserved pattern.
+    # Every value of one byte decodes to four valid codes, or is rejected
+    # exactly when one of its 2-bit fields is the reserved pattern 10; a field
+    # holds the code as 2-bit two's complement (00 = 0, 01 = +1, 11 = -1).
     for b in range(256):
         fields = [(b >> (2 * j)) & 3 for j in range(4)]
-        codes, st = oracle.unpack(np.array([[b]], np.uint8), 4, oracle.TERNARY2)
+        row = np.zeros((1, 16), np.uint8)
+        row[0, 0] = b
+        codes, st = oracle.unpack(row, 64, oracle.TERNARY2)
         if 2 in fields:
             assert st == oracle.ERESERVED
-        else:
-            assert st == oracle.OK
-            assert set(codes.ravel().tolist()) <= {-1, 0, 1}
-            assert oracle.pack(codes, oracle.TERNARY2)[0, 0] == b
+            continue
+        assert st == oracle.OK
+        got = sorted(codes.ravel().tolist())
+        want = sorted([{0: 0, 1: 1, 3: -1}[f] for f in fields] + [0] * 60)
+        assert got == want
+        assert oracle.pack(codes, oracle.TERNARY2, 16)[0, 0] == b
 
 
 def test_int4_byte_table_exhaustive():
     for b in range(256):
         nib = [b & 15, b >> 4]
-        codes, st = oracle.unpack(np.array([[b]], np.uint8), 2, oracle.INT4)
+        row = np.zeros((1, 16), np.uint8)
+        row[0, 0] = b
+        codes, st = oracle.unpack(row, 32, oracle.INT4)
         if 8 in nib:
             assert st == oracle.ERESERVED
-        else:
-            assert st == oracle.OK
-            # two's complement: value = nibble - 16 when the top bit is set
-            assert codes.ravel().tolist() == [v - 16 if v >= 8 else v for v in nib]
-            assert oracle.pack(codes, oracle.INT4)[0, 0] == b
+            continue
+        assert st == oracle.OK
+        # two's complement: value = nibble - 16 when the top bit is set
+        want = sorted([v - 16 if v >= 8 else v for v in nib] + [0] * 30)
+        assert sorted(codes.ravel().tolist()) == want
+        assert oracle.pack(codes, oracle.INT4, 16)[0, 0] == b
 
 
-@pytest.mark.parametrize("fmt,K", [(oracle.TERNARY2, 5), (oracle.BINARY1, 5), (oracle.INT4, 5)])
-def test_nonzero_padding_rejected(fmt, K):
-    codes = np.ones((2, K), np.int8)
-    packed = oracle.pack(codes, fmt, oracle.row_bytes(fmt, K) + 16)
-    bad = packed.copy()
-    bad[1, -1] = 1
-    assert oracle.unpack(bad, K, fmt)[1] == oracle.ERESERVED
-    bad = packed.copy()
-    bits = {oracle.TERNARY2: 2, oracle.BINARY1: 1, oracle.INT4: 4}[fmt] * K
-    bad[0, bits // 8] |= 1 << (bits % 8)  # first bit past the last code
-    assert oracle.unpack(bad, K, fmt)[1] == oracle.ERESERVED
-
+@pytest.mark.parametrize("fmt", [oracle.TERNARY2, oracle.BINARY1, oracle.INT4])
+@pytest.mark.parametrize("K", [5, 13, 33])
+def test_unowned_bits_rejected(fmt, K):
+    # Packing all -1 sets every bit a code owns; any other bit of the row
+    # (inside the last partly used word, or in the stride padding) must be
+    # rejected as non-canonical.
+    codes = -np.ones((2, K), np.int8)
+    ldp = oracle.row_bytes(fmt, K) + 16
+    packed = oracle.pack(codes, fmt, ldp)
+    assert oracle.unpack(packed, K, fmt)[1] == oracle.OK
+    free = np.argwhere(np.unpackbits(packed[1], bitorder="little") == 0).ravel()
+    assert free.size > 0
+    for bit in (free[0], free[-1]):
+        bad = packed.copy()
+        bad[1, bit // 8] |= np.uint8(1 << (bit % 8))
+        assert oracle.unpack(bad, K, fmt)[1] == oracle.ERESERVED
 
 # --------------------------------------------------------------------------
 # activation quantiser
