@@ -1,0 +1,179 @@
+"""B200-native low-bit-weight linear layer (BitNet-style BitLinear).
+
+The operator and its sources are stated in ``include/lowbit.h``; every step
+runs in the CUDA kernels of ``liblowbit.so`` (sm_100a).  This module only
+marshals arguments: it takes torch tensors (device memory and the current
+stream come from PyTorch), calls the C ABI through ctypes, and turns a
+non-OK status into ``LowbitError``.  There is no CPU fallback: if the built
+library is missing, importing a function raises.
+
+Functions carry the ABI's names::
+
+    packed, s_w = lowbit_pack(w, fmt, eps=1e-5)
+    codes       = lowbit_unpack(packed, K, fmt)
+    q, s_x      = lowbit_act_quant(x, eps=0.0)
+    y           = lowbit_linear(q, s_x, packed, s_w, fmt, N, out_dtype)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+TERNARY2, BINARY1, INT4 = 0, 1, 2
+F32, BF16, I32 = 0, 1, 2
+
+STATUS_NAMES = {
+    0: "LOWBIT_OK", 1: "LOWBIT_ERR_INVALID_ARG", 2: "LOWBIT_ERR_ALIGNMENT", 3: "LOWBIT_ERR_UNSUPPORTED",
+    4: "LOWBIT_ERR_OVERFLOW_BOUND", 5: "LOWBIT_ERR_NONFINITE", 6: "LOWBIT_ERR_RESERVED_CODE",
+    7: "LOWBIT_ERR_TIMEOUT", 8: "LOWBIT_ERR_CUDA",
+}
+OK, ERR_INVALID_ARG, ERR_ALIGNMENT, ERR_UNSUPPORTED, ERR_OVERFLOW_BOUND = 0, 1, 2, 3, 4
+ERR_NONFINITE, ERR_RESERVED_CODE, ERR_TIMEOUT, ERR_CUDA = 5, 6, 7, 8
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblowbit.so")
+
+# (name, restype, argtypes) of every entry point declared in include/lowbit.h
+_P, _I64, _I32, _F, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+ABI = {
+    "lowbit_packed_row_bytes": (_SZ, [_I32, _I64]),
+    "lowbit_packed_ld": (_SZ, [_I32, _I64]),
+    "lowbit_scale_count": (_I64, [_I32, _I64]),
+    "lowbit_max_k": (_I64, [_I32]),
+    "lowbit_pack_workspace_bytes": (_SZ, [_I32, _I64]),
+    "lowbit_pack": (_I32, [_P, _I64, _I64, _I64, _I32, _F, _P, _I64, _P, _P, _SZ, _P, _P]),
+    "lowbit_unpack": (_I32, [_P, _I64, _I64, _I64, _I32, _P, _I64, _P, _P]),
+    "lowbit_act_quant": (_I32, [_P, _I32, _I64, _I64, _I64, _F, _P, _I64, _P, _P, _P]),
+    "lowbit_linear": (_I32, [_P, _I64, _P, _I64, _I64, _P, _I64, _P, _I32, _I64, _P, _I32, _I64, _P, _P]),
+    "lowbit_linear_path": (_I32, [_P, _I64, _P, _I64, _I64, _P, _I64, _P, _I32, _I64, _P, _I32, _I64, _I32,
+                                  _P, _P]),
+    "lowbit_status_string": (ctypes.c_char_p, [_I32]),
+    "lowbit_version": (_I32, []),
+}
+
+
+class LowbitError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m binary_weight_transformer_b200._build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in ABI.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _check(st: int, what: str):
+    if st != OK:
+        raise LowbitError(st, what)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def packed_row_bytes(fmt: int, K: int) -> int:
+    return int(lib().lowbit_packed_row_bytes(fmt, K))
+
+
+def packed_ld(fmt: int, K: int) -> int:
+    return int(lib().lowbit_packed_ld(fmt, K))
+
+
+def scale_count(fmt: int, N: int) -> int:
+    return int(lib().lowbit_scale_count(fmt, N))
+
+
+def max_k(fmt: int) -> int:
+    return int(lib().lowbit_max_k(fmt))
+
+
+def status_flags(status_tensor) -> list[int]:
+    """Decode a device status word (bit 1<<s per status s) into status values."""
+    v = int(status_tensor.item())
+    return [s for s in range(1, 9) if v & (1 << s)]
+
+
+def lowbit_pack(w, fmt: int, eps: float = 1e-5, packed=None, s_w=None, ldp: int | None = None,
+                workspace=None, status=None, stream=None):
+    """Quantise and pack fp32 weights w[N, K] (CUDA tensor, unit inner stride)."""
+    import torch
+    N, K = w.shape
+    if ldp is None:
+        ldp = packed_ld(fmt, K)
+    if packed is None:
+        packed = torch.empty((N, ldp), dtype=torch.uint8, device=w.device)
+    if s_w is None:
+        s_w = torch.empty(scale_count(fmt, N), dtype=torch.float32, device=w.device)
+    need = int(lib().lowbit_pack_workspace_bytes(fmt, N))
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=w.device)
+    st = lib().lowbit_pack(_ptr(w), N, K, w.stride(0), fmt, eps, _ptr(packed), packed.stride(0), _ptr(s_w),
+                           _ptr(workspace), need, _ptr(status), _stream(stream))
+    _check(st, "lowbit_pack")
+    return packed, s_w
+
+
+def lowbit_unpack(packed, K: int, fmt: int, codes=None, status=None, stream=None):
+    import torch
+    N = packed.shape[0]
+    if codes is None:
+        codes = torch.empty((N, K), dtype=torch.int8, device=packed.device)
+    st = lib().lowbit_unpack(_ptr(packed), packed.stride(0), N, K, fmt, _ptr(codes), codes.stride(0),
+                             _ptr(status), _stream(stream))
+    _check(st, "lowbit_unpack")
+    return codes
+
+
+def lowbit_act_quant(x, eps: float = 0.0, q=None, s_x=None, status=None, stream=None):
+    """Per-token absmax int8 codes of x[M, K] (fp32 or bf16 CUDA tensor)."""
+    import torch
+    M, K = x.shape
+    xdt = {torch.float32: F32, torch.bfloat16: BF16}[x.dtype]
+    if q is None:
+        q = torch.empty((M, (K + 15) // 16 * 16), dtype=torch.int8, device=x.device)
+    if s_x is None:
+        s_x = torch.empty(M, dtype=torch.float32, device=x.device)
+    st = lib().lowbit_act_quant(_ptr(x), xdt, M, K, x.stride(0), eps, _ptr(q), q.stride(0), _ptr(s_x),
+                                _ptr(status), _stream(stream))
+    _check(st, "lowbit_act_quant")
+    return q, s_x
+
+
+def lowbit_linear(q, s_x, packed, s_w, fmt: int, N: int, out_dtype: int = F32, K: int | None = None,
+                  y=None, status=None, stream=None, path: int = 0):
+    """y[M, N] from int8 codes q[M, >=K] and a packed artifact (see lowbit.h).
+
+    ``path`` 0 picks the kernel by M; 1 forces the GEMV, 2 the tensor-core GEMM."""
+    import torch
+    M = q.shape[0]
+    if K is None:
+        K = q.shape[1]
+    if y is None:
+        dt = {F32: torch.float32, BF16: torch.bfloat16, I32: torch.int32}[out_dtype]
+        y = torch.empty((M, N), dtype=dt, device=q.device)
+    st = lib().lowbit_linear_path(_ptr(q), q.stride(0), _ptr(s_x), M, K, _ptr(packed), packed.stride(0),
+                                  _ptr(s_w), fmt, N, _ptr(y), out_dtype, y.stride(0), path, _ptr(status),
+                                  _stream(stream))
+    _check(st, "lowbit_linear")
+    return y

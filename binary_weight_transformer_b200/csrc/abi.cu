@@ -1,0 +1,226 @@
+// abi.cu -- the C ABI: argument checks on the host, then kernel dispatch.
+//
+// Every check here runs before any launch, so a rejected call launches
+// nothing.  The operator definitions are stated in include/lowbit.h.
+#include <climits>
+#include <cstdio>
+
+#include "lowbit_internal.cuh"
+
+namespace lowbit {
+
+lowbit_status act_quant_launch(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx, float eps,
+                               int8_t *q, int64_t ldq, float *s_x, int32_t *status, cudaStream_t st);
+lowbit_status pack_launch(const float *w, int64_t N, int64_t K, int64_t ldw, lowbit_format f, float eps,
+                          uint8_t *packed, int64_t ldp, float *s_w, void *workspace, int32_t *status,
+                          cudaStream_t st);
+lowbit_status unpack_launch(const uint8_t *packed, int64_t ldp, int64_t N, int64_t K, lowbit_format f,
+                            int8_t *codes, int64_t ldc, int32_t *status, cudaStream_t st);
+lowbit_status gemv_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
+                          const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
+                          lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, cudaStream_t st);
+lowbit_status gemm_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
+                          const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
+                          lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int32_t *status,
+                          cudaStream_t st);
+
+lowbit_status launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
+}
+
+namespace {
+
+struct DeviceInfo {
+    int sms = 0;
+    int major = 0;
+    int minor = 0;
+    bool ok = false;
+};
+
+const DeviceInfo &device_info()
+{
+    static DeviceInfo cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        static DeviceInfo none;
+        return none;
+    }
+    DeviceInfo &d = cache[dev];
+    if (!d.ok) {
+        cudaDeviceProp p;
+        if (cudaGetDeviceProperties(&p, dev) == cudaSuccess) {
+            d.sms = p.multiProcessorCount;
+            d.major = p.major;
+            d.minor = p.minor;
+            d.ok = true;
+        }
+    }
+    return d;
+}
+
+// The kernels are built for sm_100a only.
+lowbit_status check_device()
+{
+    const DeviceInfo &d = device_info();
+    if (!d.ok) return LOWBIT_ERR_CUDA;
+    if (d.major != 10 || d.minor != 0) return LOWBIT_ERR_UNSUPPORTED;
+    return LOWBIT_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool valid_format(lowbit_format f) { return f == LOWBIT_TERNARY2 || f == LOWBIT_BINARY1 || f == LOWBIT_INT4; }
+
+}  // namespace
+
+int device_sm_count()
+{
+    const DeviceInfo &d = device_info();
+    return d.ok ? d.sms : 148;
+}
+
+}  // namespace lowbit
+
+using namespace lowbit;
+
+extern "C" {
+
+size_t lowbit_packed_row_bytes(lowbit_format f, int64_t K)
+{
+    if (K <= 0) return 0;
+    switch (f) {
+    case LOWBIT_TERNARY2: return static_cast<size_t>(4 * ((K + 15) / 16));
+    case LOWBIT_BINARY1: return static_cast<size_t>((K + 7) / 8);
+    case LOWBIT_INT4: return static_cast<size_t>(4 * ((K + 7) / 8));
+    default: return 0;
+    }
+}
+
+size_t lowbit_packed_ld(lowbit_format f, int64_t K)
+{
+    const size_t rb = lowbit_packed_row_bytes(f, K);
+    return (rb + 15) / 16 * 16;
+}
+
+int64_t lowbit_scale_count(lowbit_format f, int64_t N)
+{
+    if (N <= 0 || !valid_format(f)) return 0;
+    return f == LOWBIT_TERNARY2 ? 1 : N;
+}
+
+int64_t lowbit_max_k(lowbit_format f)
+{
+    // The kernels accumulate (c << S) * q: 2^31 / (128 * 64) - 1 for ternary
+    // and binary, 2^31 / (128 * 16 * 7) for 4-bit codes.
+    switch (f) {
+    case LOWBIT_TERNARY2:
+    case LOWBIT_BINARY1: return (static_cast<int64_t>(INT32_MAX) / (128 * 64));
+    case LOWBIT_INT4: return (static_cast<int64_t>(INT32_MAX) / (128 * 16 * 7));
+    default: return 0;
+    }
+}
+
+size_t lowbit_pack_workspace_bytes(lowbit_format f, int64_t N)
+{
+    if (f != LOWBIT_TERNARY2 || N <= 0) return 0;
+    return (static_cast<size_t>(N) * 8 + 255) / 256 * 256;
+}
+
+lowbit_status lowbit_pack(const float *w, int64_t N, int64_t K, int64_t ldw, lowbit_format f, float eps,
+                          uint8_t *packed, int64_t ldp, float *s_w, void *workspace, size_t workspace_bytes,
+                          int32_t *status_dev, void *stream)
+{
+    if (!valid_format(f) || w == nullptr || packed == nullptr || s_w == nullptr) return LOWBIT_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0 || ldw < K || !(eps >= 0.0f) || eps > 3.0e38f) return LOWBIT_ERR_INVALID_ARG;
+    if (ldp < static_cast<int64_t>(lowbit_packed_row_bytes(f, K))) return LOWBIT_ERR_INVALID_ARG;
+    if (N > INT32_MAX || K > INT32_MAX) return LOWBIT_ERR_INVALID_ARG;
+    if (ldp % 16 != 0 || !aligned(packed, 16) || !aligned(w, 4) || !aligned(s_w, 4)) return LOWBIT_ERR_ALIGNMENT;
+    const size_t need = lowbit_pack_workspace_bytes(f, N);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LOWBIT_ERR_INVALID_ARG;
+    if (need > 0 && !aligned(workspace, 8)) return LOWBIT_ERR_ALIGNMENT;
+    const lowbit_status d = check_device();
+    if (d != LOWBIT_OK) return d;
+    return pack_launch(w, N, K, ldw, f, eps, packed, ldp, s_w, workspace, status_dev,
+                       static_cast<cudaStream_t>(stream));
+}
+
+lowbit_status lowbit_unpack(const uint8_t *packed, int64_t ldp, int64_t N, int64_t K, lowbit_format f,
+                            int8_t *codes, int64_t ldc, int32_t *status_dev, void *stream)
+{
+    if (!valid_format(f) || packed == nullptr || codes == nullptr) return LOWBIT_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0 || ldc < K || ldp < static_cast<int64_t>(lowbit_packed_row_bytes(f, K)))
+        return LOWBIT_ERR_INVALID_ARG;
+    if (ldp % 16 != 0 || !aligned(packed, 16)) return LOWBIT_ERR_ALIGNMENT;
+    const lowbit_status d = check_device();
+    if (d != LOWBIT_OK) return d;
+    return unpack_launch(packed, ldp, N, K, f, codes, ldc, status_dev, static_cast<cudaStream_t>(stream));
+}
+
+lowbit_status lowbit_act_quant(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx, float eps,
+                               int8_t *q, int64_t ldq, float *s_x, int32_t *status_dev, void *stream)
+{
+    if (x == nullptr || q == nullptr || s_x == nullptr) return LOWBIT_ERR_INVALID_ARG;
+    if (xdt != LOWBIT_F32 && xdt != LOWBIT_BF16) return LOWBIT_ERR_INVALID_ARG;
+    if (M <= 0 || K <= 0 || ldx < K || ldq < K || !(eps >= 0.0f) || eps > 3.0e38f) return LOWBIT_ERR_INVALID_ARG;
+    if (M > INT32_MAX) return LOWBIT_ERR_INVALID_ARG;
+    const int64_t esz = xdt == LOWBIT_F32 ? 4 : 2;
+    if (!aligned(x, 16) || (ldx * esz) % 16 != 0 || !aligned(q, 16) || ldq % 16 != 0 || !aligned(s_x, 4))
+        return LOWBIT_ERR_ALIGNMENT;
+    const lowbit_status d = check_device();
+    if (d != LOWBIT_OK) return d;
+    return act_quant_launch(x, xdt, M, K, ldx, eps, q, ldq, s_x, status_dev, static_cast<cudaStream_t>(stream));
+}
+
+lowbit_status lowbit_linear_path(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
+                                 const uint8_t *packed, int64_t ldp, const float *s_w, lowbit_format f, int64_t N,
+                                 void *y, lowbit_dtype ydt, int64_t ldy, int path, int32_t *status_dev,
+                                 void *stream)
+{
+    if (!valid_format(f) || q == nullptr || s_x == nullptr || packed == nullptr || s_w == nullptr || y == nullptr)
+        return LOWBIT_ERR_INVALID_ARG;
+    if (ydt != LOWBIT_F32 && ydt != LOWBIT_BF16 && ydt != LOWBIT_I32) return LOWBIT_ERR_INVALID_ARG;
+    if (path < 0 || path > 2) return LOWBIT_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0 || ldq < K || ldy < N) return LOWBIT_ERR_INVALID_ARG;
+    if (M > INT32_MAX || N > INT32_MAX) return LOWBIT_ERR_INVALID_ARG;
+    const int64_t rb = static_cast<int64_t>(lowbit_packed_row_bytes(f, K));
+    if (ldp < rb) return LOWBIT_ERR_INVALID_ARG;
+    if (K > lowbit_max_k(f)) return LOWBIT_ERR_OVERFLOW_BOUND;
+    const int64_t esz = ydt == LOWBIT_BF16 ? 2 : 4;
+    if (!aligned(q, 16) || ldq % 16 != 0 || !aligned(packed, 16) || ldp % 16 != 0 || !aligned(s_x, 4) ||
+        !aligned(s_w, 4) || !aligned(y, static_cast<uintptr_t>(esz)))
+        return LOWBIT_ERR_ALIGNMENT;
+    const lowbit_status d = check_device();
+    if (d != LOWBIT_OK) return d;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool use_gemv = path == 1 || (path == 0 && M <= 16);
+    if (use_gemv) return gemv_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, st);
+    return gemm_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, status_dev, st);
+}
+
+lowbit_status lowbit_linear(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
+                            const uint8_t *packed, int64_t ldp, const float *s_w, lowbit_format f, int64_t N,
+                            void *y, lowbit_dtype ydt, int64_t ldy, int32_t *status_dev, void *stream)
+{
+    return lowbit_linear_path(q, ldq, s_x, M, K, packed, ldp, s_w, f, N, y, ydt, ldy, 0, status_dev, stream);
+}
+
+const char *lowbit_status_string(lowbit_status s)
+{
+    switch (s) {
+    case LOWBIT_OK: return "ok";
+    case LOWBIT_ERR_INVALID_ARG: return "invalid argument";
+    case LOWBIT_ERR_ALIGNMENT: return "misaligned pointer or leading dimension";
+    case LOWBIT_ERR_UNSUPPORTED: return "unsupported (needs an sm_100 device)";
+    case LOWBIT_ERR_OVERFLOW_BOUND: return "K exceeds the int32 accumulator bound";
+    case LOWBIT_ERR_NONFINITE: return "non-finite input";
+    case LOWBIT_ERR_RESERVED_CODE: return "reserved code pattern or non-zero unowned bit";
+    case LOWBIT_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case LOWBIT_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+    }
+}
+
+int lowbit_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,216 @@
+// act_quant.cu -- per-token absmax int8 activation codes.
+//
+// "M8.8 - Native Binary and Ternary Transformers", section 0x05C (signed
+// per-token A8: gamma_t = max|x_t|, reconstruction scale gamma_t/127, an
+// all-zero row has zero codes and zero scale) and section 0x02C/0x02E (round
+// to nearest, ties to even).  Per element: q = clip(rint((x*127) /
+// (gamma_t + eps)), -128, 127) with one fp32 multiply and one IEEE fp32
+// divide.
+//
+// One HBM pass: a group of TPR threads owns a row, loads it into registers
+// with 16-byte non-allocating loads, reduces the row's absmax with warp
+// shuffles (plus shared memory across warps when TPR > 32), then quantises
+// from registers.  The max is taken on the fp32 bit pattern of |x|, which
+// orders non-negative floats exactly and puts Inf/NaN above every finite
+// value, so one test of gamma_t detects a non-finite row.
+#include "lowbit_internal.cuh"
+
+namespace lowbit {
+namespace {
+
+constexpr int kVPT = 8;  // 16-byte vectors per thread held in registers
+
+template <typename T> struct In;
+template <> struct In<float> {
+    static constexpr int kPerVec = 4;
+    __device__ static float get(const uint4 &v, int i)
+    {
+        uint32_t w = (&v.x)[i];
+        return __uint_as_float(w);
+    }
+    __device__ static float scalar(const void *p, int64_t i)
+    {
+        return static_cast<const float *>(p)[i];
+    }
+};
+template <> struct In<__nv_bfloat16> {
+    static constexpr int kPerVec = 8;
+    __device__ static float get(const uint4 &v, int i)
+    {
+        uint32_t w = (&v.x)[i >> 1];
+        uint32_t h = (i & 1) ? (w >> 16) : (w & 0xffffu);
+        return __uint_as_float(h << 16);
+    }
+    __device__ static float scalar(const void *p, int64_t i)
+    {
+        uint16_t h = static_cast<const uint16_t *>(p)[i];
+        return __uint_as_float(static_cast<uint32_t>(h) << 16);
+    }
+};
+
+__device__ __forceinline__ int8_t quant_one(float x, float d)
+{
+    float t = rintf(__fdiv_rn(__fmul_rn(x, 127.0f), d));
+    t = fminf(fmaxf(t, -128.0f), 127.0f);
+    return static_cast<int8_t>(static_cast<int>(t));
+}
+
+// Max of a uint32 over the TPR threads that own one row.
+template <int TPR>
+__device__ __forceinline__ uint32_t row_max(uint32_t v, uint32_t *red)
+{
+#pragma unroll
+    for (int o = (TPR < 32 ? TPR : 32) / 2; o > 0; o >>= 1)
+        v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if constexpr (TPR > 32) {
+        constexpr int kWarps = TPR / 32;
+        const int lane = threadIdx.x & 31;
+        const int warp_in_row = (threadIdx.x % TPR) / 32;
+        const int row_slot = threadIdx.x / TPR;
+        if (lane == 0) red[row_slot * kWarps + warp_in_row] = v;
+        __syncthreads();
+        v = red[row_slot * kWarps];
+#pragma unroll
+        for (int i = 1; i < kWarps; ++i) v = max(v, red[row_slot * kWarps + i]);
+    }
+    return v;
+}
+
+// Rows whose 16-byte vectors fit TPR*kVPT registers: one global read.
+template <typename T, int TPR>
+__global__ void __launch_bounds__(TPR > 256 ? TPR : 256)
+act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, float eps,
+               int8_t *__restrict__ q, int64_t ldq, float *__restrict__ s_x, int32_t *status)
+{
+    constexpr int kThreads = TPR > 256 ? TPR : 256;
+    constexpr int kRows = kThreads / TPR;
+    constexpr int E = In<T>::kPerVec;
+    __shared__ uint32_t red[kThreads / 32];
+
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * kRows + threadIdx.x / TPR;
+    const int r = threadIdx.x % TPR;
+    const bool live = row < M;
+    const int64_t nvec = K / E;
+    const char *xrow = static_cast<const char *>(x) + (live ? row : 0) * ldx * sizeof(T);
+
+    uint4 buf[kVPT];
+    uint32_t amax = 0;
+#pragma unroll
+    for (int i = 0; i < kVPT; ++i) {
+        const int64_t v = r + static_cast<int64_t>(i) * TPR;
+        if (live && v < nvec) {
+            buf[i] = ld_stream_u4(xrow + v * 16);
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                amax = max(amax, __float_as_uint(In<T>::get(buf[i], e)) & 0x7fffffffu);
+        }
+    }
+    // Tail elements past the last whole vector, one per thread.
+    const int64_t tail0 = nvec * E;
+    float tail_x = 0.0f;
+    const bool has_tail = live && (tail0 + r < K) && r < E;
+    if (has_tail) {
+        tail_x = In<T>::scalar(xrow, tail0 + r);
+        amax = max(amax, __float_as_uint(tail_x) & 0x7fffffffu);
+    }
+    amax = row_max<TPR>(amax, red);
+    if (!live) return;
+
+    const float g = __uint_as_float(amax);
+    const bool bad = !finite_bits(amax) || !finite_bits(__float_as_uint(__fmul_rn(g, 127.0f)));
+    if (bad && r == 0) report(status, LOWBIT_ERR_NONFINITE);
+    const float d = __fadd_rn(g, eps);
+    int8_t *qrow = q + row * ldq;
+
+#pragma unroll
+    for (int i = 0; i < kVPT; ++i) {
+        const int64_t v = r + static_cast<int64_t>(i) * TPR;
+        if (v < nvec) {
+            if constexpr (E == 4) {
+                uint32_t out = 0;
+                if (amax != 0) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        out |= static_cast<uint32_t>(static_cast<uint8_t>(quant_one(In<T>::get(buf[i], e), d))) << (8 * e);
+                }
+                *reinterpret_cast<uint32_t *>(qrow + v * 4) = out;
+            } else {
+                uint32_t lo = 0, hi = 0;
+                if (amax != 0) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        lo |= static_cast<uint32_t>(static_cast<uint8_t>(quant_one(In<T>::get(buf[i], e), d))) << (8 * e);
+                        hi |= static_cast<uint32_t>(static_cast<uint8_t>(quant_one(In<T>::get(buf[i], e + 4), d))) << (8 * e);
+                    }
+                }
+                *reinterpret_cast<uint2 *>(qrow + v * 8) = make_uint2(lo, hi);
+            }
+        }
+    }
+    if (has_tail) qrow[tail0 + r] = amax != 0 ? quant_one(tail_x, d) : 0;
+    if (r == 0) s_x[row] = amax != 0 ? __fdiv_rn(g, 127.0f) : 0.0f;
+}
+
+// Rows too long for registers: a max pass, then a quantise pass (the second
+// read mostly hits L2).  One 256-thread block per row.
+template <typename T>
+__global__ void __launch_bounds__(256)
+act_quant_long(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, float eps,
+               int8_t *__restrict__ q, int64_t ldq, float *__restrict__ s_x, int32_t *status)
+{
+    __shared__ uint32_t red[8];
+    const int64_t row = blockIdx.x;
+    const char *xrow = static_cast<const char *>(x) + row * ldx * sizeof(T);
+    uint32_t amax = 0;
+    for (int64_t k = threadIdx.x; k < K; k += 256)
+        amax = max(amax, __float_as_uint(In<T>::scalar(xrow, k)) & 0x7fffffffu);
+    amax = row_max<256>(amax, red);
+    const float g = __uint_as_float(amax);
+    const bool bad = !finite_bits(amax) || !finite_bits(__float_as_uint(__fmul_rn(g, 127.0f)));
+    if (bad && threadIdx.x == 0) report(status, LOWBIT_ERR_NONFINITE);
+    const float d = __fadd_rn(g, eps);
+    int8_t *qrow = q + row * ldq;
+    for (int64_t k = threadIdx.x; k < K; k += 256)
+        qrow[k] = amax != 0 ? quant_one(In<T>::scalar(xrow, k), d) : 0;
+    if (threadIdx.x == 0) s_x[row] = amax != 0 ? __fdiv_rn(g, 127.0f) : 0.0f;
+}
+
+template <typename T>
+lowbit_status launch(const void *x, int64_t M, int64_t K, int64_t ldx, float eps, int8_t *q,
+                     int64_t ldq, float *s_x, int32_t *status, cudaStream_t st)
+{
+    constexpr int E = In<T>::kPerVec;
+    const int64_t nvec = K / E;
+    auto grid_for = [&](int tpr) {
+        const int rows = (tpr > 256 ? tpr : 256) / tpr;
+        return static_cast<unsigned>((M + rows - 1) / rows);
+    };
+#define LOWBIT_AQ(TPR)                                                                          \
+    if (nvec <= static_cast<int64_t>(TPR) * kVPT) {                                             \
+        act_quant_regs<T, TPR><<<grid_for(TPR), (TPR > 256 ? TPR : 256), 0, st>>>(              \
+            x, M, K, ldx, eps, q, ldq, s_x, status);                                            \
+        return launch_status();                                                                 \
+    }
+    LOWBIT_AQ(8)
+    LOWBIT_AQ(32)
+    LOWBIT_AQ(64)
+    LOWBIT_AQ(128)
+    LOWBIT_AQ(256)
+    LOWBIT_AQ(512)
+    LOWBIT_AQ(1024)
+#undef LOWBIT_AQ
+    act_quant_long<T><<<static_cast<unsigned>(M), 256, 0, st>>>(x, M, K, ldx, eps, q, ldq, s_x, status);
+    return launch_status();
+}
+
+}  // namespace
+
+lowbit_status act_quant_launch(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                               float eps, int8_t *q, int64_t ldq, float *s_x, int32_t *status,
+                               cudaStream_t st)
+{
+    if (xdt == LOWBIT_F32) return launch<float>(x, M, K, ldx, eps, q, ldq, s_x, status, st);
+    return launch<__nv_bfloat16>(x, M, K, ldx, eps, q, ldq, s_x, status, st);
+}
+
+}  // namespace lowbit

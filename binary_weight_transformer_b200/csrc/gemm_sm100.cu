@@ -1,0 +1,537 @@
+// gemm_sm100.cu -- tensor-core GEMM for many tokens (prefill), sm_100a.
+//
+// "M8.8 - Native Binary and Ternary Transformers" 0x09B: prefill has a large
+// token dimension and is a dense contraction, so the integer dot runs on the
+// 5th-generation tensor cores (tcgen05.mma kind::i8, s8 x s8 -> s32 in tensor
+// memory).  0x09A: unpacking to bytes and calling a generic GEMM would not
+// execute the intended operator, so the kernel consumes the packed artifact
+// directly: packed weight tiles arrive in shared memory by TMA and are
+// expanded there, tile by tile, into the int8 operand the MMA reads; the
+// unpacked matrix never exists in global memory.
+//
+// CTA tile 128 tokens x 256 output features, K step 128.  Warp roles:
+//   warp 0      TMA producer: activation tile (128x128 int8, 128B swizzle)
+//               and packed weight tile (256 rows x 128 codes) per stage;
+//   warp 1      TMEM allocation and the MMA issuer (one thread);
+//   warps 2-5   expanders: packed codes -> int8 (c << S) in the UMMA
+//               K-major 128B-swizzled layout;
+//   warps 6-9   epilogue: tcgen05.ld of the s32 accumulators, acc >> S,
+//               y = float(acc) * (s_w * s_x), fp32 / bf16 / int32 stores.
+// Accumulators are double-buffered in tensor memory (2 x 256 columns) so the
+// epilogue of one tile overlaps the MMAs of the next; CTAs are persistent.
+// Every mbarrier wait is bounded in time; on expiry the CTA records
+// LOWBIT_ERR_TIMEOUT, drains its copies and MMAs, frees tensor memory and
+// returns.
+#include <cuda.h>
+
+#include "lowbit_internal.cuh"
+
+namespace lowbit {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;
+constexpr int UMMA_K = 32;
+constexpr int A_BYTES = BM * BK;
+constexpr int E_BYTES = BN * BK;
+constexpr int kThreads = 320;
+constexpr int kExpThreads = 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
+
+template <int FMT> constexpr int packed_bytes_per_kblock() { return BK * Fmt<FMT>::kBits / 8; }
+template <int FMT> constexpr int stages() { return FMT == kI4 ? 3 : 4; }
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long globaltimer()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+
+// Bounded wait: true once the phase with `parity` has completed; false if the
+// CTA aborted or `limit_ns` passed (then the timeout is recorded).
+__device__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int32_t *status,
+                         unsigned long long limit_ns = kWaitNs)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > limit_ns) {
+                *abort_flag = 1;
+                report(status, LOWBIT_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 consecutive 32-bit accumulator columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&v)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, K-major, 128-byte swizzle: rows of 128 B,
+// groups of 8 rows 1024 B apart (stride byte offset), version 1 (sm_100).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(1u) << 16;              // leading byte offset (unused for swizzled K-major)
+    d |= static_cast<uint64_t>(1024u >> 4) << 32;      // stride byte offset
+    d |= static_cast<uint64_t>(1u) << 46;              // descriptor version
+    d |= static_cast<uint64_t>(2u) << 61;              // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor: s32 accumulate, s8 x s8, both K-major, M=128, N=256.
+constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+                            (static_cast<uint32_t>(BM >> 4) << 24);
+
+// ---------------------------------------------------------------------------
+// Expansion of one stage: 256 rows x 128 codes, one (row, 16-code chunk) per
+// thread and step; output row r chunk c goes to r*128 + ((c ^ (r%8)) * 16),
+// the 128B-swizzle pattern the TMA uses for the activation tile.
+// ---------------------------------------------------------------------------
+template <int FMT>
+__device__ __forceinline__ void expand_stage(const uint8_t *P, uint8_t *E, int et)
+{
+    constexpr int PB = packed_bytes_per_kblock<FMT>();
+    const int c = et & 7;
+#pragma unroll 4
+    for (int r = et >> 3; r < BN; r += kExpThreads / 8) {
+        uint4 out;
+        if constexpr (FMT == kT2) {
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(P + r * PB + c * 4);
+            out = make_uint4(t2_expand(w, 0), t2_expand(w, 1), t2_expand(w, 2), t2_expand(w, 3));
+        } else if constexpr (FMT == kI4) {
+            const uint2 w = *reinterpret_cast<const uint2 *>(P + r * PB + c * 8);
+            out = make_uint4(i4_expand(w.x, 0), i4_expand(w.x, 1), i4_expand(w.y, 0), i4_expand(w.y, 1));
+        } else {
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(P + r * PB + (c >> 1) * 4) >> (16 * (c & 1));
+            out = make_uint4(b1_expand_nibble(w & 0xFu), b1_expand_nibble((w >> 4) & 0xFu),
+                             b1_expand_nibble((w >> 8) & 0xFu), b1_expand_nibble((w >> 12) & 0xFu));
+        }
+        *reinterpret_cast<uint4 *>(E + r * 128 + ((c ^ (r & 7)) << 4)) = out;
+    }
+}
+
+template <int OUT>
+__device__ __forceinline__ void store_row32(void *y, int64_t row, int64_t ldy, int64_t n0, int64_t N,
+                                            const uint32_t (&v)[32], int shift, const float *s_w, bool sw_per_row,
+                                            float sx, bool vec_ok)
+{
+    const bool full = (n0 + 32 <= N);
+    if constexpr (OUT == LOWBIT_I32) {
+        int32_t *yr = static_cast<int32_t *>(y) + row * ldy + n0;
+        if (full && vec_ok) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<int4 *>(yr + i) =
+                    make_int4(static_cast<int32_t>(v[i]) >> shift, static_cast<int32_t>(v[i + 1]) >> shift,
+                              static_cast<int32_t>(v[i + 2]) >> shift, static_cast<int32_t>(v[i + 3]) >> shift);
+        } else {
+            for (int i = 0; i < 32 && n0 + i < N; ++i) yr[i] = static_cast<int32_t>(v[i]) >> shift;
+        }
+    } else {
+        float f[32];
+        const float sw0 = s_w[0];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float sw = sw_per_row ? ((n0 + i < N) ? __ldg(s_w + n0 + i) : 0.0f) : sw0;
+            f[i] = rescale(static_cast<int32_t>(v[i]) >> shift, sw, sx);
+        }
+        if constexpr (OUT == LOWBIT_F32) {
+            float *yr = static_cast<float *>(y) + row * ldy + n0;
+            if (full && vec_ok) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 4)
+                    *reinterpret_cast<float4 *>(yr + i) = make_float4(f[i], f[i + 1], f[i + 2], f[i + 3]);
+            } else {
+                for (int i = 0; i < 32 && n0 + i < N; ++i) yr[i] = f[i];
+            }
+        } else {
+            __nv_bfloat16 *yr = static_cast<__nv_bfloat16 *>(y) + row * ldy + n0;
+            if (full && vec_ok) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 8) {
+                    uint4 pk;
+                    uint32_t *pw = &pk.x;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(f[i + 2 * j], f[i + 2 * j + 1]);
+                        pw[j] = *reinterpret_cast<const uint32_t *>(&b2);
+                    }
+                    *reinterpret_cast<uint4 *>(yr + i) = pk;
+                }
+            } else {
+                for (int i = 0; i < 32 && n0 + i < N; ++i) yr[i] = __float2bfloat16_rn(f[i]);
+            }
+        }
+    }
+}
+
+template <int FMT, int OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_p,
+            const float *__restrict__ s_x, const float *__restrict__ s_w, int64_t M, int64_t N, int64_t K,
+            void *__restrict__ y, int64_t ldy, int vec_ok, int32_t *status)
+{
+    constexpr int S = stages<FMT>();
+    constexpr int PB = packed_bytes_per_kblock<FMT>();
+    constexpr int P_BYTES = BN * PB;
+    constexpr int kShift = Fmt<FMT>::kShift;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = base;                       // S x 16 KB
+    uint8_t *sE = sA + S * A_BYTES;           // S x 32 KB
+    uint8_t *sP = sE + S * E_BYTES;           // S x P_BYTES
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sP + S * P_BYTES);
+    uint64_t *full_tma = bars;
+    uint64_t *full_exp = bars + S;
+    uint64_t *empty = bars + 2 * S;
+    uint64_t *acc_full = bars + 3 * S;
+    uint64_t *acc_empty = bars + 3 * S + 2;
+    uint64_t *drain = bars + 3 * S + 4;
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(bars + 3 * S + 5);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 3 * S + 6);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full_tma[s], 1);
+            mbar_init(&full_exp[s], kExpThreads);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_p)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(const_cast<uint32_t *>(tmem_slot))), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int64_t num_m = (M + BM - 1) / BM;
+    const int64_t num_n = (N + BN - 1) / BN;
+    const int64_t num_tiles = num_m * num_n;
+    const int nkb = static_cast<int>((K + BK - 1) / BK);
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            uint32_t g = 0;  // global k-block counter
+            bool ok = true;
+            for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int m0 = static_cast<int>((tile % num_m) * BM);
+                const int n0 = static_cast<int>((tile / num_m) * BN);
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % S;
+                    const uint32_t ph = (g / S) & 1u;
+                    if (!wait_bar(&empty[s], ph ^ 1u, abort_flag, status)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&full_tma[s], A_BYTES + P_BYTES);
+                    tma_load_2d(sA + s * A_BYTES, &map_a, &full_tma[s], kb * BK, m0);
+                    tma_load_2d(sP + s * P_BYTES, &map_p, &full_tma[s], kb * PB, n0);
+                }
+            }
+            if (!ok) {
+                // Let copies already issued land before the CTA leaves.
+                for (uint32_t i = 0; i < S && i < g; ++i) {
+                    const uint32_t gi = g - 1 - i;
+                    wait_bar(&full_tma[gi % S], (gi / S) & 1u, abort_flag, nullptr, 100000000ull);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            uint32_t g = 0;
+            uint32_t t = 0;
+            bool ok = true;
+            for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++t) {
+                const int b = t & 1;
+                const uint32_t aph = (t >> 1) & 1u;
+                if (!wait_bar(&acc_empty[b], aph ^ 1u, abort_flag, status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BN);
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % S;
+                    const uint32_t ph = (g / S) & 1u;
+                    if (!wait_bar(&full_tma[s], ph, abort_flag, status) ||
+                        !wait_bar(&full_exp[s], ph, abort_flag, status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(sA + s * A_BYTES);
+                    const uint32_t e_addr = smem_u32(sE + s * E_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < BK / UMMA_K; ++kk)
+                        tc_mma_i8(d_tmem, sw128_desc(a_addr + kk * UMMA_K), sw128_desc(e_addr + kk * UMMA_K),
+                                  kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                    tc_commit(&empty[s]);
+                }
+                if (!ok) break;
+                tc_commit(&acc_full[b]);
+            }
+            // All MMAs this thread issued are complete once `drain` flips.
+            tc_commit(drain);
+            wait_bar(drain, 0, abort_flag, nullptr, 100000000ull);
+        }
+    } else if (warp < 6) {
+        // ---------------- expanders ----------------
+        const int et = threadIdx.x - 64;
+        uint32_t g = 0;
+        bool ok = true;
+        for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (int kb = 0; kb < nkb; ++kb, ++g) {
+                const int s = g % S;
+                const uint32_t ph = (g / S) & 1u;
+                if (!wait_bar(&full_tma[s], ph, abort_flag, status)) { ok = false; break; }
+                expand_stage<FMT>(sP + s * P_BYTES, sE + s * E_BYTES, et);
+                // Each writer orders its generic-proxy stores before the
+                // tensor core's async-proxy reads, then arrives.
+                fence_proxy_async_smem();
+                mbar_arrive(&full_exp[s]);
+            }
+        }
+    } else {
+        // ---------------- epilogue ----------------
+        const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+        const bool sw_per_row = (FMT != kT2);
+        uint32_t t = 0;
+        for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t) {
+            const int b = t & 1;
+            const uint32_t aph = (t >> 1) & 1u;
+            // One lane waits and the warp follows its verdict, so the
+            // .sync.aligned TMEM loads below always run converged.
+            int ready = 0;
+            if (lane == 0) ready = wait_bar(&acc_full[b], aph, abort_flag, status) ? 1 : 0;
+            ready = __shfl_sync(0xffffffffu, ready, 0);
+            if (!ready) break;
+            tc_fence_after();
+            const int64_t m0 = (tile % num_m) * BM;
+            const int64_t n0 = (tile / num_m) * BN;
+            const int64_t row = m0 + quarter * 32 + lane;
+            const float sx = row < M ? s_x[row] : 0.0f;
+#pragma unroll 1
+            for (int cc = 0; cc < BN / 32; ++cc) {
+                uint32_t v[32];
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                       static_cast<uint32_t>(b * BN + cc * 32);
+                tmem_ld_32cols(taddr, v);
+                const int64_t nc = n0 + cc * 32;
+                if (row < M && nc < N)
+                    store_row32<OUT>(y, row, ldy, nc, N, v, kShift, s_w, sw_per_row, sx, vec_ok != 0);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[b]);
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<EncodeTiledFn>(nullptr);
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+bool make_map_2d(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_t outer, uint64_t stride_bytes,
+                 uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {stride_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estride[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims, strides, box, estride,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int FMT>
+constexpr size_t smem_bytes()
+{
+    return 1024 + stages<FMT>() * (A_BYTES + E_BYTES + BN * packed_bytes_per_kblock<FMT>()) + 3 * stages<FMT>() * 8 +
+           64;
+}
+
+template <int FMT, int OUT>
+lowbit_status launch_t(const CUtensorMap &ma, const CUtensorMap &mp, const float *s_x, const float *s_w,
+                       int64_t M, int64_t N, int64_t K, void *y, int64_t ldy, int vec_ok, int32_t *status,
+                       cudaStream_t st)
+{
+    constexpr size_t smem = smem_bytes<FMT>();
+    static bool configured[64] = {};  // the attribute is set once per device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LOWBIT_ERR_CUDA;
+    if (!configured[dev]) {
+        if (cudaFuncSetAttribute(gemm_kernel<FMT, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem)) != cudaSuccess)
+            return LOWBIT_ERR_CUDA;
+        configured[dev] = true;
+    }
+    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int64_t sms = device_sm_count();
+    const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
+    gemm_kernel<FMT, OUT><<<grid, kThreads, smem, st>>>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, status);
+    return launch_status();
+}
+
+template <int FMT>
+lowbit_status launch_fmt(const CUtensorMap &ma, const CUtensorMap &mp, const float *s_x, const float *s_w,
+                         int64_t M, int64_t N, int64_t K, void *y, lowbit_dtype ydt, int64_t ldy, int vec_ok,
+                         int32_t *status, cudaStream_t st)
+{
+    if (ydt == LOWBIT_F32) return launch_t<FMT, LOWBIT_F32>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, status, st);
+    if (ydt == LOWBIT_BF16) return launch_t<FMT, LOWBIT_BF16>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, status, st);
+    return launch_t<FMT, LOWBIT_I32>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, status, st);
+}
+
+}  // namespace tc
+
+lowbit_status gemm_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
+                          const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
+                          lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int32_t *status,
+                          cudaStream_t st)
+{
+    using namespace tc;
+    CUtensorMap ma, mp;
+    if (!make_map_2d(&ma, q, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(ldq), BK,
+                     BM, CU_TENSOR_MAP_SWIZZLE_128B))
+        return LOWBIT_ERR_CUDA;
+    const uint32_t pb = f == LOWBIT_TERNARY2 ? packed_bytes_per_kblock<kT2>()
+                        : f == LOWBIT_BINARY1 ? packed_bytes_per_kblock<kB1>()
+                                              : packed_bytes_per_kblock<kI4>();
+    if (!make_map_2d(&mp, packed, static_cast<uint64_t>(row_bytes), static_cast<uint64_t>(N),
+                     static_cast<uint64_t>(ldp), pb, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return LOWBIT_ERR_CUDA;
+    const int64_t esz = ydt == LOWBIT_BF16 ? 2 : 4;
+    const int vec_ok = ((reinterpret_cast<uintptr_t>(y) & 15u) == 0 && (ldy * esz) % 16 == 0) ? 1 : 0;
+    if (f == LOWBIT_TERNARY2) return launch_fmt<kT2>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, status, st);
+    if (f == LOWBIT_BINARY1) return launch_fmt<kB1>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, status, st);
+    return launch_fmt<kI4>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, status, st);
+}
+
+}  // namespace lowbit

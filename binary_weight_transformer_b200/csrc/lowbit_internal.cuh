@@ -1,0 +1,98 @@
+// lowbit_internal.cuh -- device helpers shared by the library's kernels.
+//
+// Code expansion.  Every kernel turns packed weight codes into int8x4 words
+// that hold (c << S) for four consecutive codes, S = 6 for ternary and binary
+// and S = 4 for 4-bit codes.  Shifting the field to the top of its byte makes
+// the sign extension free; the integer dot then carries a factor 2^S that the
+// epilogue removes with an exact arithmetic shift (the sum is a multiple of
+// 2^S).  The int32 bound becomes |acc| * 2^S < 2^31, which is why
+// lowbit_max_k is 2^31 / (128 * 64) - 1 for ternary and binary and
+// 2^31 / (128 * 16 * 7) for 4-bit codes.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "../../include/lowbit.h"
+
+namespace lowbit {
+
+constexpr int kT2 = LOWBIT_TERNARY2;
+constexpr int kB1 = LOWBIT_BINARY1;
+constexpr int kI4 = LOWBIT_INT4;
+
+template <int FMT> struct Fmt;
+// Ternary: 16 codes per 32-bit word, plane order (byte (k%16)%4, field (k%16)/4).
+template <> struct Fmt<kT2> {
+    static constexpr int kBits = 2;
+    static constexpr int kShift = 6;
+    static constexpr int kCodesPerWord = 16;
+};
+// Binary: 32 codes per word, bit k (little-bit-first bytes), 1 = -1.
+template <> struct Fmt<kB1> {
+    static constexpr int kBits = 1;
+    static constexpr int kShift = 6;
+    static constexpr int kCodesPerWord = 32;
+};
+// 4-bit: 8 codes per word, plane order (byte (k%8)%4, nibble (k%8)/4).
+template <> struct Fmt<kI4> {
+    static constexpr int kBits = 4;
+    static constexpr int kShift = 4;
+    static constexpr int kCodesPerWord = 8;
+};
+
+// Four ternary codes 4j..4j+3 of word w as int8 (64*c): move field j of each
+// byte to bits 7..6 of that byte.
+__device__ __forceinline__ uint32_t t2_expand(uint32_t w, int j)
+{
+    return (w << (6 - 2 * j)) & 0xC0C0C0C0u;
+}
+
+// Four 4-bit codes 4h..4h+3 of word w as int8 (16*c): nibble h of each byte
+// moved to the high nibble.
+__device__ __forceinline__ uint32_t i4_expand(uint32_t w, int h)
+{
+    return h == 0 ? ((w << 4) & 0xF0F0F0F0u) : (w & 0xF0F0F0F0u);
+}
+
+// Four binary codes from the low 4 bits of `nib`: bit m goes to bit 7 of byte
+// m (one multiply by 2^7 + 2^14 + 2^21 + 2^28 spreads the four bits without
+// carries), then bit 6 is set in every byte: 0x40 = +64, 0xC0 = -64.
+__device__ __forceinline__ uint32_t b1_expand_nibble(uint32_t nib)
+{
+    return ((nib * 0x10204080u) & 0x80808080u) | 0x40404040u;
+}
+
+__device__ __forceinline__ void report(int32_t *status, int code)
+{
+    if (status != nullptr) atomicOr(status, 1 << code);
+}
+
+__device__ __forceinline__ bool finite_bits(uint32_t u) { return (u & 0x7f800000u) != 0x7f800000u; }
+
+// 16-byte streaming load that does not allocate in L1 (weights are read once
+// per launch).
+__device__ __forceinline__ uint4 ld_stream_u4(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// Output conversion shared by the epilogues: y = float(acc) * (s_w * s_x)
+// with the two scales multiplied first, each product one fp32 rounding.
+__device__ __forceinline__ float rescale(int32_t acc, float sw, float sx)
+{
+    return __fmul_rn(__int2float_rn(acc), __fmul_rn(sw, sx));
+}
+
+}  // namespace lowbit
+
+// Host-side launch helpers (defined in abi.cu, used by every kernel file).
+namespace lowbit {
+lowbit_status launch_status();
+int device_sm_count();
+}

@@ -1,0 +1,190 @@
+/*
+ * lowbit.h -- C ABI of the B200 (sm_100a) low-bit-weight linear layer.
+ *
+ * The operator is the BitLinear forward of a BitNet-style transformer,
+ *
+ *     acc[t,n] = sum_k q[t,k] * c[n,k]            (int32)
+ *     y[t,n]   = float(acc[t,n]) * (s_w[n] * s_x[t])
+ *
+ * with weight codes c ternary {-1,0,+1}, binary {-1,+1} or 4-bit {-7..+7}
+ * and per-token int8 activation codes q.  Sources, by page title and section:
+ *
+ *   "M8.8 - Native Binary and Ternary Transformers": 0x02C-0x02E (activation
+ *     codes, integer accumulation, rescale), 0x05A-0x05D (absmean ternary
+ *     codes, per-token A8 codes, the add/subtract kernel), 0x06E (binary sign
+ *     rule and little-bit-first packing), 0x09A-0x09C (operation ledger,
+ *     decode vs prefill, the INT32 bound, the reference decoder).
+ *   "Atomic-1Bit" README: the add/sub/skip rule; four ternary codes per byte.
+ *   "T4NT-0.5B" model card: tanh(w/3)*3 clipping, 15 symmetric levels.
+ *
+ * Conventions for every call below
+ *   - All array pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates nothing and keeps no per-call state.
+ *   - Sizes are elements unless named *_bytes; leading dimensions (ld*) are
+ *     the distance between consecutive rows, row-major, K contiguous.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call is asynchronous on that stream; nothing synchronises the host.
+ *   - Argument errors are found on the host before any launch and returned
+ *     as a lowbit_status; nothing is launched then.
+ *   - Data errors found on the device (a non-finite input, a reserved code, a
+ *     pipeline wait that ran out) are OR-ed into `*status_dev` as the bit
+ *     (1u << status) when `status_dev` is not NULL (a device int32 the caller
+ *     zeroes and reads back).  With NULL they are not reported.
+ */
+#ifndef LOWBIT_H
+#define LOWBIT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Weight code formats.  Packed layouts (row n starts at byte n*ldp; every bit
+ * that no code owns must be zero):
+ *   LOWBIT_TERNARY2  2-bit two's-complement fields 00 = 0, 01 = +1, 11 = -1,
+ *                    10 reserved; four codes per byte.  Inside each
+ *                    little-endian 32-bit word of 16 codes, code k sits in
+ *                    byte (k%16)%4, field (k%16)/4 (bits 8*byte + 2*field).
+ *                    One scale per tensor.
+ *   LOWBIT_BINARY1   bit k%8 of byte k/8 is 1 for -1 and 0 for +1
+ *                    (little-bit-first, M8.8 0x06E).  One scale per row.
+ *   LOWBIT_INT4      4-bit two's-complement fields, 1000 reserved; inside each
+ *                    32-bit word of 8 codes, code k sits in byte (k%8)%4,
+ *                    nibble (k%8)/4.  One scale per row. */
+typedef enum lowbit_format {
+    LOWBIT_TERNARY2 = 0,
+    LOWBIT_BINARY1 = 1,
+    LOWBIT_INT4 = 2
+} lowbit_format;
+
+typedef enum lowbit_dtype {
+    LOWBIT_F32 = 0,  /* IEEE fp32 */
+    LOWBIT_BF16 = 1, /* bfloat16, fp32 rounded to nearest even */
+    LOWBIT_I32 = 2   /* raw int32 accumulators (outputs only) */
+} lowbit_dtype;
+
+typedef enum lowbit_status {
+    LOWBIT_OK = 0,
+    LOWBIT_ERR_INVALID_ARG = 1,     /* null pointer, size <= 0, ld too small, bad enum */
+    LOWBIT_ERR_ALIGNMENT = 2,       /* pointer or leading dimension misaligned */
+    LOWBIT_ERR_UNSUPPORTED = 3,     /* valid but not implemented (e.g. no sm_100 device) */
+    LOWBIT_ERR_OVERFLOW_BOUND = 4,  /* K beyond the int32 accumulator bound */
+    LOWBIT_ERR_NONFINITE = 5,       /* device: NaN/Inf input (or x*127 overflow) */
+    LOWBIT_ERR_RESERVED_CODE = 6,   /* device: reserved pattern or non-zero unowned bit */
+    LOWBIT_ERR_TIMEOUT = 7,         /* device: a pipeline wait gave up */
+    LOWBIT_ERR_CUDA = 8             /* a CUDA runtime call or launch failed */
+} lowbit_status;
+
+/* Bytes a packed row needs (its logical extent): TERNARY2 4*ceil(K/16),
+ * BINARY1 ceil(K/8), INT4 4*ceil(K/8).  0 for a bad format or K <= 0. */
+size_t lowbit_packed_row_bytes(lowbit_format f, int64_t K);
+
+/* Smallest valid row stride for packed weights: the row bytes rounded up to
+ * a multiple of 16. */
+size_t lowbit_packed_ld(lowbit_format f, int64_t K);
+
+/* Number of fp32 weight scales: 1 for TERNARY2 (per tensor, M8.8 0x05A),
+ * N for BINARY1 and INT4 (per output row).  0 for bad arguments. */
+int64_t lowbit_scale_count(lowbit_format f, int64_t N);
+
+/* Largest K lowbit_linear accepts for a format: the worst case
+ * |acc| = 128 * max|c| * K must stay inside int32 (M8.8 0x09C). */
+int64_t lowbit_max_k(lowbit_format f);
+
+/* Device workspace lowbit_pack needs: 8*N bytes (rounded to 256) for
+ * TERNARY2, whose per-tensor scale is a two-stage fixed-order sum; 0 for the
+ * other formats. */
+size_t lowbit_pack_workspace_bytes(lowbit_format f, int64_t N);
+
+/* lowbit_pack -- quantise fp32 weights W[N,K] (row stride ldw elements) into
+ * codes and pack them (done once per weight, off the hot path; M8.8 0x04D:
+ * export freezes codes and scales).
+ *   TERNARY2 (M8.8 0x05A-0x05B): gamma = mean|W| over the tensor, summed in
+ *     fp64 row by row (k ascending) then over rows (n ascending), rounded once
+ *     to fp32; c = clip(rint(w / (gamma + eps)), -1, 1) with an fp32 divide
+ *     and nearest-even rounding; s_w[0] = gamma.  eps >= 0 (1e-5 in M8.8).
+ *   BINARY1 (M8.8 0x06E, 0x02B): c = +1 if w >= 0 (both zeros) else -1;
+ *     s_w[n] = mean_k |W[n,k]| (fp64 sum, k ascending, rounded once).
+ *     eps is ignored.
+ *   INT4 (T4NT-0.5B): w_c = 3*tanh(w/3) evaluated in fp64 by a fixed operation
+ *     sequence (Taylor series of expm1 with a Cody-Waite split of ln 2) and
+ *     rounded once to fp32; s_w[n] = max_k |w_c| / 7; c = clip(rint(w_c /
+ *     s_w[n]), -7, 7); a zero row gives s_w = 0 and zero codes.  eps ignored.
+ * Outputs: packed[N, ldp] bytes (ldp >= lowbit_packed_row_bytes, multiple of
+ * 16, 16-byte aligned base; unowned bits written zero), s_w[lowbit_scale_count]
+ * fp32.  `workspace` must hold lowbit_pack_workspace_bytes(f, N) bytes of
+ * device memory (may be NULL when that is 0).  A non-finite weight sets
+ * LOWBIT_ERR_NONFINITE in *status_dev; the artifact is then unspecified. */
+lowbit_status lowbit_pack(const float *w, int64_t N, int64_t K, int64_t ldw,
+                          lowbit_format f, float eps,
+                          uint8_t *packed, int64_t ldp, float *s_w,
+                          void *workspace, size_t workspace_bytes,
+                          int32_t *status_dev, void *stream);
+
+/* lowbit_unpack -- decode packed[N, ldp] into int8 codes[N, ldc] (ldc >= K).
+ * A reserved field or a non-zero unowned bit sets LOWBIT_ERR_RESERVED_CODE in
+ * *status_dev (M8.8 0x0BB: reserved patterns reject); such a code decodes as
+ * 0.  Used by tests and tools, not by the hot path. */
+lowbit_status lowbit_unpack(const uint8_t *packed, int64_t ldp, int64_t N, int64_t K,
+                            lowbit_format f, int8_t *codes, int64_t ldc,
+                            int32_t *status_dev, void *stream);
+
+/* lowbit_act_quant -- per-token absmax int8 quantisation (M8.8 0x05C):
+ *   gamma_t = max_k |x[t,k]|;
+ *   gamma_t == 0:  q[t,:] = 0, s_x[t] = 0;
+ *   else           q = clip(rint((x * 127) / (gamma_t + eps)), -128, 127)
+ *                  (fp32 multiply, fp32 IEEE divide, nearest even),
+ *                  s_x[t] = gamma_t / 127.
+ * x is fp32 or bf16 (xdt = LOWBIT_F32 | LOWBIT_BF16), [M, K] with row stride
+ * ldx elements; x must be 16-byte aligned and ldx*sizeof(x) a multiple of 16.
+ * q is int8 [M, ldq], 16-byte aligned, ldq a multiple of 16, ldq >= K; bytes
+ * of q past K are left untouched.  s_x is fp32 [M].  eps >= 0 (0 in the
+ * configurations this library is measured on).  A non-finite x, or an x*127
+ * that overflows fp32, sets LOWBIT_ERR_NONFINITE; that row is unspecified. */
+lowbit_status lowbit_act_quant(const void *x, lowbit_dtype xdt, int64_t M, int64_t K,
+                               int64_t ldx, float eps, int8_t *q, int64_t ldq, float *s_x,
+                               int32_t *status_dev, void *stream);
+
+/* lowbit_linear -- the low-bit linear layer on int8 activation codes:
+ *   acc[t,n] = sum_{k<K} q[t,k] * c[n,k]  (exact int32: add/sub/skip for
+ *              ternary and binary codes, Atomic-1Bit README, M8.8 0x05D)
+ *   y[t,n]   = acc[t,n]                          (ydt = LOWBIT_I32)
+ *            = float(acc) * (s_w[n or 0] * s_x[t]) (LOWBIT_F32; the two scales
+ *              are multiplied first, both products fp32, M8.8 0x02D)
+ *            = that fp32 value rounded to bf16, nearest even (LOWBIT_BF16).
+ * Inputs: q int8 [M, ldq] and packed [N, ldp] as above (16-byte aligned bases,
+ * ldq and ldp multiples of 16), s_x fp32 [M], s_w fp32 [lowbit_scale_count].
+ * Output y [M, ldy], ldy >= N, aligned to its element size.  Bytes of q past
+ * K are ignored.  K <= lowbit_max_k(f), else LOWBIT_ERR_OVERFLOW_BOUND.
+ * M <= 16 runs the packed-weight GEMV kernel; larger M runs the tcgen05
+ * tensor-core GEMM (int8 MMA, accumulators in tensor memory). */
+lowbit_status lowbit_linear(const int8_t *q, int64_t ldq, const float *s_x,
+                            int64_t M, int64_t K,
+                            const uint8_t *packed, int64_t ldp, const float *s_w,
+                            lowbit_format f, int64_t N,
+                            void *y, lowbit_dtype ydt, int64_t ldy,
+                            int32_t *status_dev, void *stream);
+
+/* Same operator with the kernel chosen by the caller: path 0 = automatic (as
+ * lowbit_linear), 1 = packed-weight GEMV (any M), 2 = tensor-core GEMM (any
+ * M).  Lets tests and benchmarks reach both kernels at every size. */
+lowbit_status lowbit_linear_path(const int8_t *q, int64_t ldq, const float *s_x,
+                                 int64_t M, int64_t K,
+                                 const uint8_t *packed, int64_t ldp, const float *s_w,
+                                 lowbit_format f, int64_t N,
+                                 void *y, lowbit_dtype ydt, int64_t ldy,
+                                 int path, int32_t *status_dev, void *stream);
+
+/* Human-readable name of a status value (static string). */
+const char *lowbit_status_string(lowbit_status s);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int lowbit_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOWBIT_H */

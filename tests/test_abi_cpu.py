@@ -1,0 +1,147 @@
+"""The C ABI without a GPU: library loading, exported symbols, size helpers
+and host-side argument checks.
+
+No call here reaches a kernel launch: every call with fake device pointers
+carries at least one argument the host rejects first.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import binary_weight_transformer_b200 as bwt
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lowbit.h")
+FAKE = 0x10000  # 64 KB-aligned, never dereferenced
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(lowbit_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from binary_weight_transformer_b200 import _build
+    _build.build()
+    return bwt.lib()
+
+
+def test_library_exports_every_declared_function(lib):
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    # and the binding types each of them
+    assert set(names) <= set(bwt.ABI)
+
+
+def test_size_helpers(lib):
+    assert bwt.packed_row_bytes(bwt.TERNARY2, 2560) == 640
+    assert bwt.packed_row_bytes(bwt.TERNARY2, 17) == 8  # 4 * ceil(17/16)
+    assert bwt.packed_row_bytes(bwt.BINARY1, 17) == 3
+    assert bwt.packed_row_bytes(bwt.INT4, 9) == 8
+    assert bwt.packed_ld(bwt.BINARY1, 17) == 16
+    assert bwt.packed_ld(bwt.INT4, 3584) == 1792
+    assert bwt.packed_row_bytes(bwt.TERNARY2, 0) == 0
+    assert bwt.scale_count(bwt.TERNARY2, 768) == 1
+    assert bwt.scale_count(bwt.BINARY1, 768) == 768
+    assert bwt.scale_count(bwt.INT4, 0) == 0
+    assert bwt.max_k(bwt.TERNARY2) == 2**31 // (128 * 64) - 1
+    assert bwt.max_k(bwt.INT4) == (2**31 - 1) // (128 * 16 * 7)
+    assert lib.lowbit_pack_workspace_bytes(bwt.TERNARY2, 9728) == 9728 * 8
+    assert lib.lowbit_pack_workspace_bytes(bwt.BINARY1, 9728) == 0
+    assert lib.lowbit_status_string(7) == b"device pipeline wait timed out"
+    assert lib.lowbit_version() >= 100
+
+
+def _linear(lib, **kw):
+    a = dict(q=FAKE, ldq=256, s_x=FAKE, M=4, K=256, packed=FAKE, ldp=64, s_w=FAKE, fmt=bwt.TERNARY2,
+             N=8, y=FAKE, ydt=bwt.F32, ldy=8, path=0)
+    a.update(kw)
+    return lib.lowbit_linear_path(a["q"], a["ldq"], a["s_x"], a["M"], a["K"], a["packed"], a["ldp"], a["s_w"],
+                                  a["fmt"], a["N"], a["y"], a["ydt"], a["ldy"], a["path"], None, None)
+
+
+def test_linear_rejects_bad_arguments(lib):
+    assert _linear(lib, q=None) == bwt.ERR_INVALID_ARG
+    assert _linear(lib, M=0) == bwt.ERR_INVALID_ARG
+    assert _linear(lib, N=-1) == bwt.ERR_INVALID_ARG
+    assert _linear(lib, ldq=128) == bwt.ERR_INVALID_ARG          # ldq < K
+    assert _linear(lib, ldy=7) == bwt.ERR_INVALID_ARG            # ldy < N
+    assert _linear(lib, ldp=48) == bwt.ERR_INVALID_ARG           # ldp < row bytes
+    assert _linear(lib, fmt=3) == bwt.ERR_INVALID_ARG
+    assert _linear(lib, ydt=7) == bwt.ERR_INVALID_ARG
+    assert _linear(lib, path=3) == bwt.ERR_INVALID_ARG
+    assert _linear(lib, q=FAKE + 8) == bwt.ERR_ALIGNMENT
+    assert _linear(lib, ldq=264) == bwt.ERR_ALIGNMENT
+    assert _linear(lib, ldp=72) == bwt.ERR_ALIGNMENT
+    assert _linear(lib, y=FAKE + 2) == bwt.ERR_ALIGNMENT
+    big = bwt.max_k(bwt.TERNARY2) + 1
+    assert _linear(lib, K=big, ldq=(big + 15) // 16 * 16,
+                   ldp=bwt.packed_ld(bwt.TERNARY2, big)) == bwt.ERR_OVERFLOW_BOUND
+    k4 = bwt.max_k(bwt.INT4) + 1
+    assert _linear(lib, fmt=bwt.INT4, K=k4, ldq=(k4 + 15) // 16 * 16,
+                   ldp=bwt.packed_ld(bwt.INT4, k4)) == bwt.ERR_OVERFLOW_BOUND
+
+
+def test_act_quant_rejects_bad_arguments(lib):
+    f = lib.lowbit_act_quant
+    assert f(None, bwt.F32, 4, 64, 64, 0.0, FAKE, 64, FAKE, None, None) == bwt.ERR_INVALID_ARG
+    assert f(FAKE, 5, 4, 64, 64, 0.0, FAKE, 64, FAKE, None, None) == bwt.ERR_INVALID_ARG
+    assert f(FAKE, bwt.F32, 0, 64, 64, 0.0, FAKE, 64, FAKE, None, None) == bwt.ERR_INVALID_ARG
+    assert f(FAKE, bwt.F32, 4, 64, 32, 0.0, FAKE, 64, FAKE, None, None) == bwt.ERR_INVALID_ARG
+    assert f(FAKE, bwt.F32, 4, 64, 64, -1.0, FAKE, 64, FAKE, None, None) == bwt.ERR_INVALID_ARG
+    assert f(FAKE, bwt.F32, 4, 64, 64, float("nan"), FAKE, 64, FAKE, None, None) == bwt.ERR_INVALID_ARG
+    assert f(FAKE + 4, bwt.F32, 4, 64, 64, 0.0, FAKE, 64, FAKE, None, None) == bwt.ERR_ALIGNMENT
+    assert f(FAKE, bwt.F32, 4, 64, 65, 0.0, FAKE, 64, FAKE, None, None) == bwt.ERR_ALIGNMENT
+    assert f(FAKE, bwt.BF16, 4, 64, 68, 0.0, FAKE, 64, FAKE, None, None) == bwt.ERR_ALIGNMENT
+    assert f(FAKE, bwt.F32, 4, 64, 64, 0.0, FAKE, 72, FAKE, None, None) == bwt.ERR_ALIGNMENT
+
+
+def test_pack_rejects_bad_arguments(lib):
+    f = lib.lowbit_pack
+    need = lib.lowbit_pack_workspace_bytes(bwt.TERNARY2, 8)
+    ok = dict(w=FAKE, N=8, K=64, ldw=64, fmt=bwt.TERNARY2, eps=1e-5, packed=FAKE, ldp=16, s_w=FAKE,
+              ws=FAKE, wsb=need)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["w"], a["N"], a["K"], a["ldw"], a["fmt"], a["eps"], a["packed"], a["ldp"], a["s_w"],
+                 a["ws"], a["wsb"], None, None)
+    assert call(w=None) == bwt.ERR_INVALID_ARG
+    assert call(ldw=32) == bwt.ERR_INVALID_ARG
+    assert call(ldp=8) == bwt.ERR_INVALID_ARG
+    assert call(ws=None) == bwt.ERR_INVALID_ARG
+    assert call(wsb=need - 1) == bwt.ERR_INVALID_ARG
+    assert call(eps=-1e-5) == bwt.ERR_INVALID_ARG
+    assert call(ldp=24) == bwt.ERR_ALIGNMENT
+    assert call(packed=FAKE + 4) == bwt.ERR_ALIGNMENT
+
+
+def test_unpack_rejects_bad_arguments(lib):
+    f = lib.lowbit_unpack
+    assert f(None, 16, 4, 64, bwt.TERNARY2, FAKE, 64, None, None) == bwt.ERR_INVALID_ARG
+    assert f(FAKE, 16, 4, 64, bwt.TERNARY2, FAKE, 32, None, None) == bwt.ERR_INVALID_ARG
+    assert f(FAKE, 8, 4, 64, bwt.TERNARY2, FAKE, 64, None, None) == bwt.ERR_INVALID_ARG
+    assert f(FAKE, 24, 4, 64, bwt.TERNARY2, FAKE, 64, None, None) == bwt.ERR_ALIGNMENT
+
+
+def test_oracle_and_library_share_no_code():
+    # The oracle is a separate C file built by gcc; the CUDA library never
+    # includes or links it, and it never includes the library's headers.
+    orc = open(os.path.join(ROOT, "oracle", "lowbit_oracle.c")).read()
+    includes = re.findall(r"^\s*#\s*include\s*[<\"]([^>\"]+)", orc, flags=re.M)
+    assert sorted(includes) == ["math.h", "omp.h", "stdint.h", "stdlib.h", "string.h"]
+    csrc = os.path.join(ROOT, "binary_weight_transformer_b200", "csrc")
+    for fn in os.listdir(csrc):
+        text = open(os.path.join(csrc, fn)).read()
+        assert "oracle" not in text.lower(), fn
+    pkg = os.path.join(ROOT, "binary_weight_transformer_b200")
+    for fn in os.listdir(pkg):
+        if fn.endswith(".py"):
+            assert "import oracle" not in open(os.path.join(pkg, fn)).read(), fn

@@ -1,0 +1,359 @@
+"""Parity of the CUDA path with the oracle (needs a B200).
+
+Both sides get the same seeded inputs (binary_weight_transformer_b200.workloads).
+Codes, packed bytes, scales, int8 activations and int32 accumulators must be
+bit-identical.  Floating outputs must meet the stated tolerances: fp32 within
+1e-6 relative, bf16 within 1 unit in the last place.  Both sides also use the
+same operation order, so the float outputs are additionally checked for bit
+equality in separate tests.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from binary_weight_transformer_b200 import workloads as wls
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():  # pragma: no cover - CPU runs deselect -m gpu
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import binary_weight_transformer_b200 as bwt  # noqa: E402
+
+DEV = "cuda:0"
+FMTS = [bwt.TERNARY2, bwt.BINARY1, bwt.INT4]
+FMT_IDS = {bwt.TERNARY2: "ternary", bwt.BINARY1: "binary", bwt.INT4: "int4"}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from binary_weight_transformer_b200 import _build
+    _build.build()
+    oracle.build()
+    bwt.lib()
+
+
+def status_word():
+    return torch.zeros(1, dtype=torch.int32, device=DEV)
+
+
+def bf16_bits(t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def ulp_distance_bf16(a_bits, b_bits):
+    """Distance in bf16 units in the last place (monotone integer mapping)."""
+    def key(b):
+        b = b.astype(np.int32)
+        return np.where(b & 0x8000, -(b & 0x7FFF), b)
+    return np.abs(key(a_bits) - key(b_bits))
+
+
+def gpu_pack(w, fmt, eps=1e-5, extra_ld=0):
+    wt = torch.from_numpy(w).to(DEV)
+    ldp = bwt.packed_ld(fmt, w.shape[1]) + extra_ld
+    st = status_word()
+    packed, s_w = bwt.lowbit_pack(wt, fmt, eps, ldp=ldp, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    return packed, s_w
+
+
+def gpu_act(x_np, bf16=False, eps=0.0):
+    if bf16:
+        xt = torch.from_numpy(x_np.view(np.int16)).to(DEV).view(torch.bfloat16)
+    else:
+        xt = torch.from_numpy(x_np).to(DEV)
+    st = status_word()
+    q, s_x = bwt.lowbit_act_quant(xt, eps, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    return q, s_x
+
+
+# ---------------------------------------------------------------------------
+# activation quantiser
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bf16", [False, True], ids=["f32", "bf16"])
+@pytest.mark.parametrize("M,K", [(1, 192), (7, 200), (3, 9728), (257, 2560), (5, 13), (64, 3),
+                                 (9, 65536 + 24)])
+@pytest.mark.parametrize("eps", [0.0, 1e-5])
+def test_act_quant_bit_exact(M, K, bf16, eps):
+    x = wls.normal_activations(100 + M + K, M, K, 0.01, 8.0)
+    x[0, :] = 0.0  # an all-zero row: zero codes and zero scale
+    if bf16:
+        x = wls.to_bf16_bits(x)
+    q, s_x = gpu_act(x, bf16, eps)
+    q_o, s_o = oracle.act_quant(x, eps, bf16_bits=bf16)
+    assert np.array_equal(q.cpu().numpy()[:, :K], q_o)
+    assert np.array_equal(s_x.cpu().numpy().view(np.uint32), s_o.view(np.uint32))
+
+
+def test_act_quant_flags_nonfinite():
+    x = np.ones((4, 64), np.float32)
+    x[2, 5] = np.nan
+    x[3, 7] = 1e37  # x * 127 overflows fp32
+    xt = torch.from_numpy(x).to(DEV)
+    st = status_word()
+    bwt.lowbit_act_quant(xt, 0.0, status=st)
+    torch.cuda.synchronize()
+    assert bwt.status_flags(st) == [bwt.ERR_NONFINITE]
+
+
+# ---------------------------------------------------------------------------
+# packer / unpacker
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
+@pytest.mark.parametrize("N,K", [(768, 192), (37, 101), (5, 7), (1, 4096), (96, 1000), (300, 33)])
+def test_pack_bit_exact(fmt, N, K):
+    w = wls.normal_weights(200 + N + K, N, K)
+    if fmt == bwt.INT4:
+        w[0] = 0.0  # a zero row: zero scale, zero codes
+        w[1] *= 100.0  # tanh clipping bends strongly
+    packed, s_w = gpu_pack(w, fmt, extra_ld=16)
+    codes, s_o = oracle.quantize(w, fmt, 1e-5)
+    p_o = oracle.pack(codes, fmt, packed.shape[1])
+    assert np.array_equal(packed.cpu().numpy(), p_o)
+    assert np.array_equal(s_w.cpu().numpy().view(np.uint32), s_o.view(np.uint32))
+
+
+@pytest.mark.parametrize("fmt,N,K", [(bwt.TERNARY2, 9728, 2560), (bwt.TERNARY2, 2560, 9728),
+                                     (bwt.INT4, 3584, 1280), (bwt.INT4, 1280, 3584),
+                                     (bwt.BINARY1, 2048, 192)], ids=str)
+def test_pack_full_size_bit_exact(fmt, N, K):
+    w = wls.normal_weights(300 + K, N, K)
+    packed, s_w = gpu_pack(w, fmt)
+    codes, s_o = oracle.quantize(w, fmt, 1e-5)
+    assert np.array_equal(packed.cpu().numpy(), oracle.pack(codes, fmt, packed.shape[1]))
+    assert np.array_equal(s_w.cpu().numpy().view(np.uint32), s_o.view(np.uint32))
+
+
+def test_pack_ternary_eps_zero_tie():
+    # M8.8 §0x05A tie rule: w/gamma = 0.5 exactly rounds to 0 (nearest even).
+    w = np.array([[0.25, -0.75, 0.5, -0.5]], np.float32)
+    packed, s_w = gpu_pack(w, bwt.TERNARY2, eps=0.0)
+    codes = bwt.lowbit_unpack(packed, 4, bwt.TERNARY2).cpu().numpy()
+    assert s_w.item() == 0.5
+    assert codes.tolist() == [[0, -1, 1, -1]]
+
+
+def test_pack_flags_nonfinite():
+    w = np.ones((3, 40), np.float32)
+    w[1, 3] = np.inf
+    for fmt in FMTS:
+        wt = torch.from_numpy(w).to(DEV)
+        st = status_word()
+        bwt.lowbit_pack(wt, fmt, status=st)
+        torch.cuda.synchronize()
+        assert bwt.status_flags(st) == [bwt.ERR_NONFINITE], fmt
+
+
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
+def test_unpack_roundtrip_and_reserved(fmt):
+    N, K = 50, 77
+    w = wls.normal_weights(400 + fmt, N, K)
+    packed, _ = gpu_pack(w, fmt)
+    codes_o, _ = oracle.quantize(w, fmt)
+    st = status_word()
+    codes = bwt.lowbit_unpack(packed, K, fmt, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert np.array_equal(codes.cpu().numpy(), codes_o)
+    # a non-zero padding byte is rejected
+    bad = packed.clone()
+    bad[3, -1] = 1
+    st.zero_()
+    bwt.lowbit_unpack(bad, K, fmt, status=st)
+    torch.cuda.synchronize()
+    assert bwt.status_flags(st) == [bwt.ERR_RESERVED_CODE]
+    if fmt != bwt.BINARY1:
+        # a reserved field (10 / 1000) inside the extent is rejected
+        bad = packed.clone()
+        bad[4, 0] = (bad[4, 0] & ~0x3 if fmt == bwt.TERNARY2 else bad[4, 0] & ~0xF) | \
+            (0x2 if fmt == bwt.TERNARY2 else 0x8)
+        st.zero_()
+        bwt.lowbit_unpack(bad, K, fmt, status=st)
+        torch.cuda.synchronize()
+        assert bwt.status_flags(st) == [bwt.ERR_RESERVED_CODE]
+
+
+# ---------------------------------------------------------------------------
+# linear: both kernels, every format and output type
+# ---------------------------------------------------------------------------
+
+def run_case(fmt, M, N, K, path, out, seed, zero_w=False, x_bf16=False):
+    w = wls.normal_weights(seed, N, K)
+    if zero_w:
+        w[:] = 0.0
+    x = wls.normal_activations(seed + 1, M, K, 0.01, 8.0)
+    if x_bf16:
+        x = wls.to_bf16_bits(x)
+    packed, s_w = gpu_pack(w, fmt)
+    q, s_x = gpu_act(x, x_bf16)
+    st = status_word()
+    y = bwt.lowbit_linear(q, s_x, packed, s_w, fmt, N, out, K=K, status=st, path=path)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    codes, s_wo = oracle.quantize(w, fmt, 1e-5)
+    q_o, s_xo = oracle.act_quant(x, 0.0, bf16_bits=x_bf16)
+    acc = oracle.int_dot(q_o, codes, fmt, nthreads=oracle.max_threads())
+    return y, acc, s_wo, s_xo
+
+
+SHAPES = [(1, 768, 192), (3, 257, 200), (16, 96, 1000), (17, 300, 192), (129, 513, 384), (300, 768, 1040),
+          (5, 33, 16), (200, 1, 4000)]
+
+
+@pytest.mark.parametrize("path", [1, 2], ids=["gemv", "gemm"])
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
+@pytest.mark.parametrize("M,N,K", SHAPES, ids=str)
+def test_linear_int32_accumulators_bit_exact(path, fmt, M, N, K):
+    y, acc, _, _ = run_case(fmt, M, N, K, path, bwt.I32, 500 + M + N + K)
+    assert np.array_equal(y.cpu().numpy().astype(np.int64), acc)
+
+
+@pytest.mark.parametrize("path", [1, 2], ids=["gemv", "gemm"])
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
+@pytest.mark.parametrize("M,N,K", SHAPES[:6], ids=str)
+def test_linear_f32_within_tolerance(path, fmt, M, N, K):
+    y, acc, s_w, s_x = run_case(fmt, M, N, K, path, bwt.F32, 600 + M + N + K)
+    ref = oracle.rescale(acc, s_w, s_x, "f32")
+    got = y.cpu().numpy()
+    denom = np.maximum(np.abs(ref), np.finfo(np.float32).tiny)
+    assert np.max(np.abs(got - ref) / denom) <= 1e-6
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("path", [1, 2], ids=["gemv", "gemm"])
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
+@pytest.mark.parametrize("M,N,K", SHAPES[:6], ids=str)
+def test_linear_bf16_within_one_ulp(path, fmt, M, N, K):
+    y, acc, s_w, s_x = run_case(fmt, M, N, K, path, bwt.BF16, 700 + M + N + K, x_bf16=True)
+    ref = oracle.rescale(acc, s_w, s_x, "bf16")
+    got = bf16_bits(y)
+    assert ulp_distance_bf16(got, ref).max() <= 1
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("path", [1, 2], ids=["gemv", "gemm"])
+def test_linear_degenerate_weights(path):
+    # all-zero weights: gamma = 0, every code 0, y = 0
+    y, acc, _, _ = run_case(bwt.TERNARY2, 20, 64, 256, path, bwt.F32, 800, zero_w=True)
+    assert not acc.any()
+    assert not y.cpu().numpy().any()
+
+
+@pytest.mark.parametrize("path", [1, 2], ids=["gemv", "gemm"])
+def test_linear_all_plus_one_gives_row_sums(path):
+    # ternary codes all +1: acc[t, n] = sum_k q[t, k] (add/sub/skip rule)
+    M, N, K = 19, 40, 320
+    w = np.full((N, K), 0.5, np.float32)
+    x = wls.normal_activations(801, M, K)
+    packed, s_w = gpu_pack(w, bwt.TERNARY2)
+    q, s_x = gpu_act(x)
+    y = bwt.lowbit_linear(q, s_x, packed, s_w, bwt.TERNARY2, N, bwt.I32, K=K, path=path)
+    rows = q.cpu().numpy()[:, :K].astype(np.int64).sum(axis=1)
+    assert np.array_equal(y.cpu().numpy(), np.repeat(rows[:, None], N, axis=1))
+
+
+def test_linear_ignores_bytes_of_q_past_k():
+    M, N, K = 40, 70, 200
+    for path in (1, 2):
+        for fmt in FMTS:
+            w = wls.normal_weights(810 + fmt, N, K)
+            x = wls.normal_activations(811, M, K)
+            packed, s_w = gpu_pack(w, fmt)
+            q, s_x = gpu_act(x)
+            ref = bwt.lowbit_linear(q, s_x, packed, s_w, fmt, N, bwt.I32, K=K, path=path).cpu()
+            q2 = q.clone()
+            q2[:, K:] = 77  # garbage in the stride padding
+            got = bwt.lowbit_linear(q2, s_x, packed, s_w, fmt, N, bwt.I32, K=K, path=path).cpu()
+            assert torch.equal(got, ref)
+
+
+# ---------------------------------------------------------------------------
+# the workloads at full size, in the configuration bench.py times
+# ---------------------------------------------------------------------------
+
+def test_single_ternary_full():
+    wl = wls.WORKLOADS["single_ternary"]
+    m = wl.matrices[0]
+    M = wl.Ms[0]
+    w = wls.workload_weights(wl, 0)
+    x = wls.workload_activations(wl, 0, M)
+    packed, s_w = gpu_pack(w, wl.fmt)
+    q, s_x = gpu_act(x)
+    y = bwt.lowbit_linear(q, s_x, packed, s_w, wl.fmt, m.N, bwt.F32, K=m.K)
+    codes, s_wo = oracle.quantize(w, wl.fmt, 1e-5)
+    q_o, s_xo = oracle.act_quant(x)
+    ref, _ = oracle.linear(q_o, s_xo, oracle.pack(codes, wl.fmt), s_wo, wl.fmt, m.K)
+    got = y.cpu().numpy()
+    assert np.max(np.abs(got - ref) / np.maximum(np.abs(ref), 1e-30)) <= 1e-6
+
+
+def _sampled_rows(M, n=48, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(M, size=min(n, M), replace=False).tolist())
+    rows |= {0, M - 1}
+    return np.array(sorted(rows))
+
+
+@pytest.mark.parametrize("name", ["ternary_4b", "t4nt_int4"])
+def test_sweep_workloads_sampled(name):
+    wl = wls.WORKLOADS[name]
+    for mi, m in enumerate(wl.matrices):
+        w = wls.workload_weights(wl, mi)
+        packed, s_w = gpu_pack(w, wl.fmt)
+        codes, s_wo = oracle.quantize(w, wl.fmt, 1e-5)
+        assert np.array_equal(s_w.cpu().numpy().view(np.uint32), s_wo.view(np.uint32))
+        bf = wl.x_dtype == wls.BF16
+        for M in wl.Ms:
+            x = wls.workload_activations(wl, mi, M)
+            q, s_x = gpu_act(x, bf)
+            y = bwt.lowbit_linear(q, s_x, packed, s_w, wl.fmt, m.N, bwt.BF16, K=m.K)
+            rows = _sampled_rows(M)
+            q_o, s_xo = oracle.act_quant(x[rows], 0.0, bf16_bits=bf)
+            assert np.array_equal(q.cpu().numpy()[rows, :m.K], q_o)
+            acc = oracle.int_dot(q_o, codes, wl.fmt, nthreads=oracle.max_threads())
+            ref = oracle.rescale(acc, s_wo, s_xo, "bf16")
+            got = bf16_bits(y)[rows]
+            assert ulp_distance_bf16(got, ref).max() <= 1, (name, mi, M)
+
+
+def test_impeto_binary_stack_sampled():
+    wl = wls.WORKLOADS["impeto_binary"]
+    M = wl.Ms[0]
+    for mi in (0, 1, 4, 6, len(wl.matrices) - 1):  # q, k, gate, down, head
+        m = wl.matrices[mi]
+        w = wls.workload_weights(wl, mi)
+        x = wls.workload_activations(wl, mi, M)
+        packed, s_w = gpu_pack(w, wl.fmt)
+        q, s_x = gpu_act(x)
+        y = bwt.lowbit_linear(q, s_x, packed, s_w, wl.fmt, m.N, bwt.F32, K=m.K)
+        rows = _sampled_rows(M, 64, mi)
+        codes, s_wo = oracle.quantize(w, wl.fmt, 1e-5)
+        q_o, s_xo = oracle.act_quant(x[rows])
+        acc = oracle.int_dot(q_o, codes, wl.fmt, nthreads=oracle.max_threads())
+        ref = oracle.rescale(acc, s_wo, s_xo, "f32")
+        got = y.cpu().numpy()[rows]
+        assert np.max(np.abs(got - ref) / np.maximum(np.abs(ref), 1e-30)) <= 1e-6
+
+
+def test_atomic_stack_full():
+    wl = wls.WORKLOADS["atomic_stack"]
+    for mi in (0, 1, 2, 3, len(wl.matrices) - 1):
+        m = wl.matrices[mi]
+        w = wls.workload_weights(wl, mi)
+        packed, s_w = gpu_pack(w, wl.fmt)
+        codes, s_wo = oracle.quantize(w, wl.fmt, 1e-5)
+        for M in wl.Ms:
+            x = wls.workload_activations(wl, mi, M)
+            q, s_x = gpu_act(x)
+            y = bwt.lowbit_linear(q, s_x, packed, s_w, wl.fmt, m.N, bwt.BF16, K=m.K)
+            q_o, s_xo = oracle.act_quant(x)
+            acc = oracle.int_dot(q_o, codes, wl.fmt, nthreads=oracle.max_threads())
+            ref = oracle.rescale(acc, s_wo, s_xo, "bf16")
+            assert ulp_distance_bf16(bf16_bits(y), ref).max() <= 1
