@@ -165,7 +165,7 @@ lowbit_status lowbit_act_quant(const void *x, lowbit_dtype xdt, int64_t M, int64
     if (M <= 0 || K <= 0 || ldx < K || ldq < K || !(eps >= 0.0f) || eps > 3.0e38f) return LOWBIT_ERR_INVALID_ARG;
     if (M > INT32_MAX) return LOWBIT_ERR_INVALID_ARG;
     const int64_t esz = xdt == LOWBIT_F32 ? 4 : 2;
-    if (!aligned(x, 16) || (ldx * esz) % 16 != 0 || !aligned(q, 16) || ldq % 16 != 0 || !aligned(s_x, 4))
+    if (!aligned(x, static_cast<uintptr_t>(esz)) || !aligned(q, 16) || ldq % 16 != 0 || !aligned(s_x, 4))
         return LOWBIT_ERR_ALIGNMENT;
     const lowbit_status d = check_device();
     if (d != LOWBIT_OK) return d;

@@ -151,8 +151,9 @@ act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
     if (r == 0) s_x[row] = amax != 0 ? __fdiv_rn(g, 127.0f) : 0.0f;
 }
 
-// Rows too long for registers: a max pass, then a quantise pass (the second
-// read mostly hits L2).  One 256-thread block per row.
+// Rows too long for registers, or rows without 16-byte alignment: a max
+// pass, then a quantise pass (the second read mostly hits L2), with scalar
+// loads.  One 256-thread block per row.
 template <typename T>
 __global__ void __launch_bounds__(256)
 act_quant_long(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, float eps,
@@ -181,6 +182,13 @@ lowbit_status launch(const void *x, int64_t M, int64_t K, int64_t ldx, float eps
 {
     constexpr int E = In<T>::kPerVec;
     const int64_t nvec = K / E;
+    // 16-byte vector loads need a 16-byte aligned base and row stride; any
+    // other layout takes the scalar-load kernel.
+    const bool vec_ok = (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (ldx * static_cast<int64_t>(sizeof(T))) % 16 == 0;
+    if (!vec_ok) {
+        act_quant_long<T><<<static_cast<unsigned>(M), 256, 0, st>>>(x, M, K, ldx, eps, q, ldq, s_x, status);
+        return launch_status();
+    }
     auto grid_for = [&](int tpr) {
         const int rows = (tpr > 256 ? tpr : 256) / tpr;
         return static_cast<unsigned>((M + rows - 1) / rows);

@@ -138,7 +138,8 @@ lowbit_status lowbit_unpack(const uint8_t *packed, int64_t ldp, int64_t N, int64
  *                  (fp32 multiply, fp32 IEEE divide, nearest even),
  *                  s_x[t] = gamma_t / 127.
  * x is fp32 or bf16 (xdt = LOWBIT_F32 | LOWBIT_BF16), [M, K] with row stride
- * ldx elements; x must be 16-byte aligned and ldx*sizeof(x) a multiple of 16.
+ * ldx elements, aligned to its element size (rows that start on 16-byte
+ * boundaries take the one-pass vector kernel, others a two-pass scalar one).
  * q is int8 [M, ldq], 16-byte aligned, ldq a multiple of 16, ldq >= K; bytes
  * of q past K are left untouched.  s_x is fp32 [M].  eps >= 0 (0 in the
  * configurations this library is measured on).  A non-finite x, or an x*127

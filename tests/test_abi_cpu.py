@@ -96,9 +96,9 @@ def test_act_quant_rejects_bad_arguments(lib):
     assert f(FAKE, bwt.F32, 4, 64, 32, 0.0, FAKE, 64, FAKE, None, None) == bwt.ERR_INVALID_ARG
     assert f(FAKE, bwt.F32, 4, 64, 64, -1.0, FAKE, 64, FAKE, None, None) == bwt.ERR_INVALID_ARG
     assert f(FAKE, bwt.F32, 4, 64, 64, float("nan"), FAKE, 64, FAKE, None, None) == bwt.ERR_INVALID_ARG
-    assert f(FAKE + 4, bwt.F32, 4, 64, 64, 0.0, FAKE, 64, FAKE, None, None) == bwt.ERR_ALIGNMENT
-    assert f(FAKE, bwt.F32, 4, 64, 65, 0.0, FAKE, 64, FAKE, None, None) == bwt.ERR_ALIGNMENT
-    assert f(FAKE, bwt.BF16, 4, 64, 68, 0.0, FAKE, 64, FAKE, None, None) == bwt.ERR_ALIGNMENT
+    assert f(FAKE + 2, bwt.F32, 4, 64, 64, 0.0, FAKE, 64, FAKE, None, None) == bwt.ERR_ALIGNMENT
+    assert f(FAKE + 1, bwt.BF16, 4, 64, 64, 0.0, FAKE, 64, FAKE, None, None) == bwt.ERR_ALIGNMENT
+    assert f(FAKE, bwt.F32, 4, 64, 64, 0.0, FAKE + 8, 64, FAKE, None, None) == bwt.ERR_ALIGNMENT
     assert f(FAKE, bwt.F32, 4, 64, 64, 0.0, FAKE, 72, FAKE, None, None) == bwt.ERR_ALIGNMENT
 
 
