@@ -41,6 +41,7 @@ ABI = {
     "lowbit_max_k": (_I64, [_I32]),
     "lowbit_pack_workspace_bytes": (_SZ, [_I32, _I64]),
     "lowbit_pack": (_I32, [_P, _I64, _I64, _I64, _I32, _F, _P, _I64, _P, _P, _SZ, _P, _P]),
+    "lowbit_pack_ternary_noalloc": (_I32, [_P, _I64, _I64, _I64, _F, _P, _I64, _P, _P, _P]),
     "lowbit_unpack": (_I32, [_P, _I64, _I64, _I64, _I32, _P, _I64, _P, _P]),
     "lowbit_act_quant": (_I32, [_P, _I32, _I64, _I64, _I64, _F, _P, _I64, _P, _P, _P]),
     "lowbit_linear": (_I32, [_P, _I64, _P, _I64, _I64, _P, _I64, _P, _I32, _I64, _P, _I32, _I64, _P, _P]),
@@ -131,6 +132,24 @@ def lowbit_pack(w, fmt: int, eps: float = 1e-5, packed=None, s_w=None, ldp: int 
     st = lib().lowbit_pack(_ptr(w), N, K, w.stride(0), fmt, eps, _ptr(packed), packed.stride(0), _ptr(s_w),
                            _ptr(workspace), need, _ptr(status), _stream(stream))
     _check(st, "lowbit_pack")
+    return packed, s_w
+
+
+def lowbit_pack_ternary_noalloc(w, eps: float = 1e-5, packed=None, s_w=None, ldp: int | None = None,
+                                status=None, stream=None):
+    """Ternary pack that allocates nothing in the library (see lowbit.h);
+    output tensors are still the caller's."""
+    import torch
+    N, K = w.shape
+    if ldp is None:
+        ldp = packed_ld(TERNARY2, K)
+    if packed is None:
+        packed = torch.empty((N, ldp), dtype=torch.uint8, device=w.device)
+    if s_w is None:
+        s_w = torch.empty(1, dtype=torch.float32, device=w.device)
+    st = lib().lowbit_pack_ternary_noalloc(_ptr(w), N, K, w.stride(0), eps, _ptr(packed), packed.stride(0),
+                                           _ptr(s_w), _ptr(status), _stream(stream))
+    _check(st, "lowbit_pack_ternary_noalloc")
     return packed, s_w
 
 

@@ -91,8 +91,11 @@ __device__ __forceinline__ float rescale(int32_t acc, float sw, float sx)
 
 }  // namespace lowbit
 
-// Host-side launch helpers (defined in abi.cu, used by every kernel file).
+// Host-side launch helpers (defined in abi.cu and pack.cu).
 namespace lowbit {
 lowbit_status launch_status();
 int device_sm_count();
+lowbit_status pack_launch(const float *w, int64_t N, int64_t K, int64_t ldw, lowbit_format f, float eps,
+                          uint8_t *packed, int64_t ldp, float *s_w, void *workspace, int32_t *status,
+                          cudaStream_t st);
 }

@@ -14,6 +14,8 @@
 //     max|w_c|/7, 15 levels.  tanh is evaluated here in fp64 by a fixed
 //     sequence (see tanh_fixed) rather than by a library call, so the result
 //     does not depend on a math library's last bit.
+#include <mutex>
+
 #include "lowbit_internal.cuh"
 
 namespace lowbit {
@@ -241,3 +243,66 @@ lowbit_status unpack_launch(const uint8_t *packed, int64_t ldp, int64_t N, int64
 }
 
 }  // namespace lowbit
+
+// ---------------------------------------------------------------------------
+// Ternary packing without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory when they pack: runtimes that fix
+// their device-memory budget at start-up and forbid allocation afterwards, and
+// hosts whose device memory belongs to another allocator that a plain C caller
+// cannot reach (a cudaFree would also synchronise the whole device, stalling
+// their other streams).  For them the fixed-order row sums that the ternary
+// scale needs live in a file-scope device array instead of a workspace.
+// The array is at most kNoAllocMaxRows fp64 values (512 KB) and every GPU
+// that loads the library keeps it until the process exits.
+// ---------------------------------------------------------------------------
+namespace lowbit {
+namespace {
+
+constexpr int64_t kNoAllocMaxRows = LOWBIT_NOALLOC_MAX_ROWS;
+static __device__ __align__(256) double g_noalloc_row_sums[kNoAllocMaxRows];
+
+// Device address of g_noalloc_row_sums, looked up once per device with that
+// device current.  In host code the array's name is only a host-side stand-in,
+// so the kernels must be given this address, never the name.
+double *noalloc_scratch(int dev)
+{
+    static std::mutex mu;
+    static double *addr[64] = {};
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_row_sums) != cudaSuccess || p == nullptr) return nullptr;
+        addr[dev] = static_cast<double *>(p);
+    }
+    return addr[dev];
+}
+
+}  // namespace
+}  // namespace lowbit
+
+extern "C" lowbit_status lowbit_pack_ternary_noalloc(const float *w, int64_t N, int64_t K, int64_t ldw, float eps,
+                                                     uint8_t *packed, int64_t ldp, float *s_w,
+                                                     int32_t *status_dev, void *stream)
+{
+    using namespace lowbit;
+    if (w == nullptr || packed == nullptr || s_w == nullptr) return LOWBIT_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0 || ldw < K || !(eps >= 0.0f) || eps > 3.0e38f) return LOWBIT_ERR_INVALID_ARG;
+    if (N > kNoAllocMaxRows || K > INT32_MAX) return LOWBIT_ERR_INVALID_ARG;
+    if (ldp < static_cast<int64_t>(4 * ((K + 15) / 16))) return LOWBIT_ERR_INVALID_ARG;
+    if (ldp % 16 != 0 || (reinterpret_cast<uintptr_t>(packed) & 15u) != 0 ||
+        (reinterpret_cast<uintptr_t>(w) & 3u) != 0 || (reinterpret_cast<uintptr_t>(s_w) & 3u) != 0)
+        return LOWBIT_ERR_ALIGNMENT;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LOWBIT_ERR_CUDA;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    if (prop.major != 10 || prop.minor != 0) return LOWBIT_ERR_UNSUPPORTED;
+    double *rows = noalloc_scratch(dev);
+    if (rows == nullptr) return LOWBIT_ERR_CUDA;
+    // Every row sum the call reads (rows 0..N-1) is written earlier in the
+    // same call, so nothing left by a previous call is ever read and the
+    // array needs no clearing.
+    return pack_launch(w, N, K, ldw, LOWBIT_TERNARY2, eps, packed, ldp, s_w, rows, status_dev,
+                       static_cast<cudaStream_t>(stream));
+}

@@ -123,6 +123,31 @@ lowbit_status lowbit_pack(const float *w, int64_t N, int64_t K, int64_t ldw,
                           void *workspace, size_t workspace_bytes,
                           int32_t *status_dev, void *stream);
 
+/* Largest N lowbit_pack_ternary_noalloc accepts. */
+#define LOWBIT_NOALLOC_MAX_ROWS 65536
+
+/* lowbit_pack_ternary_noalloc -- lowbit_pack for LOWBIT_TERNARY2 that
+ * allocates nothing and takes no workspace.  (The pages have no counterpart:
+ * this is a deployment variant of the same packer.)  It is for callers that
+ * cannot allocate device memory at packing time: runtimes whose device-memory
+ * budget is fixed at start-up, and hosts whose device memory belongs to an
+ * allocator a C caller cannot reach (a cudaFree would also synchronise the
+ * device and stall their other streams).  The per-row sums of the ternary
+ * scale go to a static device array of LOWBIT_NOALLOC_MAX_ROWS doubles
+ * (512 KB) that every GPU loading the library keeps until exit.
+ *   - N > LOWBIT_NOALLOC_MAX_ROWS returns LOWBIT_ERR_INVALID_ARG; other
+ *     arguments, outputs and errors are exactly those of lowbit_pack.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls share the one array: calls that may overlap on the GPU (on
+ *     different streams, or from several host threads) race and must be
+ *     serialised by the caller.  Each call writes every entry it reads, so
+ *     the contents left by an earlier call never matter. */
+lowbit_status lowbit_pack_ternary_noalloc(const float *w, int64_t N, int64_t K, int64_t ldw,
+                                          float eps, uint8_t *packed, int64_t ldp, float *s_w,
+                                          int32_t *status_dev, void *stream);
+
 /* lowbit_unpack -- decode packed[N, ldp] into int8 codes[N, ldc] (ldc >= K).
  * A reserved field or a non-zero unowned bit sets LOWBIT_ERR_RESERVED_CODE in
  * *status_dev (M8.8 0x0BB: reserved patterns reject); such a code decodes as
