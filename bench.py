@@ -118,13 +118,19 @@ class Point:
         self.ops = 2 * M * m.N * m.K
 
 
-def build_state(wl, device, pool_bytes_target, torch, bwt):
-    """Pack the weights (off the timed path) into a rotating pool and create
-    the activation, code and output buffers."""
+def select_points(wl, only_M=None):
     points = []
     for mi, m in enumerate(wl.matrices):
         for M in sorted(wl.Ms, reverse=True):
-            points.append(Point(mi, m, M))
+            if only_M is None or M in only_M:
+                points.append(Point(mi, m, M))
+    return points
+
+
+def build_state(wl, device, pool_bytes_target, torch, bwt, only_M=None, pool_copies=None):
+    """Pack the weights (off the timed path) into a rotating pool and create
+    the activation, code and output buffers."""
+    points = select_points(wl, only_M)
     packs = []
     for mi, m in enumerate(wl.matrices):
         w = torch.from_numpy(wls.workload_weights(wl, mi)).to(device)
@@ -132,7 +138,7 @@ def build_state(wl, device, pool_bytes_target, torch, bwt):
         packs.append((packed, s_w))
         del w
     per_set = sum(p[0].numel() for p in packs)
-    copies = max(2, int(np.ceil(pool_bytes_target / per_set)))
+    copies = pool_copies or max(2, int(np.ceil(pool_bytes_target / per_set)))
     pool = [[(p.clone(), s) for (p, s) in packs] for _ in range(copies)]
     xs, qs, sxs, ys = {}, {}, {}, {}
     for pt in points:
@@ -162,7 +168,8 @@ def run_gpu_arm(args, wl):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     ydt = bwt.BF16 if wl.y_dtype == wls.BF16 else bwt.F32
-    points, pool, xs, qs, sxs, ys = build_state(wl, device, 3 * L2_BYTES, torch, bwt)
+    only_M = set(int(v) for v in args.points.split(",")) if args.points else None
+    points, pool, xs, qs, sxs, ys = build_state(wl, device, 3 * L2_BYTES, torch, bwt, only_M, args.pool_copies)
     stream = torch.cuda.current_stream()
     counter = [0]
 
@@ -172,13 +179,15 @@ def run_gpu_arm(args, wl):
             key = (pt.mi, pt.M)
             packed, s_w = pool[counter[0] % len(pool)][pt.mi]
             counter[0] += 1
-            bwt.lowbit_act_quant(xs[key], 0.0, q=qs[key], s_x=sxs[key], stream=stream)
             if events is not None:
                 events[i][0].record(stream)
+            bwt.lowbit_act_quant(xs[key], 0.0, q=qs[key], s_x=sxs[key], stream=stream)
+            if events is not None:
+                events[i][1].record(stream)
             bwt.lowbit_linear(qs[key], sxs[key], packed, s_w, wl.fmt, pt.m.N, ydt, K=pt.m.K, y=ys[key],
                               stream=stream)
             if events is not None:
-                events[i][1].record(stream)
+                events[i][2].record(stream)
             launches += 2  # act quant + one linear kernel (GEMV for M <= 16, else GEMM)
         return launches
 
@@ -186,7 +195,7 @@ def run_gpu_arm(args, wl):
         step()
     torch.cuda.synchronize()
 
-    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in points]
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in points]
            for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
@@ -211,13 +220,13 @@ def run_gpu_arm(args, wl):
         elapsed_ms = float(t.item())
 
     # per-point device times (ms per launch, averaged over the timed steps)
-    per_point = []
+    per_point, per_act = [], []
     for i, pt in enumerate(points):
-        ms = statistics.mean(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(args.steps))
-        per_point.append(ms)
+        per_act.append(statistics.mean(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(args.steps)))
+        per_point.append(statistics.mean(evs[s][i][1].elapsed_time(evs[s][i][2]) for s in range(args.steps)))
 
     # end to end through the public API with host buffers (pinned), one replica
-    e2e = run_e2e(args, wl, points, pool, qs, sxs, ys, torch, bwt, stream, ydt)
+    e2e = None if args.no_e2e else run_e2e(args, wl, points, pool, qs, sxs, ys, torch, bwt, stream, ydt)
 
     if world > 1:
         torch.distributed.destroy_process_group()
@@ -234,10 +243,14 @@ def run_gpu_arm(args, wl):
     pts_out = []
     gemv_bytes = gemv_ms = 0.0
     big_ops = big_ms = 0.0
-    for pt, ms in zip(points, per_point):
+    xbytes = 2 if wl.x_dtype == wls.BF16 else 4
+    for pt, ms, ams in zip(points, per_point, per_act):
         fmt_bits = {wls.TERNARY2: 2, wls.BINARY1: 1, wls.INT4: 4}[wl.fmt]
         packed_bytes = pt.m.N * pt.m.K * fmt_bits // 8
-        d = {"matrix": f"{pt.m.K}->{pt.m.N}", "M": pt.M, "kernel": pt.kernel, "us": round(ms * 1e3, 2)}
+        act_bytes = pt.M * pt.m.K * (xbytes + 1) + 4 * pt.M
+        d = {"matrix": f"{pt.m.K}->{pt.m.N}", "M": pt.M, "kernel": pt.kernel, "us": round(ms * 1e3, 2),
+             "act_quant_us": round(ams * 1e3, 2),
+             "act_quant_gbs": round(act_bytes / (ams * 1e-3) / 1e9, 1)}
         if pt.M <= 16:
             gbs = packed_bytes / (ms * 1e-3) / 1e9
             d.update(packed_gbs=round(gbs, 1), frac_hbm=round(gbs / hbm, 3))
@@ -372,7 +385,7 @@ def oracle_sample_step(wl, rows_per_point, nthreads, cache):
 def run_cpu_baseline(wl, seconds_target):
     import oracle
     oracle.build()
-    nthreads = os.cpu_count() or 1
+    nthreads = oracle.max_threads()
     cache = {}
     rows = 1
     oracle_sample_step(wl, rows, nthreads, cache)  # warm: quantise weights
@@ -401,7 +414,7 @@ def run_reference_arm(args, wl):
         return None
     import oracle
     oracle.build()
-    nthreads = os.cpu_count() or 1
+    nthreads = oracle.max_threads()
     cache = {}
     rows = 16
     oracle_sample_step(wl, rows, nthreads, cache)
@@ -437,6 +450,10 @@ def main(argv=None):
     ap.add_argument("--workload", default="ternary_4b", choices=sorted(wls.WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--points", default=None, help="comma-separated subset of the sweep's M values")
+    ap.add_argument("--pool-copies", type=int, default=None,
+                    help="number of packed weight copies to rotate over (default: enough to exceed 3x L2)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -385,8 +385,8 @@ int orc_act_quant_bf16(const uint16_t *x, long M, long K, long ldx, float eps,
  * adds the activation, c = -1 subtracts it, c = 0 skips it.  4-bit codes
  * multiply.  The worst case |acc| <= 128 * cmax * K must fit int32
  * [M8.8 §0x09C]: K > INT32_MAX / (128 * cmax) returns ORC_EOVERFLOW.
- * Rows t are independent; nthreads > 1 splits them across OpenMP threads
- * without changing any result. */
+ * Every (t, n) pair is independent; nthreads > 1 splits the pairs across
+ * OpenMP threads without changing any result. */
 int orc_int_dot(const int8_t *q, long ldq, const int8_t *codes, long M, long N, long K,
                 int fmt, int64_t *acc, int nthreads)
 {
@@ -395,11 +395,11 @@ int orc_int_dot(const int8_t *q, long ldq, const int8_t *codes, long M, long N, 
     if (K > 2147483647L / (128L * cmax)) return ORC_EOVERFLOW;
 #ifdef _OPENMP
     if (nthreads < 1) nthreads = 1;
-#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#pragma omp parallel for collapse(2) schedule(static) num_threads(nthreads)
 #endif
     for (long t = 0; t < M; ++t) {
-        const int8_t *qt = q + t * ldq;
         for (long n = 0; n < N; ++n) {
+            const int8_t *qt = q + t * ldq;
             const int8_t *cn = codes + n * K;
             int64_t a = 0;
             if (fmt == ORC_INT4) {
