@@ -21,7 +21,7 @@ INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE,
-          "--expt-relaxed-constexpr", "-Xptxas", "-v"]
+          "-Xptxas", "-v"]
 PER_FILE = {"pack.cu": ["-fmad=false"]}
 
 

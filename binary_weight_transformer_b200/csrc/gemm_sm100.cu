@@ -38,10 +38,19 @@ constexpr int E_BYTES = BN * BK;
 constexpr int kThreads = 320;
 constexpr int kExpThreads = 128;
 constexpr uint32_t kTmemCols = 512;
-constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
+// Wait bound in SM clock cycles: 4e9 cycles is about 2 s at the B200's clocks.
+constexpr long long kWaitCycles = 4000000000ll;
 
-template <int FMT> constexpr int packed_bytes_per_kblock() { return BK * Fmt<FMT>::kBits / 8; }
-template <int FMT> constexpr int stages() { return FMT == kI4 ? 3 : 4; }
+template <int FMT> __host__ __device__ constexpr int packed_bytes_per_kblock() { return BK * Fmt<FMT>::kBits / 8; }
+// Ring depths: TMA stages (activation tile + packed tile) and expanded-tile
+// stages, chosen to fit 227 KB of shared memory with the epilogue staging.
+template <int FMT> __host__ __device__ constexpr int tma_stages() { return FMT == kI4 ? 4 : (FMT == kT2 ? 5 : 6); }
+constexpr int kExpStages = 2;
+// Epilogue staging: per epilogue warp, 32 rows of one 32-column chunk, rows
+// padded by 16 bytes so the row-wise writes and the column-wise reads are
+// free of bank conflicts.
+template <int OUT> __host__ __device__ constexpr int stage_row_bytes() { return OUT == LOWBIT_BF16 ? 80 : 144; }
+template <int OUT> __host__ __device__ constexpr int stage_warp_bytes() { return 32 * stage_row_bytes<OUT>(); }
 
 // ---------------------------------------------------------------------------
 // PTX wrappers
@@ -51,12 +60,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p)
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ unsigned long long globaltimer()
-{
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
 {
@@ -89,17 +92,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 
 
 // Bounded wait: true once the phase with `parity` has completed; false if the
-// CTA aborted or `limit_ns` passed (then the timeout is recorded).
+// CTA aborted or `limit` SM cycles passed (then the timeout is recorded).
 __device__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int32_t *status,
-                         unsigned long long limit_ns = kWaitNs)
+                         long long limit = kWaitCycles)
 {
     if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = globaltimer();
+    const long long t0 = clock64();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 63u) == 0) {
             if (*abort_flag) return false;
-            if (globaltimer() - t0 > limit_ns) {
+            if (clock64() - t0 > limit) {
                 *abort_flag = 1;
                 report(status, LOWBIT_ERR_TIMEOUT);
                 return false;
@@ -119,6 +122,19 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -174,86 +190,137 @@ constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<ui
                             (static_cast<uint32_t>(BM >> 4) << 24);
 
 // ---------------------------------------------------------------------------
-// Expansion of one stage: 256 rows x 128 codes, one (row, 16-code chunk) per
-// thread and step; output row r chunk c goes to r*128 + ((c ^ (r%8)) * 16),
-// the 128B-swizzle pattern the TMA uses for the activation tile.
+// Expansion of one stage: 256 rows x 128 codes.  Each thread loads 16 bytes of
+// packed codes at a time (ld.shared.v4) and writes whole 16-code chunks of the
+// int8 tile (st.shared.v4); chunk c of row r goes to r*128 + ((c ^ (r%8))*16),
+// the 128B-swizzle pattern the TMA uses for the activation tile.  Within every
+// group of 8 lanes the loads cover 128 contiguous bytes and the stores hit 8
+// distinct 16-byte bank groups, so neither conflicts.
 // ---------------------------------------------------------------------------
 template <int FMT>
-__device__ __forceinline__ void expand_stage(const uint8_t *P, uint8_t *E, int et)
+__device__ __forceinline__ void expand_stage(uint32_t P, uint32_t E, int et)
 {
-    constexpr int PB = packed_bytes_per_kblock<FMT>();
-    const int c = et & 7;
-#pragma unroll 4
-    for (int r = et >> 3; r < BN; r += kExpThreads / 8) {
-        uint4 out;
-        if constexpr (FMT == kT2) {
-            const uint32_t w = *reinterpret_cast<const uint32_t *>(P + r * PB + c * 4);
-            out = make_uint4(t2_expand(w, 0), t2_expand(w, 1), t2_expand(w, 2), t2_expand(w, 3));
-        } else if constexpr (FMT == kI4) {
-            const uint2 w = *reinterpret_cast<const uint2 *>(P + r * PB + c * 8);
-            out = make_uint4(i4_expand(w.x, 0), i4_expand(w.x, 1), i4_expand(w.y, 0), i4_expand(w.y, 1));
-        } else {
-            const uint32_t w = *reinterpret_cast<const uint32_t *>(P + r * PB + (c >> 1) * 4) >> (16 * (c & 1));
-            out = make_uint4(b1_expand_nibble(w & 0xFu), b1_expand_nibble((w >> 4) & 0xFu),
-                             b1_expand_nibble((w >> 8) & 0xFu), b1_expand_nibble((w >> 12) & 0xFu));
+    if constexpr (FMT == kT2) {
+        // 32 packed bytes per row: item = (row, half), half = 4 chunks.
+#pragma unroll
+        for (int j = 0; j < (BN * 2) / kExpThreads; ++j) {
+            const int i = et + kExpThreads * j;
+            const int r = i >> 1, h = i & 1;
+            const uint4 w = lds128(P + r * 32 + h * 16);
+            const uint32_t rowE = E + r * 128;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t wk = (&w.x)[k];
+                const int c = 4 * h + k;
+                sts128(rowE + ((c ^ (r & 7)) << 4),
+                       make_uint4(t2_expand(wk, 0), t2_expand(wk, 1), t2_expand(wk, 2), t2_expand(wk, 3)));
+            }
         }
-        *reinterpret_cast<uint4 *>(E + r * 128 + ((c ^ (r & 7)) << 4)) = out;
+    } else if constexpr (FMT == kI4) {
+        // 64 packed bytes per row: item = (row, quarter), quarter = 2 chunks.
+#pragma unroll
+        for (int j = 0; j < (BN * 4) / kExpThreads; ++j) {
+            const int i = et + kExpThreads * j;
+            const int r = i >> 2, qd = i & 3;
+            const uint4 w = lds128(P + r * 64 + qd * 16);
+            const uint32_t rowE = E + r * 128;
+            sts128(rowE + (((2 * qd) ^ (r & 7)) << 4),
+                   make_uint4(i4_expand(w.x, 0), i4_expand(w.x, 1), i4_expand(w.y, 0), i4_expand(w.y, 1)));
+            sts128(rowE + (((2 * qd + 1) ^ (r & 7)) << 4),
+                   make_uint4(i4_expand(w.z, 0), i4_expand(w.z, 1), i4_expand(w.w, 0), i4_expand(w.w, 1)));
+        }
+    } else {
+        // 16 packed bytes per row: item = row, 8 chunks of 16 codes (16 bits).
+#pragma unroll
+        for (int j = 0; j < BN / kExpThreads; ++j) {
+            const int r = et + kExpThreads * j;
+            const uint4 w = lds128(P + r * 16);
+            const uint32_t rowE = E + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint32_t h = (&w.x)[c >> 1] >> (16 * (c & 1));
+                sts128(rowE + ((c ^ (r & 7)) << 4),
+                       make_uint4(b1_expand_nibble(h & 0xFu), b1_expand_nibble((h >> 4) & 0xFu),
+                                  b1_expand_nibble((h >> 8) & 0xFu), b1_expand_nibble((h >> 12) & 0xFu)));
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Epilogue for one 32-column chunk of one warp's 32 rows.
+// v[i] is the accumulator of (row = this lane, column nc + i).
+// ---------------------------------------------------------------------------
+template <int OUT>
+__device__ __forceinline__ uint32_t out_word(const uint32_t (&v)[32], const float (&sw)[32], float sx, int shift,
+                                             int j)
+{
+    if constexpr (OUT == LOWBIT_I32) {
+        return static_cast<uint32_t>(static_cast<int32_t>(v[j]) >> shift);
+    } else if constexpr (OUT == LOWBIT_F32) {
+        return __float_as_uint(rescale(static_cast<int32_t>(v[j]) >> shift, sw[j], sx));
+    } else {
+        const float a = rescale(static_cast<int32_t>(v[2 * j]) >> shift, sw[2 * j], sx);
+        const float b = rescale(static_cast<int32_t>(v[2 * j + 1]) >> shift, sw[2 * j + 1], sx);
+        const __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
+        return *reinterpret_cast<const uint32_t *>(&p);
     }
 }
 
 template <int OUT>
-__device__ __forceinline__ void store_row32(void *y, int64_t row, int64_t ldy, int64_t n0, int64_t N,
-                                            const uint32_t (&v)[32], int shift, const float *s_w, bool sw_per_row,
-                                            float sx, bool vec_ok)
+__device__ __forceinline__ void epilogue_chunk(const uint32_t (&v)[32], const float (&sw)[32], float sx, int shift,
+                                               void *__restrict__ y, int64_t ldy, int64_t row0, int64_t M,
+                                               int64_t nc, int64_t N, bool vec_ok, uint32_t stage, int lane)
 {
-    const bool full = (n0 + 32 <= N);
-    if constexpr (OUT == LOWBIT_I32) {
-        int32_t *yr = static_cast<int32_t *>(y) + row * ldy + n0;
-        if (full && vec_ok) {
+    constexpr int kWords = OUT == LOWBIT_BF16 ? 16 : 32;   // 32-bit words per row of the chunk
+    constexpr int kEsz = OUT == LOWBIT_BF16 ? 2 : 4;
+    constexpr int RS = stage_row_bytes<OUT>();
+    const int64_t row = row0 + lane;
+    if (vec_ok && nc + 32 <= N) {
+        // rows -> staging (row-wise), then staging -> global (column pieces)
 #pragma unroll
-            for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<int4 *>(yr + i) =
-                    make_int4(static_cast<int32_t>(v[i]) >> shift, static_cast<int32_t>(v[i + 1]) >> shift,
-                              static_cast<int32_t>(v[i + 2]) >> shift, static_cast<int32_t>(v[i + 3]) >> shift);
-        } else {
-            for (int i = 0; i < 32 && n0 + i < N; ++i) yr[i] = static_cast<int32_t>(v[i]) >> shift;
+        for (int p = 0; p < kWords / 4; ++p)
+            sts128(stage + lane * RS + p * 16,
+                   make_uint4(out_word<OUT>(v, sw, sx, shift, 4 * p), out_word<OUT>(v, sw, sx, shift, 4 * p + 1),
+                              out_word<OUT>(v, sw, sx, shift, 4 * p + 2), out_word<OUT>(v, sw, sx, shift, 4 * p + 3)));
+        __syncwarp();
+        constexpr int kPieces = kWords / 4;        // 16-byte pieces per row
+        constexpr int kRowsPerPass = 32 / kPieces;
+#pragma unroll
+        for (int pass = 0; pass < kPieces; ++pass) {
+            const int r = pass * kRowsPerPass + lane / kPieces;
+            const int piece = lane % kPieces;
+            const uint4 val = lds128(stage + r * RS + piece * 16);
+            if (row0 + r < M) {
+                char *dst = static_cast<char *>(y) + ((row0 + r) * ldy + nc) * kEsz + piece * 16;
+                *reinterpret_cast<uint4 *>(dst) = val;
+            }
         }
-    } else {
-        float f[32];
-        const float sw0 = s_w[0];
+        __syncwarp();
+    } else if (row < M) {
+        // ragged column tail or unaligned output: element stores
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            const float sw = sw_per_row ? ((n0 + i < N) ? __ldg(s_w + n0 + i) : 0.0f) : sw0;
-            f[i] = rescale(static_cast<int32_t>(v[i]) >> shift, sw, sx);
-        }
-        if constexpr (OUT == LOWBIT_F32) {
-            float *yr = static_cast<float *>(y) + row * ldy + n0;
-            if (full && vec_ok) {
-#pragma unroll
-                for (int i = 0; i < 32; i += 4)
-                    *reinterpret_cast<float4 *>(yr + i) = make_float4(f[i], f[i + 1], f[i + 2], f[i + 3]);
-            } else {
-                for (int i = 0; i < 32 && n0 + i < N; ++i) yr[i] = f[i];
-            }
-        } else {
-            __nv_bfloat16 *yr = static_cast<__nv_bfloat16 *>(y) + row * ldy + n0;
-            if (full && vec_ok) {
-#pragma unroll
-                for (int i = 0; i < 32; i += 8) {
-                    uint4 pk;
-                    uint32_t *pw = &pk.x;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(f[i + 2 * j], f[i + 2 * j + 1]);
-                        pw[j] = *reinterpret_cast<const uint32_t *>(&b2);
-                    }
-                    *reinterpret_cast<uint4 *>(yr + i) = pk;
+            if (nc + i < N) {
+                const int32_t a = static_cast<int32_t>(v[i]) >> shift;
+                if constexpr (OUT == LOWBIT_I32) {
+                    static_cast<int32_t *>(y)[row * ldy + nc + i] = a;
+                } else if constexpr (OUT == LOWBIT_F32) {
+                    static_cast<float *>(y)[row * ldy + nc + i] = rescale(a, sw[i], sx);
+                } else {
+                    static_cast<__nv_bfloat16 *>(y)[row * ldy + nc + i] = __float2bfloat16_rn(rescale(a, sw[i], sx));
                 }
-            } else {
-                for (int i = 0; i < 32 && n0 + i < N; ++i) yr[i] = __float2bfloat16_rn(f[i]);
             }
         }
     }
+}
+
+template <int FMT, int OUT>
+__host__ __device__ constexpr size_t smem_bytes()
+{
+    return 1024 + static_cast<size_t>(tma_stages<FMT>()) * (A_BYTES + BN * packed_bytes_per_kblock<FMT>()) +
+           static_cast<size_t>(kExpStages) * E_BYTES + 4 * stage_warp_bytes<OUT>() +
+           8 * (2 * tma_stages<FMT>() + 2 * kExpStages + 8);
 }
 
 template <int FMT, int OUT>
@@ -262,34 +329,40 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
             const float *__restrict__ s_x, const float *__restrict__ s_w, int64_t M, int64_t N, int64_t K,
             void *__restrict__ y, int64_t ldy, int vec_ok, int32_t *status)
 {
-    constexpr int S = stages<FMT>();
+    constexpr int ST = tma_stages<FMT>();
+    constexpr int SE = kExpStages;
     constexpr int PB = packed_bytes_per_kblock<FMT>();
     constexpr int P_BYTES = BN * PB;
     constexpr int kShift = Fmt<FMT>::kShift;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sA = base;                       // S x 16 KB
-    uint8_t *sE = sA + S * A_BYTES;           // S x 32 KB
-    uint8_t *sP = sE + S * E_BYTES;           // S x P_BYTES
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sP + S * P_BYTES);
+    uint8_t *sA = base;                        // ST x 16 KB, 1024-aligned
+    uint8_t *sE = sA + ST * A_BYTES;           // SE x 32 KB, 1024-aligned
+    uint8_t *sP = sE + SE * E_BYTES;           // ST x P_BYTES
+    uint8_t *sStage = sP + ST * P_BYTES;       // 4 x epilogue staging
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sStage + 4 * stage_warp_bytes<OUT>());
     uint64_t *full_tma = bars;
-    uint64_t *full_exp = bars + S;
-    uint64_t *empty = bars + 2 * S;
-    uint64_t *acc_full = bars + 3 * S;
-    uint64_t *acc_empty = bars + 3 * S + 2;
-    uint64_t *drain = bars + 3 * S + 4;
-    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(bars + 3 * S + 5);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 3 * S + 6);
+    uint64_t *empty_tma = bars + ST;
+    uint64_t *full_exp = bars + 2 * ST;
+    uint64_t *empty_exp = bars + 2 * ST + SE;
+    uint64_t *acc_full = bars + 2 * ST + 2 * SE;
+    uint64_t *acc_empty = acc_full + 2;
+    uint64_t *drain = acc_full + 4;
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(acc_full + 5);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(acc_full + 6);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
+        for (int s = 0; s < ST; ++s) {
             mbar_init(&full_tma[s], 1);
+            mbar_init(&empty_tma[s], 1);
+        }
+        for (int s = 0; s < SE; ++s) {
             mbar_init(&full_exp[s], kExpThreads);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty_exp[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
@@ -325,9 +398,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
                 const int m0 = static_cast<int>((tile % num_m) * BM);
                 const int n0 = static_cast<int>((tile / num_m) * BN);
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
-                    const int s = g % S;
-                    const uint32_t ph = (g / S) & 1u;
-                    if (!wait_bar(&empty[s], ph ^ 1u, abort_flag, status)) { ok = false; break; }
+                    const int s = g % ST;
+                    const uint32_t ph = (g / ST) & 1u;
+                    if (!wait_bar(&empty_tma[s], ph ^ 1u, abort_flag, status)) { ok = false; break; }
                     mbar_arrive_expect_tx(&full_tma[s], A_BYTES + P_BYTES);
                     tma_load_2d(sA + s * A_BYTES, &map_a, &full_tma[s], kb * BK, m0);
                     tma_load_2d(sP + s * P_BYTES, &map_p, &full_tma[s], kb * PB, n0);
@@ -335,9 +408,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
             }
             if (!ok) {
                 // Let copies already issued land before the CTA leaves.
-                for (uint32_t i = 0; i < S && i < g; ++i) {
+                for (uint32_t i = 0; i < ST && i < g; ++i) {
                     const uint32_t gi = g - 1 - i;
-                    wait_bar(&full_tma[gi % S], (gi / S) & 1u, abort_flag, nullptr, 100000000ull);
+                    wait_bar(&full_tma[gi % ST], (gi / ST) & 1u, abort_flag, nullptr, 200000000ll);
                 }
             }
         }
@@ -354,47 +427,50 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BN);
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
-                    const int s = g % S;
-                    const uint32_t ph = (g / S) & 1u;
-                    if (!wait_bar(&full_tma[s], ph, abort_flag, status) ||
-                        !wait_bar(&full_exp[s], ph, abort_flag, status)) { ok = false; break; }
+                    const int s1 = g % ST, s2 = g % SE;
+                    if (!wait_bar(&full_tma[s1], (g / ST) & 1u, abort_flag, status) ||
+                        !wait_bar(&full_exp[s2], (g / SE) & 1u, abort_flag, status)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a_addr = smem_u32(sA + s * A_BYTES);
-                    const uint32_t e_addr = smem_u32(sE + s * E_BYTES);
+                    const uint32_t a_addr = smem_u32(sA + s1 * A_BYTES);
+                    const uint32_t e_addr = smem_u32(sE + s2 * E_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < BK / UMMA_K; ++kk)
                         tc_mma_i8(d_tmem, sw128_desc(a_addr + kk * UMMA_K), sw128_desc(e_addr + kk * UMMA_K),
                                   kIdesc, (kb | kk) != 0 ? 1u : 0u);
-                    tc_commit(&empty[s]);
+                    tc_commit(&empty_tma[s1]);
+                    tc_commit(&empty_exp[s2]);
                 }
                 if (!ok) break;
                 tc_commit(&acc_full[b]);
             }
             // All MMAs this thread issued are complete once `drain` flips.
             tc_commit(drain);
-            wait_bar(drain, 0, abort_flag, nullptr, 100000000ull);
+            wait_bar(drain, 0, abort_flag, nullptr, 200000000ll);
         }
     } else if (warp < 6) {
         // ---------------- expanders ----------------
         const int et = threadIdx.x - 64;
+        const uint32_t p_base = smem_u32(sP);
+        const uint32_t e_base = smem_u32(sE);
         uint32_t g = 0;
         bool ok = true;
         for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
             for (int kb = 0; kb < nkb; ++kb, ++g) {
-                const int s = g % S;
-                const uint32_t ph = (g / S) & 1u;
-                if (!wait_bar(&full_tma[s], ph, abort_flag, status)) { ok = false; break; }
-                expand_stage<FMT>(sP + s * P_BYTES, sE + s * E_BYTES, et);
+                const int s1 = g % ST, s2 = g % SE;
+                if (!wait_bar(&full_tma[s1], (g / ST) & 1u, abort_flag, status) ||
+                    !wait_bar(&empty_exp[s2], ((g / SE) & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
+                expand_stage<FMT>(p_base + s1 * P_BYTES, e_base + s2 * E_BYTES, et);
                 // Each writer orders its generic-proxy stores before the
                 // tensor core's async-proxy reads, then arrives.
                 fence_proxy_async_smem();
-                mbar_arrive(&full_exp[s]);
+                mbar_arrive(&full_exp[s2]);
             }
         }
     } else {
         // ---------------- epilogue ----------------
         const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
-        const bool sw_per_row = (FMT != kT2);
+        const uint32_t stage = smem_u32(sStage) + static_cast<uint32_t>((warp - 6) * stage_warp_bytes<OUT>());
+        const float sw_tensor = (FMT == kT2) ? s_w[0] : 0.0f;
         uint32_t t = 0;
         for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t) {
             const int b = t & 1;
@@ -408,17 +484,22 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
             tc_fence_after();
             const int64_t m0 = (tile % num_m) * BM;
             const int64_t n0 = (tile / num_m) * BN;
-            const int64_t row = m0 + quarter * 32 + lane;
-            const float sx = row < M ? s_x[row] : 0.0f;
+            const int64_t row0 = m0 + quarter * 32;
+            const float sx = (row0 + lane < M) ? s_x[row0 + lane] : 0.0f;
 #pragma unroll 1
             for (int cc = 0; cc < BN / 32; ++cc) {
+                const int64_t nc = n0 + cc * 32;
                 uint32_t v[32];
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                        static_cast<uint32_t>(b * BN + cc * 32);
                 tmem_ld_32cols(taddr, v);
-                const int64_t nc = n0 + cc * 32;
-                if (row < M && nc < N)
-                    store_row32<OUT>(y, row, ldy, nc, N, v, kShift, s_w, sw_per_row, sx, vec_ok != 0);
+                if (nc < N) {
+                    float sw[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        sw[i] = (FMT == kT2) ? sw_tensor : ((nc + i < N) ? __ldg(s_w + nc + i) : 0.0f);
+                    epilogue_chunk<OUT>(v, sw, sx, kShift, y, ldy, row0, M, nc, N, vec_ok != 0, stage, lane);
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -470,19 +551,13 @@ bool make_map_2d(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_t out
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int FMT>
-constexpr size_t smem_bytes()
-{
-    return 1024 + stages<FMT>() * (A_BYTES + E_BYTES + BN * packed_bytes_per_kblock<FMT>()) + 3 * stages<FMT>() * 8 +
-           64;
-}
-
 template <int FMT, int OUT>
 lowbit_status launch_t(const CUtensorMap &ma, const CUtensorMap &mp, const float *s_x, const float *s_w,
                        int64_t M, int64_t N, int64_t K, void *y, int64_t ldy, int vec_ok, int32_t *status,
                        cudaStream_t st)
 {
-    constexpr size_t smem = smem_bytes<FMT>();
+    constexpr size_t smem = smem_bytes<FMT, OUT>();
+    static_assert(smem <= 232448, "shared memory budget");
     static bool configured[64] = {};  // the attribute is set once per device
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LOWBIT_ERR_CUDA;

@@ -14,7 +14,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
-#include "../../include/lowbit.h"
+#include "lowbit.h"
 
 namespace lowbit {
 
