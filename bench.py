@@ -109,6 +109,61 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# CUDA runtime events that can live inside a captured graph
+# ---------------------------------------------------------------------------
+class GraphEvents:
+    """cudaEvent objects recorded with cudaEventRecordExternal, so that a
+    recording made during stream capture becomes an event-record node that
+    timestamps the graph's execution (a plain record inside a capture only
+    orders work)."""
+    EXTERNAL = 0x1
+
+    def __init__(self):
+        import ctypes
+        import torch
+        torch.cuda.init()
+        self.ct = ctypes
+        self.rt = self._find_cudart()
+        self.rt.cudaEventCreate.argtypes = [ctypes.c_void_p]
+        self.rt.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
+        self.rt.cudaEventElapsedTime.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+        self.rt.cudaEventDestroy.argtypes = [ctypes.c_void_p]
+        self.events = []
+
+    @staticmethod
+    def _find_cudart():
+        import ctypes
+        with open("/proc/self/maps") as f:
+            for line in f:
+                path = line.split()[-1] if "/" in line else ""
+                if "libcudart.so" in path:
+                    return ctypes.CDLL(path)
+        return ctypes.CDLL("libcudart.so.12")
+
+    def new(self):
+        ev = self.ct.c_void_p()
+        if self.rt.cudaEventCreate(self.ct.byref(ev)) != 0:
+            raise RuntimeError("cudaEventCreate failed")
+        self.events.append(ev)
+        return ev
+
+    def record(self, ev, stream):
+        if self.rt.cudaEventRecordWithFlags(ev, self.ct.c_void_p(stream.cuda_stream), self.EXTERNAL) != 0:
+            raise RuntimeError("cudaEventRecordWithFlags failed")
+
+    def elapsed_ms(self, a, b):
+        out = self.ct.c_float()
+        if self.rt.cudaEventElapsedTime(self.ct.byref(out), a, b) != 0:
+            raise RuntimeError("cudaEventElapsedTime failed")
+        return out.value
+
+    def close(self):
+        for ev in self.events:
+            self.rt.cudaEventDestroy(ev)
+        self.events = []
+
+
+# ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
 class Point:
@@ -139,6 +194,8 @@ def build_state(wl, device, pool_bytes_target, torch, bwt, only_M=None, pool_cop
         del w
     per_set = sum(p[0].numel() for p in packs)
     copies = pool_copies or max(2, int(np.ceil(pool_bytes_target / per_set)))
+    # every launch of a step reads its own copy, so a step never re-reads
+    # weights from L2: at least one copy per point
     pool = [[(p.clone(), s) for (p, s) in packs] for _ in range(copies)]
     xs, qs, sxs, ys = {}, {}, {}, {}
     for pt in points:
@@ -171,32 +228,47 @@ def run_gpu_arm(args, wl):
     only_M = set(int(v) for v in args.points.split(",")) if args.points else None
     points, pool, xs, qs, sxs, ys = build_state(wl, device, 3 * L2_BYTES, torch, bwt, only_M, args.pool_copies)
     stream = torch.cuda.current_stream()
-    counter = [0]
+    gev = GraphEvents()
+    n_sets = len(pool)
 
-    def step(events=None):
+    def step(s, events=None):
+        """One pass of the hot path; weights come from pool set s (each point
+        of the step reads its own copy).  `events` adds external event-record
+        nodes around every launch."""
+        st = torch.cuda.current_stream()
         launches = 0
         for i, pt in enumerate(points):
             key = (pt.mi, pt.M)
-            packed, s_w = pool[counter[0] % len(pool)][pt.mi]
-            counter[0] += 1
+            packed, s_w = pool[(s * len(points) + i) % n_sets][pt.mi]
             if events is not None:
-                events[i][0].record(stream)
-            bwt.lowbit_act_quant(xs[key], 0.0, q=qs[key], s_x=sxs[key], stream=stream)
+                gev.record(events[i][0], st)
+            bwt.lowbit_act_quant(xs[key], 0.0, q=qs[key], s_x=sxs[key])
             if events is not None:
-                events[i][1].record(stream)
-            bwt.lowbit_linear(qs[key], sxs[key], packed, s_w, wl.fmt, pt.m.N, ydt, K=pt.m.K, y=ys[key],
-                              stream=stream)
+                gev.record(events[i][1], st)
+            bwt.lowbit_linear(qs[key], sxs[key], packed, s_w, wl.fmt, pt.m.N, ydt, K=pt.m.K, y=ys[key])
             if events is not None:
-                events[i][2].record(stream)
+                gev.record(events[i][2], st)
             launches += 2  # act quant + one linear kernel (GEMV for M <= 16, else GEMM)
         return launches
 
-    for _ in range(args.warmup):
-        step()
+    # eager warm-up (sets kernel attributes, loads modules), then one captured
+    # graph per timed step, each with its own events
+    for w in range(args.warmup):
+        step(w)
+    torch.cuda.synchronize()
+    evs = [[[gev.new() for _ in range(3)] for _ in points] for _ in range(args.steps)]
+    graphs = []
+    launches_per_step = 0
+    for s_ in range(args.steps):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            launches_per_step = step(s_, evs[s_])
+        graphs.append(g)
+    torch.cuda.synchronize()
+    for w in range(min(args.warmup, len(graphs))):
+        graphs[w].replay()
     torch.cuda.synchronize()
 
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in points]
-           for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
     if world > 1:
@@ -205,12 +277,12 @@ def run_gpu_arm(args, wl):
     sampler.start()
     time.sleep(0.3)
     t_start.record(stream)
-    launches = 0
-    for s in range(args.steps):
-        launches += step(evs[s])
+    for g in graphs:
+        g.replay()
     t_end.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
+    launches = launches_per_step * args.steps
     if world > 1:
         torch.distributed.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
@@ -222,8 +294,10 @@ def run_gpu_arm(args, wl):
     # per-point device times (ms per launch, averaged over the timed steps)
     per_point, per_act = [], []
     for i, pt in enumerate(points):
-        per_act.append(statistics.mean(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(args.steps)))
-        per_point.append(statistics.mean(evs[s][i][1].elapsed_time(evs[s][i][2]) for s in range(args.steps)))
+        per_act.append(statistics.mean(gev.elapsed_ms(evs[s][i][0], evs[s][i][1]) for s in range(args.steps)))
+        per_point.append(statistics.mean(gev.elapsed_ms(evs[s][i][1], evs[s][i][2]) for s in range(args.steps)))
+    del graphs
+    gev.close()
 
     # end to end through the public API with host buffers (pinned), one replica
     e2e = None if args.no_e2e else run_e2e(args, wl, points, pool, qs, sxs, ys, torch, bwt, stream, ydt)
@@ -295,7 +369,9 @@ def run_gpu_arm(args, wl):
         "dtype": "int8 x ternary -> int32 (bf16 in/out)" if wl.fmt == wls.TERNARY2 else "int8 x low-bit -> int32",
         "data": "synthetic (seeded N(0,1) activations with outliers, N(0,0.02) weights)",
         "config": {"workload": f"{wl.name}: " + ", ".join(f"{m.K}->{m.N}" for m in wl.matrices)
-                   + f" x M in {sorted(wl.Ms, reverse=True)}",
+                   + f" x M in {sorted(set(pt.M for pt in points), reverse=True)}",
+                   "timing": "each timed step is a CUDA graph replay; per-kernel times from event-record nodes "
+                             "around each launch",
                    "parallelism": f"replicas x{world} (token batches, no collective)",
                    "l2": f"weights rotate over {len(pool)} packed copies ({len(pool) * sum(p[0].numel() for p in pool[0]) / 2**20:.0f} MiB > L2); "
                          "activations at M=8192 exceed L2"},

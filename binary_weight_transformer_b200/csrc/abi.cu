@@ -193,7 +193,9 @@ lowbit_status lowbit_linear_path(const int8_t *q, int64_t ldq, const float *s_x,
     const lowbit_status d = check_device();
     if (d != LOWBIT_OK) return d;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const bool use_gemv = path == 1 || (path == 0 && M <= 16);
+    // Up to 4 tokens the dp4a GEMV streams weights fastest; from 5 on its
+    // int8 MACs outgrow the CUDA cores and the tensor-core GEMM wins.
+    const bool use_gemv = path == 1 || (path == 0 && M <= 4);
     if (use_gemv) return gemv_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, st);
     return gemm_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, status_dev, st);
 }

@@ -55,6 +55,27 @@ __device__ __forceinline__ int8_t quant_one(float x, float d)
     return static_cast<int8_t>(static_cast<int>(t));
 }
 
+// Same codes as quant_one without a divide or a conversion instruction per
+// element.  With t = x*127 (rounded), rd = RN(1/d) and u = RN(t*rd): since
+// |t| <= 127*gamma <= 127*d, |u - t/d| <= 127*(2^-24 + 2^-24 + 2^-48) < 1.6e-5,
+// and the IEEE quotient z = RN(t/d) is within half an ulp of t/d, < 4e-6 for
+// |z| < 128: |u - z| < 2e-5.  So u and z round to the same integer unless u
+// lies near a midpoint k + 1/2; elements within 1e-4 of one (about 2 in 10^4)
+// take the divide.  Rounding uses the IEEE nearest-even addition
+// v = u + 1.5*2^23: for |u| < 2^22 the sum is exact to the unit, v - 1.5*2^23
+// is rint(u), and the low byte of v's bit pattern is that integer in two's
+// complement.  |u| <= 127.00002 here, so no clamp is needed (M8.8 0x05C
+// clips to [-128, 127]; with eps >= 0 the codes never leave [-127, 127]).
+__device__ __forceinline__ uint32_t quant_byte(float x, float d, float rd)
+{
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    const float t = __fmul_rn(x, 127.0f);
+    const float u = __fmul_rn(t, rd);
+    float v = __fadd_rn(u, kMagic);
+    if (fabsf(__fsub_rn(u, __fsub_rn(v, kMagic))) > 0.4999f) v = __fadd_rn(__fdiv_rn(t, d), kMagic);
+    return __float_as_uint(v) & 0xFFu;
+}
+
 // Max of a uint32 over the TPR threads that own one row.
 template <int TPR>
 __device__ __forceinline__ uint32_t row_max(uint32_t v, uint32_t *red)
@@ -120,6 +141,7 @@ act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
     const bool bad = !finite_bits(amax) || !finite_bits(__float_as_uint(__fmul_rn(g, 127.0f)));
     if (bad && r == 0) report(status, LOWBIT_ERR_NONFINITE);
     const float d = __fadd_rn(g, eps);
+    const float rd = __frcp_rn(d);
     int8_t *qrow = q + row * ldq;
 
 #pragma unroll
@@ -131,7 +153,7 @@ act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
                 if (amax != 0) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        out |= static_cast<uint32_t>(static_cast<uint8_t>(quant_one(In<T>::get(buf[i], e), d))) << (8 * e);
+                        out |= quant_byte(In<T>::get(buf[i], e), d, rd) << (8 * e);
                 }
                 *reinterpret_cast<uint32_t *>(qrow + v * 4) = out;
             } else {
@@ -139,15 +161,15 @@ act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
                 if (amax != 0) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        lo |= static_cast<uint32_t>(static_cast<uint8_t>(quant_one(In<T>::get(buf[i], e), d))) << (8 * e);
-                        hi |= static_cast<uint32_t>(static_cast<uint8_t>(quant_one(In<T>::get(buf[i], e + 4), d))) << (8 * e);
+                        lo |= quant_byte(In<T>::get(buf[i], e), d, rd) << (8 * e);
+                        hi |= quant_byte(In<T>::get(buf[i], e + 4), d, rd) << (8 * e);
                     }
                 }
                 *reinterpret_cast<uint2 *>(qrow + v * 8) = make_uint2(lo, hi);
             }
         }
     }
-    if (has_tail) qrow[tail0 + r] = amax != 0 ? quant_one(tail_x, d) : 0;
+    if (has_tail) qrow[tail0 + r] = amax != 0 ? static_cast<int8_t>(quant_byte(tail_x, d, rd)) : 0;
     if (r == 0) s_x[row] = amax != 0 ? __fdiv_rn(g, 127.0f) : 0.0f;
 }
 

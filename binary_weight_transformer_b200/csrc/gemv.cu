@@ -100,7 +100,10 @@ __device__ __forceinline__ void store_out(void *y, int64_t idx, int32_t acc, flo
     }
 }
 
-template <int FMT, int MT, int OUT>
+// Each warp takes R consecutive rows and U 16-byte chunks per lane of each:
+// all R*U weight loads are issued before any of them is used, so a batch of
+// rows costs one DRAM round trip, and the grid is sized to run in one wave.
+template <int FMT, int MT, int U, int R, int OUT>
 __global__ void __launch_bounds__(kWarps * 32)
 gemv_kernel(const int8_t *__restrict__ q, int64_t ldq, const float *__restrict__ s_x, int M, int64_t K,
             const uint8_t *__restrict__ packed, int64_t ldp, int64_t nchunks, const float *__restrict__ s_w,
@@ -110,47 +113,86 @@ gemv_kernel(const int8_t *__restrict__ q, int64_t ldq, const float *__restrict__
     constexpr int kCodesPerChunk = 4 * F::kCodesPerWord;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    for (int64_t row = static_cast<int64_t>(blockIdx.x) * kWarps + warp; row < N;
-         row += static_cast<int64_t>(gridDim.x) * kWarps) {
-        const uint8_t *prow = packed + row * ldp;
-        int32_t acc[MT];
+    for (int64_t row0 = (static_cast<int64_t>(blockIdx.x) * kWarps + warp) * R; row0 < N;
+         row0 += static_cast<int64_t>(gridDim.x) * kWarps * R) {
+        int32_t acc[R][MT];
 #pragma unroll
-        for (int t = 0; t < MT; ++t) acc[t] = 0;
-        for (int64_t c = lane; c < nchunks; c += 32) {
-            const uint4 wv = ld_stream_u4(prow + c * 16);
-            const int64_t k0 = c * kCodesPerChunk;
+        for (int r = 0; r < R; ++r)
 #pragma unroll
-            for (int t = 0; t < MT; ++t)
-                if (t < M) acc[t] = chunk_dot<FMT>(wv, q + t * ldq, k0, K, acc[t]);
+            for (int t = 0; t < MT; ++t) acc[r][t] = 0;
+        for (int64_t c0 = 0; c0 < nchunks; c0 += 32 * U) {
+            uint4 wv[R][U];
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int64_t c = c0 + lane + 32 * u;
+                    wv[r][u] = (c < nchunks && row0 + r < N) ? ld_stream_u4(packed + (row0 + r) * ldp + c * 16)
+                                                             : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t c = c0 + lane + 32 * u;
+                if (c < nchunks) {
+#pragma unroll
+                    for (int r = 0; r < R; ++r)
+#pragma unroll
+                        for (int t = 0; t < MT; ++t)
+                            if (t < M)
+                                acc[r][t] = chunk_dot<FMT>(wv[r][u], q + t * ldq, c * kCodesPerChunk, K, acc[r][t]);
+                }
+            }
         }
-        const float sw = s_w[FMT == kT2 ? 0 : row];
 #pragma unroll
-        for (int t = 0; t < MT; ++t) {
-            int32_t v = acc[t];
+        for (int r = 0; r < R; ++r) {
+            const int64_t row = row0 + r;
+            const float sw = (row < N) ? s_w[FMT == kT2 ? 0 : row] : 0.0f;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == t && t < M) store_out<OUT>(y, t * ldy + row, v >> F::kShift, sw, s_x[t]);
+            for (int t = 0; t < MT; ++t) {
+                int32_t v = acc[r][t];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (lane == t && t < M && row < N) store_out<OUT>(y, t * ldy + row, v >> F::kShift, sw, s_x[t]);
+            }
         }
     }
 }
 
-template <int FMT, int MT>
+template <int FMT, int MT, int U, int R>
 lowbit_status launch_mt(const int8_t *q, int64_t ldq, const float *s_x, int M, int64_t K,
-                        const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w, int64_t N,
+                        const uint8_t *packed, int64_t ldp, int64_t nchunks, const float *s_w, int64_t N,
                         void *y, lowbit_dtype ydt, int64_t ldy, cudaStream_t st)
 {
-    const int64_t nchunks = (row_bytes + 15) / 16;
-    int64_t blocks = (N + kWarps - 1) / kWarps;
+    int64_t blocks = (N + kWarps * R - 1) / (kWarps * R);
     const int64_t cap = static_cast<int64_t>(device_sm_count()) * 16;
     if (blocks > cap) blocks = cap;
     const dim3 grid(static_cast<unsigned>(blocks)), block(kWarps * 32);
     if (ydt == LOWBIT_F32)
-        gemv_kernel<FMT, MT, LOWBIT_F32><<<grid, block, 0, st>>>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ldy);
+        gemv_kernel<FMT, MT, U, R, LOWBIT_F32><<<grid, block, 0, st>>>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ldy);
     else if (ydt == LOWBIT_BF16)
-        gemv_kernel<FMT, MT, LOWBIT_BF16><<<grid, block, 0, st>>>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ldy);
+        gemv_kernel<FMT, MT, U, R, LOWBIT_BF16><<<grid, block, 0, st>>>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ldy);
     else
-        gemv_kernel<FMT, MT, LOWBIT_I32><<<grid, block, 0, st>>>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ldy);
+        gemv_kernel<FMT, MT, U, R, LOWBIT_I32><<<grid, block, 0, st>>>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ldy);
     return launch_status();
+}
+
+// Pick U (chunks per lane in flight) from the row length and R (rows per
+// warp) so that the grid fills the GPU in about one wave of 2 blocks per SM.
+template <int FMT, int MT>
+lowbit_status launch_u(const int8_t *q, int64_t ldq, const float *s_x, int M, int64_t K,
+                       const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w, int64_t N,
+                       void *y, lowbit_dtype ydt, int64_t ldy, cudaStream_t st)
+{
+    const int64_t nchunks = (row_bytes + 15) / 16;
+    const int64_t slots = static_cast<int64_t>(device_sm_count()) * 2 * kWarps;  // warps in one wave
+    if (nchunks <= 64) {
+        if (MT == 1 && N >= 4 * slots)
+            return launch_mt<FMT, MT, 2, 4>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ydt, ldy, st);
+        if (MT <= 4 && N >= 2 * slots)
+            return launch_mt<FMT, MT, 2, 2>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ydt, ldy, st);
+        return launch_mt<FMT, MT, 2, 1>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ydt, ldy, st);
+    }
+    return launch_mt<FMT, MT, 8, 1>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ydt, ldy, st);
 }
 
 template <int FMT>
@@ -158,11 +200,9 @@ lowbit_status launch_fmt(const int8_t *q, int64_t ldq, const float *s_x, int M, 
                          const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w, int64_t N,
                          void *y, lowbit_dtype ydt, int64_t ldy, cudaStream_t st)
 {
-    if (M <= 1) return launch_mt<FMT, 1>(q, ldq, s_x, M, K, packed, ldp, row_bytes, s_w, N, y, ydt, ldy, st);
-    if (M <= 2) return launch_mt<FMT, 2>(q, ldq, s_x, M, K, packed, ldp, row_bytes, s_w, N, y, ydt, ldy, st);
-    if (M <= 4) return launch_mt<FMT, 4>(q, ldq, s_x, M, K, packed, ldp, row_bytes, s_w, N, y, ydt, ldy, st);
-    if (M <= 8) return launch_mt<FMT, 8>(q, ldq, s_x, M, K, packed, ldp, row_bytes, s_w, N, y, ydt, ldy, st);
-    return launch_mt<FMT, 16>(q, ldq, s_x, M, K, packed, ldp, row_bytes, s_w, N, y, ydt, ldy, st);
+    if (M <= 1) return launch_u<FMT, 1>(q, ldq, s_x, M, K, packed, ldp, row_bytes, s_w, N, y, ydt, ldy, st);
+    if (M <= 4) return launch_u<FMT, 4>(q, ldq, s_x, M, K, packed, ldp, row_bytes, s_w, N, y, ydt, ldy, st);
+    return launch_u<FMT, 16>(q, ldq, s_x, M, K, packed, ldp, row_bytes, s_w, N, y, ydt, ldy, st);
 }
 
 }  // namespace

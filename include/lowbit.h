@@ -184,7 +184,7 @@ lowbit_status lowbit_act_quant(const void *x, lowbit_dtype xdt, int64_t M, int64
  * ldq and ldp multiples of 16), s_x fp32 [M], s_w fp32 [lowbit_scale_count].
  * Output y [M, ldy], ldy >= N, aligned to its element size.  Bytes of q past
  * K are ignored.  K <= lowbit_max_k(f), else LOWBIT_ERR_OVERFLOW_BOUND.
- * M <= 16 runs the packed-weight GEMV kernel; larger M runs the tcgen05
+ * M <= 4 runs the packed-weight GEMV kernel; larger M runs the tcgen05
  * tensor-core GEMM (int8 MMA, accumulators in tensor memory). */
 lowbit_status lowbit_linear(const int8_t *q, int64_t ldq, const float *s_x,
                             int64_t M, int64_t K,
