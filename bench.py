@@ -53,6 +53,27 @@ def dist_env():
     return rank, world, local
 
 
+def shard_range(M: int, rank: int, world: int):
+    """Token rows [start, stop) of rank `rank` when M rows are split across
+    `world` ranks as evenly as possible (per-token quantisation makes every
+    row independent, so the shards need no exchange)."""
+    base, extra = divmod(M, world)
+    start = rank * base + min(rank, extra)
+    return start, start + base + (1 if rank < extra else 0)
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest `value` over all ranks of the default process group (the
+    whole-job time is the slowest rank's); returns `value` without a group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------------------
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
@@ -285,11 +306,7 @@ def run_gpu_arm(args, wl):
     launches = launches_per_step * args.steps
     if world > 1:
         torch.distributed.barrier()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), device)
 
     # per-point device times (ms per launch, averaged over the timed steps)
     per_point, per_act = [], []

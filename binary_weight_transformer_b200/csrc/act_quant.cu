@@ -18,33 +18,37 @@
 namespace lowbit {
 namespace {
 
-constexpr int kVPT = 8;  // 16-byte vectors per thread held in registers
+constexpr int kVPT = 4;  // 16-byte vectors per thread held in registers
 
 template <typename T> struct In;
 template <> struct In<float> {
     static constexpr int kPerVec = 4;
-    __device__ static float get(const uint4 &v, int i)
+    __device__ static float get(const uint4 &v, int i) { return __uint_as_float((&v.x)[i]); }
+    __device__ static float scalar(const void *p, int64_t i) { return static_cast<const float *>(p)[i]; }
+    // max of |x| bits over one vector (a non-finite value sorts above all finite ones)
+    __device__ static uint32_t absmax_bits(const uint4 &v)
     {
-        uint32_t w = (&v.x)[i];
-        return __uint_as_float(w);
-    }
-    __device__ static float scalar(const void *p, int64_t i)
-    {
-        return static_cast<const float *>(p)[i];
+        return max(max(v.x & 0x7fffffffu, v.y & 0x7fffffffu), max(v.z & 0x7fffffffu, v.w & 0x7fffffffu));
     }
 };
 template <> struct In<__nv_bfloat16> {
     static constexpr int kPerVec = 8;
     __device__ static float get(const uint4 &v, int i)
     {
-        uint32_t w = (&v.x)[i >> 1];
-        uint32_t h = (i & 1) ? (w >> 16) : (w & 0xffffu);
-        return __uint_as_float(h << 16);
+        const uint32_t w = (&v.x)[i >> 1];
+        return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
     }
     __device__ static float scalar(const void *p, int64_t i)
     {
-        uint16_t h = static_cast<const uint16_t *>(p)[i];
+        const uint16_t h = static_cast<const uint16_t *>(p)[i];
         return __uint_as_float(static_cast<uint32_t>(h) << 16);
+    }
+    // 16-bit lane-wise max of the |x| bit patterns, then the larger half
+    __device__ static uint32_t absmax_bits(const uint4 &v)
+    {
+        const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7fff7fffu, v.y & 0x7fff7fffu),
+                                    __vmaxu2(v.z & 0x7fff7fffu, v.w & 0x7fff7fffu));
+        return max(m << 16, m & 0xffff0000u);
     }
 };
 
@@ -55,25 +59,37 @@ __device__ __forceinline__ int8_t quant_one(float x, float d)
     return static_cast<int8_t>(static_cast<int>(t));
 }
 
-// Same codes as quant_one without a divide or a conversion instruction per
-// element.  With t = x*127 (rounded), rd = RN(1/d) and u = RN(t*rd): since
-// |t| <= 127*gamma <= 127*d, |u - t/d| <= 127*(2^-24 + 2^-24 + 2^-48) < 1.6e-5,
-// and the IEEE quotient z = RN(t/d) is within half an ulp of t/d, < 4e-6 for
-// |z| < 128: |u - z| < 2e-5.  So u and z round to the same integer unless u
-// lies near a midpoint k + 1/2; elements within 1e-4 of one (about 2 in 10^4)
-// take the divide.  Rounding uses the IEEE nearest-even addition
-// v = u + 1.5*2^23: for |u| < 2^22 the sum is exact to the unit, v - 1.5*2^23
-// is rint(u), and the low byte of v's bit pattern is that integer in two's
-// complement.  |u| <= 127.00002 here, so no clamp is needed (M8.8 0x05C
-// clips to [-128, 127]; with eps >= 0 the codes never leave [-127, 127]).
-__device__ __forceinline__ uint32_t quant_byte(float x, float d, float rd)
+// Codes for four values without a divide or a conversion instruction each.
+// The exact code is rint(z), z = RN(t/d), t = RN(127x).  With c = RN(127 *
+// RN(1/d)) and u = RN(x*c), |u - t/d| <= (127|x|/d) * 4 * 2^-24 < 3.1e-5 and
+// |z - t/d| <= 2^-18 < 3.9e-6 (|z| < 128), so |u - z| < 3.5e-5: u and z round
+// to the same integer unless u lies within that distance of a midpoint
+// k + 1/2.  Rounding uses the IEEE nearest-even addition v = u + 1.5*2^23,
+// exact to the unit for |u| < 2^22: v - 1.5*2^23 is rint(u) and the low byte
+// of v's bit pattern is the code in two's complement.  A value within 1e-4
+// of a midpoint (about 2 in 10^4) sets `near`; the caller then redoes the
+// four values with the IEEE divide.  |u| <= 127.0001, so no clamp is needed.
+__device__ __forceinline__ uint32_t quant4(float x0, float x1, float x2, float x3, float c, bool &near)
 {
     constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-    const float t = __fmul_rn(x, 127.0f);
-    const float u = __fmul_rn(t, rd);
-    float v = __fadd_rn(u, kMagic);
-    if (fabsf(__fsub_rn(u, __fsub_rn(v, kMagic))) > 0.4999f) v = __fadd_rn(__fdiv_rn(t, d), kMagic);
-    return __float_as_uint(v) & 0xFFu;
+    const float u0 = __fmul_rn(x0, c), u1 = __fmul_rn(x1, c), u2 = __fmul_rn(x2, c), u3 = __fmul_rn(x3, c);
+    const float v0 = __fadd_rn(u0, kMagic), v1 = __fadd_rn(u1, kMagic);
+    const float v2 = __fadd_rn(u2, kMagic), v3 = __fadd_rn(u3, kMagic);
+    near |= fabsf(__fsub_rn(u0, __fsub_rn(v0, kMagic))) > 0.4999f;
+    near |= fabsf(__fsub_rn(u1, __fsub_rn(v1, kMagic))) > 0.4999f;
+    near |= fabsf(__fsub_rn(u2, __fsub_rn(v2, kMagic))) > 0.4999f;
+    near |= fabsf(__fsub_rn(u3, __fsub_rn(v3, kMagic))) > 0.4999f;
+    const uint32_t lo = __byte_perm(__float_as_uint(v0), __float_as_uint(v1), 0x0040);
+    const uint32_t hi = __byte_perm(__float_as_uint(v2), __float_as_uint(v3), 0x0040);
+    return __byte_perm(lo, hi, 0x5410);
+}
+
+__device__ __forceinline__ uint32_t quant4_exact(float x0, float x1, float x2, float x3, float d)
+{
+    return static_cast<uint32_t>(static_cast<uint8_t>(quant_one(x0, d))) |
+           (static_cast<uint32_t>(static_cast<uint8_t>(quant_one(x1, d))) << 8) |
+           (static_cast<uint32_t>(static_cast<uint8_t>(quant_one(x2, d))) << 16) |
+           (static_cast<uint32_t>(static_cast<uint8_t>(quant_one(x3, d))) << 24);
 }
 
 // Max of a uint32 over the TPR threads that own one row.
@@ -121,9 +137,7 @@ act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
         const int64_t v = r + static_cast<int64_t>(i) * TPR;
         if (live && v < nvec) {
             buf[i] = ld_stream_u4(xrow + v * 16);
-#pragma unroll
-            for (int e = 0; e < E; ++e)
-                amax = max(amax, __float_as_uint(In<T>::get(buf[i], e)) & 0x7fffffffu);
+            amax = max(amax, In<T>::absmax_bits(buf[i]));
         }
     }
     // Tail elements past the last whole vector, one per thread.
@@ -141,35 +155,34 @@ act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
     const bool bad = !finite_bits(amax) || !finite_bits(__float_as_uint(__fmul_rn(g, 127.0f)));
     if (bad && r == 0) report(status, LOWBIT_ERR_NONFINITE);
     const float d = __fadd_rn(g, eps);
-    const float rd = __frcp_rn(d);
+    const float c = __fmul_rn(127.0f, __frcp_rn(d));
     int8_t *qrow = q + row * ldq;
 
 #pragma unroll
     for (int i = 0; i < kVPT; ++i) {
         const int64_t v = r + static_cast<int64_t>(i) * TPR;
         if (v < nvec) {
+            const uint4 &b = buf[i];
             if constexpr (E == 4) {
-                uint32_t out = 0;
-                if (amax != 0) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        out |= quant_byte(In<T>::get(buf[i], e), d, rd) << (8 * e);
-                }
+                bool near = false;
+                uint32_t out = quant4(In<T>::get(b, 0), In<T>::get(b, 1), In<T>::get(b, 2), In<T>::get(b, 3), c, near);
+                if (near) out = quant4_exact(In<T>::get(b, 0), In<T>::get(b, 1), In<T>::get(b, 2), In<T>::get(b, 3), d);
+                if (amax == 0) out = 0;
                 *reinterpret_cast<uint32_t *>(qrow + v * 4) = out;
             } else {
-                uint32_t lo = 0, hi = 0;
-                if (amax != 0) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        lo |= quant_byte(In<T>::get(buf[i], e), d, rd) << (8 * e);
-                        hi |= quant_byte(In<T>::get(buf[i], e + 4), d, rd) << (8 * e);
-                    }
+                bool near = false;
+                uint32_t lo = quant4(In<T>::get(b, 0), In<T>::get(b, 1), In<T>::get(b, 2), In<T>::get(b, 3), c, near);
+                uint32_t hi = quant4(In<T>::get(b, 4), In<T>::get(b, 5), In<T>::get(b, 6), In<T>::get(b, 7), c, near);
+                if (near) {
+                    lo = quant4_exact(In<T>::get(b, 0), In<T>::get(b, 1), In<T>::get(b, 2), In<T>::get(b, 3), d);
+                    hi = quant4_exact(In<T>::get(b, 4), In<T>::get(b, 5), In<T>::get(b, 6), In<T>::get(b, 7), d);
                 }
+                if (amax == 0) lo = hi = 0;
                 *reinterpret_cast<uint2 *>(qrow + v * 8) = make_uint2(lo, hi);
             }
         }
     }
-    if (has_tail) qrow[tail0 + r] = amax != 0 ? static_cast<int8_t>(quant_byte(tail_x, d, rd)) : 0;
+    if (has_tail) qrow[tail0 + r] = amax != 0 ? quant_one(tail_x, d) : 0;
     if (r == 0) s_x[row] = amax != 0 ? __fdiv_rn(g, 127.0f) : 0.0f;
 }
 

@@ -518,6 +518,241 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
 }
 
 // ---------------------------------------------------------------------------
+// Split-K over a thread-block cluster, for problems with fewer output tiles
+// than SMs (few tokens, or few output features).  The C CTAs of a cluster
+// share one output tile; CTA s accumulates k-blocks [s*nkb/C, (s+1)*nkb/C)
+// into tensor memory.  The partial tiles are then reduce-scattered through
+// distributed shared memory: CTA s receives every peer's partial sums for
+// columns [s*W, (s+1)*W), W = 256/C, adds them (int32 addition is exact, so
+// the result equals the unsplit accumulation bit for bit) and runs the
+// epilogue for those columns.  No global scratch memory is used.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t map_to_peer(uint32_t saddr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void st_cluster128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+template <int FMT, int OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_p,
+                   const float *__restrict__ s_x, const float *__restrict__ s_w, int64_t M, int64_t N, int64_t K,
+                   void *__restrict__ y, int64_t ldy, int vec_ok, int C, int32_t *status)
+{
+    constexpr int ST = tma_stages<FMT>();
+    constexpr int SE = kExpStages;
+    constexpr int PB = packed_bytes_per_kblock<FMT>();
+    constexpr int P_BYTES = BN * PB;
+    constexpr int kShift = Fmt<FMT>::kShift;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = base;
+    uint8_t *sE = sA + ST * A_BYTES;
+    uint8_t *sP = sE + SE * E_BYTES;
+    uint8_t *sStage = sP + ST * P_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sStage + 4 * stage_warp_bytes<OUT>());
+    uint64_t *full_tma = bars;
+    uint64_t *empty_tma = bars + ST;
+    uint64_t *full_exp = bars + 2 * ST;
+    uint64_t *empty_exp = bars + 2 * ST + SE;
+    uint64_t *acc_full = bars + 2 * ST + 2 * SE;
+    uint64_t *drain = acc_full + 4;
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(acc_full + 5);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(acc_full + 6);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t srank = cluster_rank();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(&full_tma[s], 1);
+            mbar_init(&empty_tma[s], 1);
+        }
+        for (int s = 0; s < SE; ++s) {
+            mbar_init(&full_exp[s], kExpThreads);
+            mbar_init(&empty_exp[s], 1);
+        }
+        mbar_init(&acc_full[0], 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_p)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(const_cast<uint32_t *>(tmem_slot))), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int64_t num_m = (M + BM - 1) / BM;
+    const int64_t tile = blockIdx.x / C;
+    const int m0 = static_cast<int>((tile % num_m) * BM);
+    const int n0 = static_cast<int>((tile / num_m) * BN);
+    const int nkb = static_cast<int>((K + BK - 1) / BK);
+    const int kb_begin = static_cast<int>((static_cast<int64_t>(srank) * nkb) / C);
+    const int kb_end = static_cast<int>((static_cast<int64_t>(srank + 1) * nkb) / C);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t g = 0;
+            bool ok = true;
+            for (int kb = kb_begin; kb < kb_end; ++kb, ++g) {
+                const int s = g % ST;
+                if (!wait_bar(&empty_tma[s], ((g / ST) & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
+                mbar_arrive_expect_tx(&full_tma[s], A_BYTES + P_BYTES);
+                tma_load_2d(sA + s * A_BYTES, &map_a, &full_tma[s], kb * BK, m0);
+                tma_load_2d(sP + s * P_BYTES, &map_p, &full_tma[s], kb * PB, n0);
+            }
+            if (!ok) {
+                for (uint32_t i = 0; i < ST && i < g; ++i) {
+                    const uint32_t gi = g - 1 - i;
+                    wait_bar(&full_tma[gi % ST], (gi / ST) & 1u, abort_flag, nullptr, 200000000ll);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            uint32_t g = 0;
+            bool ok = true;
+            for (int kb = kb_begin; kb < kb_end; ++kb, ++g) {
+                const int s1 = g % ST, s2 = g % SE;
+                if (!wait_bar(&full_tma[s1], (g / ST) & 1u, abort_flag, status) ||
+                    !wait_bar(&full_exp[s2], (g / SE) & 1u, abort_flag, status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t a_addr = smem_u32(sA + s1 * A_BYTES);
+                const uint32_t e_addr = smem_u32(sE + s2 * E_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < BK / UMMA_K; ++kk)
+                    tc_mma_i8(tmem_base, sw128_desc(a_addr + kk * UMMA_K), sw128_desc(e_addr + kk * UMMA_K), kIdesc,
+                              (g | kk) != 0 ? 1u : 0u);
+                tc_commit(&empty_tma[s1]);
+                tc_commit(&empty_exp[s2]);
+            }
+            if (ok) tc_commit(&acc_full[0]);
+            tc_commit(drain);
+            wait_bar(drain, 0, abort_flag, nullptr, 200000000ll);
+        }
+    } else if (warp < 6) {
+        const int et = threadIdx.x - 64;
+        const uint32_t p_base = smem_u32(sP);
+        const uint32_t e_base = smem_u32(sE);
+        uint32_t g = 0;
+        for (int kb = kb_begin; kb < kb_end; ++kb, ++g) {
+            const int s1 = g % ST, s2 = g % SE;
+            if (!wait_bar(&full_tma[s1], (g / ST) & 1u, abort_flag, status) ||
+                !wait_bar(&empty_exp[s2], ((g / SE) & 1u) ^ 1u, abort_flag, status)) break;
+            expand_stage<FMT>(p_base + s1 * P_BYTES, e_base + s2 * E_BYTES, et);
+            fence_proxy_async_smem();
+            mbar_arrive(&full_exp[s2]);
+        }
+    }
+    int ready = 1;
+    if (warp >= 6) {
+        int r = 0;
+        if (lane == 0) r = wait_bar(&acc_full[0], 0, abort_flag, status) ? 1 : 0;
+        ready = __shfl_sync(0xffffffffu, r, 0);
+        tc_fence_after();
+    }
+    __syncwarp();
+
+    // Every CTA of the cluster is done with its pipeline buffers: from here
+    // they hold the received partial tiles.
+    const int W = BN / C;                       // columns each CTA finishes
+    const int RB = 4 * W + 16;                  // receive row stride (padded)
+    const uint32_t recv = smem_u32(sA);
+    cluster_sync_all();
+    const int quarter = warp & 3;
+    const int row_in_tile = quarter * 32 + lane;
+    const int64_t row = m0 + row_in_tile;
+    if (warp >= 6) {
+        for (int j = 0; j < C; ++j) {
+            for (int cc = 0; cc < W / 32; ++cc) {
+                uint32_t v[32];
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                       static_cast<uint32_t>(j * W + cc * 32);
+                tmem_ld_32cols(taddr, v);
+                if (!ready) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = 0;
+                }
+                if (row < M) {
+                    const uint32_t dst = map_to_peer(
+                        recv + static_cast<uint32_t>((srank * BM + row_in_tile) * RB + cc * 128), static_cast<uint32_t>(j));
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) st_cluster128(dst + p * 16, v[4 * p], v[4 * p + 1], v[4 * p + 2], v[4 * p + 3]);
+                }
+            }
+        }
+    }
+    cluster_sync_all();
+    if (warp >= 6) {
+        const uint32_t stage = smem_u32(sStage) + static_cast<uint32_t>((warp - 6) * stage_warp_bytes<OUT>());
+        const float sx = row < M ? s_x[row] : 0.0f;
+        const float sw_tensor = (FMT == kT2) ? s_w[0] : 0.0f;
+        for (int cc = 0; cc < W / 32; ++cc) {
+            uint32_t v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0;
+            if (row < M) {
+                for (int s = 0; s < C; ++s) {
+                    const uint32_t src = recv + static_cast<uint32_t>((s * BM + row_in_tile) * RB + cc * 128);
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        const uint4 a = lds128(src + p * 16);
+                        v[4 * p] += a.x;
+                        v[4 * p + 1] += a.y;
+                        v[4 * p + 2] += a.z;
+                        v[4 * p + 3] += a.w;
+                    }
+                }
+            }
+            const int64_t nc = n0 + static_cast<int64_t>(srank) * W + cc * 32;
+            if (nc < N) {
+                float sw[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    sw[i] = (FMT == kT2) ? sw_tensor : ((nc + i < N) ? __ldg(s_w + nc + i) : 0.0f);
+                epilogue_chunk<OUT>(v, sw, sx, kShift, y, ldy, m0 + quarter * 32, M, nc, N, vec_ok != 0, stage, lane);
+            }
+        }
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -569,6 +804,38 @@ lowbit_status launch_t(const CUtensorMap &ma, const CUtensorMap &mp, const float
     }
     const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int64_t sms = device_sm_count();
+    const int nkb = static_cast<int>((K + BK - 1) / BK);
+    // Split K over a cluster when the tiles leave most SMs idle: the largest
+    // C in {2, 4, 8} that keeps every split at least 2 k-blocks deep and the
+    // whole grid within one wave.
+    int C = 1;
+    for (int c = 2; c <= 8; c *= 2)
+        if (tiles * c <= sms && nkb >= 2 * c) C = c;
+    if (C > 1) {
+        static bool configured_split[64] = {};
+        if (!configured_split[dev]) {
+            if (cudaFuncSetAttribute(gemm_splitk_kernel<FMT, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem)) != cudaSuccess)
+                return LOWBIT_ERR_CUDA;
+            configured_split[dev] = true;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(tiles * C));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(C);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, gemm_splitk_kernel<FMT, OUT>, ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, C,
+                               status) != cudaSuccess)
+            return LOWBIT_ERR_CUDA;
+        return launch_status();
+    }
     const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
     gemm_kernel<FMT, OUT><<<grid, kThreads, smem, st>>>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, status);
     return launch_status();

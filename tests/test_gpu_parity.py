@@ -203,8 +203,11 @@ def run_case(fmt, M, N, K, path, out, seed, zero_w=False, x_bf16=False):
     return y, acc, s_wo, s_xo
 
 
+# Includes shapes that take the cluster split-K path of the GEMM (few output
+# tiles, deep K): (16, 96, 1000), (300, 768, 1040), (200, 1, 4000),
+# (64, 500, 4096), (130, 1000, 2000).
 SHAPES = [(1, 768, 192), (3, 257, 200), (16, 96, 1000), (17, 300, 192), (129, 513, 384), (300, 768, 1040),
-          (5, 33, 16), (200, 1, 4000)]
+          (5, 33, 16), (200, 1, 4000), (64, 500, 4096), (130, 1000, 2000)]
 
 
 @pytest.mark.parametrize("path", [1, 2], ids=["gemv", "gemm"])
@@ -217,7 +220,7 @@ def test_linear_int32_accumulators_bit_exact(path, fmt, M, N, K):
 
 @pytest.mark.parametrize("path", [1, 2], ids=["gemv", "gemm"])
 @pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
-@pytest.mark.parametrize("M,N,K", SHAPES[:6], ids=str)
+@pytest.mark.parametrize("M,N,K", SHAPES[:6] + SHAPES[8:], ids=str)
 def test_linear_f32_within_tolerance(path, fmt, M, N, K):
     y, acc, s_w, s_x = run_case(fmt, M, N, K, path, bwt.F32, 600 + M + N + K)
     ref = oracle.rescale(acc, s_w, s_x, "f32")
@@ -229,7 +232,7 @@ def test_linear_f32_within_tolerance(path, fmt, M, N, K):
 
 @pytest.mark.parametrize("path", [1, 2], ids=["gemv", "gemm"])
 @pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
-@pytest.mark.parametrize("M,N,K", SHAPES[:6], ids=str)
+@pytest.mark.parametrize("M,N,K", SHAPES[:6] + SHAPES[8:], ids=str)
 def test_linear_bf16_within_one_ulp(path, fmt, M, N, K):
     y, acc, s_w, s_x = run_case(fmt, M, N, K, path, bwt.BF16, 700 + M + N + K, x_bf16=True)
     ref = oracle.rescale(acc, s_w, s_x, "bf16")
