@@ -183,7 +183,8 @@ def lowbit_linear(q, s_x, packed, s_w, fmt: int, N: int, out_dtype: int = F32, K
                   y=None, status=None, stream=None, path: int = 0):
     """y[M, N] from int8 codes q[M, >=K] and a packed artifact (see lowbit.h).
 
-    ``path`` 0 picks the kernel by M; 1 forces the GEMV, 2 the tensor-core GEMM."""
+    ``path`` 0 picks the kernel by M; 1 forces the GEMV, 2 the tensor-core GEMM
+    with the expanded tile in shared memory, 3 the one with it in tensor memory."""
     import torch
     M = q.shape[0]
     if K is None:

@@ -1,0 +1,431 @@
+// gemm_ts.cu -- tensor-core GEMM with the weight operand in tensor memory.
+//
+// Same operator as gemm_sm100.cu ("M8.8 - Native Binary and Ternary
+// Transformers" 0x02D, 0x09A-0x09B): acc = sum_k q[t,k] c[n,k] on the
+// 5th-generation tensor cores, the packed artifact consumed directly.  Here
+// the operands are swapped: the MMA's A operand is a 128-row tile of weight
+// codes and B is a tile of up to 224 tokens, so that
+//
+//   D[n, t] (TMEM, s32) += A[n, k] (TMEM, int8) * B[t, k] (smem, int8).
+//
+// Expander warps read their row's packed codes from the TMA-staged tile,
+// expand them in registers and write them straight into tensor memory with
+// tcgen05.st (one 32-column store per row and K step): the expanded operand
+// never passes through shared memory, which leaves shared-memory bandwidth
+// to the TMA and the MMA's reads of the token tile.
+//
+// Warp roles: 0 TMA producer; 1 TMEM allocation and MMA issue; 2-5 expanders
+// (warp w owns TMEM lanes 32*(w%4)..+31 = weight rows); 6-9 epilogue.
+// TMEM columns: two accumulator buffers of 224 and two A stages of 32.
+// Every mbarrier wait is bounded (see tc_common.cuh).
+#include "tc_common.cuh"
+
+namespace lowbit {
+namespace ts {
+
+using namespace tc;
+
+constexpr int BW = 128;         // weight rows per tile (MMA M)
+constexpr int BT = 224;         // largest token tile (MMA N)
+constexpr int BK = 128;         // K per stage
+constexpr int kThreads = 320;
+constexpr int kACols = BK / 4;  // TMEM columns per A stage (4 int8 per column)
+constexpr int kAStages = 2;
+constexpr int kDCols = BT;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kStages = 5;      // TMA stages: token tile + packed tile
+
+template <int FMT> __host__ __device__ constexpr int packed_row_kblock() { return BK * Fmt<FMT>::kBits / 8; }
+constexpr int Q_BYTES = BT * BK;  // largest token tile
+template <int FMT> __host__ __device__ constexpr int p_bytes() { return BW * packed_row_kblock<FMT>(); }
+template <int OUT> __host__ __device__ constexpr int stage_row_bytes() { return OUT == LOWBIT_BF16 ? 80 : 144; }
+template <int OUT> __host__ __device__ constexpr int stage_warp_bytes() { return 32 * stage_row_bytes<OUT>(); }
+
+template <int FMT, int OUT>
+__host__ __device__ constexpr size_t smem_bytes()
+{
+    return 1024 + static_cast<size_t>(kStages) * (Q_BYTES + p_bytes<FMT>()) + 4 * stage_warp_bytes<OUT>() +
+           8 * (2 * kStages + 2 * kAStages + 8);
+}
+
+__device__ __forceinline__ void tmem_st_32cols(uint32_t taddr, const uint32_t (&v)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+          "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+          "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// D (TMEM) += A (TMEM) * B (smem descriptor)^T, s8 x s8 -> s32.
+__device__ __forceinline__ void tc_mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Instruction descriptor: s32 accumulate, s8 x s8, both K-major, M = 128, N = nt.
+__device__ __forceinline__ uint32_t idesc_for(int nt)
+{
+    return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(nt >> 3) << 17) |
+           (static_cast<uint32_t>(BW >> 4) << 24);
+}
+
+// One weight row's 128 codes of one K step, expanded to 32 int8x4 words of
+// (c << S) in K order.
+template <int FMT>
+__device__ __forceinline__ void expand_row(uint32_t prow, uint32_t (&w)[32])
+{
+    if constexpr (FMT == kT2) {
+        // 32 packed bytes = 8 words of 16 codes.
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint4 p = lds128(prow + h * 16);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int g = 0; g < 4; ++g) w[16 * h + 4 * j + g] = t2_expand((&p.x)[j], g);
+        }
+    } else if constexpr (FMT == kI4) {
+        // 64 packed bytes = 16 words of 8 codes.
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const uint4 p = lds128(prow + h * 16);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                w[8 * h + 2 * j] = i4_expand((&p.x)[j], 0);
+                w[8 * h + 2 * j + 1] = i4_expand((&p.x)[j], 1);
+            }
+        }
+    } else {
+        // 16 packed bytes = 4 words of 32 codes.
+        const uint4 p = lds128(prow);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int m = 0; m < 8; ++m) w[8 * j + m] = b1_expand_nibble(((&p.x)[j] >> (4 * m)) & 0xFu);
+    }
+}
+
+// Epilogue of one 32-token chunk for this warp's 32 weight rows.  v[i] is the
+// accumulator of (row n = this lane, token t0 + i).  The values go through a
+// per-warp staging tile (token-major, rows padded by 16 bytes) so that the
+// global stores are 64-byte (bf16) or 128-byte (fp32, int32) row segments.
+template <int OUT>
+__device__ __forceinline__ void store_chunk(const uint32_t (&v)[32], float sw, const float *__restrict__ s_x,
+                                            int shift, void *__restrict__ y, int64_t ldy, int64_t t0, int64_t M,
+                                            int64_t n0, int64_t N, bool vec_ok, uint32_t stage, int lane)
+{
+    constexpr int kEsz = OUT == LOWBIT_BF16 ? 2 : 4;
+    constexpr int RS = stage_row_bytes<OUT>();
+    const int64_t n = n0 + lane;
+    if (vec_ok && n0 + 32 <= N) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int32_t a = static_cast<int32_t>(v[i]) >> shift;
+            const uint32_t addr = stage + i * RS + lane * kEsz;
+            if constexpr (OUT == LOWBIT_I32) {
+                asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
+            } else {
+                const float sx = (t0 + i < M) ? __ldg(s_x + t0 + i) : 0.0f;
+                const float f = rescale(a, sw, sx);
+                if constexpr (OUT == LOWBIT_F32) {
+                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(__float_as_uint(f)) : "memory");
+                } else {
+                    const __nv_bfloat16 b = __float2bfloat16_rn(f);
+                    asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(*reinterpret_cast<const uint16_t *>(&b))
+                                 : "memory");
+                }
+            }
+        }
+        __syncwarp();
+        constexpr int kPieces = 32 * kEsz / 16;     // 16-byte pieces per token row
+        constexpr int kRowsPerPass = 32 / kPieces;
+#pragma unroll
+        for (int pass = 0; pass < kPieces; ++pass) {
+            const int r = pass * kRowsPerPass + lane / kPieces;
+            const int piece = lane % kPieces;
+            const uint4 val = lds128(stage + r * RS + piece * 16);
+            if (t0 + r < M) {
+                char *dst = static_cast<char *>(y) + ((t0 + r) * ldy + n0) * kEsz + piece * 16;
+                *reinterpret_cast<uint4 *>(dst) = val;
+            }
+        }
+        __syncwarp();
+    } else if (n < N) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if (t0 + i < M) {
+                const int32_t a = static_cast<int32_t>(v[i]) >> shift;
+                const int64_t idx = (t0 + i) * ldy + n;
+                if constexpr (OUT == LOWBIT_I32) {
+                    static_cast<int32_t *>(y)[idx] = a;
+                } else if constexpr (OUT == LOWBIT_F32) {
+                    static_cast<float *>(y)[idx] = rescale(a, sw, s_x[t0 + i]);
+                } else {
+                    static_cast<__nv_bfloat16 *>(y)[idx] = __float2bfloat16_rn(rescale(a, sw, s_x[t0 + i]));
+                }
+            }
+        }
+    }
+}
+
+template <int FMT, int OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_ts_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_p,
+               const float *__restrict__ s_x, const float *__restrict__ s_w, int64_t M, int64_t N, int64_t K,
+               void *__restrict__ y, int64_t ldy, int vec_ok, int nt, int32_t *status)
+{
+    constexpr int PB = packed_row_kblock<FMT>();
+    constexpr int P_BYTES = p_bytes<FMT>();
+    constexpr int kShift = Fmt<FMT>::kShift;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = base;                          // kStages x 28 KB, 1024-aligned
+    uint8_t *sP = sQ + kStages * Q_BYTES;        // kStages x P_BYTES
+    uint8_t *sStage = sP + kStages * P_BYTES;    // 4 x epilogue staging
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sStage + 4 * stage_warp_bytes<OUT>());
+    uint64_t *full_tma = bars;
+    uint64_t *empty_tma = bars + kStages;
+    uint64_t *full_a = bars + 2 * kStages;
+    uint64_t *empty_a = full_a + kAStages;
+    uint64_t *acc_full = empty_a + kAStages;
+    uint64_t *acc_empty = acc_full + 2;
+    uint64_t *drain = acc_full + 4;
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(acc_full + 5);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(acc_full + 6);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full_tma[s], 1);
+            mbar_init(&empty_tma[s], 1);
+        }
+        for (int s = 0; s < kAStages; ++s) {
+            mbar_init(&full_a[s], 128);
+            mbar_init(&empty_a[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_q)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_p)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(const_cast<uint32_t *>(tmem_slot))), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t a_col0 = 2 * kDCols;          // first A stage column
+
+    const int64_t num_w = (N + BW - 1) / BW;
+    const int64_t num_t = (M + nt - 1) / nt;
+    const int64_t num_tiles = num_w * num_t;
+    const int nkb = static_cast<int>((K + BK - 1) / BK);
+    const uint32_t q_bytes = static_cast<uint32_t>(nt) * BK;
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            uint32_t g = 0;
+            bool ok = true;
+            for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int w0 = static_cast<int>((tile % num_w) * BW);
+                const int t0 = static_cast<int>((tile / num_w) * nt);
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % kStages;
+                    if (!wait_bar(&empty_tma[s], ((g / kStages) & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&full_tma[s], q_bytes + P_BYTES);
+                    tma_load_2d(sQ + s * Q_BYTES, &map_q, &full_tma[s], kb * BK, t0);
+                    tma_load_2d(sP + s * P_BYTES, &map_p, &full_tma[s], kb * PB, w0);
+                }
+            }
+            if (!ok) {
+                for (uint32_t i = 0; i < kStages && i < g; ++i) {
+                    const uint32_t gi = g - 1 - i;
+                    wait_bar(&full_tma[gi % kStages], (gi / kStages) & 1u, abort_flag, nullptr, 200000000ll);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            const uint32_t idesc = idesc_for(nt);
+            uint32_t g = 0;
+            uint32_t t = 0;
+            bool ok = true;
+            for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++t) {
+                const int b = t & 1;
+                if (!wait_bar(&acc_empty[b], ((t >> 1) & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * kDCols);
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s1 = g % kStages, s2 = g % kAStages;
+                    if (!wait_bar(&full_tma[s1], (g / kStages) & 1u, abort_flag, status) ||
+                        !wait_bar(&full_a[s2], (g / kAStages) & 1u, abort_flag, status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t q_addr = smem_u32(sQ + s1 * Q_BYTES);
+                    const uint32_t a_tmem = tmem_base + a_col0 + static_cast<uint32_t>(s2 * kACols);
+#pragma unroll
+                    for (int kk = 0; kk < BK / UMMA_K; ++kk)
+                        tc_mma_i8_ts(d_tmem, a_tmem + kk * (UMMA_K / 4), sw128_desc(q_addr + kk * UMMA_K), idesc,
+                                     (kb | kk) != 0 ? 1u : 0u);
+                    tc_commit(&empty_tma[s1]);
+                    tc_commit(&empty_a[s2]);
+                }
+                if (!ok) break;
+                tc_commit(&acc_full[b]);
+            }
+            tc_commit(drain);
+            wait_bar(drain, 0, abort_flag, nullptr, 200000000ll);
+        }
+    } else if (warp < 6) {
+        // ---------------- expanders: packed -> TMEM ----------------
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;             // weight row within the tile
+        const uint32_t p_base = smem_u32(sP);
+        uint32_t g = 0;
+        bool ok = true;
+        for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (int kb = 0; kb < nkb; ++kb, ++g) {
+                const int s1 = g % kStages, s2 = g % kAStages;
+                int ready = 0;
+                if (lane == 0)
+                    ready = (wait_bar(&full_tma[s1], (g / kStages) & 1u, abort_flag, status) &&
+                             wait_bar(&empty_a[s2], ((g / kAStages) & 1u) ^ 1u, abort_flag, status)) ? 1 : 0;
+                ready = __shfl_sync(0xffffffffu, ready, 0);
+                if (!ready) { ok = false; break; }
+                tc_fence_after();
+                uint32_t w[32];
+                expand_row<FMT>(p_base + s1 * P_BYTES + r * PB, w);
+                tmem_st_32cols(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + a_col0 +
+                                   static_cast<uint32_t>(s2 * kACols), w);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&full_a[s2]);
+            }
+        }
+    } else {
+        // ---------------- epilogue ----------------
+        const int quarter = warp & 3;
+        const uint32_t stage = smem_u32(sStage) + static_cast<uint32_t>((warp - 6) * stage_warp_bytes<OUT>());
+        uint32_t t = 0;
+        for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t) {
+            const int b = t & 1;
+            int ready = 0;
+            if (lane == 0) ready = wait_bar(&acc_full[b], (t >> 1) & 1u, abort_flag, status) ? 1 : 0;
+            ready = __shfl_sync(0xffffffffu, ready, 0);
+            if (!ready) break;
+            tc_fence_after();
+            const int64_t n0 = (tile % num_w) * BW + quarter * 32;
+            const int64_t t0 = (tile / num_w) * nt;
+            const int64_t n = n0 + lane;
+            const float sw = (n < N) ? s_w[FMT == kT2 ? 0 : n] : 0.0f;
+#pragma unroll 1
+            for (int cc = 0; cc < nt / 32; ++cc) {
+                uint32_t v[32];
+                tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                   static_cast<uint32_t>(b * kDCols + cc * 32), v);
+                const int64_t tc0 = t0 + cc * 32;
+                if (tc0 < M && n0 < N)
+                    store_chunk<OUT>(v, sw, s_x, kShift, y, ldy, tc0, M, n0, N, vec_ok != 0, stage, lane);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[b]);
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+template <int FMT, int OUT>
+lowbit_status launch_t(const CUtensorMap &mq, const CUtensorMap &mp, const float *s_x, const float *s_w, int64_t M,
+                       int64_t N, int64_t K, void *y, int64_t ldy, int vec_ok, int nt, int32_t *status,
+                       cudaStream_t st)
+{
+    constexpr size_t smem = smem_bytes<FMT, OUT>();
+    static_assert(smem <= 232448, "shared memory budget");
+    static bool configured[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LOWBIT_ERR_CUDA;
+    if (!configured[dev]) {
+        if (cudaFuncSetAttribute(gemm_ts_kernel<FMT, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem)) != cudaSuccess)
+            return LOWBIT_ERR_CUDA;
+        configured[dev] = true;
+    }
+    const int64_t tiles = ((N + BW - 1) / BW) * ((M + nt - 1) / nt);
+    const int64_t sms = device_sm_count();
+    const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
+    gemm_ts_kernel<FMT, OUT><<<grid, kThreads, smem, st>>>(mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt, status);
+    return launch_status();
+}
+
+template <int FMT>
+lowbit_status launch_fmt(const CUtensorMap &mq, const CUtensorMap &mp, const float *s_x, const float *s_w,
+                         int64_t M, int64_t N, int64_t K, void *y, lowbit_dtype ydt, int64_t ldy, int vec_ok,
+                         int nt, int32_t *status, cudaStream_t st)
+{
+    if (ydt == LOWBIT_F32) return launch_t<FMT, LOWBIT_F32>(mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt, status, st);
+    if (ydt == LOWBIT_BF16) return launch_t<FMT, LOWBIT_BF16>(mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt, status, st);
+    return launch_t<FMT, LOWBIT_I32>(mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt, status, st);
+}
+
+}  // namespace ts
+
+// Token tile: 224 for many tokens, else M rounded up to a multiple of 32.
+lowbit_status gemm_ts_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
+                             const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
+                             lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int32_t *status,
+                             cudaStream_t st)
+{
+    using namespace ts;
+    const int nt = M >= BT ? BT : static_cast<int>((M + 31) / 32 * 32);
+    CUtensorMap mq, mp;
+    if (!make_map_2d(&mq, q, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(ldq), BK,
+                     static_cast<uint32_t>(nt), CU_TENSOR_MAP_SWIZZLE_128B))
+        return LOWBIT_ERR_CUDA;
+    const uint32_t pb = f == LOWBIT_TERNARY2 ? packed_row_kblock<kT2>()
+                        : f == LOWBIT_BINARY1 ? packed_row_kblock<kB1>()
+                                              : packed_row_kblock<kI4>();
+    if (!make_map_2d(&mp, packed, static_cast<uint64_t>(row_bytes), static_cast<uint64_t>(N),
+                     static_cast<uint64_t>(ldp), pb, BW, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return LOWBIT_ERR_CUDA;
+    const int64_t esz = ydt == LOWBIT_BF16 ? 2 : 4;
+    const int vec_ok = ((reinterpret_cast<uintptr_t>(y) & 15u) == 0 && (ldy * esz) % 16 == 0) ? 1 : 0;
+    if (f == LOWBIT_TERNARY2) return launch_fmt<kT2>(mq, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, nt, status, st);
+    if (f == LOWBIT_BINARY1) return launch_fmt<kB1>(mq, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, nt, status, st);
+    return launch_fmt<kI4>(mq, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, nt, status, st);
+}
+
+}  // namespace lowbit

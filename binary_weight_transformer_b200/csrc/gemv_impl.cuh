@@ -212,7 +212,7 @@ gemv_smem_kernel(const int8_t *__restrict__ q, int64_t ldq, const float *__restr
 {
     using F = Fmt<FMT>;
     constexpr int QP = QPieces<FMT>::value;
-    extern __shared__ uint4 qs[];  // [M][nchunks * QP]
+    extern __shared__ uint4 qs[];  // [M][QP][nchunks]: piece-major, so lanes read consecutive pieces
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int64_t row0 = (static_cast<int64_t>(blockIdx.x) * kWarps + warp) * R;
@@ -236,8 +236,8 @@ gemv_smem_kernel(const int8_t *__restrict__ q, int64_t ldq, const float *__restr
             }
         if (c0 == 0) {
             for (int64_t i = threadIdx.x; i < M * qpieces; i += blockDim.x) {
-                const int64_t t = i / qpieces, p = i % qpieces;
-                qs[i] = load_q16(q + t * ldq, p * 16, K);
+                const int64_t t = i / qpieces, j = i % qpieces;   // j = chunk * QP + piece
+                qs[t * qpieces + (j % QP) * nchunks + j / QP] = load_q16(q + t * ldq, j * 16, K);
             }
             __syncthreads();
         }
@@ -250,7 +250,7 @@ gemv_smem_kernel(const int8_t *__restrict__ q, int64_t ldq, const float *__restr
                     if (t < M) {
                         uint4 qv[QP];
 #pragma unroll
-                        for (int p = 0; p < QP; ++p) qv[p] = qs[t * qpieces + c * QP + p];
+                        for (int p = 0; p < QP; ++p) qv[p] = qs[t * qpieces + p * nchunks + c];
 #pragma unroll
                         for (int r = 0; r < R; ++r) acc[r][t] = chunk_dot_regs<FMT>(wv[r][u], qv, acc[r][t]);
                     }

@@ -184,8 +184,11 @@ lowbit_status lowbit_act_quant(const void *x, lowbit_dtype xdt, int64_t M, int64
  * ldq and ldp multiples of 16), s_x fp32 [M], s_w fp32 [lowbit_scale_count].
  * Output y [M, ldy], ldy >= N, aligned to its element size.  Bytes of q past
  * K are ignored.  K <= lowbit_max_k(f), else LOWBIT_ERR_OVERFLOW_BOUND.
- * M <= 4 runs the packed-weight GEMV kernel; larger M runs the tcgen05
- * tensor-core GEMM (int8 MMA, accumulators in tensor memory). */
+ * M <= 4 runs the packed-weight GEMV kernel; larger M runs a tcgen05
+ * tensor-core GEMM (int8 MMA, accumulators in tensor memory): with the
+ * expanded weight tile in shared memory and K split over a cluster when the
+ * output tiles are few (5 <= M < 512), with the weight tile in tensor memory
+ * from M = 512. */
 lowbit_status lowbit_linear(const int8_t *q, int64_t ldq, const float *s_x,
                             int64_t M, int64_t K,
                             const uint8_t *packed, int64_t ldp, const float *s_w,
@@ -194,8 +197,10 @@ lowbit_status lowbit_linear(const int8_t *q, int64_t ldq, const float *s_x,
                             int32_t *status_dev, void *stream);
 
 /* Same operator with the kernel chosen by the caller: path 0 = automatic (as
- * lowbit_linear), 1 = packed-weight GEMV (any M), 2 = tensor-core GEMM (any
- * M).  Lets tests and benchmarks reach both kernels at every size. */
+ * lowbit_linear), 1 = packed-weight GEMV (any M), 2 = tensor-core GEMM with
+ * the expanded weight tile in shared memory (any M), 3 = tensor-core GEMM
+ * with the expanded weight tile in tensor memory (any M).  Lets tests and
+ * benchmarks reach every kernel at every size. */
 lowbit_status lowbit_linear_path(const int8_t *q, int64_t ldq, const float *s_x,
                                  int64_t M, int64_t K,
                                  const uint8_t *packed, int64_t ldp, const float *s_w,
