@@ -197,11 +197,16 @@ gemm_ts_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     uint8_t *sP = sQ + kStages * Q_BYTES;        // kStages x P_BYTES
     uint8_t *sStage = sP + kStages * P_BYTES;    // 4 x epilogue staging
     uint64_t *bars = reinterpret_cast<uint64_t *>(sStage + 4 * stage_warp_bytes<OUT>());
+    // full_tma[s]: the TMA stage's token and packed tiles have landed.
+    // full_a[s2]: A stage s2 holds the expanded weights of a K step, and the
+    //   expanders saw that step's TMA stage complete, so one wait on full_a
+    //   orders the MMA after both (release/acquire through the expanders).
+    // mma_done[s]: the MMAs of the K step that used TMA stage s are complete;
+    //   it frees that TMA stage and, two K steps later, the A stage.
     uint64_t *full_tma = bars;
-    uint64_t *empty_tma = bars + kStages;
+    uint64_t *mma_done = bars + kStages;
     uint64_t *full_a = bars + 2 * kStages;
-    uint64_t *empty_a = full_a + kAStages;
-    uint64_t *acc_full = empty_a + kAStages;
+    uint64_t *acc_full = full_a + 2 * kAStages;
     uint64_t *acc_empty = acc_full + 2;
     uint64_t *drain = acc_full + 4;
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(acc_full + 5);
@@ -213,12 +218,9 @@ gemm_ts_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full_tma[s], 1);
-            mbar_init(&empty_tma[s], 1);
+            mbar_init(&mma_done[s], 1);
         }
-        for (int s = 0; s < kAStages; ++s) {
-            mbar_init(&full_a[s], 128);
-            mbar_init(&empty_a[s], 1);
-        }
+        for (int s = 0; s < kAStages; ++s) mbar_init(&full_a[s], 128);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
             mbar_init(&acc_empty[b], 4);
@@ -256,7 +258,7 @@ gemm_ts_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 const int t0 = static_cast<int>((tile / num_w) * nt);
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
                     const int s = g % kStages;
-                    if (!wait_bar(&empty_tma[s], ((g / kStages) & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
+                    if (!wait_bar(&mma_done[s], ((g / kStages) & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
                     mbar_arrive_expect_tx(&full_tma[s], q_bytes + P_BYTES);
                     tma_load_2d(sQ + s * Q_BYTES, &map_q, &full_tma[s], kb * BK, t0);
                     tma_load_2d(sP + s * P_BYTES, &map_p, &full_tma[s], kb * PB, w0);
@@ -273,6 +275,9 @@ gemm_ts_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             const uint32_t idesc = idesc_for(nt);
+            // K-major SW128 descriptor of TMA stage 0; stage s and K slice kk
+            // add (s * Q_BYTES + kk * 32) / 16 to its start-address field.
+            const uint64_t qdesc0 = sw128_desc(smem_u32(sQ));
             uint32_t g = 0;
             uint32_t t = 0;
             bool ok = true;
@@ -283,17 +288,15 @@ gemm_ts_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * kDCols);
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
                     const int s1 = g % kStages, s2 = g % kAStages;
-                    if (!wait_bar(&full_tma[s1], (g / kStages) & 1u, abort_flag, status) ||
-                        !wait_bar(&full_a[s2], (g / kAStages) & 1u, abort_flag, status)) { ok = false; break; }
+                    if (!wait_bar(&full_a[s2], (g / kAStages) & 1u, abort_flag, status)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t q_addr = smem_u32(sQ + s1 * Q_BYTES);
+                    const uint64_t qdesc = qdesc0 + static_cast<uint64_t>((s1 * Q_BYTES) >> 4);
                     const uint32_t a_tmem = tmem_base + a_col0 + static_cast<uint32_t>(s2 * kACols);
 #pragma unroll
                     for (int kk = 0; kk < BK / UMMA_K; ++kk)
-                        tc_mma_i8_ts(d_tmem, a_tmem + kk * (UMMA_K / 4), sw128_desc(q_addr + kk * UMMA_K), idesc,
-                                     (kb | kk) != 0 ? 1u : 0u);
-                    tc_commit(&empty_tma[s1]);
-                    tc_commit(&empty_a[s2]);
+                        tc_mma_i8_ts(d_tmem, a_tmem + kk * (UMMA_K / 4), qdesc + static_cast<uint64_t>(kk * (UMMA_K >> 4)),
+                                     idesc, (kb | kk) != 0 ? 1u : 0u);
+                    tc_commit(&mma_done[s1]);
                 }
                 if (!ok) break;
                 tc_commit(&acc_full[b]);
@@ -311,10 +314,16 @@ gemm_ts_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
             for (int kb = 0; kb < nkb; ++kb, ++g) {
                 const int s1 = g % kStages, s2 = g % kAStages;
+                // A stage s2 is free once the MMAs of K step g - kAStages
+                // are complete (mma_done of that step's TMA stage).
                 int ready = 0;
-                if (lane == 0)
-                    ready = (wait_bar(&full_tma[s1], (g / kStages) & 1u, abort_flag, status) &&
-                             wait_bar(&empty_a[s2], ((g / kAStages) & 1u) ^ 1u, abort_flag, status)) ? 1 : 0;
+                if (lane == 0) {
+                    ready = wait_bar(&full_tma[s1], (g / kStages) & 1u, abort_flag, status) ? 1 : 0;
+                    if (ready && g >= static_cast<uint32_t>(kAStages)) {
+                        const uint32_t gp = g - kAStages;
+                        ready = wait_bar(&mma_done[gp % kStages], (gp / kStages) & 1u, abort_flag, status) ? 1 : 0;
+                    }
+                }
                 ready = __shfl_sync(0xffffffffu, ready, 0);
                 if (!ready) { ok = false; break; }
                 tc_fence_after();
