@@ -184,7 +184,8 @@ def lowbit_linear(q, s_x, packed, s_w, fmt: int, N: int, out_dtype: int = F32, K
     """y[M, N] from int8 codes q[M, >=K] and a packed artifact (see lowbit.h).
 
     ``path`` 0 picks the kernel by M; 1 forces the GEMV, 2 the tensor-core GEMM
-    with the expanded tile in shared memory, 3 the one with it in tensor memory."""
+    with the expanded tile in shared memory, 3 the one with it in tensor memory,
+    4 the tensor-memory one on SM pairs (256 weight rows per MMA)."""
     import torch
     M = q.shape[0]
     if K is None:

@@ -29,6 +29,11 @@ lowbit_status gemm_ts_launch(const int8_t *q, int64_t ldq, const float *s_x, int
                              lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int32_t *status,
                              cudaStream_t st);
 
+lowbit_status gemm_ts_pair_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
+                                  const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
+                                  lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy,
+                                  int32_t *status, cudaStream_t st);
+
 lowbit_status launch_status()
 {
     return cudaGetLastError() == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
@@ -185,7 +190,7 @@ lowbit_status lowbit_linear_path(const int8_t *q, int64_t ldq, const float *s_x,
     if (!valid_format(f) || q == nullptr || s_x == nullptr || packed == nullptr || s_w == nullptr || y == nullptr)
         return LOWBIT_ERR_INVALID_ARG;
     if (ydt != LOWBIT_F32 && ydt != LOWBIT_BF16 && ydt != LOWBIT_I32) return LOWBIT_ERR_INVALID_ARG;
-    if (path < 0 || path > 3) return LOWBIT_ERR_INVALID_ARG;
+    if (path < 0 || path > 4) return LOWBIT_ERR_INVALID_ARG;
     if (M <= 0 || N <= 0 || K <= 0 || ldq < K || ldy < N) return LOWBIT_ERR_INVALID_ARG;
     if (M > INT32_MAX || N > INT32_MAX) return LOWBIT_ERR_INVALID_ARG;
     const int64_t rb = static_cast<int64_t>(lowbit_packed_row_bytes(f, K));
@@ -205,6 +210,8 @@ lowbit_status lowbit_linear_path(const int8_t *q, int64_t ldq, const float *s_x,
     // From 512 tokens the tensor-memory variant (weights as the MMA's A
     // operand in TMEM) is as fast or faster; below it the shared-memory
     // variant, which splits K over a cluster when tiles are few, wins.
+    if (path == 4)
+        return gemm_ts_pair_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, status_dev, st);
     if (path == 3 || (path == 0 && M >= 512))
         return gemm_ts_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, status_dev, st);
     return gemm_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, status_dev, st);

@@ -314,21 +314,22 @@ gemm_ts_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
             for (int kb = 0; kb < nkb; ++kb, ++g) {
                 const int s1 = g % kStages, s2 = g % kAStages;
-                // A stage s2 is free once the MMAs of K step g - kAStages
-                // are complete (mma_done of that step's TMA stage).
                 int ready = 0;
-                if (lane == 0) {
-                    ready = wait_bar(&full_tma[s1], (g / kStages) & 1u, abort_flag, status) ? 1 : 0;
-                    if (ready && g >= static_cast<uint32_t>(kAStages)) {
-                        const uint32_t gp = g - kAStages;
-                        ready = wait_bar(&mma_done[gp % kStages], (gp / kStages) & 1u, abort_flag, status) ? 1 : 0;
-                    }
+                if (lane == 0) ready = wait_bar(&full_tma[s1], (g / kStages) & 1u, abort_flag, status) ? 1 : 0;
+                ready = __shfl_sync(0xffffffffu, ready, 0);
+                if (!ready) { ok = false; break; }
+                // Expand in registers first: only the TMEM store waits for the
+                // A stage, which is free once the MMAs of K step g - kAStages
+                // are complete (mma_done of that step's TMA stage).
+                uint32_t w[32];
+                expand_row<FMT>(p_base + s1 * P_BYTES + r * PB, w);
+                if (lane == 0 && g >= static_cast<uint32_t>(kAStages)) {
+                    const uint32_t gp = g - kAStages;
+                    ready = wait_bar(&mma_done[gp % kStages], (gp / kStages) & 1u, abort_flag, status) ? 1 : 0;
                 }
                 ready = __shfl_sync(0xffffffffu, ready, 0);
                 if (!ready) { ok = false; break; }
                 tc_fence_after();
-                uint32_t w[32];
-                expand_row<FMT>(p_base + s1 * P_BYTES + r * PB, w);
                 tmem_st_32cols(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + a_col0 +
                                    static_cast<uint32_t>(s2 * kACols), w);
                 tmem_wait_st();
@@ -410,6 +411,315 @@ lowbit_status launch_fmt(const CUtensorMap &mq, const CUtensorMap &mp, const flo
     return launch_t<FMT, LOWBIT_I32>(mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt, status, st);
 }
 
+
+// ---------------------------------------------------------------------------
+// SM-pair variant (tcgen05 cta_group::2).
+//
+// A cluster of two CTAs computes a 256-row weight tile: each CTA expands its
+// 128 rows into its own tensor memory, and the MMA (issued by the even CTA
+// for both) has M = 256.  The token tile's N columns are split between the
+// two CTAs' shared memory, N/2 each, so that each SM stages and reads half the
+// token bytes of the single-CTA kernel per MAC; the L2 -> SM traffic per MAC
+// drops the same way.  Each CTA's tensor memory holds the accumulators of its
+// own 128 weight rows for all N tokens, and each CTA runs its own epilogue.
+//
+// Barriers (every CTA holds all of them; the even CTA's full_a and acc_empty
+// collect the arrivals of both):
+//   full_tma[s]   local TMA completion (token half + packed rows)
+//   full_a[s2]    even CTA: 4 expander warps x 2 CTAs wrote A stage s2 and saw
+//                 their TMA stage complete
+//   mma_done[s]   both CTAs, multicast commit: the MMAs of the K step that used
+//                 TMA stage s are done (frees the TMA stage, and two K steps
+//                 later the A stage)
+//   acc_full[b]   both CTAs, multicast commit: accumulator buffer b is final
+//   acc_empty[b]  even CTA: 4 epilogue warps x 2 CTAs have drained buffer b
+// ---------------------------------------------------------------------------
+constexpr int kPairStages = 8;
+constexpr int QH_BYTES = (BT / 2) * BK;  // largest token half tile
+
+template <int FMT, int OUT>
+__host__ __device__ constexpr size_t smem_bytes_pair()
+{
+    return 1024 + static_cast<size_t>(kPairStages) * (QH_BYTES + p_bytes<FMT>()) + 4 * stage_warp_bytes<OUT>() +
+           8 * (2 * kPairStages + kAStages + 8);
+}
+
+__device__ __forceinline__ void tc_mma_i8_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on the barrier at this shared-memory offset in both CTAs of the pair
+// once the pair's MMAs issued so far are complete.
+__device__ __forceinline__ void tc_commit_pair_both(uint64_t *bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+        ::"r"(smem_u32(bar)), "h"(static_cast<uint16_t>(0x3)) : "memory");
+}
+
+__device__ __forceinline__ void tc_commit_pair_self(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ uint32_t idesc_pair(int nt)
+{
+    return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(nt >> 3) << 17) |
+           (static_cast<uint32_t>((2 * BW) >> 4) << 24);
+}
+
+template <int FMT, int OUT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+gemm_ts_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_p,
+                    const float *__restrict__ s_x, const float *__restrict__ s_w, int64_t M, int64_t N, int64_t K,
+                    void *__restrict__ y, int64_t ldy, int vec_ok, int nt, int32_t *status)
+{
+    constexpr int PB = packed_row_kblock<FMT>();
+    constexpr int P_BYTES = p_bytes<FMT>();
+    constexpr int kShift = Fmt<FMT>::kShift;
+    constexpr int S = kPairStages;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = base;                      // S x 14 KB token halves, 1024-aligned
+    uint8_t *sP = sQ + S * QH_BYTES;         // S x P_BYTES packed rows
+    uint8_t *sStage = sP + S * P_BYTES;      // 4 x epilogue staging
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sStage + 4 * stage_warp_bytes<OUT>());
+    uint64_t *full_tma = bars;
+    uint64_t *mma_done = bars + S;
+    uint64_t *full_a = bars + 2 * S;
+    uint64_t *acc_full = full_a + kAStages;
+    uint64_t *acc_empty = acc_full + 2;
+    uint64_t *drain = acc_full + 4;
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(acc_full + 5);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(acc_full + 6);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full_tma[s], 1);
+            mbar_init(&mma_done[s], 1);
+        }
+        for (int s = 0; s < kAStages; ++s) mbar_init(&full_a[s], 8);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 8);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_q)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_p)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(const_cast<uint32_t *>(tmem_slot))), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // both CTAs' barriers exist before any remote arrive
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t a_col0 = 2 * kDCols;
+
+    const int64_t num_w = (N + 2 * BW - 1) / (2 * BW);  // 256-row weight tiles
+    const int64_t num_t = (M + nt - 1) / nt;
+    const int64_t num_tiles = num_w * num_t;
+    const int64_t pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+    const int nkb = static_cast<int>((K + BK - 1) / BK);
+    const int half = nt / 2;
+    const uint32_t qh_bytes = static_cast<uint32_t>(half) * BK;
+
+    if (warp == 0) {
+        // ---------------- TMA producer (both CTAs) ----------------
+        if (lane == 0) {
+            uint32_t g = 0;
+            bool ok = true;
+            for (int64_t tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+                const int w0 = static_cast<int>((tile % num_w) * 2 * BW + rank * BW);
+                const int t0 = static_cast<int>((tile / num_w) * nt + rank * half);
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % S;
+                    if (!wait_bar(&mma_done[s], ((g / S) & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&full_tma[s], qh_bytes + P_BYTES);
+                    tma_load_2d(sQ + s * QH_BYTES, &map_q, &full_tma[s], kb * BK, t0);
+                    tma_load_2d(sP + s * P_BYTES, &map_p, &full_tma[s], kb * PB, w0);
+                }
+            }
+            if (!ok) {
+                for (uint32_t i = 0; i < static_cast<uint32_t>(S) && i < g; ++i) {
+                    const uint32_t gi = g - 1 - i;
+                    wait_bar(&full_tma[gi % S], (gi / S) & 1u, abort_flag, nullptr, 200000000ll);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (even CTA) ----------------
+        if (leader && lane == 0) {
+            const uint32_t idesc = idesc_pair(nt);
+            const uint64_t qdesc0 = sw128_desc(smem_u32(sQ));
+            uint32_t g = 0;
+            uint32_t t = 0;
+            bool ok = true;
+            for (int64_t tile = pair; tile < num_tiles && ok; tile += num_pairs, ++t) {
+                const int b = t & 1;
+                if (!wait_bar(&acc_empty[b], ((t >> 1) & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * kDCols);
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s1 = g % S, s2 = g % kAStages;
+                    if (!wait_bar(&full_a[s2], (g / kAStages) & 1u, abort_flag, status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t qdesc = qdesc0 + static_cast<uint64_t>((s1 * QH_BYTES) >> 4);
+                    const uint32_t a_tmem = tmem_base + a_col0 + static_cast<uint32_t>(s2 * kACols);
+#pragma unroll
+                    for (int kk = 0; kk < BK / UMMA_K; ++kk)
+                        tc_mma_i8_ts_pair(d_tmem, a_tmem + kk * (UMMA_K / 4),
+                                          qdesc + static_cast<uint64_t>(kk * (UMMA_K >> 4)), idesc,
+                                          (kb | kk) != 0 ? 1u : 0u);
+                    tc_commit_pair_both(&mma_done[s1]);
+                }
+                if (!ok) break;
+                tc_commit_pair_both(&acc_full[b]);
+            }
+            tc_commit_pair_self(drain);
+            wait_bar(drain, 0, abort_flag, nullptr, 200000000ll);
+        }
+    } else if (warp < 6) {
+        // ---------------- expanders: packed -> own TMEM ----------------
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const uint32_t p_base = smem_u32(sP);
+        const uint32_t full_a_leader = map_to_peer(smem_u32(full_a), 0);
+        uint32_t g = 0;
+        bool ok = true;
+        for (int64_t tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+            for (int kb = 0; kb < nkb; ++kb, ++g) {
+                const int s1 = g % S, s2 = g % kAStages;
+                int ready = 0;
+                if (lane == 0) ready = wait_bar(&full_tma[s1], (g / S) & 1u, abort_flag, status) ? 1 : 0;
+                ready = __shfl_sync(0xffffffffu, ready, 0);
+                if (!ready) { ok = false; break; }
+                uint32_t w[32];
+                expand_row<FMT>(p_base + s1 * P_BYTES + r * PB, w);
+                if (lane == 0 && g >= static_cast<uint32_t>(kAStages)) {
+                    const uint32_t gp = g - kAStages;
+                    ready = wait_bar(&mma_done[gp % S], (gp / S) & 1u, abort_flag, status) ? 1 : 0;
+                }
+                ready = __shfl_sync(0xffffffffu, ready, 0);
+                if (!ready) { ok = false; break; }
+                tc_fence_after();
+                tmem_st_32cols(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + a_col0 +
+                                   static_cast<uint32_t>(s2 * kACols), w);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(full_a_leader + static_cast<uint32_t>(s2 * 8));
+            }
+        }
+    } else {
+        // ---------------- epilogue: own 128 weight rows ----------------
+        const int quarter = warp & 3;
+        const uint32_t stage = smem_u32(sStage) + static_cast<uint32_t>((warp - 6) * stage_warp_bytes<OUT>());
+        const uint32_t acc_empty_leader = map_to_peer(smem_u32(acc_empty), 0);
+        uint32_t t = 0;
+        for (int64_t tile = pair; tile < num_tiles; tile += num_pairs, ++t) {
+            const int b = t & 1;
+            int ready = 0;
+            if (lane == 0) ready = wait_bar(&acc_full[b], (t >> 1) & 1u, abort_flag, status) ? 1 : 0;
+            ready = __shfl_sync(0xffffffffu, ready, 0);
+            if (!ready) break;
+            tc_fence_after();
+            const int64_t n0 = (tile % num_w) * 2 * BW + rank * BW + quarter * 32;
+            const int64_t t0 = (tile / num_w) * nt;
+            const int64_t n = n0 + lane;
+            const float sw = (n < N) ? s_w[FMT == kT2 ? 0 : n] : 0.0f;
+#pragma unroll 1
+            for (int cc = 0; cc < nt / 32; ++cc) {
+                uint32_t v[32];
+                tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                   static_cast<uint32_t>(b * kDCols + cc * 32), v);
+                const int64_t tc0 = t0 + cc * 32;
+                if (tc0 < M && n0 < N)
+                    store_chunk<OUT>(v, sw, s_x, kShift, y, ldy, tc0, M, n0, N, vec_ok != 0, stage, lane);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(acc_empty_leader + static_cast<uint32_t>(b * 8));
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // the pair's MMAs and remote arrivals are over
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+template <int FMT, int OUT>
+lowbit_status launch_pair_t(const CUtensorMap &mq, const CUtensorMap &mp, const float *s_x, const float *s_w,
+                            int64_t M, int64_t N, int64_t K, void *y, int64_t ldy, int vec_ok, int nt,
+                            int32_t *status, cudaStream_t st)
+{
+    constexpr size_t smem = smem_bytes_pair<FMT, OUT>();
+    static_assert(smem <= 232448, "shared memory budget");
+    static int max_pairs[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LOWBIT_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    if (max_pairs[dev] == 0) {
+        if (cudaFuncSetAttribute(gemm_ts_pair_kernel<FMT, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem)) != cudaSuccess)
+            return LOWBIT_ERR_CUDA;
+        // Pairs that can be resident at once (the GPCs decide how many SM
+        // pairs exist); the persistent grid never exceeds it.
+        cfg.gridDim = dim3(2 * static_cast<unsigned>(device_sm_count() / 2));
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_ts_pair_kernel<FMT, OUT>, &cfg) != cudaSuccess || n <= 0)
+            return LOWBIT_ERR_CUDA;
+        max_pairs[dev] = n;
+    }
+    const int64_t tiles = ((N + 2 * BW - 1) / (2 * BW)) * ((M + nt - 1) / nt);
+    const int64_t pairs = tiles < max_pairs[dev] ? tiles : max_pairs[dev];
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    if (cudaLaunchKernelEx(&cfg, gemm_ts_pair_kernel<FMT, OUT>, mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt,
+                           status) != cudaSuccess)
+        return LOWBIT_ERR_CUDA;
+    return launch_status();
+}
+
+template <int FMT>
+lowbit_status launch_pair_fmt(const CUtensorMap &mq, const CUtensorMap &mp, const float *s_x, const float *s_w,
+                              int64_t M, int64_t N, int64_t K, void *y, lowbit_dtype ydt, int64_t ldy, int vec_ok,
+                              int nt, int32_t *status, cudaStream_t st)
+{
+    if (ydt == LOWBIT_F32)
+        return launch_pair_t<FMT, LOWBIT_F32>(mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt, status, st);
+    if (ydt == LOWBIT_BF16)
+        return launch_pair_t<FMT, LOWBIT_BF16>(mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt, status, st);
+    return launch_pair_t<FMT, LOWBIT_I32>(mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt, status, st);
+}
+
 }  // namespace ts
 
 // Token tile: 224 for many tokens, else M rounded up to a multiple of 32.
@@ -437,4 +747,34 @@ lowbit_status gemm_ts_launch(const int8_t *q, int64_t ldq, const float *s_x, int
     return launch_fmt<kI4>(mq, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, nt, status, st);
 }
 
+}  // namespace lowbit
+
+namespace lowbit {
+// SM-pair variant: token tile as above (224, or M rounded up to 32), each CTA
+// of the pair staging half of it.
+lowbit_status gemm_ts_pair_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
+                                  const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
+                                  lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy,
+                                  int32_t *status, cudaStream_t st)
+{
+    using namespace ts;
+    const int nt = M >= BT ? BT : static_cast<int>((M + 31) / 32 * 32);
+    CUtensorMap mq, mp;
+    if (!make_map_2d(&mq, q, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(ldq), BK,
+                     static_cast<uint32_t>(nt / 2), CU_TENSOR_MAP_SWIZZLE_128B))
+        return LOWBIT_ERR_CUDA;
+    const uint32_t pb = f == LOWBIT_TERNARY2 ? packed_row_kblock<kT2>()
+                        : f == LOWBIT_BINARY1 ? packed_row_kblock<kB1>()
+                                              : packed_row_kblock<kI4>();
+    if (!make_map_2d(&mp, packed, static_cast<uint64_t>(row_bytes), static_cast<uint64_t>(N),
+                     static_cast<uint64_t>(ldp), pb, BW, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return LOWBIT_ERR_CUDA;
+    const int64_t esz = ydt == LOWBIT_BF16 ? 2 : 4;
+    const int vec_ok = ((reinterpret_cast<uintptr_t>(y) & 15u) == 0 && (ldy * esz) % 16 == 0) ? 1 : 0;
+    if (f == LOWBIT_TERNARY2)
+        return launch_pair_fmt<kT2>(mq, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, nt, status, st);
+    if (f == LOWBIT_BINARY1)
+        return launch_pair_fmt<kB1>(mq, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, nt, status, st);
+    return launch_pair_fmt<kI4>(mq, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, nt, status, st);
+}
 }  // namespace lowbit

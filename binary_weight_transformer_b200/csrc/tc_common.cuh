@@ -54,10 +54,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 }
 
 
+// Arrive on a barrier given by its shared::cluster address, which may be in
+// another CTA of the cluster (see map_to_peer).  Default semantics (release
+// at CTA scope): a cluster-scope release costs about a thousand cycles per
+// arrival here.  What the waiter needs ordered before it is either tensor
+// memory written by this thread (completed by tcgen05.wait::st and fenced by
+// tcgen05.fence::before_thread_sync) or TMA data whose completion this
+// thread observed on its own barrier.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 // Bounded wait: true once the phase with `parity` has completed; false if the
 // CTA aborted or `limit` SM cycles passed (then the timeout is recorded).
 __device__ inline bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int32_t *status,
-                         long long limit = kWaitCycles)
+                                long long limit = kWaitCycles)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();

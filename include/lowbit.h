@@ -199,8 +199,10 @@ lowbit_status lowbit_linear(const int8_t *q, int64_t ldq, const float *s_x,
 /* Same operator with the kernel chosen by the caller: path 0 = automatic (as
  * lowbit_linear), 1 = packed-weight GEMV (any M), 2 = tensor-core GEMM with
  * the expanded weight tile in shared memory (any M), 3 = tensor-core GEMM
- * with the expanded weight tile in tensor memory (any M).  Lets tests and
- * benchmarks reach every kernel at every size. */
+ * with the expanded weight tile in tensor memory (any M), 4 = the same on
+ * pairs of SMs (one MMA covers 256 weight rows; any M).  Other values return
+ * LOWBIT_ERR_INVALID_ARG.  Lets tests and benchmarks reach every kernel at
+ * every size. */
 lowbit_status lowbit_linear_path(const int8_t *q, int64_t ldq, const float *s_x,
                                  int64_t M, int64_t K,
                                  const uint8_t *packed, int64_t ldp, const float *s_w,

@@ -210,7 +210,7 @@ SHAPES = [(1, 768, 192), (3, 257, 200), (16, 96, 1000), (17, 300, 192), (129, 51
           (5, 33, 16), (200, 1, 4000), (64, 500, 4096), (130, 1000, 2000)]
 
 
-@pytest.mark.parametrize("path", [1, 2, 3], ids=["gemv", "gemm", "gemm_ts"])
+@pytest.mark.parametrize("path", [1, 2, 3, 4], ids=["gemv", "gemm", "gemm_ts", "gemm_ts_pair"])
 @pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
 @pytest.mark.parametrize("M,N,K", SHAPES, ids=str)
 def test_linear_int32_accumulators_bit_exact(path, fmt, M, N, K):
@@ -218,7 +218,7 @@ def test_linear_int32_accumulators_bit_exact(path, fmt, M, N, K):
     assert np.array_equal(y.cpu().numpy().astype(np.int64), acc)
 
 
-@pytest.mark.parametrize("path", [1, 2, 3], ids=["gemv", "gemm", "gemm_ts"])
+@pytest.mark.parametrize("path", [1, 2, 3, 4], ids=["gemv", "gemm", "gemm_ts", "gemm_ts_pair"])
 @pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
 @pytest.mark.parametrize("M,N,K", SHAPES[:6] + SHAPES[8:], ids=str)
 def test_linear_f32_within_tolerance(path, fmt, M, N, K):
@@ -230,7 +230,7 @@ def test_linear_f32_within_tolerance(path, fmt, M, N, K):
     assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
 
 
-@pytest.mark.parametrize("path", [1, 2, 3], ids=["gemv", "gemm", "gemm_ts"])
+@pytest.mark.parametrize("path", [1, 2, 3, 4], ids=["gemv", "gemm", "gemm_ts", "gemm_ts_pair"])
 @pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
 @pytest.mark.parametrize("M,N,K", SHAPES[:6] + SHAPES[8:], ids=str)
 def test_linear_bf16_within_one_ulp(path, fmt, M, N, K):
@@ -241,7 +241,7 @@ def test_linear_bf16_within_one_ulp(path, fmt, M, N, K):
     assert np.array_equal(got, ref)
 
 
-@pytest.mark.parametrize("path", [1, 2, 3], ids=["gemv", "gemm", "gemm_ts"])
+@pytest.mark.parametrize("path", [1, 2, 3, 4], ids=["gemv", "gemm", "gemm_ts", "gemm_ts_pair"])
 def test_linear_degenerate_weights(path):
     # all-zero weights: gamma = 0, every code 0, y = 0
     y, acc, _, _ = run_case(bwt.TERNARY2, 20, 64, 256, path, bwt.F32, 800, zero_w=True)
@@ -249,7 +249,7 @@ def test_linear_degenerate_weights(path):
     assert not y.cpu().numpy().any()
 
 
-@pytest.mark.parametrize("path", [1, 2, 3], ids=["gemv", "gemm", "gemm_ts"])
+@pytest.mark.parametrize("path", [1, 2, 3, 4], ids=["gemv", "gemm", "gemm_ts", "gemm_ts_pair"])
 def test_linear_all_plus_one_gives_row_sums(path):
     # ternary codes all +1: acc[t, n] = sum_k q[t, k] (add/sub/skip rule)
     M, N, K = 19, 40, 320
