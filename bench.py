@@ -149,10 +149,22 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
+def dispatched_kernel(M):
+    """The kernel lowbit_linear picks for M tokens (same rule as the library):
+    the packed-weight GEMV up to 4 tokens, the tensor-core GEMM with the
+    weight tile expanded into shared memory (cluster split-K when output tiles
+    are few) below 512, the one with it in tensor memory from 512."""
+    if M <= 4:
+        return "gemv_smem_kernel"
+    return "gemm_kernel/gemm_splitk_kernel" if M < 512 else "gemm_ts_kernel"
+
+
 class Point:
     def __init__(self, mi, m, M):
         self.mi, self.m, self.M = mi, m, M
-        self.kernel = "gemv" if M <= 16 else "gemm"
+        self.kernel = dispatched_kernel(M)
+        # up to 16 tokens the packed weights dominate the bytes: HBM-bound
+        self.bound = "hbm" if M <= 16 else "tensor"
         self.ops = 2 * M * m.N * m.K
 
 
@@ -315,7 +327,7 @@ def run_gpu_arm(args, wl):
         d = {"matrix": f"{pt.m.K}->{pt.m.N}", "M": pt.M, "kernel": pt.kernel, "us": round(ms * 1e3, 2),
              "act_quant_us": round(ams * 1e3, 2),
              "act_quant_gbs": round(act_bytes / (ams * 1e-3) / 1e9, 1)}
-        if pt.M <= 16:
+        if pt.bound == "hbm":
             gbs = packed_bytes / (ms * 1e-3) / 1e9
             d.update(packed_gbs=round(gbs, 1), frac_hbm=round(gbs / hbm, 3))
             gemv_bytes += packed_bytes
@@ -329,16 +341,16 @@ def run_gpu_arm(args, wl):
 
     # dominant kernel: the tensor-core GEMM at the largest M (about 60% of the
     # step); the launch reported is the first matrix's, the one profiled
-    big = [i for i, pt in enumerate(points) if pt.kernel == "gemm"]
+    big = [i for i, pt in enumerate(points) if pt.bound == "tensor"]
     dom_i = min(big, key=lambda i: (-points[i].M, i)) if big else max(range(len(points)), key=lambda i: per_point[i])
     dom, dom_ms = points[dom_i], per_point[dom_i]
-    if dom.kernel == "gemm":
+    if dom.bound == "tensor":
         achieved = dom.ops / (dom_ms * 1e-3) / 1e12
         roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(int8_peak, 1),
                     "unit": "TOPS", "frac": round(achieved / int8_peak, 4),
-                    "traffic": profiled_traffic("gemm_kernel_ternary_4b_M8192.md", "gemm_sm100.cu")
+                    "traffic": profiled_traffic("gemm_ts_kernel_ternary_4b_M8192.md", "gemm_ts.cu")
                     if (wl.name == "ternary_4b" and dom.M == 8192 and dom.mi == 0) else None,
-                    "kernel": f"lowbit gemm_kernel, M={dom.M} {dom.m.K}->{dom.m.N}",
+                    "kernel": f"lowbit {dom.kernel}, M={dom.M} {dom.m.K}->{dom.m.N}",
                     "peak_note": f"int8 = 2 x bf16 sustained ({peak_kind})"}
     else:
         fmt_bits = {wls.TERNARY2: 2, wls.BINARY1: 1, wls.INT4: 4}[wl.fmt]
@@ -346,7 +358,7 @@ def run_gpu_arm(args, wl):
         achieved = byts / (dom_ms * 1e-3) / 1e9
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                     "frac": round(achieved / hbm, 4), "traffic": None,
-                    "kernel": f"lowbit gemv_kernel, M={dom.M}", "peak_note": peak_kind}
+                    "kernel": f"lowbit {dom.kernel}, M={dom.M}", "peak_note": peak_kind}
 
     cpu = run_cpu_baseline(wl, args.cpu_seconds) if (rank == 0 and world == 1 and not args.no_cpu) else None
     line = {
