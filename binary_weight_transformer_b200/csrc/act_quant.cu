@@ -123,6 +123,8 @@ act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
     constexpr int kRows = kThreads / TPR;
     constexpr int E = In<T>::kPerVec;
     __shared__ uint32_t red[kThreads / 32];
+    pdl_wait();
+    pdl_trigger();
 
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kRows + threadIdx.x / TPR;
     const int r = threadIdx.x % TPR;
@@ -195,6 +197,8 @@ act_quant_long(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
                int8_t *__restrict__ q, int64_t ldq, float *__restrict__ s_x, int32_t *status)
 {
     __shared__ uint32_t red[8];
+    pdl_wait();
+    pdl_trigger();
     const int64_t row = blockIdx.x;
     const char *xrow = static_cast<const char *>(x) + row * ldx * sizeof(T);
     uint32_t amax = 0;
@@ -221,8 +225,8 @@ lowbit_status launch(const void *x, int64_t M, int64_t K, int64_t ldx, float eps
     // other layout takes the scalar-load kernel.
     const bool vec_ok = (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (ldx * static_cast<int64_t>(sizeof(T))) % 16 == 0;
     if (!vec_ok) {
-        act_quant_long<T><<<static_cast<unsigned>(M), 256, 0, st>>>(x, M, K, ldx, eps, q, ldq, s_x, status);
-        return launch_status();
+        return launch_pdl(act_quant_long<T>, dim3(static_cast<unsigned>(M)), dim3(256), 0, st, 0, x, M, K, ldx, eps,
+                          q, ldq, s_x, status);
     }
     auto grid_for = [&](int tpr) {
         const int rows = (tpr > 256 ? tpr : 256) / tpr;
@@ -230,9 +234,8 @@ lowbit_status launch(const void *x, int64_t M, int64_t K, int64_t ldx, float eps
     };
 #define LOWBIT_AQ(TPR)                                                                          \
     if (nvec <= static_cast<int64_t>(TPR) * kVPT) {                                             \
-        act_quant_regs<T, TPR><<<grid_for(TPR), (TPR > 256 ? TPR : 256), 0, st>>>(              \
-            x, M, K, ldx, eps, q, ldq, s_x, status);                                            \
-        return launch_status();                                                                 \
+        return launch_pdl(act_quant_regs<T, TPR>, dim3(grid_for(TPR)), dim3(TPR > 256 ? TPR : 256), \
+                          0, st, 0, x, M, K, ldx, eps, q, ldq, s_x, status);                    \
     }
     LOWBIT_AQ(8)
     LOWBIT_AQ(32)
@@ -242,8 +245,8 @@ lowbit_status launch(const void *x, int64_t M, int64_t K, int64_t ldx, float eps
     LOWBIT_AQ(512)
     LOWBIT_AQ(1024)
 #undef LOWBIT_AQ
-    act_quant_long<T><<<static_cast<unsigned>(M), 256, 0, st>>>(x, M, K, ldx, eps, q, ldq, s_x, status);
-    return launch_status();
+    return launch_pdl(act_quant_long<T>, dim3(static_cast<unsigned>(M)), dim3(256), 0, st, 0, x, M, K, ldx, eps, q,
+                      ldq, s_x, status);
 }
 
 }  // namespace

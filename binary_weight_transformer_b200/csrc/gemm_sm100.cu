@@ -245,6 +245,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // Global memory is touched only after the previous kernel on the stream
+    // has completed (programmatic dependent launch, see pdl_wait).
+    pdl_wait();
+    pdl_trigger();
 
     const int64_t num_m = (M + BM - 1) / BM;
     const int64_t num_n = (N + BN - 1) / BN;
@@ -446,6 +450,10 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // Global memory is touched only after the previous kernel on the stream
+    // has completed (programmatic dependent launch, see pdl_wait).
+    pdl_wait();
+    pdl_trigger();
 
     const int64_t num_m = (M + BM - 1) / BM;
     const int64_t tile = blockIdx.x / C;
@@ -625,26 +633,12 @@ lowbit_status launch_t(const CUtensorMap &ma, const CUtensorMap &mp, const float
                 return LOWBIT_ERR_CUDA;
             configured_split[dev] = true;
         }
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(static_cast<unsigned>(tiles * C));
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = static_cast<unsigned>(C);
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, gemm_splitk_kernel<FMT, OUT>, ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, C,
-                               status) != cudaSuccess)
-            return LOWBIT_ERR_CUDA;
-        return launch_status();
+        return launch_pdl(gemm_splitk_kernel<FMT, OUT>, dim3(static_cast<unsigned>(tiles * C)), dim3(kThreads), smem,
+                          st, static_cast<unsigned>(C), ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, C, status);
     }
     const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
-    gemm_kernel<FMT, OUT><<<grid, kThreads, smem, st>>>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, status);
-    return launch_status();
+    return launch_pdl(gemm_kernel<FMT, OUT>, dim3(grid), dim3(kThreads), smem, st, 0, ma, mp, s_x, s_w, M, N, K, y,
+                      ldy, vec_ok, status);
 }
 
 template <int FMT>

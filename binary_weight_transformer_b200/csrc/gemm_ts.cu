@@ -240,6 +240,10 @@ gemm_ts_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // Global memory is touched only after the previous kernel on the stream
+    // has completed (programmatic dependent launch, see pdl_wait).
+    pdl_wait();
+    pdl_trigger();
     const uint32_t a_col0 = 2 * kDCols;          // first A stage column
 
     const int64_t num_w = (N + BW - 1) / BW;
@@ -397,8 +401,8 @@ lowbit_status launch_t(const CUtensorMap &mq, const CUtensorMap &mp, const float
     const int64_t tiles = ((N + BW - 1) / BW) * ((M + nt - 1) / nt);
     const int64_t sms = device_sm_count();
     const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
-    gemm_ts_kernel<FMT, OUT><<<grid, kThreads, smem, st>>>(mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt, status);
-    return launch_status();
+    return launch_pdl(gemm_ts_kernel<FMT, OUT>, dim3(grid), dim3(kThreads), smem, st, 0, mq, mp, s_x, s_w, M, N, K,
+                      y, ldy, vec_ok, nt, status);
 }
 
 template <int FMT>
@@ -533,6 +537,10 @@ gemm_ts_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
     cluster_sync_all();  // both CTAs' barriers exist before any remote arrive
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // Global memory is touched only after the previous kernel on the stream
+    // has completed (programmatic dependent launch, see pdl_wait).
+    pdl_wait();
+    pdl_trigger();
     const uint32_t a_col0 = 2 * kDCols;
 
     const int64_t num_w = (N + 2 * BW - 1) / (2 * BW);  // 256-row weight tiles
@@ -701,11 +709,8 @@ lowbit_status launch_pair_t(const CUtensorMap &mq, const CUtensorMap &mp, const 
     }
     const int64_t tiles = ((N + 2 * BW - 1) / (2 * BW)) * ((M + nt - 1) / nt);
     const int64_t pairs = tiles < max_pairs[dev] ? tiles : max_pairs[dev];
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-    if (cudaLaunchKernelEx(&cfg, gemm_ts_pair_kernel<FMT, OUT>, mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt,
-                           status) != cudaSuccess)
-        return LOWBIT_ERR_CUDA;
-    return launch_status();
+    return launch_pdl(gemm_ts_pair_kernel<FMT, OUT>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kThreads), smem,
+                      st, 0, mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt, status);
 }
 
 template <int FMT>

@@ -115,6 +115,8 @@ gemv_kernel(const int8_t *__restrict__ q, int64_t ldq, const float *__restrict__
     constexpr int kCodesPerChunk = 4 * F::kCodesPerWord;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    pdl_wait();
+    pdl_trigger();
     for (int64_t row0 = (static_cast<int64_t>(blockIdx.x) * kWarps + warp) * R; row0 < N;
          row0 += static_cast<int64_t>(gridDim.x) * kWarps * R) {
         int32_t acc[R][MT];
@@ -217,6 +219,8 @@ gemv_smem_kernel(const int8_t *__restrict__ q, int64_t ldq, const float *__restr
     const int lane = threadIdx.x & 31;
     const int64_t row0 = (static_cast<int64_t>(blockIdx.x) * kWarps + warp) * R;
     const int64_t qpieces = nchunks * QP;
+    pdl_wait();
+    pdl_trigger();
 
     int32_t acc[R][MT];
 #pragma unroll
@@ -296,12 +300,14 @@ lowbit_status launch_smem(const int8_t *q, int64_t ldq, const float *s_x, int M,
     const int64_t blocks = (N + kWarps * R - 1) / (kWarps * R);
     const dim3 g(static_cast<unsigned>(blocks)), b(kWarps * 32);
     if (ydt == LOWBIT_F32)
-        gemv_smem_kernel<FMT, MT, U, R, LOWBIT_F32><<<g, b, smem, st>>>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ldy);
+        return launch_pdl(gemv_smem_kernel<FMT, MT, U, R, LOWBIT_F32>, g, b, smem, st, 0, q, ldq, s_x, M, K, packed, ldp,
+                          nchunks, s_w, N, y, ldy);
     else if (ydt == LOWBIT_BF16)
-        gemv_smem_kernel<FMT, MT, U, R, LOWBIT_BF16><<<g, b, smem, st>>>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ldy);
+        return launch_pdl(gemv_smem_kernel<FMT, MT, U, R, LOWBIT_BF16>, g, b, smem, st, 0, q, ldq, s_x, M, K, packed, ldp,
+                          nchunks, s_w, N, y, ldy);
     else
-        gemv_smem_kernel<FMT, MT, U, R, LOWBIT_I32><<<g, b, smem, st>>>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ldy);
-    return launch_status();
+        return launch_pdl(gemv_smem_kernel<FMT, MT, U, R, LOWBIT_I32>, g, b, smem, st, 0, q, ldq, s_x, M, K, packed, ldp,
+                          nchunks, s_w, N, y, ldy);
 }
 
 // Long rows whose activations do not fit the shared-memory staging: the
@@ -316,12 +322,14 @@ lowbit_status launch_global(const int8_t *q, int64_t ldq, const float *s_x, int 
     if (blocks > cap) blocks = cap;
     const dim3 grid(static_cast<unsigned>(blocks)), block(kWarps * 32);
     if (ydt == LOWBIT_F32)
-        gemv_kernel<FMT, MT, 8, 1, LOWBIT_F32><<<grid, block, 0, st>>>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ldy);
+        return launch_pdl(gemv_kernel<FMT, MT, 8, 1, LOWBIT_F32>, grid, block, 0, st, 0, q, ldq, s_x, M, K, packed, ldp,
+                          nchunks, s_w, N, y, ldy);
     else if (ydt == LOWBIT_BF16)
-        gemv_kernel<FMT, MT, 8, 1, LOWBIT_BF16><<<grid, block, 0, st>>>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ldy);
+        return launch_pdl(gemv_kernel<FMT, MT, 8, 1, LOWBIT_BF16>, grid, block, 0, st, 0, q, ldq, s_x, M, K, packed, ldp,
+                          nchunks, s_w, N, y, ldy);
     else
-        gemv_kernel<FMT, MT, 8, 1, LOWBIT_I32><<<grid, block, 0, st>>>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ldy);
-    return launch_status();
+        return launch_pdl(gemv_kernel<FMT, MT, 8, 1, LOWBIT_I32>, grid, block, 0, st, 0, q, ldq, s_x, M, K, packed, ldp,
+                          nchunks, s_w, N, y, ldy);
 }
 
 // One launch for up to 4 tokens.  U (16-byte chunks per lane in flight) comes

@@ -11,6 +11,7 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -89,12 +90,52 @@ __device__ __forceinline__ float rescale(int32_t acc, float sw, float sx)
     return __fmul_rn(__int2float_rn(acc), __fmul_rn(sw, sx));
 }
 
+// Programmatic dependent launch.  The hot-path kernels are launched with
+// programmatic stream serialization, so a kernel may start while the one
+// before it on the stream is still running.  pdl_wait() blocks until that
+// kernel has completed and its memory operations are visible; every kernel
+// calls it before its first global-memory access (activations, weights,
+// outputs, status word), so the order of memory effects is exactly the
+// stream order and only the launch and the prologue (barrier set-up, tensor
+// memory allocation) overlap the previous kernel.  pdl_trigger() allows the
+// next kernel to be launched.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 }  // namespace lowbit
 
 // Host-side launch helpers (defined in abi.cu and pack.cu).
 namespace lowbit {
 lowbit_status launch_status();
 int device_sm_count();
+
+// Launch with programmatic stream serialization (see pdl_wait); cluster_x > 0
+// also sets the cluster size for kernels without compiled-in cluster dims.
+template <typename... KArgs, typename... Args>
+inline lowbit_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                unsigned cluster_x, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    unsigned n = 1;
+    if (cluster_x > 0) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = cluster_x;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        n = 2;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    return launch_status();
+}
 lowbit_status pack_launch(const float *w, int64_t N, int64_t K, int64_t ldw, lowbit_format f, float eps,
                           uint8_t *packed, int64_t ldp, float *s_w, void *workspace, int32_t *status,
                           cudaStream_t st);
