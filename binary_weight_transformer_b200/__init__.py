@@ -21,6 +21,7 @@ import os
 
 TERNARY2, BINARY1, INT4 = 0, 1, 2
 F32, BF16, I32 = 0, 1, 2
+WEIGHTS_STABLE = 1  # LOWBIT_LINEAR_WEIGHTS_STABLE
 
 STATUS_NAMES = {
     0: "LOWBIT_OK", 1: "LOWBIT_ERR_INVALID_ARG", 2: "LOWBIT_ERR_ALIGNMENT", 3: "LOWBIT_ERR_UNSUPPORTED",
@@ -47,6 +48,8 @@ ABI = {
     "lowbit_linear": (_I32, [_P, _I64, _P, _I64, _I64, _P, _I64, _P, _I32, _I64, _P, _I32, _I64, _P, _P]),
     "lowbit_linear_path": (_I32, [_P, _I64, _P, _I64, _I64, _P, _I64, _P, _I32, _I64, _P, _I32, _I64, _I32,
                                   _P, _P]),
+    "lowbit_linear_ex": (_I32, [_P, _I64, _P, _I64, _I64, _P, _I64, _P, _I32, _I64, _P, _I32, _I64, _I32,
+                                ctypes.c_uint, _P, _P]),
     "lowbit_status_string": (ctypes.c_char_p, [_I32]),
     "lowbit_version": (_I32, []),
 }
@@ -180,12 +183,15 @@ def lowbit_act_quant(x, eps: float = 0.0, q=None, s_x=None, status=None, stream=
 
 
 def lowbit_linear(q, s_x, packed, s_w, fmt: int, N: int, out_dtype: int = F32, K: int | None = None,
-                  y=None, status=None, stream=None, path: int = 0):
+                  y=None, status=None, stream=None, path: int = 0, weights_stable: bool = False):
     """y[M, N] from int8 codes q[M, >=K] and a packed artifact (see lowbit.h).
 
     ``path`` 0 picks the kernel by M; 1 forces the GEMV, 2 the tensor-core GEMM
     with the expanded tile in shared memory, 3 the one with it in tensor memory,
-    4 the tensor-memory one on SM pairs (256 weight rows per MMA)."""
+    4 the tensor-memory one on SM pairs (256 weight rows per MMA).
+    ``weights_stable`` passes LOWBIT_LINEAR_WEIGHTS_STABLE: the kernel that
+    precedes this call on the stream does not write ``packed`` or ``s_w``, so
+    weight reads may start before it finishes."""
     import torch
     M = q.shape[0]
     if K is None:
@@ -193,8 +199,8 @@ def lowbit_linear(q, s_x, packed, s_w, fmt: int, N: int, out_dtype: int = F32, K
     if y is None:
         dt = {F32: torch.float32, BF16: torch.bfloat16, I32: torch.int32}[out_dtype]
         y = torch.empty((M, N), dtype=dt, device=q.device)
-    st = lib().lowbit_linear_path(_ptr(q), q.stride(0), _ptr(s_x), M, K, _ptr(packed), packed.stride(0),
-                                  _ptr(s_w), fmt, N, _ptr(y), out_dtype, y.stride(0), path, _ptr(status),
-                                  _stream(stream))
+    st = lib().lowbit_linear_ex(_ptr(q), q.stride(0), _ptr(s_x), M, K, _ptr(packed), packed.stride(0),
+                                _ptr(s_w), fmt, N, _ptr(y), out_dtype, y.stride(0), path,
+                                WEIGHTS_STABLE if weights_stable else 0, _ptr(status), _stream(stream))
     _check(st, "lowbit_linear")
     return y

@@ -18,16 +18,17 @@ lowbit_status unpack_launch(const uint8_t *packed, int64_t ldp, int64_t N, int64
                             int8_t *codes, int64_t ldc, int32_t *status, cudaStream_t st);
 lowbit_status gemv_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
                           const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
-                          lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, cudaStream_t st);
+                          lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int prefetch,
+                          cudaStream_t st);
 lowbit_status gemm_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
                           const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
-                          lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int32_t *status,
-                          cudaStream_t st);
+                          lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int prefetch,
+                          int32_t *status, cudaStream_t st);
 
 lowbit_status gemm_ts_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
                              const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
-                             lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int32_t *status,
-                             cudaStream_t st);
+                             lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int prefetch,
+                             int32_t *status, cudaStream_t st);
 
 lowbit_status gemm_ts_pair_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
                                   const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
@@ -182,11 +183,13 @@ lowbit_status lowbit_act_quant(const void *x, lowbit_dtype xdt, int64_t M, int64
     return act_quant_launch(x, xdt, M, K, ldx, eps, q, ldq, s_x, status_dev, static_cast<cudaStream_t>(stream));
 }
 
-lowbit_status lowbit_linear_path(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
-                                 const uint8_t *packed, int64_t ldp, const float *s_w, lowbit_format f, int64_t N,
-                                 void *y, lowbit_dtype ydt, int64_t ldy, int path, int32_t *status_dev,
-                                 void *stream)
+lowbit_status lowbit_linear_ex(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
+                               const uint8_t *packed, int64_t ldp, const float *s_w, lowbit_format f, int64_t N,
+                               void *y, lowbit_dtype ydt, int64_t ldy, int path, unsigned flags,
+                               int32_t *status_dev, void *stream)
 {
+    if ((flags & ~static_cast<unsigned>(LOWBIT_LINEAR_WEIGHTS_STABLE)) != 0) return LOWBIT_ERR_INVALID_ARG;
+    const int prefetch = (flags & LOWBIT_LINEAR_WEIGHTS_STABLE) != 0 ? 1 : 0;
     if (!valid_format(f) || q == nullptr || s_x == nullptr || packed == nullptr || s_w == nullptr || y == nullptr)
         return LOWBIT_ERR_INVALID_ARG;
     if (ydt != LOWBIT_F32 && ydt != LOWBIT_BF16 && ydt != LOWBIT_I32) return LOWBIT_ERR_INVALID_ARG;
@@ -206,15 +209,23 @@ lowbit_status lowbit_linear_path(const int8_t *q, int64_t ldq, const float *s_x,
     // Up to 4 tokens the dp4a GEMV streams weights fastest; from 5 on its
     // int8 MACs outgrow the CUDA cores and the tensor-core GEMM wins.
     const bool use_gemv = path == 1 || (path == 0 && M <= 4);
-    if (use_gemv) return gemv_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, st);
+    if (use_gemv) return gemv_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, st);
     // From 512 tokens the tensor-memory variant (weights as the MMA's A
     // operand in TMEM) is as fast or faster; below it the shared-memory
     // variant, which splits K over a cluster when tiles are few, wins.
     if (path == 4)
         return gemm_ts_pair_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, status_dev, st);
     if (path == 3 || (path == 0 && M >= 512))
-        return gemm_ts_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, status_dev, st);
-    return gemm_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, status_dev, st);
+        return gemm_ts_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
+    return gemm_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
+}
+
+lowbit_status lowbit_linear_path(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
+                                 const uint8_t *packed, int64_t ldp, const float *s_w, lowbit_format f, int64_t N,
+                                 void *y, lowbit_dtype ydt, int64_t ldy, int path, int32_t *status_dev,
+                                 void *stream)
+{
+    return lowbit_linear_ex(q, ldq, s_x, M, K, packed, ldp, s_w, f, N, y, ydt, ldy, path, 0u, status_dev, stream);
 }
 
 lowbit_status lowbit_linear(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,

@@ -189,7 +189,7 @@ template <int FMT, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_p,
             const float *__restrict__ s_x, const float *__restrict__ s_w, int64_t M, int64_t N, int64_t K,
-            void *__restrict__ y, int64_t ldy, int vec_ok, int32_t *status)
+            void *__restrict__ y, int64_t ldy, int vec_ok, int prefetch, int32_t *status)
 {
     constexpr int ST = tma_stages<FMT>();
     constexpr int SE = kExpStages;
@@ -246,8 +246,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     // Global memory is touched only after the previous kernel on the stream
-    // has completed (programmatic dependent launch, see pdl_wait).
-    pdl_wait();
+    // has completed (programmatic dependent launch, see pdl_wait).  With
+    // prefetch the TMA thread first starts the packed-weight half of its
+    // first stages (the caller vouches that the previous kernel does not
+    // write the weights) and waits after that.
+    if (prefetch == 0 || threadIdx.x != 0) pdl_wait();
     pdl_trigger();
 
     const int64_t num_m = (M + BM - 1) / BM;
@@ -260,12 +263,28 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
         if (lane == 0) {
             uint32_t g = 0;  // global k-block counter
             bool ok = true;
+            uint32_t npre = 0;  // stages whose weight half was started before the wait
+            if (prefetch != 0) {
+                if (blockIdx.x < num_tiles) {
+                    const int n0 = static_cast<int>((blockIdx.x / num_m) * BN);
+                    npre = static_cast<uint32_t>(nkb < ST ? nkb : ST);
+                    for (uint32_t i = 0; i < npre; ++i) {
+                        mbar_arrive_expect_tx(&full_tma[i], A_BYTES + P_BYTES);
+                        tma_load_2d(sP + i * P_BYTES, &map_p, &full_tma[i], static_cast<int>(i) * PB, n0);
+                    }
+                }
+                pdl_wait();
+            }
             for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 const int m0 = static_cast<int>((tile % num_m) * BM);
                 const int n0 = static_cast<int>((tile / num_m) * BN);
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
                     const int s = g % ST;
                     const uint32_t ph = (g / ST) & 1u;
+                    if (g < npre) {
+                        tma_load_2d(sA + s * A_BYTES, &map_a, &full_tma[s], kb * BK, m0);
+                        continue;
+                    }
                     if (!wait_bar(&empty_tma[s], ph ^ 1u, abort_flag, status)) { ok = false; break; }
                     mbar_arrive_expect_tx(&full_tma[s], A_BYTES + P_BYTES);
                     tma_load_2d(sA + s * A_BYTES, &map_a, &full_tma[s], kb * BK, m0);
@@ -397,7 +416,7 @@ template <int FMT, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_p,
                    const float *__restrict__ s_x, const float *__restrict__ s_w, int64_t M, int64_t N, int64_t K,
-                   void *__restrict__ y, int64_t ldy, int vec_ok, int C, int32_t *status)
+                   void *__restrict__ y, int64_t ldy, int vec_ok, int C, int prefetch, int32_t *status)
 {
     constexpr int ST = tma_stages<FMT>();
     constexpr int SE = kExpStages;
@@ -451,8 +470,11 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     // Global memory is touched only after the previous kernel on the stream
-    // has completed (programmatic dependent launch, see pdl_wait).
-    pdl_wait();
+    // has completed (programmatic dependent launch, see pdl_wait).  With
+    // prefetch the TMA thread first starts the packed-weight half of its
+    // first stages (the caller vouches that the previous kernel does not
+    // write the weights) and waits after that.
+    if (prefetch == 0 || threadIdx.x != 0) pdl_wait();
     pdl_trigger();
 
     const int64_t num_m = (M + BM - 1) / BM;
@@ -467,8 +489,22 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
         if (lane == 0) {
             uint32_t g = 0;
             bool ok = true;
+            uint32_t npre = 0;  // stages whose weight half was started before the wait
+            if (prefetch != 0) {
+                const int nloc = kb_end - kb_begin;
+                npre = static_cast<uint32_t>(nloc < ST ? nloc : ST);
+                for (uint32_t i = 0; i < npre; ++i) {
+                    mbar_arrive_expect_tx(&full_tma[i], A_BYTES + P_BYTES);
+                    tma_load_2d(sP + i * P_BYTES, &map_p, &full_tma[i], (kb_begin + static_cast<int>(i)) * PB, n0);
+                }
+                pdl_wait();
+            }
             for (int kb = kb_begin; kb < kb_end; ++kb, ++g) {
                 const int s = g % ST;
+                if (g < npre) {
+                    tma_load_2d(sA + s * A_BYTES, &map_a, &full_tma[s], kb * BK, m0);
+                    continue;
+                }
                 if (!wait_bar(&empty_tma[s], ((g / ST) & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
                 mbar_arrive_expect_tx(&full_tma[s], A_BYTES + P_BYTES);
                 tma_load_2d(sA + s * A_BYTES, &map_a, &full_tma[s], kb * BK, m0);
@@ -602,8 +638,8 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
 // ---------------------------------------------------------------------------
 template <int FMT, int OUT>
 lowbit_status launch_t(const CUtensorMap &ma, const CUtensorMap &mp, const float *s_x, const float *s_w,
-                       int64_t M, int64_t N, int64_t K, void *y, int64_t ldy, int vec_ok, int32_t *status,
-                       cudaStream_t st)
+                       int64_t M, int64_t N, int64_t K, void *y, int64_t ldy, int vec_ok, int prefetch,
+                       int32_t *status, cudaStream_t st)
 {
     constexpr size_t smem = smem_bytes<FMT, OUT>();
     static_assert(smem <= 232448, "shared memory budget");
@@ -634,29 +670,32 @@ lowbit_status launch_t(const CUtensorMap &ma, const CUtensorMap &mp, const float
             configured_split[dev] = true;
         }
         return launch_pdl(gemm_splitk_kernel<FMT, OUT>, dim3(static_cast<unsigned>(tiles * C)), dim3(kThreads), smem,
-                          st, static_cast<unsigned>(C), ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, C, status);
+                          st, static_cast<unsigned>(C), ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, C, prefetch,
+                          status);
     }
     const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
     return launch_pdl(gemm_kernel<FMT, OUT>, dim3(grid), dim3(kThreads), smem, st, 0, ma, mp, s_x, s_w, M, N, K, y,
-                      ldy, vec_ok, status);
+                      ldy, vec_ok, prefetch, status);
 }
 
 template <int FMT>
 lowbit_status launch_fmt(const CUtensorMap &ma, const CUtensorMap &mp, const float *s_x, const float *s_w,
                          int64_t M, int64_t N, int64_t K, void *y, lowbit_dtype ydt, int64_t ldy, int vec_ok,
-                         int32_t *status, cudaStream_t st)
+                         int prefetch, int32_t *status, cudaStream_t st)
 {
-    if (ydt == LOWBIT_F32) return launch_t<FMT, LOWBIT_F32>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, status, st);
-    if (ydt == LOWBIT_BF16) return launch_t<FMT, LOWBIT_BF16>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, status, st);
-    return launch_t<FMT, LOWBIT_I32>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, status, st);
+    if (ydt == LOWBIT_F32)
+        return launch_t<FMT, LOWBIT_F32>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, st);
+    if (ydt == LOWBIT_BF16)
+        return launch_t<FMT, LOWBIT_BF16>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, st);
+    return launch_t<FMT, LOWBIT_I32>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, st);
 }
 
 }  // namespace tc
 
 lowbit_status gemm_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
                           const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
-                          lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int32_t *status,
-                          cudaStream_t st)
+                          lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int prefetch,
+                          int32_t *status, cudaStream_t st)
 {
     using namespace tc;
     CUtensorMap ma, mp;
@@ -671,9 +710,9 @@ lowbit_status gemm_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_
         return LOWBIT_ERR_CUDA;
     const int64_t esz = ydt == LOWBIT_BF16 ? 2 : 4;
     const int vec_ok = ((reinterpret_cast<uintptr_t>(y) & 15u) == 0 && (ldy * esz) % 16 == 0) ? 1 : 0;
-    if (f == LOWBIT_TERNARY2) return launch_fmt<kT2>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, status, st);
-    if (f == LOWBIT_BINARY1) return launch_fmt<kB1>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, status, st);
-    return launch_fmt<kI4>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, status, st);
+    if (f == LOWBIT_TERNARY2) return launch_fmt<kT2>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, st);
+    if (f == LOWBIT_BINARY1) return launch_fmt<kB1>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, st);
+    return launch_fmt<kI4>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, st);
 }
 
 }  // namespace lowbit

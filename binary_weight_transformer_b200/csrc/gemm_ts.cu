@@ -185,7 +185,7 @@ template <int FMT, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_ts_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_p,
                const float *__restrict__ s_x, const float *__restrict__ s_w, int64_t M, int64_t N, int64_t K,
-               void *__restrict__ y, int64_t ldy, int vec_ok, int nt, int32_t *status)
+               void *__restrict__ y, int64_t ldy, int vec_ok, int nt, int prefetch, int32_t *status)
 {
     constexpr int PB = packed_row_kblock<FMT>();
     constexpr int P_BYTES = p_bytes<FMT>();
@@ -241,8 +241,11 @@ gemm_ts_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     // Global memory is touched only after the previous kernel on the stream
-    // has completed (programmatic dependent launch, see pdl_wait).
-    pdl_wait();
+    // has completed (programmatic dependent launch, see pdl_wait).  With
+    // prefetch the TMA thread first starts the packed-weight half of its
+    // first stages (the caller vouches that the previous kernel does not
+    // write the weights) and waits after that.
+    if (prefetch == 0 || threadIdx.x != 0) pdl_wait();
     pdl_trigger();
     const uint32_t a_col0 = 2 * kDCols;          // first A stage column
 
@@ -257,11 +260,27 @@ gemm_ts_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         if (lane == 0) {
             uint32_t g = 0;
             bool ok = true;
+            uint32_t npre = 0;  // stages whose weight half was started before the wait
+            if (prefetch != 0) {
+                if (blockIdx.x < num_tiles) {
+                    const int w0 = static_cast<int>((blockIdx.x % num_w) * BW);
+                    npre = static_cast<uint32_t>(nkb < kStages ? nkb : kStages);
+                    for (uint32_t i = 0; i < npre; ++i) {
+                        mbar_arrive_expect_tx(&full_tma[i], q_bytes + P_BYTES);
+                        tma_load_2d(sP + i * P_BYTES, &map_p, &full_tma[i], static_cast<int>(i) * PB, w0);
+                    }
+                }
+                pdl_wait();
+            }
             for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 const int w0 = static_cast<int>((tile % num_w) * BW);
                 const int t0 = static_cast<int>((tile / num_w) * nt);
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
                     const int s = g % kStages;
+                    if (g < npre) {
+                        tma_load_2d(sQ + s * Q_BYTES, &map_q, &full_tma[s], kb * BK, t0);
+                        continue;
+                    }
                     if (!wait_bar(&mma_done[s], ((g / kStages) & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
                     mbar_arrive_expect_tx(&full_tma[s], q_bytes + P_BYTES);
                     tma_load_2d(sQ + s * Q_BYTES, &map_q, &full_tma[s], kb * BK, t0);
@@ -384,7 +403,7 @@ gemm_ts_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
 
 template <int FMT, int OUT>
 lowbit_status launch_t(const CUtensorMap &mq, const CUtensorMap &mp, const float *s_x, const float *s_w, int64_t M,
-                       int64_t N, int64_t K, void *y, int64_t ldy, int vec_ok, int nt, int32_t *status,
+                       int64_t N, int64_t K, void *y, int64_t ldy, int vec_ok, int nt, int prefetch, int32_t *status,
                        cudaStream_t st)
 {
     constexpr size_t smem = smem_bytes<FMT, OUT>();
@@ -402,17 +421,19 @@ lowbit_status launch_t(const CUtensorMap &mq, const CUtensorMap &mp, const float
     const int64_t sms = device_sm_count();
     const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
     return launch_pdl(gemm_ts_kernel<FMT, OUT>, dim3(grid), dim3(kThreads), smem, st, 0, mq, mp, s_x, s_w, M, N, K,
-                      y, ldy, vec_ok, nt, status);
+                      y, ldy, vec_ok, nt, prefetch, status);
 }
 
 template <int FMT>
 lowbit_status launch_fmt(const CUtensorMap &mq, const CUtensorMap &mp, const float *s_x, const float *s_w,
                          int64_t M, int64_t N, int64_t K, void *y, lowbit_dtype ydt, int64_t ldy, int vec_ok,
-                         int nt, int32_t *status, cudaStream_t st)
+                         int nt, int prefetch, int32_t *status, cudaStream_t st)
 {
-    if (ydt == LOWBIT_F32) return launch_t<FMT, LOWBIT_F32>(mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt, status, st);
-    if (ydt == LOWBIT_BF16) return launch_t<FMT, LOWBIT_BF16>(mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt, status, st);
-    return launch_t<FMT, LOWBIT_I32>(mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt, status, st);
+    if (ydt == LOWBIT_F32)
+        return launch_t<FMT, LOWBIT_F32>(mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt, prefetch, status, st);
+    if (ydt == LOWBIT_BF16)
+        return launch_t<FMT, LOWBIT_BF16>(mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt, prefetch, status, st);
+    return launch_t<FMT, LOWBIT_I32>(mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt, prefetch, status, st);
 }
 
 
@@ -730,8 +751,8 @@ lowbit_status launch_pair_fmt(const CUtensorMap &mq, const CUtensorMap &mp, cons
 // Token tile: 224 for many tokens, else M rounded up to a multiple of 32.
 lowbit_status gemm_ts_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
                              const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
-                             lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int32_t *status,
-                             cudaStream_t st)
+                             lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int prefetch,
+                             int32_t *status, cudaStream_t st)
 {
     using namespace ts;
     const int nt = M >= BT ? BT : static_cast<int>((M + 31) / 32 * 32);
@@ -747,9 +768,9 @@ lowbit_status gemm_ts_launch(const int8_t *q, int64_t ldq, const float *s_x, int
         return LOWBIT_ERR_CUDA;
     const int64_t esz = ydt == LOWBIT_BF16 ? 2 : 4;
     const int vec_ok = ((reinterpret_cast<uintptr_t>(y) & 15u) == 0 && (ldy * esz) % 16 == 0) ? 1 : 0;
-    if (f == LOWBIT_TERNARY2) return launch_fmt<kT2>(mq, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, nt, status, st);
-    if (f == LOWBIT_BINARY1) return launch_fmt<kB1>(mq, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, nt, status, st);
-    return launch_fmt<kI4>(mq, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, nt, status, st);
+    if (f == LOWBIT_TERNARY2) return launch_fmt<kT2>(mq, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, nt, prefetch, status, st);
+    if (f == LOWBIT_BINARY1) return launch_fmt<kB1>(mq, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, nt, prefetch, status, st);
+    return launch_fmt<kI4>(mq, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, nt, prefetch, status, st);
 }
 
 }  // namespace lowbit

@@ -109,13 +109,16 @@ template <int FMT, int MT, int U, int R, int OUT>
 __global__ void __launch_bounds__(kWarps * 32)
 gemv_kernel(const int8_t *__restrict__ q, int64_t ldq, const float *__restrict__ s_x, int M, int64_t K,
             const uint8_t *__restrict__ packed, int64_t ldp, int64_t nchunks, const float *__restrict__ s_w,
-            int64_t N, void *__restrict__ y, int64_t ldy)
+            int64_t N, void *__restrict__ y, int64_t ldy, int prefetch)
 {
     using F = Fmt<FMT>;
     constexpr int kCodesPerChunk = 4 * F::kCodesPerWord;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    pdl_wait();
+    // With prefetch the first weight loads are issued before the wait for the
+    // previous kernel (the caller vouches that it does not write the weights).
+    bool waited = prefetch == 0;
+    if (waited) pdl_wait();
     pdl_trigger();
     for (int64_t row0 = (static_cast<int64_t>(blockIdx.x) * kWarps + warp) * R; row0 < N;
          row0 += static_cast<int64_t>(gridDim.x) * kWarps * R) {
@@ -134,6 +137,10 @@ gemv_kernel(const int8_t *__restrict__ q, int64_t ldq, const float *__restrict__
                     wv[r][u] = (c < nchunks && row0 + r < N) ? ld_stream_u4(packed + (row0 + r) * ldp + c * 16)
                                                              : make_uint4(0, 0, 0, 0);
                 }
+            if (!waited) {
+                pdl_wait();
+                waited = true;
+            }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int64_t c = c0 + lane + 32 * u;
@@ -210,7 +217,7 @@ template <int FMT, int MT, int U, int R, int OUT>
 __global__ void __launch_bounds__(kWarps * 32)
 gemv_smem_kernel(const int8_t *__restrict__ q, int64_t ldq, const float *__restrict__ s_x, int M, int64_t K,
                  const uint8_t *__restrict__ packed, int64_t ldp, int64_t nchunks, const float *__restrict__ s_w,
-                 int64_t N, void *__restrict__ y, int64_t ldy)
+                 int64_t N, void *__restrict__ y, int64_t ldy, int prefetch)
 {
     using F = Fmt<FMT>;
     constexpr int QP = QPieces<FMT>::value;
@@ -219,7 +226,9 @@ gemv_smem_kernel(const int8_t *__restrict__ q, int64_t ldq, const float *__restr
     const int lane = threadIdx.x & 31;
     const int64_t row0 = (static_cast<int64_t>(blockIdx.x) * kWarps + warp) * R;
     const int64_t qpieces = nchunks * QP;
-    pdl_wait();
+    // With prefetch the first weight loads are issued before the wait for the
+    // previous kernel (the caller vouches that it does not write the weights).
+    if (prefetch == 0) pdl_wait();
     pdl_trigger();
 
     int32_t acc[R][MT];
@@ -239,6 +248,7 @@ gemv_smem_kernel(const int8_t *__restrict__ q, int64_t ldq, const float *__restr
                                                          : make_uint4(0, 0, 0, 0);
             }
         if (c0 == 0) {
+            if (prefetch != 0) pdl_wait();
             for (int64_t i = threadIdx.x; i < M * qpieces; i += blockDim.x) {
                 const int64_t t = i / qpieces, j = i % qpieces;   // j = chunk * QP + piece
                 qs[t * qpieces + (j % QP) * nchunks + j / QP] = load_q16(q + t * ldq, j * 16, K);
@@ -281,7 +291,7 @@ constexpr int64_t kGemvSmemMax = 96 * 1024;
 template <int FMT, int MT, int U, int R>
 lowbit_status launch_smem(const int8_t *q, int64_t ldq, const float *s_x, int M, int64_t K, const uint8_t *packed,
                           int64_t ldp, int64_t nchunks, const float *s_w, int64_t N, void *y, lowbit_dtype ydt,
-                          int64_t ldy, size_t smem, cudaStream_t st)
+                          int64_t ldy, size_t smem, int prefetch, cudaStream_t st)
 {
     static bool configured[64] = {};
     int dev = 0;
@@ -301,13 +311,13 @@ lowbit_status launch_smem(const int8_t *q, int64_t ldq, const float *s_x, int M,
     const dim3 g(static_cast<unsigned>(blocks)), b(kWarps * 32);
     if (ydt == LOWBIT_F32)
         return launch_pdl(gemv_smem_kernel<FMT, MT, U, R, LOWBIT_F32>, g, b, smem, st, 0, q, ldq, s_x, M, K, packed, ldp,
-                          nchunks, s_w, N, y, ldy);
+                          nchunks, s_w, N, y, ldy, prefetch);
     else if (ydt == LOWBIT_BF16)
         return launch_pdl(gemv_smem_kernel<FMT, MT, U, R, LOWBIT_BF16>, g, b, smem, st, 0, q, ldq, s_x, M, K, packed, ldp,
-                          nchunks, s_w, N, y, ldy);
+                          nchunks, s_w, N, y, ldy, prefetch);
     else
         return launch_pdl(gemv_smem_kernel<FMT, MT, U, R, LOWBIT_I32>, g, b, smem, st, 0, q, ldq, s_x, M, K, packed, ldp,
-                          nchunks, s_w, N, y, ldy);
+                          nchunks, s_w, N, y, ldy, prefetch);
 }
 
 // Long rows whose activations do not fit the shared-memory staging: the
@@ -315,7 +325,7 @@ lowbit_status launch_smem(const int8_t *q, int64_t ldq, const float *s_x, int M,
 template <int FMT, int MT>
 lowbit_status launch_global(const int8_t *q, int64_t ldq, const float *s_x, int M, int64_t K,
                             const uint8_t *packed, int64_t ldp, int64_t nchunks, const float *s_w, int64_t N,
-                            void *y, lowbit_dtype ydt, int64_t ldy, cudaStream_t st)
+                            void *y, lowbit_dtype ydt, int64_t ldy, int prefetch, cudaStream_t st)
 {
     int64_t blocks = (N + kWarps - 1) / kWarps;
     const int64_t cap = static_cast<int64_t>(device_sm_count()) * 16;
@@ -323,13 +333,13 @@ lowbit_status launch_global(const int8_t *q, int64_t ldq, const float *s_x, int 
     const dim3 grid(static_cast<unsigned>(blocks)), block(kWarps * 32);
     if (ydt == LOWBIT_F32)
         return launch_pdl(gemv_kernel<FMT, MT, 8, 1, LOWBIT_F32>, grid, block, 0, st, 0, q, ldq, s_x, M, K, packed, ldp,
-                          nchunks, s_w, N, y, ldy);
+                          nchunks, s_w, N, y, ldy, prefetch);
     else if (ydt == LOWBIT_BF16)
         return launch_pdl(gemv_kernel<FMT, MT, 8, 1, LOWBIT_BF16>, grid, block, 0, st, 0, q, ldq, s_x, M, K, packed, ldp,
-                          nchunks, s_w, N, y, ldy);
+                          nchunks, s_w, N, y, ldy, prefetch);
     else
         return launch_pdl(gemv_kernel<FMT, MT, 8, 1, LOWBIT_I32>, grid, block, 0, st, 0, q, ldq, s_x, M, K, packed, ldp,
-                          nchunks, s_w, N, y, ldy);
+                          nchunks, s_w, N, y, ldy, prefetch);
 }
 
 // One launch for up to 4 tokens.  U (16-byte chunks per lane in flight) comes
@@ -338,33 +348,33 @@ lowbit_status launch_global(const int8_t *q, int64_t ldq, const float *s_x, int 
 template <int FMT, int MT>
 lowbit_status launch_tokens(const int8_t *q, int64_t ldq, const float *s_x, int M, int64_t K,
                             const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w, int64_t N,
-                            void *y, lowbit_dtype ydt, int64_t ldy, cudaStream_t st)
+                            void *y, lowbit_dtype ydt, int64_t ldy, int prefetch, cudaStream_t st)
 {
     const int64_t nchunks = (row_bytes + 15) / 16;
     const int64_t smem_i = static_cast<int64_t>(M) * nchunks * QPieces<FMT>::value * 16;
     if (smem_i > kGemvSmemMax)
-        return launch_global<FMT, MT>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ydt, ldy, st);
+        return launch_global<FMT, MT>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ydt, ldy, prefetch, st);
     const size_t smem = static_cast<size_t>(smem_i);
     const int64_t slots = static_cast<int64_t>(device_sm_count()) * 2 * kWarps;  // warps in one wave
     if (nchunks <= 64) {
         if constexpr (MT == 1) {
             if (N >= 4 * slots)
-                return launch_smem<FMT, MT, 2, 4>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ydt, ldy, smem, st);
+                return launch_smem<FMT, MT, 2, 4>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ydt, ldy, smem, prefetch, st);
         }
         if (N >= 2 * slots)
-            return launch_smem<FMT, MT, 2, 2>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ydt, ldy, smem, st);
-        return launch_smem<FMT, MT, 2, 1>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ydt, ldy, smem, st);
+            return launch_smem<FMT, MT, 2, 2>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ydt, ldy, smem, prefetch, st);
+        return launch_smem<FMT, MT, 2, 1>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ydt, ldy, smem, prefetch, st);
     }
     if (nchunks <= 160)
-        return launch_smem<FMT, MT, 5, 1>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ydt, ldy, smem, st);
-    return launch_smem<FMT, MT, 8, 1>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ydt, ldy, smem, st);
+        return launch_smem<FMT, MT, 5, 1>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ydt, ldy, smem, prefetch, st);
+    return launch_smem<FMT, MT, 8, 1>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ydt, ldy, smem, prefetch, st);
 }
 
 // Tokens are processed in groups of up to 4, one launch per group.
 template <int FMT>
 lowbit_status gemv_launch_fmt(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
                               const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w, int64_t N,
-                              void *y, lowbit_dtype ydt, int64_t ldy, cudaStream_t st)
+                              void *y, lowbit_dtype ydt, int64_t ldy, int prefetch, cudaStream_t st)
 {
     const int64_t esz = (ydt == LOWBIT_BF16) ? 2 : 4;
     for (int64_t t0 = 0; t0 < M; t0 += 4) {
@@ -373,8 +383,8 @@ lowbit_status gemv_launch_fmt(const int8_t *q, int64_t ldq, const float *s_x, in
         const float *sg = s_x + t0;
         void *yg = static_cast<char *>(y) + t0 * ldy * esz;
         const lowbit_status s = (m == 1)
-            ? launch_tokens<FMT, 1>(qg, ldq, sg, m, K, packed, ldp, row_bytes, s_w, N, yg, ydt, ldy, st)
-            : launch_tokens<FMT, 4>(qg, ldq, sg, m, K, packed, ldp, row_bytes, s_w, N, yg, ydt, ldy, st);
+            ? launch_tokens<FMT, 1>(qg, ldq, sg, m, K, packed, ldp, row_bytes, s_w, N, yg, ydt, ldy, prefetch, st)
+            : launch_tokens<FMT, 4>(qg, ldq, sg, m, K, packed, ldp, row_bytes, s_w, N, yg, ydt, ldy, prefetch, st);
         if (s != LOWBIT_OK) return s;
     }
     return LOWBIT_OK;

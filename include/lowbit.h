@@ -210,6 +210,30 @@ lowbit_status lowbit_linear_path(const int8_t *q, int64_t ldq, const float *s_x,
                                  void *y, lowbit_dtype ydt, int64_t ldy,
                                  int path, int32_t *status_dev, void *stream);
 
+/* Flag for lowbit_linear_ex: the caller guarantees that the packed artifact
+ * and s_w are not written by the kernel that immediately precedes this call
+ * on `stream` (nor concurrently by any other stream).  The library launches
+ * its kernels so that they may start while the preceding kernel is still
+ * running, and every kernel waits for that kernel to finish before touching
+ * activations, outputs or the status word.  With this flag the weight bytes,
+ * which do not depend on it, are requested before that wait, which hides the
+ * memory latency of the first weight tiles behind the previous kernel.  In
+ * a decode or prefill loop the preceding kernel is lowbit_act_quant or
+ * another linear layer, so the guarantee holds; directly after lowbit_pack of
+ * the same weights it does not. */
+#define LOWBIT_LINEAR_WEIGHTS_STABLE 1u
+
+/* lowbit_linear_path with launch flags (0 or LOWBIT_LINEAR_WEIGHTS_STABLE);
+ * other flag bits return LOWBIT_ERR_INVALID_ARG.  Results are identical for
+ * every flag value. */
+lowbit_status lowbit_linear_ex(const int8_t *q, int64_t ldq, const float *s_x,
+                               int64_t M, int64_t K,
+                               const uint8_t *packed, int64_t ldp, const float *s_w,
+                               lowbit_format f, int64_t N,
+                               void *y, lowbit_dtype ydt, int64_t ldy,
+                               int path, unsigned flags,
+                               int32_t *status_dev, void *stream);
+
 /* Human-readable name of a status value (static string). */
 const char *lowbit_status_string(lowbit_status s);
 

@@ -88,6 +88,16 @@ def test_linear_rejects_bad_arguments(lib):
                    ldp=bwt.packed_ld(bwt.INT4, k4)) == bwt.ERR_OVERFLOW_BOUND
 
 
+def test_linear_ex_rejects_unknown_flags(lib):
+    f = lib.lowbit_linear_ex
+    args = [FAKE, 256, FAKE, 4, 256, FAKE, 64, FAKE, bwt.TERNARY2, 8, FAKE, bwt.F32, 8, 0]
+    for flags in (2, 4, 0x80000000, 0xFFFFFFFF):
+        assert f(*args, flags, None, None) == bwt.ERR_INVALID_ARG
+    bad = list(args)
+    bad[0] = None                                   # q = NULL with a valid flag
+    assert f(*bad, bwt.WEIGHTS_STABLE, None, None) == bwt.ERR_INVALID_ARG
+
+
 def test_act_quant_rejects_bad_arguments(lib):
     f = lib.lowbit_act_quant
     assert f(None, bwt.F32, 4, 64, 64, 0.0, FAKE, 64, FAKE, None, None) == bwt.ERR_INVALID_ARG

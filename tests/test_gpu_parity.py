@@ -184,7 +184,7 @@ def test_unpack_roundtrip_and_reserved(fmt):
 # linear: both kernels, every format and output type
 # ---------------------------------------------------------------------------
 
-def run_case(fmt, M, N, K, path, out, seed, zero_w=False, x_bf16=False):
+def run_case(fmt, M, N, K, path, out, seed, zero_w=False, x_bf16=False, weights_stable=False):
     w = wls.normal_weights(seed, N, K)
     if zero_w:
         w[:] = 0.0
@@ -194,7 +194,8 @@ def run_case(fmt, M, N, K, path, out, seed, zero_w=False, x_bf16=False):
     packed, s_w = gpu_pack(w, fmt)
     q, s_x = gpu_act(x, x_bf16)
     st = status_word()
-    y = bwt.lowbit_linear(q, s_x, packed, s_w, fmt, N, out, K=K, status=st, path=path)
+    y = bwt.lowbit_linear(q, s_x, packed, s_w, fmt, N, out, K=K, status=st, path=path,
+                          weights_stable=weights_stable)
     torch.cuda.synchronize()
     assert st.item() == 0
     codes, s_wo = oracle.quantize(w, fmt, 1e-5)
@@ -239,6 +240,21 @@ def test_linear_bf16_within_one_ulp(path, fmt, M, N, K):
     got = bf16_bits(y)
     assert ulp_distance_bf16(got, ref).max() <= 1
     assert np.array_equal(got, ref)
+
+
+# LOWBIT_LINEAR_WEIGHTS_STABLE: weight reads start before the wait for the
+# preceding kernel (here the act quant that produced q, launched just before
+# on the same stream); the results must not change.  Shapes cover the GEMV
+# (one and several token groups), the cluster split-K GEMM, the persistent
+# GEMM, and the tensor-memory GEMM with more tiles than SMs.
+@pytest.mark.parametrize("path", [0, 1, 2, 3], ids=["auto", "gemv", "gemm", "gemm_ts"])
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
+@pytest.mark.parametrize("M,N,K", [(1, 2560, 768), (9, 300, 1000), (130, 1000, 2000), (600, 4000, 640)], ids=str)
+def test_linear_weights_stable_bit_exact(path, fmt, M, N, K):
+    if path == 1 and M > 16:
+        pytest.skip("GEMV path kept to decode sizes")
+    y, acc, _, _ = run_case(fmt, M, N, K, path, bwt.I32, 900 + M + N + K, weights_stable=True)
+    assert np.array_equal(y.cpu().numpy().astype(np.int64), acc)
 
 
 @pytest.mark.parametrize("path", [1, 2, 3, 4], ids=["gemv", "gemm", "gemm_ts", "gemm_ts_pair"])
