@@ -563,9 +563,12 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
     __syncwarp();
 
     // Every CTA of the cluster is done with its pipeline buffers: from here
-    // they hold the received partial tiles.
+    // they hold the received partial tiles, piece-major: 16-byte piece p
+    // (4 columns) of 32-column chunk cc of row r from source rank s sits at
+    // ((s * NC + cc) * 8 + p) * BM + r, so that the 32 lanes (rows) of one
+    // remote store instruction write 512 contiguous bytes.
     const int W = BN / C;                       // columns each CTA finishes
-    const int RB = 4 * W + 16;                  // receive row stride (padded)
+    const int NC = W / 32;                      // 32-column chunks per slice
     const uint32_t recv = smem_u32(sA);
     cluster_sync_all();
     const int quarter = warp & 3;
@@ -584,9 +587,12 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
                 }
                 if (row < M) {
                     const uint32_t dst = map_to_peer(
-                        recv + static_cast<uint32_t>((srank * BM + row_in_tile) * RB + cc * 128), static_cast<uint32_t>(j));
+                        recv + static_cast<uint32_t>(((static_cast<int>(srank) * NC + cc) * 8 * BM + row_in_tile) * 16),
+                        static_cast<uint32_t>(j));
 #pragma unroll
-                    for (int p = 0; p < 8; ++p) st_cluster128(dst + p * 16, v[4 * p], v[4 * p + 1], v[4 * p + 2], v[4 * p + 3]);
+                    for (int p = 0; p < 8; ++p)
+                        st_cluster128(dst + static_cast<uint32_t>(p * BM * 16), v[4 * p], v[4 * p + 1], v[4 * p + 2],
+                                      v[4 * p + 3]);
                 }
             }
         }
@@ -602,10 +608,10 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
             for (int i = 0; i < 32; ++i) v[i] = 0;
             if (row < M) {
                 for (int s = 0; s < C; ++s) {
-                    const uint32_t src = recv + static_cast<uint32_t>((s * BM + row_in_tile) * RB + cc * 128);
+                    const uint32_t src = recv + static_cast<uint32_t>(((s * NC + cc) * 8 * BM + row_in_tile) * 16);
 #pragma unroll
                     for (int p = 0; p < 8; ++p) {
-                        const uint4 a = lds128(src + p * 16);
+                        const uint4 a = lds128(src + static_cast<uint32_t>(p * BM * 16));
                         v[4 * p] += a.x;
                         v[4 * p + 1] += a.y;
                         v[4 * p + 2] += a.z;
