@@ -149,20 +149,32 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
-def dispatched_kernel(M):
-    """The kernel lowbit_linear picks for M tokens (same rule as the library):
-    the packed-weight GEMV up to 4 tokens, the tensor-core GEMM with the
-    weight tile expanded into shared memory (cluster split-K when output tiles
-    are few) below 512, the one with it in tensor memory from 512."""
+def dispatched_kernel(M, N, row_bytes):
+    """The kernel lowbit_linear picks (same rule as the library): the
+    packed-weight GEMV up to 4 tokens; warp-level MMAs up to 16 tokens when
+    rows are short or N is large; the tensor-core GEMM with the weight tile
+    expanded into shared memory (cluster split-K when output tiles are few)
+    below 512 tokens; the one with it in tensor memory from 512."""
     if M <= 4:
         return "gemv_smem_kernel"
+    if M <= 16 and (row_bytes <= 512 or N >= 3200):
+        return "skinny_mma_kernel/stream_mma_kernel"
     return "gemm_kernel/gemm_splitk_kernel" if M < 512 else "gemm_ts_kernel"
 
 
+def packed_row_bytes(fmt, K):
+    """Bytes of one packed weight row (lowbit_packed_row_bytes)."""
+    if fmt == wls.TERNARY2:
+        return 4 * ((K + 15) // 16)
+    if fmt == wls.BINARY1:
+        return (K + 7) // 8
+    return 4 * ((K + 7) // 8)
+
+
 class Point:
-    def __init__(self, mi, m, M):
+    def __init__(self, mi, m, M, fmt):
         self.mi, self.m, self.M = mi, m, M
-        self.kernel = dispatched_kernel(M)
+        self.kernel = dispatched_kernel(M, m.N, packed_row_bytes(fmt, m.K))
         # up to 16 tokens the packed weights dominate the bytes: HBM-bound
         self.bound = "hbm" if M <= 16 else "tensor"
         self.ops = 2 * M * m.N * m.K
@@ -173,7 +185,7 @@ def select_points(wl, only_M=None):
     for mi, m in enumerate(wl.matrices):
         for M in sorted(wl.Ms, reverse=True):
             if only_M is None or M in only_M:
-                points.append(Point(mi, m, M))
+                points.append(Point(mi, m, M, wl.fmt))
     return points
 
 

@@ -30,6 +30,11 @@ lowbit_status gemm_ts_launch(const int8_t *q, int64_t ldq, const float *s_x, int
                              lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int prefetch,
                              int32_t *status, cudaStream_t st);
 
+lowbit_status skinny_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
+                            const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
+                            lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int prefetch,
+                            int32_t *status, cudaStream_t st);
+
 lowbit_status gemm_ts_pair_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
                                   const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
                                   lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy,
@@ -193,8 +198,9 @@ lowbit_status lowbit_linear_ex(const int8_t *q, int64_t ldq, const float *s_x, i
     if (!valid_format(f) || q == nullptr || s_x == nullptr || packed == nullptr || s_w == nullptr || y == nullptr)
         return LOWBIT_ERR_INVALID_ARG;
     if (ydt != LOWBIT_F32 && ydt != LOWBIT_BF16 && ydt != LOWBIT_I32) return LOWBIT_ERR_INVALID_ARG;
-    if (path < 0 || path > 4) return LOWBIT_ERR_INVALID_ARG;
+    if (path < 0 || path > 5) return LOWBIT_ERR_INVALID_ARG;
     if (M <= 0 || N <= 0 || K <= 0 || ldq < K || ldy < N) return LOWBIT_ERR_INVALID_ARG;
+    if (path == 5 && M > 16) return LOWBIT_ERR_INVALID_ARG;
     if (M > INT32_MAX || N > INT32_MAX) return LOWBIT_ERR_INVALID_ARG;
     const int64_t rb = static_cast<int64_t>(lowbit_packed_row_bytes(f, K));
     if (ldp < rb) return LOWBIT_ERR_INVALID_ARG;
@@ -207,9 +213,16 @@ lowbit_status lowbit_linear_ex(const int8_t *q, int64_t ldq, const float *s_x, i
     if (d != LOWBIT_OK) return d;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // Up to 4 tokens the dp4a GEMV streams weights fastest; from 5 on its
-    // int8 MACs outgrow the CUDA cores and the tensor-core GEMM wins.
+    // int8 MACs outgrow the CUDA cores and tensor-core MMAs win.
     const bool use_gemv = path == 1 || (path == 0 && M <= 4);
     if (use_gemv) return gemv_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, st);
+    // 5 to 16 tokens: warp-level tensor-core MMAs on register fragments
+    // where they were measured faster than the split-K GEMM: rows of at most
+    // 512 packed bytes (one round of register loads), or at least 100 blocks
+    // of 32 output rows.  Longer rows with fewer blocks stay on the GEMM.
+    const bool skinny_wins = rb <= 512 || N >= 3200;
+    if (path == 5 || (path == 0 && M <= 16 && skinny_wins))
+        return skinny_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
     // From 512 tokens the tensor-memory variant (weights as the MMA's A
     // operand in TMEM) is as fast or faster; below it the shared-memory
     // variant, which splits K over a cluster when tiles are few, wins.

@@ -184,11 +184,13 @@ lowbit_status lowbit_act_quant(const void *x, lowbit_dtype xdt, int64_t M, int64
  * ldq and ldp multiples of 16), s_x fp32 [M], s_w fp32 [lowbit_scale_count].
  * Output y [M, ldy], ldy >= N, aligned to its element size.  Bytes of q past
  * K are ignored.  K <= lowbit_max_k(f), else LOWBIT_ERR_OVERFLOW_BOUND.
- * M <= 4 runs the packed-weight GEMV kernel; larger M runs a tcgen05
- * tensor-core GEMM (int8 MMA, accumulators in tensor memory): with the
- * expanded weight tile in shared memory and K split over a cluster when the
- * output tiles are few (5 <= M < 512), with the weight tile in tensor memory
- * from M = 512. */
+ * M <= 4 runs the packed-weight GEMV kernel (dp4a); 5 <= M <= 16 runs
+ * warp-level tensor-core MMAs (mma.sync, int8) on weight fragments expanded
+ * in registers when rows are short (<= 512 packed bytes) or N >= 3200;
+ * otherwise, and for 17 <= M < 512, a tcgen05 tensor-core GEMM (int8 MMA,
+ * accumulators in tensor memory) with the expanded weight tile in shared
+ * memory and K split over a cluster when the output tiles are few; from
+ * M = 512 the tcgen05 GEMM with the weight tile in tensor memory. */
 lowbit_status lowbit_linear(const int8_t *q, int64_t ldq, const float *s_x,
                             int64_t M, int64_t K,
                             const uint8_t *packed, int64_t ldp, const float *s_w,
@@ -200,8 +202,9 @@ lowbit_status lowbit_linear(const int8_t *q, int64_t ldq, const float *s_x,
  * lowbit_linear), 1 = packed-weight GEMV (any M), 2 = tensor-core GEMM with
  * the expanded weight tile in shared memory (any M), 3 = tensor-core GEMM
  * with the expanded weight tile in tensor memory (any M), 4 = the same on
- * pairs of SMs (one MMA covers 256 weight rows; any M).  Other values return
- * LOWBIT_ERR_INVALID_ARG.  Lets tests and benchmarks reach every kernel at
+ * pairs of SMs (one MMA covers 256 weight rows; any M), 5 = warp-level
+ * tensor-core MMAs on register fragments (M <= 16).  Other values, and path 5
+ * with M > 16, return LOWBIT_ERR_INVALID_ARG.  Lets tests and benchmarks reach every kernel at
  * every size. */
 lowbit_status lowbit_linear_path(const int8_t *q, int64_t ldq, const float *s_x,
                                  int64_t M, int64_t K,
