@@ -77,8 +77,11 @@ def gpu_act(x_np, bf16=False, eps=0.0):
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("bf16", [False, True], ids=["f32", "bf16"])
+# Shapes cover one thread group per row for every TPR, the scalar-load path
+# (unaligned rows), rows longer than the register path (65560), many rows of
+# 16-byte vectors, and a zero row in each.
 @pytest.mark.parametrize("M,K", [(1, 192), (7, 200), (3, 9728), (257, 2560), (5, 13), (64, 3),
-                                 (9, 65536 + 24)])
+                                 (9, 65536 + 24), (300, 9728), (1000, 192), (600, 12288), (256, 24)])
 @pytest.mark.parametrize("eps", [0.0, 1e-5])
 def test_act_quant_bit_exact(M, K, bf16, eps):
     x = wls.normal_activations(100 + M + K, M, K, 0.01, 8.0)
@@ -91,15 +94,19 @@ def test_act_quant_bit_exact(M, K, bf16, eps):
     assert np.array_equal(s_x.cpu().numpy().view(np.uint32), s_o.view(np.uint32))
 
 
-def test_act_quant_flags_nonfinite():
-    x = np.ones((4, 64), np.float32)
+@pytest.mark.parametrize("M", [4, 300], ids=["regs", "ring"])
+def test_act_quant_flags_nonfinite(M):
+    x = np.ones((M, 64), np.float32)
     x[2, 5] = np.nan
     x[3, 7] = 1e37  # x * 127 overflows fp32
     xt = torch.from_numpy(x).to(DEV)
     st = status_word()
-    bwt.lowbit_act_quant(xt, 0.0, status=st)
+    q, s_x = bwt.lowbit_act_quant(xt, 0.0, status=st)
     torch.cuda.synchronize()
     assert bwt.status_flags(st) == [bwt.ERR_NONFINITE]
+    if M > 4:  # the finite rows are unaffected
+        q_o, s_o = oracle.act_quant(x[4:], 0.0)
+        assert np.array_equal(q.cpu().numpy()[4:, :64], q_o)
 
 
 # ---------------------------------------------------------------------------
