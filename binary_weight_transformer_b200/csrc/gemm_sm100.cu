@@ -41,6 +41,9 @@ template <int FMT> __host__ __device__ constexpr int packed_bytes_per_kblock() {
 // stages, chosen to fit 227 KB of shared memory with the epilogue staging.
 template <int FMT> __host__ __device__ constexpr int tma_stages() { return FMT == kI4 ? 4 : (FMT == kT2 ? 5 : 6); }
 constexpr int kExpStages = 2;
+// An expansion stage is freed by the MMA-completion barrier of the TMA stage
+// its K step used, so there must be more TMA stages than expansion stages.
+static_assert(kExpStages < 4, "fewer expansion stages than TMA stages (4 to 6)");
 // Epilogue staging: per epilogue warp, 32 rows of one 32-column chunk, rows
 // padded by 16 bytes so the row-wise writes and the column-wise reads are
 // free of bank conflicts.
@@ -205,7 +208,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
     uint8_t *sStage = sP + ST * P_BYTES;       // 4 x epilogue staging
     uint64_t *bars = reinterpret_cast<uint64_t *>(sStage + 4 * stage_warp_bytes<OUT>());
     uint64_t *full_tma = bars;
-    uint64_t *empty_tma = bars + ST;
+    uint64_t *mma_done = bars + ST;   // MMAs of the step that used TMA stage s are complete
     uint64_t *full_exp = bars + 2 * ST;
     uint64_t *empty_exp = bars + 2 * ST + SE;
     uint64_t *acc_full = bars + 2 * ST + 2 * SE;
@@ -220,11 +223,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
     if (threadIdx.x == 0) {
         for (int s = 0; s < ST; ++s) {
             mbar_init(&full_tma[s], 1);
-            mbar_init(&empty_tma[s], 1);
+            mbar_init(&mma_done[s], 1);
         }
         for (int s = 0; s < SE; ++s) {
             mbar_init(&full_exp[s], kExpThreads);
-            mbar_init(&empty_exp[s], 1);
+            mbar_init(&empty_exp[s], 1);  // unused: the expansion stage is freed by mma_done
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
@@ -285,7 +288,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
                         tma_load_2d(sA + s * A_BYTES, &map_a, &full_tma[s], kb * BK, m0);
                         continue;
                     }
-                    if (!wait_bar(&empty_tma[s], ph ^ 1u, abort_flag, status)) { ok = false; break; }
+                    if (!wait_bar(&mma_done[s], ph ^ 1u, abort_flag, status)) { ok = false; break; }
                     mbar_arrive_expect_tx(&full_tma[s], A_BYTES + P_BYTES);
                     tma_load_2d(sA + s * A_BYTES, &map_a, &full_tma[s], kb * BK, m0);
                     tma_load_2d(sP + s * P_BYTES, &map_p, &full_tma[s], kb * PB, n0);
@@ -313,8 +316,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BN);
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
                     const int s1 = g % ST, s2 = g % SE;
-                    if (!wait_bar(&full_tma[s1], (g / ST) & 1u, abort_flag, status) ||
-                        !wait_bar(&full_exp[s2], (g / SE) & 1u, abort_flag, status)) { ok = false; break; }
+                    // the expanders saw the TMA stage complete before arriving on
+                    // full_exp, so one wait orders the MMA after both
+                    if (!wait_bar(&full_exp[s2], (g / SE) & 1u, abort_flag, status)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(sA + s1 * A_BYTES);
                     const uint32_t e_addr = smem_u32(sE + s2 * E_BYTES);
@@ -322,8 +326,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
                     for (int kk = 0; kk < BK / UMMA_K; ++kk)
                         tc_mma_i8(d_tmem, sw128_desc(a_addr + kk * UMMA_K), sw128_desc(e_addr + kk * UMMA_K),
                                   kIdesc, (kb | kk) != 0 ? 1u : 0u);
-                    tc_commit(&empty_tma[s1]);
-                    tc_commit(&empty_exp[s2]);
+                    tc_commit(&mma_done[s1]);
                 }
                 if (!ok) break;
                 tc_commit(&acc_full[b]);
@@ -342,8 +345,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
         for (int64_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
             for (int kb = 0; kb < nkb; ++kb, ++g) {
                 const int s1 = g % ST, s2 = g % SE;
-                if (!wait_bar(&full_tma[s1], (g / ST) & 1u, abort_flag, status) ||
-                    !wait_bar(&empty_exp[s2], ((g / SE) & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
+                // expansion stage s2 is free once the MMAs of step g - SE are
+                // complete (mma_done of that step's TMA stage)
+                if (!wait_bar(&full_tma[s1], (g / ST) & 1u, abort_flag, status)) { ok = false; break; }
+                if (g >= static_cast<uint32_t>(SE)) {
+                    const uint32_t gp = g - SE;
+                    if (!wait_bar(&mma_done[gp % ST], (gp / ST) & 1u, abort_flag, status)) { ok = false; break; }
+                }
                 expand_stage<FMT>(p_base + s1 * P_BYTES, e_base + s2 * E_BYTES, et);
                 // Each writer orders its generic-proxy stores before the
                 // tensor core's async-proxy reads, then arrives.
@@ -432,7 +440,7 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
     uint8_t *sStage = sP + ST * P_BYTES;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sStage + 4 * stage_warp_bytes<OUT>());
     uint64_t *full_tma = bars;
-    uint64_t *empty_tma = bars + ST;
+    uint64_t *mma_done = bars + ST;   // MMAs of the step that used TMA stage s are complete
     uint64_t *full_exp = bars + 2 * ST;
     uint64_t *empty_exp = bars + 2 * ST + SE;
     uint64_t *acc_full = bars + 2 * ST + 2 * SE;
@@ -447,11 +455,11 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
     if (threadIdx.x == 0) {
         for (int s = 0; s < ST; ++s) {
             mbar_init(&full_tma[s], 1);
-            mbar_init(&empty_tma[s], 1);
+            mbar_init(&mma_done[s], 1);
         }
         for (int s = 0; s < SE; ++s) {
             mbar_init(&full_exp[s], kExpThreads);
-            mbar_init(&empty_exp[s], 1);
+            mbar_init(&empty_exp[s], 1);  // unused: the expansion stage is freed by mma_done
         }
         mbar_init(&acc_full[0], 1);
         mbar_init(drain, 1);
@@ -505,7 +513,7 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
                     tma_load_2d(sA + s * A_BYTES, &map_a, &full_tma[s], kb * BK, m0);
                     continue;
                 }
-                if (!wait_bar(&empty_tma[s], ((g / ST) & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
+                if (!wait_bar(&mma_done[s], ((g / ST) & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
                 mbar_arrive_expect_tx(&full_tma[s], A_BYTES + P_BYTES);
                 tma_load_2d(sA + s * A_BYTES, &map_a, &full_tma[s], kb * BK, m0);
                 tma_load_2d(sP + s * P_BYTES, &map_p, &full_tma[s], kb * PB, n0);
@@ -523,8 +531,7 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
             bool ok = true;
             for (int kb = kb_begin; kb < kb_end; ++kb, ++g) {
                 const int s1 = g % ST, s2 = g % SE;
-                if (!wait_bar(&full_tma[s1], (g / ST) & 1u, abort_flag, status) ||
-                    !wait_bar(&full_exp[s2], (g / SE) & 1u, abort_flag, status)) { ok = false; break; }
+                if (!wait_bar(&full_exp[s2], (g / SE) & 1u, abort_flag, status)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t a_addr = smem_u32(sA + s1 * A_BYTES);
                 const uint32_t e_addr = smem_u32(sE + s2 * E_BYTES);
@@ -532,8 +539,7 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
                 for (int kk = 0; kk < BK / UMMA_K; ++kk)
                     tc_mma_i8(tmem_base, sw128_desc(a_addr + kk * UMMA_K), sw128_desc(e_addr + kk * UMMA_K), kIdesc,
                               (g | kk) != 0 ? 1u : 0u);
-                tc_commit(&empty_tma[s1]);
-                tc_commit(&empty_exp[s2]);
+                tc_commit(&mma_done[s1]);
             }
             if (ok) tc_commit(&acc_full[0]);
             tc_commit(drain);
@@ -546,8 +552,11 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
         uint32_t g = 0;
         for (int kb = kb_begin; kb < kb_end; ++kb, ++g) {
             const int s1 = g % ST, s2 = g % SE;
-            if (!wait_bar(&full_tma[s1], (g / ST) & 1u, abort_flag, status) ||
-                !wait_bar(&empty_exp[s2], ((g / SE) & 1u) ^ 1u, abort_flag, status)) break;
+            if (!wait_bar(&full_tma[s1], (g / ST) & 1u, abort_flag, status)) break;
+            if (g >= static_cast<uint32_t>(SE)) {
+                const uint32_t gp = g - SE;
+                if (!wait_bar(&mma_done[gp % ST], (gp / ST) & 1u, abort_flag, status)) break;
+            }
             expand_stage<FMT>(p_base + s1 * P_BYTES, e_base + s2 * E_BYTES, et);
             fence_proxy_async_smem();
             mbar_arrive(&full_exp[s2]);
