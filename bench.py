@@ -149,17 +149,20 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
-def dispatched_kernel(M, N, row_bytes):
+def dispatched_kernel(M, N, row_bytes, fmt=None):
     """The kernel lowbit_linear picks (same rule as the library): the
     packed-weight GEMV up to 4 tokens; warp-level MMAs up to 16 tokens when
     rows are short or N is large; the tensor-core GEMM with the weight tile
     expanded into shared memory (cluster split-K when output tiles are few)
-    below 512 tokens; the one with it in tensor memory from 512."""
+    below 512 tokens; from 512 the SM-pair one for ternary weights and the
+    one with the weight tile in tensor memory for the others."""
     if M <= 4:
         return "gemv_smem_kernel"
     if M <= 16 and (row_bytes <= 512 or N >= 3200):
         return "skinny_mma_kernel/stream_mma_kernel"
-    return "gemm_kernel/gemm_splitk_kernel" if M < 512 else "gemm_ts_kernel"
+    if M < 512:
+        return "gemm_kernel/gemm_splitk_kernel"
+    return "gemm_pair_kernel" if fmt == wls.TERNARY2 else "gemm_ts_kernel"
 
 
 def packed_row_bytes(fmt, K):
@@ -174,7 +177,7 @@ def packed_row_bytes(fmt, K):
 class Point:
     def __init__(self, mi, m, M, fmt):
         self.mi, self.m, self.M = mi, m, M
-        self.kernel = dispatched_kernel(M, m.N, packed_row_bytes(fmt, m.K))
+        self.kernel = dispatched_kernel(M, m.N, packed_row_bytes(fmt, m.K), fmt)
         # up to 16 tokens the packed weights dominate the bytes: HBM-bound
         self.bound = "hbm" if M <= 16 else "tensor"
         self.ops = 2 * M * m.N * m.K
@@ -362,7 +365,7 @@ def run_gpu_arm(args, wl):
         achieved = dom.ops / (dom_ms * 1e-3) / 1e12
         roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(int8_peak, 1),
                     "unit": "TOPS", "frac": round(achieved / int8_peak, 4),
-                    "traffic": profiled_traffic("gemm_ts_kernel_ternary_4b_M8192.md", "gemm_ts.cu")
+                    "traffic": profiled_traffic("gemm_pair_kernel_ternary_4b_M8192.md", "gemm_sm100.cu")
                     if (wl.name == "ternary_4b" and dom.M == 8192 and dom.mi == 0) else None,
                     "kernel": f"lowbit {dom.kernel}, M={dom.M} {dom.m.K}->{dom.m.N}",
                     "peak_note": f"int8 = 2 x bf16 sustained ({peak_kind})"}

@@ -189,7 +189,8 @@ def lowbit_linear(q, s_x, packed, s_w, fmt: int, N: int, out_dtype: int = F32, K
     ``path`` 0 picks the kernel by M; 1 forces the GEMV, 2 the tensor-core GEMM
     with the expanded tile in shared memory, 3 the one with it in tensor memory,
     4 the tensor-memory one on SM pairs (256 weight rows per MMA), 5 the warp-level
-    mma.sync kernel for at most 16 tokens.
+    mma.sync kernel for at most 16 tokens, 6 the shared-memory one on SM pairs
+    (256 tokens x 256 features per MMA).
     ``weights_stable`` passes LOWBIT_LINEAR_WEIGHTS_STABLE: the kernel that
     precedes this call on the stream does not write ``packed`` or ``s_w``, so
     weight reads may start before it finishes."""

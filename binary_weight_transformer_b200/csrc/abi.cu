@@ -35,6 +35,11 @@ lowbit_status skinny_launch(const int8_t *q, int64_t ldq, const float *s_x, int6
                             lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int prefetch,
                             int32_t *status, cudaStream_t st);
 
+lowbit_status gemm_pair_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
+                               const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
+                               lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int prefetch,
+                               int32_t *status, cudaStream_t st);
+
 lowbit_status gemm_ts_pair_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
                                   const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
                                   lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy,
@@ -198,7 +203,7 @@ lowbit_status lowbit_linear_ex(const int8_t *q, int64_t ldq, const float *s_x, i
     if (!valid_format(f) || q == nullptr || s_x == nullptr || packed == nullptr || s_w == nullptr || y == nullptr)
         return LOWBIT_ERR_INVALID_ARG;
     if (ydt != LOWBIT_F32 && ydt != LOWBIT_BF16 && ydt != LOWBIT_I32) return LOWBIT_ERR_INVALID_ARG;
-    if (path < 0 || path > 5) return LOWBIT_ERR_INVALID_ARG;
+    if (path < 0 || path > 6) return LOWBIT_ERR_INVALID_ARG;
     if (M <= 0 || N <= 0 || K <= 0 || ldq < K || ldy < N) return LOWBIT_ERR_INVALID_ARG;
     if (path == 5 && M > 16) return LOWBIT_ERR_INVALID_ARG;
     if (M > INT32_MAX || N > INT32_MAX) return LOWBIT_ERR_INVALID_ARG;
@@ -223,11 +228,17 @@ lowbit_status lowbit_linear_ex(const int8_t *q, int64_t ldq, const float *s_x, i
     const bool skinny_wins = rb <= 512 || N >= 3200;
     if (path == 5 || (path == 0 && M <= 16 && skinny_wins))
         return skinny_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
-    // From 512 tokens the tensor-memory variant (weights as the MMA's A
-    // operand in TMEM) is as fast or faster; below it the shared-memory
-    // variant, which splits K over a cluster when tiles are few, wins.
+    // Below 512 tokens the shared-memory variant, which splits K over a
+    // cluster when tiles are few, wins.
+    if (path == 6)
+        return gemm_pair_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
     if (path == 4)
         return gemm_ts_pair_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, status_dev, st);
+    // From 512 tokens ternary weights run on SM pairs with the expanded tile
+    // in shared memory (measured fastest for them); 4-bit and binary weights
+    // on the tensor-memory variant.
+    if (path == 0 && M >= 512 && f == LOWBIT_TERNARY2)
+        return gemm_pair_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
     if (path == 3 || (path == 0 && M >= 512))
         return gemm_ts_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
     return gemm_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);

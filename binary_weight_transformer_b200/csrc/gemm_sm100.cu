@@ -55,20 +55,20 @@ constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<ui
                             (static_cast<uint32_t>(BM >> 4) << 24);
 
 // ---------------------------------------------------------------------------
-// Expansion of one stage: 256 rows x 128 codes.  Each thread loads 16 bytes of
+// Expansion of one stage: ROWS (256, or 128 per CTA of a pair) rows x 128 codes.  Each thread loads 16 bytes of
 // packed codes at a time (ld.shared.v4) and writes whole 16-code chunks of the
 // int8 tile (st.shared.v4); chunk c of row r goes to r*128 + ((c ^ (r%8))*16),
 // the 128B-swizzle pattern the TMA uses for the activation tile.  Within every
 // group of 8 lanes the loads cover 128 contiguous bytes and the stores hit 8
 // distinct 16-byte bank groups, so neither conflicts.
 // ---------------------------------------------------------------------------
-template <int FMT>
+template <int FMT, int ROWS = BN>
 __device__ __forceinline__ void expand_stage(uint32_t P, uint32_t E, int et)
 {
     if constexpr (FMT == kT2) {
         // 32 packed bytes per row: item = (row, half), half = 4 chunks.
 #pragma unroll
-        for (int j = 0; j < (BN * 2) / kExpThreads; ++j) {
+        for (int j = 0; j < (ROWS * 2) / kExpThreads; ++j) {
             const int i = et + kExpThreads * j;
             const int r = i >> 1, h = i & 1;
             const uint4 w = lds128(P + r * 32 + h * 16);
@@ -84,7 +84,7 @@ __device__ __forceinline__ void expand_stage(uint32_t P, uint32_t E, int et)
     } else if constexpr (FMT == kI4) {
         // 64 packed bytes per row: item = (row, quarter), quarter = 2 chunks.
 #pragma unroll
-        for (int j = 0; j < (BN * 4) / kExpThreads; ++j) {
+        for (int j = 0; j < (ROWS * 4) / kExpThreads; ++j) {
             const int i = et + kExpThreads * j;
             const int r = i >> 2, qd = i & 3;
             const uint4 w = lds128(P + r * 64 + qd * 16);
@@ -97,7 +97,7 @@ __device__ __forceinline__ void expand_stage(uint32_t P, uint32_t E, int et)
     } else {
         // 16 packed bytes per row: item = row, 8 chunks of 16 codes (16 bits).
 #pragma unroll
-        for (int j = 0; j < BN / kExpThreads; ++j) {
+        for (int j = 0; j < ROWS / kExpThreads; ++j) {
             const int r = et + kExpThreads * j;
             const uint4 w = lds128(P + r * 16);
             const uint32_t rowE = E + r * 128;
@@ -649,6 +649,315 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
 }
 
 // ---------------------------------------------------------------------------
+// SM-pair variant (tcgen05 cta_group::2): a cluster of two CTAs computes a
+// 256-token x 256-feature tile with M = 256 MMAs issued by the even CTA.  CTA r
+// stages tokens m0 + 128r (the MMA's A rows it owns) and expands features
+// n0 + 128r (its half of the B operand) into its own shared memory; each CTA's
+// tensor memory holds its 128 tokens x all 256 features, and each CTA runs the
+// epilogue for them.  Per SM and K step this stages half the expanded weights
+// of the single-CTA kernel and issues no MMAs on the odd CTA.
+//
+// Barriers (all in both CTAs; the even CTA's full_exp and acc_empty collect
+// the arrivals of both): full_tma[s] local TMA completion; full_exp[s2] 4
+// expander warps x 2 CTAs wrote expansion stage s2 and saw their TMA stage
+// complete; mma_done[s] (multicast commit) the MMAs of the K step that used
+// TMA stage s are done; acc_full[b] (multicast commit) accumulator b is final;
+// acc_empty[b] 4 epilogue warps x 2 CTAs drained accumulator b.
+// ---------------------------------------------------------------------------
+constexpr int PBM = 128;                      // tokens per CTA (the pair's MMA has M = 256)
+constexpr int PBN = 128;                      // features expanded per CTA (the pair's N = 256)
+constexpr int PE_BYTES = PBN * BK;
+template <int FMT> __host__ __device__ constexpr int pair_tma_stages() { return FMT == kI4 ? 7 : 8; }
+constexpr uint32_t kPairIdesc = (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>((2 * PBN) >> 3) << 17) |
+                                (static_cast<uint32_t>((2 * PBM) >> 4) << 24);
+
+template <int FMT, int OUT>
+__host__ __device__ constexpr size_t pair_smem_bytes()
+{
+    return 1024 + static_cast<size_t>(pair_tma_stages<FMT>()) * (A_BYTES + PBN * packed_bytes_per_kblock<FMT>()) +
+           static_cast<size_t>(kExpStages) * PE_BYTES + 4 * stage_warp_bytes<OUT>() +
+           8 * (2 * pair_tma_stages<FMT>() + kExpStages + 8);
+}
+
+__device__ __forceinline__ void tc_mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_commit_pair_both(uint64_t *bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+        ::"r"(smem_u32(bar)), "h"(static_cast<uint16_t>(0x3)) : "memory");
+}
+
+__device__ __forceinline__ void tc_commit_pair_self(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_u32(bar)) : "memory");
+}
+
+template <int FMT, int OUT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_p,
+                 const float *__restrict__ s_x, const float *__restrict__ s_w, int64_t M, int64_t N, int64_t K,
+                 void *__restrict__ y, int64_t ldy, int vec_ok, int prefetch, int32_t *status)
+{
+    constexpr int ST = pair_tma_stages<FMT>();
+    constexpr int SE = kExpStages;
+    constexpr int PB = packed_bytes_per_kblock<FMT>();
+    constexpr int P_BYTES = PBN * PB;
+    constexpr int kShift = Fmt<FMT>::kShift;
+    static_assert(SE < ST, "an expansion stage is freed through the MMA barrier of an older TMA stage");
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = base;                        // ST x 16 KB, 1024-aligned
+    uint8_t *sE = sA + ST * A_BYTES;           // SE x 16 KB, 1024-aligned
+    uint8_t *sP = sE + SE * PE_BYTES;          // ST x P_BYTES
+    uint8_t *sStage = sP + ST * P_BYTES;       // 4 x epilogue staging
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sStage + 4 * stage_warp_bytes<OUT>());
+    uint64_t *full_tma = bars;
+    uint64_t *mma_done = bars + ST;
+    uint64_t *full_exp = bars + 2 * ST;
+    uint64_t *acc_full = full_exp + SE;
+    uint64_t *acc_empty = acc_full + 2;
+    uint64_t *drain = acc_full + 4;
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(acc_full + 5);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(acc_full + 6);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(&full_tma[s], 1);
+            mbar_init(&mma_done[s], 1);
+        }
+        for (int s = 0; s < SE; ++s) mbar_init(&full_exp[s], 8);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 8);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_p)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(const_cast<uint32_t *>(tmem_slot))), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // both CTAs' barriers exist before any remote arrive
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    // Global memory is touched only after the previous kernel on the stream
+    // has completed (programmatic dependent launch, see pdl_wait); with
+    // prefetch the TMA thread starts the weight half of its first stages first.
+    if (prefetch == 0 || threadIdx.x != 0) pdl_wait();
+    pdl_trigger();
+
+    const int64_t num_m = (M + 2 * PBM - 1) / (2 * PBM);
+    const int64_t num_n = (N + 2 * PBN - 1) / (2 * PBN);
+    const int64_t num_tiles = num_m * num_n;
+    const int64_t pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+    const int nkb = static_cast<int>((K + BK - 1) / BK);
+
+    if (warp == 0) {
+        // ---------------- TMA producer (both CTAs) ----------------
+        if (lane == 0) {
+            uint32_t g = 0;
+            bool ok = true;
+            uint32_t npre = 0;
+            if (prefetch != 0) {
+                if (pair < num_tiles) {
+                    const int n0 = static_cast<int>((pair / num_m) * 2 * PBN + rank * PBN);
+                    npre = static_cast<uint32_t>(nkb < ST ? nkb : ST);
+                    for (uint32_t i = 0; i < npre; ++i) {
+                        mbar_arrive_expect_tx(&full_tma[i], A_BYTES + P_BYTES);
+                        tma_load_2d(sP + i * P_BYTES, &map_p, &full_tma[i], static_cast<int>(i) * PB, n0);
+                    }
+                }
+                pdl_wait();
+            }
+            for (int64_t tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+                const int m0 = static_cast<int>((tile % num_m) * 2 * PBM + rank * PBM);
+                const int n0 = static_cast<int>((tile / num_m) * 2 * PBN + rank * PBN);
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % ST;
+                    if (g < npre) {
+                        tma_load_2d(sA + s * A_BYTES, &map_a, &full_tma[s], kb * BK, m0);
+                        continue;
+                    }
+                    if (!wait_bar(&mma_done[s], ((g / ST) & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&full_tma[s], A_BYTES + P_BYTES);
+                    tma_load_2d(sA + s * A_BYTES, &map_a, &full_tma[s], kb * BK, m0);
+                    tma_load_2d(sP + s * P_BYTES, &map_p, &full_tma[s], kb * PB, n0);
+                }
+            }
+            if (!ok) {
+                for (uint32_t i = 0; i < ST && i < g; ++i) {
+                    const uint32_t gi = g - 1 - i;
+                    wait_bar(&full_tma[gi % ST], (gi / ST) & 1u, abort_flag, nullptr, 200000000ll);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (even CTA) ----------------
+        if (leader && lane == 0) {
+            uint32_t g = 0;
+            uint32_t t = 0;
+            bool ok = true;
+            for (int64_t tile = pair; tile < num_tiles && ok; tile += num_pairs, ++t) {
+                const int b = t & 1;
+                if (!wait_bar(&acc_empty[b], ((t >> 1) & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * 2 * PBN);
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s1 = g % ST, s2 = g % SE;
+                    if (!wait_bar(&full_exp[s2], (g / SE) & 1u, abort_flag, status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(sA + s1 * A_BYTES);
+                    const uint32_t e_addr = smem_u32(sE + s2 * PE_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < BK / UMMA_K; ++kk)
+                        tc_mma_i8_pair(d_tmem, sw128_desc(a_addr + kk * UMMA_K), sw128_desc(e_addr + kk * UMMA_K),
+                                       kPairIdesc, (kb | kk) != 0 ? 1u : 0u);
+                    tc_commit_pair_both(&mma_done[s1]);
+                }
+                if (!ok) break;
+                tc_commit_pair_both(&acc_full[b]);
+            }
+            tc_commit_pair_self(drain);
+            wait_bar(drain, 0, abort_flag, nullptr, 200000000ll);
+        }
+    } else if (warp < 6) {
+        // ---------------- expanders: own 128 features ----------------
+        const int et = threadIdx.x - 64;
+        const uint32_t p_base = smem_u32(sP);
+        const uint32_t e_base = smem_u32(sE);
+        const uint32_t full_exp_leader = map_to_peer(smem_u32(full_exp), 0);
+        uint32_t g = 0;
+        bool ok = true;
+        for (int64_t tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+            for (int kb = 0; kb < nkb; ++kb, ++g) {
+                const int s1 = g % ST, s2 = g % SE;
+                if (!wait_bar(&full_tma[s1], (g / ST) & 1u, abort_flag, status)) { ok = false; break; }
+                if (g >= static_cast<uint32_t>(SE)) {
+                    const uint32_t gp = g - SE;
+                    if (!wait_bar(&mma_done[gp % ST], (gp / ST) & 1u, abort_flag, status)) { ok = false; break; }
+                }
+                expand_stage<FMT, PBN>(p_base + s1 * P_BYTES, e_base + s2 * PE_BYTES, et);
+                // each writer orders its stores before the async proxy's reads;
+                // one arrival per warp on the even CTA's barrier
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(full_exp_leader + static_cast<uint32_t>(s2 * 8));
+            }
+        }
+    } else {
+        // ---------------- epilogue: own 128 tokens x 256 features ----------------
+        const int quarter = warp & 3;
+        const uint32_t stage = smem_u32(sStage) + static_cast<uint32_t>((warp - 6) * stage_warp_bytes<OUT>());
+        const uint32_t acc_empty_leader = map_to_peer(smem_u32(acc_empty), 0);
+        const float sw_tensor = (FMT == kT2) ? s_w[0] : 0.0f;
+        uint32_t t = 0;
+        for (int64_t tile = pair; tile < num_tiles; tile += num_pairs, ++t) {
+            const int b = t & 1;
+            int ready = 0;
+            if (lane == 0) ready = wait_bar(&acc_full[b], (t >> 1) & 1u, abort_flag, status) ? 1 : 0;
+            ready = __shfl_sync(0xffffffffu, ready, 0);
+            if (!ready) break;
+            tc_fence_after();
+            const int64_t m0 = (tile % num_m) * 2 * PBM + rank * PBM;
+            const int64_t n0 = (tile / num_m) * 2 * PBN;
+            const int64_t row0 = m0 + quarter * 32;
+            const float sx = (row0 + lane < M) ? s_x[row0 + lane] : 0.0f;
+#pragma unroll 1
+            for (int cc = 0; cc < 2 * PBN / 32; ++cc) {
+                const int64_t nc = n0 + cc * 32;
+                uint32_t v[32];
+                tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                   static_cast<uint32_t>(b * 2 * PBN + cc * 32), v);
+                if (nc < N) {
+                    float sw[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        sw[i] = (FMT == kT2) ? sw_tensor : ((nc + i < N) ? __ldg(s_w + nc + i) : 0.0f);
+                    epilogue_chunk<OUT>(v, sw, sx, kShift, y, ldy, row0, M, nc, N, vec_ok != 0, stage, lane);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(acc_empty_leader + static_cast<uint32_t>(b * 8));
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // the pair's MMAs and remote arrivals are over
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+template <int FMT, int OUT>
+lowbit_status launch_pair_t(const CUtensorMap &ma, const CUtensorMap &mp, const float *s_x, const float *s_w,
+                            int64_t M, int64_t N, int64_t K, void *y, int64_t ldy, int vec_ok, int prefetch,
+                            int32_t *status, cudaStream_t st)
+{
+    constexpr size_t smem = pair_smem_bytes<FMT, OUT>();
+    static_assert(smem <= 232448, "shared memory budget");
+    static int max_pairs[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LOWBIT_ERR_CUDA;
+    if (max_pairs[dev] == 0) {
+        if (cudaFuncSetAttribute(gemm_pair_kernel<FMT, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem)) != cudaSuccess)
+            return LOWBIT_ERR_CUDA;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * static_cast<unsigned>(device_sm_count() / 2));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<FMT, OUT>, &cfg) != cudaSuccess || n <= 0)
+            return LOWBIT_ERR_CUDA;
+        max_pairs[dev] = n;
+    }
+    const int64_t tiles = ((M + 2 * PBM - 1) / (2 * PBM)) * ((N + 2 * PBN - 1) / (2 * PBN));
+    const int64_t pairs = tiles < max_pairs[dev] ? tiles : max_pairs[dev];
+    return launch_pdl(gemm_pair_kernel<FMT, OUT>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kThreads), smem, st,
+                      0, ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status);
+}
+
+template <int FMT>
+lowbit_status launch_pair_fmt(const CUtensorMap &ma, const CUtensorMap &mp, const float *s_x, const float *s_w,
+                              int64_t M, int64_t N, int64_t K, void *y, lowbit_dtype ydt, int64_t ldy, int vec_ok,
+                              int prefetch, int32_t *status, cudaStream_t st)
+{
+    if (ydt == LOWBIT_F32)
+        return launch_pair_t<FMT, LOWBIT_F32>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, st);
+    if (ydt == LOWBIT_BF16)
+        return launch_pair_t<FMT, LOWBIT_BF16>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, st);
+    return launch_pair_t<FMT, LOWBIT_I32>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, st);
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 template <int FMT, int OUT>
@@ -730,4 +1039,32 @@ lowbit_status gemm_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_
     return launch_fmt<kI4>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, st);
 }
 
+}  // namespace lowbit
+
+namespace lowbit {
+// SM-pair variant: 128-token activation boxes and 128-row packed boxes per CTA.
+lowbit_status gemm_pair_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
+                               const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
+                               lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int prefetch,
+                               int32_t *status, cudaStream_t st)
+{
+    using namespace tc;
+    CUtensorMap ma, mp;
+    if (!make_map_2d(&ma, q, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(ldq), BK,
+                     PBM, CU_TENSOR_MAP_SWIZZLE_128B))
+        return LOWBIT_ERR_CUDA;
+    const uint32_t pb = f == LOWBIT_TERNARY2 ? packed_bytes_per_kblock<kT2>()
+                        : f == LOWBIT_BINARY1 ? packed_bytes_per_kblock<kB1>()
+                                              : packed_bytes_per_kblock<kI4>();
+    if (!make_map_2d(&mp, packed, static_cast<uint64_t>(row_bytes), static_cast<uint64_t>(N),
+                     static_cast<uint64_t>(ldp), pb, PBN, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return LOWBIT_ERR_CUDA;
+    const int64_t esz = ydt == LOWBIT_BF16 ? 2 : 4;
+    const int vec_ok = ((reinterpret_cast<uintptr_t>(y) & 15u) == 0 && (ldy * esz) % 16 == 0) ? 1 : 0;
+    if (f == LOWBIT_TERNARY2)
+        return launch_pair_fmt<kT2>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, st);
+    if (f == LOWBIT_BINARY1)
+        return launch_pair_fmt<kB1>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, st);
+    return launch_pair_fmt<kI4>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, st);
+}
 }  // namespace lowbit

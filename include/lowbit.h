@@ -190,7 +190,9 @@ lowbit_status lowbit_act_quant(const void *x, lowbit_dtype xdt, int64_t M, int64
  * otherwise, and for 17 <= M < 512, a tcgen05 tensor-core GEMM (int8 MMA,
  * accumulators in tensor memory) with the expanded weight tile in shared
  * memory and K split over a cluster when the output tiles are few; from
- * M = 512 the tcgen05 GEMM with the weight tile in tensor memory. */
+ * M = 512 a tcgen05 GEMM on pairs of SMs (cta_group::2, 256 x 256 tiles,
+ * expanded weights in shared memory) for ternary weights and the tcgen05
+ * GEMM with the weight tile in tensor memory for 4-bit and binary weights. */
 lowbit_status lowbit_linear(const int8_t *q, int64_t ldq, const float *s_x,
                             int64_t M, int64_t K,
                             const uint8_t *packed, int64_t ldp, const float *s_w,
@@ -203,8 +205,9 @@ lowbit_status lowbit_linear(const int8_t *q, int64_t ldq, const float *s_x,
  * the expanded weight tile in shared memory (any M), 3 = tensor-core GEMM
  * with the expanded weight tile in tensor memory (any M), 4 = the same on
  * pairs of SMs (one MMA covers 256 weight rows; any M), 5 = warp-level
- * tensor-core MMAs on register fragments (M <= 16).  Other values, and path 5
- * with M > 16, return LOWBIT_ERR_INVALID_ARG.  Lets tests and benchmarks reach every kernel at
+ * tensor-core MMAs on register fragments (M <= 16), 6 = tensor-core GEMM on
+ * pairs of SMs with the expanded weight tile in shared memory (any M).  Other
+ * values, and path 5 with M > 16, return LOWBIT_ERR_INVALID_ARG.  Lets tests and benchmarks reach every kernel at
  * every size. */
 lowbit_status lowbit_linear_path(const int8_t *q, int64_t ldq, const float *s_x,
                                  int64_t M, int64_t K,

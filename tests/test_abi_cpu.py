@@ -75,7 +75,7 @@ def test_linear_rejects_bad_arguments(lib):
     assert _linear(lib, ldp=48) == bwt.ERR_INVALID_ARG           # ldp < row bytes
     assert _linear(lib, fmt=3) == bwt.ERR_INVALID_ARG
     assert _linear(lib, ydt=7) == bwt.ERR_INVALID_ARG
-    assert _linear(lib, path=6) == bwt.ERR_INVALID_ARG
+    assert _linear(lib, path=7) == bwt.ERR_INVALID_ARG
     assert _linear(lib, path=5, M=17) == bwt.ERR_INVALID_ARG   # warp-MMA kernel: M <= 16
     assert _linear(lib, q=FAKE + 8) == bwt.ERR_ALIGNMENT
     assert _linear(lib, ldq=264) == bwt.ERR_ALIGNMENT

@@ -220,7 +220,7 @@ SHAPES = [(1, 768, 192), (3, 257, 200), (16, 96, 1000), (17, 300, 192), (129, 51
           (5, 33, 16), (200, 1, 4000), (64, 500, 4096), (130, 1000, 2000)]
 
 
-@pytest.mark.parametrize("path", [1, 2, 3, 4, 5], ids=["gemv", "gemm", "gemm_ts", "gemm_ts_pair", "skinny"])
+@pytest.mark.parametrize("path", [1, 2, 3, 4, 5, 6], ids=["gemv", "gemm", "gemm_ts", "gemm_ts_pair", "skinny", "gemm_pair"])
 @pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
 @pytest.mark.parametrize("M,N,K", SHAPES, ids=str)
 def test_linear_int32_accumulators_bit_exact(path, fmt, M, N, K):
@@ -228,7 +228,7 @@ def test_linear_int32_accumulators_bit_exact(path, fmt, M, N, K):
     assert np.array_equal(y.cpu().numpy().astype(np.int64), acc)
 
 
-@pytest.mark.parametrize("path", [1, 2, 3, 4, 5], ids=["gemv", "gemm", "gemm_ts", "gemm_ts_pair", "skinny"])
+@pytest.mark.parametrize("path", [1, 2, 3, 4, 5, 6], ids=["gemv", "gemm", "gemm_ts", "gemm_ts_pair", "skinny", "gemm_pair"])
 @pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
 @pytest.mark.parametrize("M,N,K", SHAPES[:6] + SHAPES[8:], ids=str)
 def test_linear_f32_within_tolerance(path, fmt, M, N, K):
@@ -240,7 +240,7 @@ def test_linear_f32_within_tolerance(path, fmt, M, N, K):
     assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
 
 
-@pytest.mark.parametrize("path", [1, 2, 3, 4, 5], ids=["gemv", "gemm", "gemm_ts", "gemm_ts_pair", "skinny"])
+@pytest.mark.parametrize("path", [1, 2, 3, 4, 5, 6], ids=["gemv", "gemm", "gemm_ts", "gemm_ts_pair", "skinny", "gemm_pair"])
 @pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
 @pytest.mark.parametrize("M,N,K", SHAPES[:6] + SHAPES[8:], ids=str)
 def test_linear_bf16_within_one_ulp(path, fmt, M, N, K):
@@ -256,7 +256,7 @@ def test_linear_bf16_within_one_ulp(path, fmt, M, N, K):
 # on the same stream); the results must not change.  Shapes cover the GEMV
 # (one and several token groups), the cluster split-K GEMM, the persistent
 # GEMM, and the tensor-memory GEMM with more tiles than SMs.
-@pytest.mark.parametrize("path", [0, 1, 2, 3, 5], ids=["auto", "gemv", "gemm", "gemm_ts", "skinny"])
+@pytest.mark.parametrize("path", [0, 1, 2, 3, 5, 6], ids=["auto", "gemv", "gemm", "gemm_ts", "skinny", "gemm_pair"])
 @pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
 @pytest.mark.parametrize("M,N,K", [(1, 2560, 768), (9, 300, 1000), (16, 2600, 2600), (130, 1000, 2000),
                                    (600, 4000, 640)], ids=str)
@@ -267,7 +267,7 @@ def test_linear_weights_stable_bit_exact(path, fmt, M, N, K):
     assert np.array_equal(y.cpu().numpy().astype(np.int64), acc)
 
 
-@pytest.mark.parametrize("path", [1, 2, 3, 4, 5], ids=["gemv", "gemm", "gemm_ts", "gemm_ts_pair", "skinny"])
+@pytest.mark.parametrize("path", [1, 2, 3, 4, 5, 6], ids=["gemv", "gemm", "gemm_ts", "gemm_ts_pair", "skinny", "gemm_pair"])
 def test_linear_degenerate_weights(path):
     # all-zero weights: gamma = 0, every code 0, y = 0
     y, acc, _, _ = run_case(bwt.TERNARY2, 16 if path == 5 else 20, 64, 256, path, bwt.F32, 800, zero_w=True)
@@ -275,7 +275,7 @@ def test_linear_degenerate_weights(path):
     assert not y.cpu().numpy().any()
 
 
-@pytest.mark.parametrize("path", [1, 2, 3, 4, 5], ids=["gemv", "gemm", "gemm_ts", "gemm_ts_pair", "skinny"])
+@pytest.mark.parametrize("path", [1, 2, 3, 4, 5, 6], ids=["gemv", "gemm", "gemm_ts", "gemm_ts_pair", "skinny", "gemm_pair"])
 def test_linear_all_plus_one_gives_row_sums(path):
     # ternary codes all +1: acc[t, n] = sum_k q[t, k] (add/sub/skip rule)
     M, N, K = (16 if path == 5 else 19), 40, 320
