@@ -77,11 +77,13 @@ def gpu_act(x_np, bf16=False, eps=0.0):
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("bf16", [False, True], ids=["f32", "bf16"])
-# Shapes cover one thread group per row for every TPR, the scalar-load path
+# Shapes cover one thread group per row for every TPR (the 1024-thread group
+# of both register builds: 9728, 12288, 16384, 24584), the scalar-load path
 # (unaligned rows), rows longer than the register path (65560), many rows of
 # 16-byte vectors, and a zero row in each.
 @pytest.mark.parametrize("M,K", [(1, 192), (7, 200), (3, 9728), (257, 2560), (5, 13), (64, 3),
-                                 (9, 65536 + 24), (300, 9728), (1000, 192), (600, 12288), (256, 24)])
+                                 (9, 65536 + 24), (300, 9728), (1000, 192), (600, 12288), (256, 24),
+                                 (33, 768), (5, 16384), (2, 24584)])
 @pytest.mark.parametrize("eps", [0.0, 1e-5])
 def test_act_quant_bit_exact(M, K, bf16, eps):
     x = wls.normal_activations(100 + M + K, M, K, 0.01, 8.0)
@@ -90,6 +92,30 @@ def test_act_quant_bit_exact(M, K, bf16, eps):
         x = wls.to_bf16_bits(x)
     q, s_x = gpu_act(x, bf16, eps)
     q_o, s_o = oracle.act_quant(x, eps, bf16_bits=bf16)
+    assert np.array_equal(q.cpu().numpy()[:, :K], q_o)
+    assert np.array_equal(s_x.cpu().numpy().view(np.uint32), s_o.view(np.uint32))
+
+
+# The deep build (five vectors per thread at 1536 resident threads) runs when
+# it halves the thread group of the wide build and M x group fills two waves
+# of the GPU, or when only it holds the row; each case is sized 10% past that
+# bound for its group: bf16 K = 320, 1280, 2560, 5120, 9728, 20480 (groups 8 to
+# 512), f32 K = 9728 (512), and rows of 3073 to 5120 vectors (1024, any M).
+@pytest.mark.parametrize("K,bf16", [(320, True), (1280, True), (2560, True), (5120, True), (9728, True),
+                                    (20480, True), (9728, False), (24584, True), (40960, True), (20480, False)])
+def test_act_quant_bit_exact_deep(K, bf16):
+    nvec = K // (8 if bf16 else 4)
+    groups = (8, 32, 64, 128, 256, 512, 1024)
+    tpr_deep = next(g for g in groups if nvec <= 5 * g)
+    tpr_wide = next((g for g in groups if nvec <= 3 * g), None)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    M = 3 if tpr_wide is None else (2 * sms * 1536 * 11 // 10 + tpr_deep - 1) // tpr_deep
+    x = wls.normal_activations(7 + K, M, K, 0.01, 8.0)
+    x[0, :] = 0.0
+    if bf16:
+        x = wls.to_bf16_bits(x)
+    q, s_x = gpu_act(x, bf16, 0.0)
+    q_o, s_o = oracle.act_quant(x, 0.0, bf16_bits=bf16)
     assert np.array_equal(q.cpu().numpy()[:, :K], q_o)
     assert np.array_equal(s_x.cpu().numpy().view(np.uint32), s_o.view(np.uint32))
 
