@@ -77,6 +77,8 @@ __device__ __forceinline__ int8_t quant_one(float x, float d)
 // of v's bit pattern is the code in two's complement.  A value within 1e-4
 // of a midpoint (about 2 in 10^4) sets `near`; the caller then redoes the
 // four values with the IEEE divide.  |u| <= 127.0001, so no clamp is needed.
+// The relative bounds need RN(1/d) and c normal and finite, i.e. d in
+// [2^-121, 2^126); outside it the caller takes the divide for every value.
 __device__ __forceinline__ uint32_t quant4(float x0, float x1, float x2, float x3, float c, bool &near)
 {
     constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
@@ -172,6 +174,8 @@ act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
     if (bad && r == 0) report(status, LOWBIT_ERR_NONFINITE);
     const float d = __fadd_rn(g, eps);
     const float c = __fmul_rn(127.0f, __frcp_rn(d));
+    // Rows with max|x| below about 3.7e-37, or an eps near the fp32 maximum.
+    const bool slow = !(d >= 0x1p-121f && d < 0x1p126f);
     int8_t *qrow = q + row * ldq;
 
 #pragma unroll
@@ -180,13 +184,13 @@ act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
         if (v < nvec) {
             const uint4 &b = buf[i];
             if constexpr (E == 4) {
-                bool near = false;
+                bool near = slow;
                 uint32_t out = quant4(In<T>::get(b, 0), In<T>::get(b, 1), In<T>::get(b, 2), In<T>::get(b, 3), c, near);
                 if (near) out = quant4_exact(In<T>::get(b, 0), In<T>::get(b, 1), In<T>::get(b, 2), In<T>::get(b, 3), d);
                 if (amax == 0) out = 0;
                 *reinterpret_cast<uint32_t *>(qrow + v * 4) = out;
             } else {
-                bool near = false;
+                bool near = slow;
                 uint32_t lo = quant4(In<T>::get(b, 0), In<T>::get(b, 1), In<T>::get(b, 2), In<T>::get(b, 3), c, near);
                 uint32_t hi = quant4(In<T>::get(b, 4), In<T>::get(b, 5), In<T>::get(b, 6), In<T>::get(b, 7), c, near);
                 if (near) {

@@ -120,6 +120,53 @@ def test_act_quant_bit_exact_deep(K, bf16):
     assert np.array_equal(s_x.cpu().numpy().view(np.uint32), s_o.view(np.uint32))
 
 
+def edge_rows(seed, M, K, eps):
+    """Rows that stress the codes' rounding: by row index mod 4, ordinary
+    N(0,1); tiny (max |x| from 1e-44 to 1e-36, subnormals included, where the
+    reciprocal of the row max is not a normal fp32); values placed within a few
+    ulp of rounding midpoints, 127x/max|x| = k + 1/2; and large (1e30 to 1e35,
+    127x still finite).  With a large eps all rows are scaled near 1e36 (and
+    clipped to 2e36, where 127x is still finite) so that the codes are not all
+    zero."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((M, K))
+    for t in range(M):
+        kind = t % 4
+        if eps > 1.0:
+            x[t] = np.clip(x[t] * 10 ** rng.uniform(35.0, 35.7), -2e36, 2e36)
+        elif kind == 1:
+            x[t] *= 10 ** rng.uniform(-44.0, -36.0)
+        elif kind == 2:
+            g = 10 ** rng.uniform(-3.0, 3.0)
+            k = rng.integers(-127, 127, K)
+            x[t] = (k + 0.5) * g / 127.0 * (1.0 + rng.uniform(-3e-7, 3e-7, K))
+            x[t, 0] = g
+        elif kind == 3:
+            x[t] *= 10 ** rng.uniform(30.0, 35.0)
+    return x.astype(np.float32)
+
+
+# eps = 0; 5e37 (d just below 2^126: the fast path); 1e38 (d above it: the
+# divide for every value).  Small M takes the wide build, large M the deep one.
+@pytest.mark.parametrize("eps", [0.0, 5e37, 1e38])
+@pytest.mark.parametrize("K,bf16,deep", [(2560, True, False), (2560, False, False), (9728, True, True),
+                                         (9728, False, True)])
+def test_act_quant_rounding_edges(K, bf16, deep, eps):
+    M = 64
+    if deep:
+        nvec = K // (8 if bf16 else 4)
+        tpr_deep = next(g for g in (8, 32, 64, 128, 256, 512, 1024) if nvec <= 5 * g)
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        M = (2 * sms * 1536 * 11 // 10 + tpr_deep - 1) // tpr_deep
+    x = edge_rows(K + int(eps > 0) + int(eps > 6e37), M, K, eps)
+    if bf16:
+        x = wls.to_bf16_bits(x)
+    q, s_x = gpu_act(x, bf16, eps)
+    q_o, s_o = oracle.act_quant(x, eps, bf16_bits=bf16)
+    assert np.array_equal(q.cpu().numpy()[:, :K], q_o)
+    assert np.array_equal(s_x.cpu().numpy().view(np.uint32), s_o.view(np.uint32))
+
+
 @pytest.mark.parametrize("M", [4, 300], ids=["regs", "ring"])
 def test_act_quant_flags_nonfinite(M):
     x = np.ones((M, 64), np.float32)
