@@ -25,6 +25,10 @@ lowbit_status gemm_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_
                           lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int prefetch,
                           int32_t *status, cudaStream_t st);
 
+// True when the shared-memory GEMM would split K over a cluster (few output
+// tiles, deep K).
+bool gemm_splits_k(int64_t M, int64_t N, int64_t K);
+
 lowbit_status gemm_ts_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
                              const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
                              lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int prefetch,
@@ -235,10 +239,18 @@ lowbit_status lowbit_linear_ex(const int8_t *q, int64_t ldq, const float *s_x, i
     if (path == 4)
         return gemm_ts_pair_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, status_dev, st);
     // From 512 tokens ternary weights run on SM pairs with the expanded tile
-    // in shared memory (measured fastest for them); 4-bit and binary weights
-    // on the tensor-memory variant.
-    if (path == 0 && M >= 512 && f == LOWBIT_TERNARY2)
+    // in shared memory (measured fastest for them), except for deep K
+    // (>= 2048) with output tiles too few to fill the GPU: there the split-K
+    // shared-memory kernel stays faster (9728->2560 at M = 512: 28.6 us vs
+    // 32.8 us; for 1024->256 at M = 1024 the pair kernel is ahead, 9.2 us vs
+    // 9.6 us).  4-bit and binary weights take the tensor-memory variant from
+    // 512 tokens (the split-K kernel measured faster for some of their shapes
+    // and slower for others).
+    if (path == 0 && M >= 512 && f == LOWBIT_TERNARY2) {
+        if (K >= 2048 && gemm_splits_k(M, N, K))
+            return gemm_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
         return gemm_pair_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
+    }
     if (path == 3 || (path == 0 && M >= 512))
         return gemm_ts_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
     return gemm_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);

@@ -37,6 +37,19 @@ constexpr int kExpThreads = 128;
 constexpr uint32_t kTmemCols = 512;
 
 template <int FMT> __host__ __device__ constexpr int packed_bytes_per_kblock() { return BK * Fmt<FMT>::kBits / 8; }
+
+// Split K over a cluster when the tiles leave most SMs idle: the largest C in
+// {2, 4, 8} that keeps every split at least 2 k-blocks deep and the whole grid
+// within one wave; 1 when no split applies.
+inline int splitk_clusters(int64_t M, int64_t N, int64_t K, int64_t sms)
+{
+    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int64_t nkb = (K + BK - 1) / BK;
+    int C = 1;
+    for (int c = 2; c <= 8; c *= 2)
+        if (tiles * c <= sms && nkb >= 2 * c) C = c;
+    return C;
+}
 // Ring depths: TMA stages (activation tile + packed tile) and expanded-tile
 // stages, chosen to fit 227 KB of shared memory with the epilogue staging.
 template <int FMT> __host__ __device__ constexpr int tma_stages() { return FMT == kI4 ? 4 : (FMT == kT2 ? 5 : 6); }
@@ -978,13 +991,7 @@ lowbit_status launch_t(const CUtensorMap &ma, const CUtensorMap &mp, const float
     }
     const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int64_t sms = device_sm_count();
-    const int nkb = static_cast<int>((K + BK - 1) / BK);
-    // Split K over a cluster when the tiles leave most SMs idle: the largest
-    // C in {2, 4, 8} that keeps every split at least 2 k-blocks deep and the
-    // whole grid within one wave.
-    int C = 1;
-    for (int c = 2; c <= 8; c *= 2)
-        if (tiles * c <= sms && nkb >= 2 * c) C = c;
+    const int C = splitk_clusters(M, N, K, sms);
     if (C > 1) {
         static bool configured_split[64] = {};
         if (!configured_split[dev]) {
@@ -1015,6 +1022,11 @@ lowbit_status launch_fmt(const CUtensorMap &ma, const CUtensorMap &mp, const flo
 }
 
 }  // namespace tc
+
+bool gemm_splits_k(int64_t M, int64_t N, int64_t K)
+{
+    return tc::splitk_clusters(M, N, K, device_sm_count()) > 1;
+}
 
 lowbit_status gemm_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
                           const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,

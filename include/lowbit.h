@@ -191,8 +191,10 @@ lowbit_status lowbit_act_quant(const void *x, lowbit_dtype xdt, int64_t M, int64
  * accumulators in tensor memory) with the expanded weight tile in shared
  * memory and K split over a cluster when the output tiles are few; from
  * M = 512 a tcgen05 GEMM on pairs of SMs (cta_group::2, 256 x 256 tiles,
- * expanded weights in shared memory) for ternary weights and the tcgen05
- * GEMM with the weight tile in tensor memory for 4-bit and binary weights. */
+ * expanded weights in shared memory) for ternary weights, except for
+ * K >= 2048 when the shared-memory GEMM would split K (that case keeps it),
+ * and the tcgen05 GEMM with the weight tile in tensor memory for 4-bit and
+ * binary weights. */
 lowbit_status lowbit_linear(const int8_t *q, int64_t ldq, const float *s_x,
                             int64_t M, int64_t K,
                             const uint8_t *packed, int64_t ldp, const float *s_w,
