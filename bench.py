@@ -149,53 +149,30 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
-def dispatched_kernel(M, N, row_bytes, fmt=None):
-    """The kernel lowbit_linear picks (same rule as the library): the
-    packed-weight GEMV up to 4 tokens; warp-level MMAs up to 16 tokens when
-    rows are short or N is large; the tensor-core GEMM with the weight tile
-    expanded into shared memory (cluster split-K when output tiles are few)
-    below 512 tokens; from 512 the SM-pair one for ternary weights and the
-    one with the weight tile in tensor memory for the others."""
-    if M <= 4:
-        return "gemv_smem_kernel"
-    if M <= 16 and (row_bytes <= 512 or N >= 3200):
-        return "skinny_mma_kernel/stream_mma_kernel"
-    if M < 512:
-        return "gemm_kernel/gemm_splitk_kernel"
-    return "gemm_pair_kernel" if fmt == wls.TERNARY2 else "gemm_ts_kernel"
-
-
-def packed_row_bytes(fmt, K):
-    """Bytes of one packed weight row (lowbit_packed_row_bytes)."""
-    if fmt == wls.TERNARY2:
-        return 4 * ((K + 15) // 16)
-    if fmt == wls.BINARY1:
-        return (K + 7) // 8
-    return 4 * ((K + 7) // 8)
-
-
 class Point:
-    def __init__(self, mi, m, M, fmt):
+    def __init__(self, mi, m, M, fmt, sm_count=148):
+        import binary_weight_transformer_b200 as bwt
         self.mi, self.m, self.M = mi, m, M
-        self.kernel = dispatched_kernel(M, m.N, packed_row_bytes(fmt, m.K), fmt)
+        # the kernel lowbit_linear dispatches to, as the library reports it
+        self.kernel = bwt.linear_kernel(M, m.N, m.K, fmt, 0, sm_count)
         # up to 16 tokens the packed weights dominate the bytes: HBM-bound
         self.bound = "hbm" if M <= 16 else "tensor"
         self.ops = 2 * M * m.N * m.K
 
 
-def select_points(wl, only_M=None):
+def select_points(wl, only_M=None, sm_count=148):
     points = []
     for mi, m in enumerate(wl.matrices):
         for M in sorted(wl.Ms, reverse=True):
             if only_M is None or M in only_M:
-                points.append(Point(mi, m, M, wl.fmt))
+                points.append(Point(mi, m, M, wl.fmt, sm_count))
     return points
 
 
 def build_state(wl, device, pool_bytes_target, torch, bwt, only_M=None, pool_copies=None):
     """Pack the weights (off the timed path) into a rotating pool and create
     the activation, code and output buffers."""
-    points = select_points(wl, only_M)
+    points = select_points(wl, only_M, torch.cuda.get_device_properties(device).multi_processor_count)
     packs = []
     for mi, m in enumerate(wl.matrices):
         w = torch.from_numpy(wls.workload_weights(wl, mi)).to(device)

@@ -50,6 +50,8 @@ ABI = {
                                   _P, _P]),
     "lowbit_linear_ex": (_I32, [_P, _I64, _P, _I64, _I64, _P, _I64, _P, _I32, _I64, _P, _I32, _I64, _I32,
                                 ctypes.c_uint, _P, _P]),
+    "lowbit_linear_kernel": (_I32, [_I64, _I64, _I64, _I32, _I32, _I32, _P]),
+    "lowbit_kernel_name": (ctypes.c_char_p, [_I32]),
     "lowbit_status_string": (ctypes.c_char_p, [_I32]),
     "lowbit_version": (_I32, []),
 }
@@ -110,6 +112,14 @@ def scale_count(fmt: int, N: int) -> int:
 
 def max_k(fmt: int) -> int:
     return int(lib().lowbit_max_k(fmt))
+
+
+def linear_kernel(M: int, N: int, K: int, fmt: int, path: int = 0, sm_count: int = 0) -> str:
+    """Name of the kernel lowbit_linear (path 0) or a forced path launches for
+    this problem on a GPU with `sm_count` SMs (0: the current device)."""
+    k = ctypes.c_int(0)
+    _check(lib().lowbit_linear_kernel(M, N, K, fmt, path, sm_count, ctypes.byref(k)), "lowbit_linear_kernel")
+    return lib().lowbit_kernel_name(k.value).decode()
 
 
 def status_flags(status_tensor) -> list[int]:

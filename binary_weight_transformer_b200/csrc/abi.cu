@@ -25,9 +25,9 @@ lowbit_status gemm_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_
                           lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int prefetch,
                           int32_t *status, cudaStream_t st);
 
-// True when the shared-memory GEMM would split K over a cluster (few output
-// tiles, deep K).
-bool gemm_splits_k(int64_t M, int64_t N, int64_t K);
+// True when the shared-memory GEMM would split K over a cluster on a GPU
+// with `sms` SMs (few output tiles, deep K).
+bool gemm_splits_k(int64_t M, int64_t N, int64_t K, int64_t sms);
 
 lowbit_status gemm_ts_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
                              const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
@@ -96,6 +96,48 @@ lowbit_status check_device()
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 bool valid_format(lowbit_format f) { return f == LOWBIT_TERNARY2 || f == LOWBIT_BINARY1 || f == LOWBIT_INT4; }
+
+// The kernel lowbit_linear_path launches for a valid problem; rb = packed
+// row bytes, sms = SMs of the GPU it runs on.
+lowbit_kernel choose_kernel(int64_t M, int64_t N, int64_t K, lowbit_format f, int64_t rb, int path, int64_t sms)
+{
+    // Up to 4 tokens the dp4a GEMV streams weights fastest; from 5 on its
+    // int8 MACs outgrow the CUDA cores and tensor-core MMAs win.
+    if (path == 1 || (path == 0 && M <= 4)) return LOWBIT_KERNEL_GEMV;
+    // 5 to 16 tokens: warp-level tensor-core MMAs on register fragments
+    // where they were measured faster than the split-K GEMM: rows of at most
+    // 512 packed bytes (one round of register loads), or at least 100 blocks
+    // of 32 output rows.  Longer rows with fewer blocks stay on the GEMM.
+    const bool skinny_wins = rb <= 512 || N >= 3200;
+    if (path == 5 || (path == 0 && M <= 16 && skinny_wins)) return LOWBIT_KERNEL_WARP_MMA;
+    if (path == 6) return LOWBIT_KERNEL_GEMM_PAIR;
+    if (path == 4) return LOWBIT_KERNEL_GEMM_TMEM_PAIR;
+    // Below 512 tokens the shared-memory variant, which splits K over a
+    // cluster when tiles are few, wins.  From 512 tokens ternary weights run
+    // on SM pairs with the expanded tile in shared memory (measured fastest
+    // for them), except for deep K (>= 2048) with output tiles too few to
+    // fill the GPU: there the split-K shared-memory kernel stays faster
+    // (9728->2560 at M = 512: 28.6 us vs 32.8 us; for 1024->256 at M = 1024
+    // the pair kernel is ahead, 9.2 us vs 9.6 us).  4-bit and binary weights
+    // take the tensor-memory variant from 512 tokens (the split-K kernel
+    // measured faster for some of their shapes and slower for others).
+    const bool splits = gemm_splits_k(M, N, K, sms);
+    if (path == 0 && M >= 512 && f == LOWBIT_TERNARY2)
+        return (K >= 2048 && splits) ? LOWBIT_KERNEL_GEMM_SPLITK : LOWBIT_KERNEL_GEMM_PAIR;
+    if (path == 3 || (path == 0 && M >= 512)) return LOWBIT_KERNEL_GEMM_TMEM;
+    return splits ? LOWBIT_KERNEL_GEMM_SPLITK : LOWBIT_KERNEL_GEMM;
+}
+
+// Checks shared by lowbit_linear_ex and lowbit_linear_kernel that depend on
+// the problem's shape only.
+lowbit_status check_linear_shape(int64_t M, int64_t N, int64_t K, lowbit_format f, int path)
+{
+    if (!valid_format(f) || path < 0 || path > 6) return LOWBIT_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0 || M > INT32_MAX || N > INT32_MAX) return LOWBIT_ERR_INVALID_ARG;
+    if (path == 5 && M > 16) return LOWBIT_ERR_INVALID_ARG;
+    if (K > lowbit_max_k(f)) return LOWBIT_ERR_OVERFLOW_BOUND;
+    return LOWBIT_OK;
+}
 
 }  // namespace
 
@@ -213,7 +255,8 @@ lowbit_status lowbit_linear_ex(const int8_t *q, int64_t ldq, const float *s_x, i
     if (M > INT32_MAX || N > INT32_MAX) return LOWBIT_ERR_INVALID_ARG;
     const int64_t rb = static_cast<int64_t>(lowbit_packed_row_bytes(f, K));
     if (ldp < rb) return LOWBIT_ERR_INVALID_ARG;
-    if (K > lowbit_max_k(f)) return LOWBIT_ERR_OVERFLOW_BOUND;
+    const lowbit_status shape = check_linear_shape(M, N, K, f, path);
+    if (shape != LOWBIT_OK) return shape;
     const int64_t esz = ydt == LOWBIT_BF16 ? 2 : 4;
     if (!aligned(q, 16) || ldq % 16 != 0 || !aligned(packed, 16) || ldp % 16 != 0 || !aligned(s_x, 4) ||
         !aligned(s_w, 4) || !aligned(y, static_cast<uintptr_t>(esz)))
@@ -221,39 +264,50 @@ lowbit_status lowbit_linear_ex(const int8_t *q, int64_t ldq, const float *s_x, i
     const lowbit_status d = check_device();
     if (d != LOWBIT_OK) return d;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // Up to 4 tokens the dp4a GEMV streams weights fastest; from 5 on its
-    // int8 MACs outgrow the CUDA cores and tensor-core MMAs win.
-    const bool use_gemv = path == 1 || (path == 0 && M <= 4);
-    if (use_gemv) return gemv_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, st);
-    // 5 to 16 tokens: warp-level tensor-core MMAs on register fragments
-    // where they were measured faster than the split-K GEMM: rows of at most
-    // 512 packed bytes (one round of register loads), or at least 100 blocks
-    // of 32 output rows.  Longer rows with fewer blocks stay on the GEMM.
-    const bool skinny_wins = rb <= 512 || N >= 3200;
-    if (path == 5 || (path == 0 && M <= 16 && skinny_wins))
+    switch (choose_kernel(M, N, K, f, rb, path, device_sm_count())) {
+    case LOWBIT_KERNEL_GEMV:
+        return gemv_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, st);
+    case LOWBIT_KERNEL_WARP_MMA:
         return skinny_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
-    // Below 512 tokens the shared-memory variant, which splits K over a
-    // cluster when tiles are few, wins.
-    if (path == 6)
+    case LOWBIT_KERNEL_GEMM_PAIR:
         return gemm_pair_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
-    if (path == 4)
+    case LOWBIT_KERNEL_GEMM_TMEM_PAIR:
         return gemm_ts_pair_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, status_dev, st);
-    // From 512 tokens ternary weights run on SM pairs with the expanded tile
-    // in shared memory (measured fastest for them), except for deep K
-    // (>= 2048) with output tiles too few to fill the GPU: there the split-K
-    // shared-memory kernel stays faster (9728->2560 at M = 512: 28.6 us vs
-    // 32.8 us; for 1024->256 at M = 1024 the pair kernel is ahead, 9.2 us vs
-    // 9.6 us).  4-bit and binary weights take the tensor-memory variant from
-    // 512 tokens (the split-K kernel measured faster for some of their shapes
-    // and slower for others).
-    if (path == 0 && M >= 512 && f == LOWBIT_TERNARY2) {
-        if (K >= 2048 && gemm_splits_k(M, N, K))
-            return gemm_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
-        return gemm_pair_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
-    }
-    if (path == 3 || (path == 0 && M >= 512))
+    case LOWBIT_KERNEL_GEMM_TMEM:
         return gemm_ts_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
-    return gemm_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
+    default:  // LOWBIT_KERNEL_GEMM or LOWBIT_KERNEL_GEMM_SPLITK: the launcher splits by the same rule
+        return gemm_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
+    }
+}
+
+lowbit_status lowbit_linear_kernel(int64_t M, int64_t N, int64_t K, lowbit_format f, int path, int sm_count,
+                                   lowbit_kernel *kernel)
+{
+    if (kernel == nullptr) return LOWBIT_ERR_INVALID_ARG;
+    const lowbit_status shape = check_linear_shape(M, N, K, f, path);
+    if (shape != LOWBIT_OK) return shape;
+    int64_t sms = sm_count;
+    if (sms <= 0) {
+        const lowbit_status d = check_device();
+        if (d != LOWBIT_OK) return d;
+        sms = device_sm_count();
+    }
+    *kernel = choose_kernel(M, N, K, f, static_cast<int64_t>(lowbit_packed_row_bytes(f, K)), path, sms);
+    return LOWBIT_OK;
+}
+
+const char *lowbit_kernel_name(lowbit_kernel k)
+{
+    switch (k) {
+    case LOWBIT_KERNEL_GEMV: return "gemv_smem_kernel/gemv_kernel";
+    case LOWBIT_KERNEL_WARP_MMA: return "skinny_mma_kernel/stream_mma_kernel";
+    case LOWBIT_KERNEL_GEMM: return "gemm_kernel";
+    case LOWBIT_KERNEL_GEMM_SPLITK: return "gemm_splitk_kernel";
+    case LOWBIT_KERNEL_GEMM_PAIR: return "gemm_pair_kernel";
+    case LOWBIT_KERNEL_GEMM_TMEM: return "gemm_ts_kernel";
+    case LOWBIT_KERNEL_GEMM_TMEM_PAIR: return "gemm_ts_pair_kernel";
+    default: return "unknown";
+    }
 }
 
 lowbit_status lowbit_linear_path(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,

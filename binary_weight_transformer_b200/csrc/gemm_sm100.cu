@@ -1023,9 +1023,9 @@ lowbit_status launch_fmt(const CUtensorMap &ma, const CUtensorMap &mp, const flo
 
 }  // namespace tc
 
-bool gemm_splits_k(int64_t M, int64_t N, int64_t K)
+bool gemm_splits_k(int64_t M, int64_t N, int64_t K, int64_t sms)
 {
-    return tc::splitk_clusters(M, N, K, device_sm_count()) > 1;
+    return tc::splitk_clusters(M, N, K, sms) > 1;
 }
 
 lowbit_status gemm_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,

@@ -242,6 +242,33 @@ lowbit_status lowbit_linear_ex(const int8_t *q, int64_t ldq, const float *s_x,
                                int path, unsigned flags,
                                int32_t *status_dev, void *stream);
 
+/* The kernels lowbit_linear_path can launch. */
+typedef enum {
+    LOWBIT_KERNEL_GEMV = 1,           /* packed-weight GEMV (dp4a), groups of up to 4 tokens */
+    LOWBIT_KERNEL_WARP_MMA = 2,       /* warp-level mma.sync on register weight fragments */
+    LOWBIT_KERNEL_GEMM = 3,           /* tcgen05 GEMM, expanded weight tile in shared memory */
+    LOWBIT_KERNEL_GEMM_SPLITK = 4,    /* the same with K split over a cluster of 2, 4 or 8 CTAs */
+    LOWBIT_KERNEL_GEMM_PAIR = 5,      /* tcgen05 GEMM on SM pairs, tile in shared memory */
+    LOWBIT_KERNEL_GEMM_TMEM = 6,      /* tcgen05 GEMM, expanded weight tile in tensor memory */
+    LOWBIT_KERNEL_GEMM_TMEM_PAIR = 7  /* the same on SM pairs */
+} lowbit_kernel;
+
+/* The kernel lowbit_linear_path(..., path, ...) launches for an M x K by
+ * K -> N problem in format f, on a GPU with sm_count SMs (sm_count <= 0: the
+ * current device, which must be a B200).  Host only: no launch and no device
+ * memory, so with sm_count > 0 it needs no GPU.  Writes *kernel and returns
+ * LOWBIT_OK; returns the status lowbit_linear_path would return for the
+ * shape (LOWBIT_ERR_INVALID_ARG for M, N or K <= 0, a path outside 0..6, path
+ * 5 with M > 16 or a null kernel; LOWBIT_ERR_OVERFLOW_BOUND for K above
+ * lowbit_max_k), or LOWBIT_ERR_CUDA / LOWBIT_ERR_UNSUPPORTED when sm_count <= 0
+ * and the device cannot be queried or is not a B200. */
+lowbit_status lowbit_linear_kernel(int64_t M, int64_t N, int64_t K, lowbit_format f, int path,
+                                   int sm_count, lowbit_kernel *kernel);
+
+/* Name of the kernel function(s) behind a lowbit_kernel value, as in a
+ * profiler's launch list (static string; "unknown" for other values). */
+const char *lowbit_kernel_name(lowbit_kernel k);
+
 /* Human-readable name of a status value (static string). */
 const char *lowbit_status_string(lowbit_status s);
 

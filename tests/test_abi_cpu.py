@@ -66,6 +66,60 @@ def _linear(lib, **kw):
                                   a["fmt"], a["N"], a["y"], a["ydt"], a["ldy"], a["path"], None, None)
 
 
+# (M, N, K, format, path, SMs) -> kernel, worked out by hand from the
+# dispatch rules (tiles of 128 tokens x 256 features, K blocks of 128):
+# GEMV up to 4 tokens; warp MMAs up to 16 when a packed row is <= 512 bytes
+# or N >= 3200; the shared-memory GEMM below 512 tokens, split over a cluster
+# of C in {2, 4, 8} when tiles * C fits the SMs and every split keeps 2 K
+# blocks; from 512, SM pairs for ternary weights (split-K kept when K >= 2048
+# and the GEMM splits) and the tensor-memory GEMM for the other formats.
+DISPATCH = [
+    ((1, 9728, 2560, bwt.TERNARY2, 0, 148), "gemv_smem_kernel/gemv_kernel"),
+    ((4, 9728, 2560, bwt.TERNARY2, 0, 148), "gemv_smem_kernel/gemv_kernel"),
+    ((16, 9728, 2560, bwt.TERNARY2, 0, 148), "skinny_mma_kernel/stream_mma_kernel"),  # N >= 3200
+    ((8, 192, 768, bwt.BINARY1, 0, 148), "skinny_mma_kernel/stream_mma_kernel"),      # 96-byte rows
+    ((16, 2560, 9728, bwt.TERNARY2, 0, 148), "gemm_splitk_kernel"),  # 2432-byte rows, 10 tiles, C = 8
+    ((128, 9728, 2560, bwt.TERNARY2, 0, 148), "gemm_splitk_kernel"),  # 38 tiles, C = 2
+    ((256, 768, 192, bwt.TERNARY2, 0, 148), "gemm_kernel"),  # 2 K blocks: no split
+    ((300, 9728, 2560, bwt.TERNARY2, 0, 148), "gemm_kernel"),  # 114 tiles: no split
+    ((8192, 9728, 2560, bwt.TERNARY2, 0, 148), "gemm_pair_kernel"),
+    ((1024, 2560, 9728, bwt.TERNARY2, 0, 148), "gemm_pair_kernel"),  # 80 tiles: no split
+    ((512, 2560, 9728, bwt.TERNARY2, 0, 148), "gemm_splitk_kernel"),  # 40 tiles, C = 2, deep K
+    ((512, 2560, 9728, bwt.TERNARY2, 0, 64), "gemm_pair_kernel"),    # 40 x 2 > 64 SMs: no split
+    ((1024, 256, 1024, bwt.TERNARY2, 0, 148), "gemm_pair_kernel"),   # splits, but K < 2048
+    ((8192, 1280, 3584, bwt.INT4, 0, 148), "gemm_ts_kernel"),
+    ((512, 1280, 3584, bwt.INT4, 0, 148), "gemm_ts_kernel"),  # splits, but not ternary
+    ((16384, 192, 768, bwt.BINARY1, 0, 148), "gemm_ts_kernel"),
+    # forced paths
+    ((300, 9728, 2560, bwt.TERNARY2, 1, 148), "gemv_smem_kernel/gemv_kernel"),
+    ((8192, 9728, 2560, bwt.TERNARY2, 2, 148), "gemm_kernel"),
+    ((2, 2560, 9728, bwt.TERNARY2, 2, 148), "gemm_splitk_kernel"),
+    ((1, 9728, 2560, bwt.INT4, 3, 148), "gemm_ts_kernel"),
+    ((64, 9728, 2560, bwt.BINARY1, 4, 148), "gemm_ts_pair_kernel"),
+    ((16, 2560, 9728, bwt.TERNARY2, 5, 148), "skinny_mma_kernel/stream_mma_kernel"),
+    ((1, 9728, 2560, bwt.TERNARY2, 6, 148), "gemm_pair_kernel"),
+]
+
+
+@pytest.mark.parametrize("args,name", DISPATCH)
+def test_linear_kernel_dispatch(lib, args, name):
+    assert bwt.linear_kernel(*args) == name
+
+
+def test_linear_kernel_rejects_bad_arguments(lib):
+    k = ctypes.c_int(0)
+    q = lib.lowbit_linear_kernel
+    assert q(16, 256, 256, bwt.TERNARY2, 7, 148, ctypes.byref(k)) == bwt.ERR_INVALID_ARG   # path
+    assert q(17, 256, 256, bwt.TERNARY2, 5, 148, ctypes.byref(k)) == bwt.ERR_INVALID_ARG   # path 5, M > 16
+    assert q(0, 256, 256, bwt.TERNARY2, 0, 148, ctypes.byref(k)) == bwt.ERR_INVALID_ARG
+    assert q(16, 256, 0, bwt.TERNARY2, 0, 148, ctypes.byref(k)) == bwt.ERR_INVALID_ARG
+    assert q(16, 256, 256, 3, 0, 148, ctypes.byref(k)) == bwt.ERR_INVALID_ARG             # format
+    assert q(16, 256, 256, bwt.TERNARY2, 0, 148, None) == bwt.ERR_INVALID_ARG
+    big = bwt.max_k(bwt.INT4) + 1
+    assert q(16, 256, big, bwt.INT4, 0, 148, ctypes.byref(k)) == bwt.ERR_OVERFLOW_BOUND
+    assert lib.lowbit_kernel_name(0) == b"unknown"
+
+
 def test_linear_rejects_bad_arguments(lib):
     assert _linear(lib, q=None) == bwt.ERR_INVALID_ARG
     assert _linear(lib, M=0) == bwt.ERR_INVALID_ARG
