@@ -346,6 +346,64 @@ def test_act_quant_bf16_equals_widened_f32():
     assert np.array_equal(q1, q2) and np.array_equal(s1, s2)
 
 
+@pytest.mark.parametrize("k", [-80, -40, 40, 80])
+def test_act_quant_power_of_two_scale_invariance(k):
+    # Multiplying a row by 2^k is exact while every value stays normal, and
+    # both the product by 127 and the division by the row max commute with
+    # it, so the codes must not change and s_x must scale by 2^k.  Rows far
+    # from 1 in magnitude are where a reciprocal of the max over- or
+    # underflows.
+    x = wls.normal_activations(53, 16, 300, 0.01, 8.0)
+    x = x[np.all(np.abs(x) > 1e-6, axis=1)]
+    xs = (x.astype(np.float64) * 2.0 ** k).astype(np.float32)
+    assert np.all(np.abs(xs) >= np.finfo(np.float32).tiny) and np.all(np.isfinite(xs * np.float32(127)))
+    q1, s1 = oracle.act_quant(x)
+    q2, s2 = oracle.act_quant(xs)
+    assert np.array_equal(q1, q2)
+    assert np.array_equal(s2.astype(np.float64), s1.astype(np.float64) * 2.0 ** k)
+
+
+def _round_f32(r):
+    """Nearest binary32 value to the rational r >= 0, ties to even, with
+    subnormals (from the IEEE 754 definition, in exact arithmetic)."""
+    from fractions import Fraction
+    if r == 0:
+        return Fraction(0)
+    e = r.numerator.bit_length() - r.denominator.bit_length()
+    if Fraction(2) ** e > r:
+        e -= 1
+    quantum = Fraction(2) ** (max(e, -126) - 23)
+    n, rem = divmod(r, quantum)
+    if rem * 2 > quantum or (rem * 2 == quantum and n % 2 == 1):
+        n += 1
+    return n * quantum
+
+
+def test_act_quant_subnormal_rows_exact():
+    # Rows whose values are subnormal or near the smallest normal: codes
+    # computed in exact rational arithmetic with explicit binary32 rounding
+    # of 127x and of the quotient, then rounding half to even.
+    from fractions import Fraction
+    rng = np.random.default_rng(54)
+    rows = [rng.standard_normal(64) * 10.0 ** e for e in (-44, -42, -40, -39, -38, -37)]
+    x = np.array(rows).astype(np.float32)
+    q, s_x = oracle.act_quant(x)
+    for t in range(x.shape[0]):
+        vals = [Fraction(float(v)) for v in x[t]]
+        g = max(abs(v) for v in vals)
+        if g == 0:
+            assert not q[t].any() and s_x[t] == 0
+            continue
+        for kk, v in enumerate(vals):
+            sign = -1 if v < 0 else 1
+            z = _round_f32(_round_f32(127 * abs(v)) / g)  # |RN(RN(127x)/g)|
+            n, rem = divmod(z, 1)
+            if rem * 2 > 1 or (rem * 2 == 1 and n % 2 == 1):
+                n += 1
+            assert q[t, kk] == sign * min(int(n), 127), (t, kk)
+        assert Fraction(float(s_x[t])) == _round_f32(g / 127)
+
+
 def test_act_quant_rejects_nonfinite():
     x = np.ones((2, 8), np.float32)
     x[1, 3] = np.inf
