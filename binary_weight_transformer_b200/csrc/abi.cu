@@ -63,31 +63,33 @@ struct DeviceInfo {
     bool ok = false;
 };
 
-const DeviceInfo &device_info()
+// Queried once per device; SM count and compute capability are published
+// together as one int (SMs in the low 16 bits, major and minor above).
+DeviceInfo device_info()
 {
-    static DeviceInfo cache[64];
+    static PerDevice cache;
+    DeviceInfo d;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
-        static DeviceInfo none;
-        return none;
-    }
-    DeviceInfo &d = cache[dev];
-    if (!d.ok) {
+    if (cudaGetDevice(&dev) != cudaSuccess) return d;
+    const int packed = cache.get(dev, [&] {
         cudaDeviceProp p;
-        if (cudaGetDeviceProperties(&p, dev) == cudaSuccess) {
-            d.sms = p.multiProcessorCount;
-            d.major = p.major;
-            d.minor = p.minor;
-            d.ok = true;
-        }
-    }
+        if (cudaGetDeviceProperties(&p, dev) != cudaSuccess || p.multiProcessorCount <= 0 ||
+            p.multiProcessorCount > 0xffff || p.major < 0 || p.major > 0x7f || p.minor < 0 || p.minor > 0xff)
+            return 0;
+        return p.multiProcessorCount | (p.minor << 16) | (p.major << 24);
+    });
+    if (packed <= 0) return d;
+    d.sms = packed & 0xffff;
+    d.minor = (packed >> 16) & 0xff;
+    d.major = (packed >> 24) & 0x7f;
+    d.ok = true;
     return d;
 }
 
 // The kernels are built for sm_100a only.
 lowbit_status check_device()
 {
-    const DeviceInfo &d = device_info();
+    const DeviceInfo d = device_info();
     if (!d.ok) return LOWBIT_ERR_CUDA;
     if (d.major != 10 || d.minor != 0) return LOWBIT_ERR_UNSUPPORTED;
     return LOWBIT_OK;
@@ -143,7 +145,7 @@ lowbit_status check_linear_shape(int64_t M, int64_t N, int64_t K, lowbit_format 
 
 int device_sm_count()
 {
-    const DeviceInfo &d = device_info();
+    const DeviceInfo d = device_info();
     return d.ok ? d.sms : 148;
 }
 

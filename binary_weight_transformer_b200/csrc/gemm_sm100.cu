@@ -936,24 +936,25 @@ lowbit_status launch_pair_t(const CUtensorMap &ma, const CUtensorMap &mp, const 
 {
     constexpr size_t smem = pair_smem_bytes<FMT, OUT>();
     static_assert(smem <= 232448, "shared memory budget");
-    static int max_pairs[64] = {};
+    // Pairs that can be resident at once, found (with the shared-memory
+    // attribute set) on the first launch on each device.
+    static PerDevice max_pairs;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LOWBIT_ERR_CUDA;
-    if (max_pairs[dev] == 0) {
+    if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    const int resident = max_pairs.get(dev, [&] {
         if (cudaFuncSetAttribute(gemm_pair_kernel<FMT, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem)) != cudaSuccess)
-            return LOWBIT_ERR_CUDA;
+            return 0;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * static_cast<unsigned>(device_sm_count() / 2));
         cfg.blockDim = dim3(kThreads);
         cfg.dynamicSmemBytes = smem;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<FMT, OUT>, &cfg) != cudaSuccess || n <= 0)
-            return LOWBIT_ERR_CUDA;
-        max_pairs[dev] = n;
-    }
+        return cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<FMT, OUT>, &cfg) == cudaSuccess ? n : 0;
+    });
+    if (resident <= 0) return LOWBIT_ERR_CUDA;
     const int64_t tiles = ((M + 2 * PBM - 1) / (2 * PBM)) * ((N + 2 * PBN - 1) / (2 * PBN));
-    const int64_t pairs = tiles < max_pairs[dev] ? tiles : max_pairs[dev];
+    const int64_t pairs = tiles < resident ? tiles : resident;
     return launch_pdl(gemm_pair_kernel<FMT, OUT>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kThreads), smem, st,
                       0, ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status);
 }
@@ -980,26 +981,24 @@ lowbit_status launch_t(const CUtensorMap &ma, const CUtensorMap &mp, const float
 {
     constexpr size_t smem = smem_bytes<FMT, OUT>();
     static_assert(smem <= 232448, "shared memory budget");
-    static bool configured[64] = {};  // the attribute is set once per device
+    static PerDevice configured;  // the attribute is set once per device
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LOWBIT_ERR_CUDA;
-    if (!configured[dev]) {
-        if (cudaFuncSetAttribute(gemm_kernel<FMT, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem)) != cudaSuccess)
-            return LOWBIT_ERR_CUDA;
-        configured[dev] = true;
-    }
+    if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    if (configured.get(dev, [&] {
+            return cudaFuncSetAttribute(gemm_kernel<FMT, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(smem)) == cudaSuccess ? 1 : 0;
+        }) <= 0)
+        return LOWBIT_ERR_CUDA;
     const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int64_t sms = device_sm_count();
     const int C = splitk_clusters(M, N, K, sms);
     if (C > 1) {
-        static bool configured_split[64] = {};
-        if (!configured_split[dev]) {
-            if (cudaFuncSetAttribute(gemm_splitk_kernel<FMT, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(smem)) != cudaSuccess)
-                return LOWBIT_ERR_CUDA;
-            configured_split[dev] = true;
-        }
+        static PerDevice configured_split;
+        if (configured_split.get(dev, [&] {
+                return cudaFuncSetAttribute(gemm_splitk_kernel<FMT, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            static_cast<int>(smem)) == cudaSuccess ? 1 : 0;
+            }) <= 0)
+            return LOWBIT_ERR_CUDA;
         return launch_pdl(gemm_splitk_kernel<FMT, OUT>, dim3(static_cast<unsigned>(tiles * C)), dim3(kThreads), smem,
                           st, static_cast<unsigned>(C), ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, C, prefetch,
                           status);

@@ -408,15 +408,14 @@ lowbit_status launch_t(const CUtensorMap &mq, const CUtensorMap &mp, const float
 {
     constexpr size_t smem = smem_bytes<FMT, OUT>();
     static_assert(smem <= 232448, "shared memory budget");
-    static bool configured[64] = {};
+    static PerDevice configured;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LOWBIT_ERR_CUDA;
-    if (!configured[dev]) {
-        if (cudaFuncSetAttribute(gemm_ts_kernel<FMT, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem)) != cudaSuccess)
-            return LOWBIT_ERR_CUDA;
-        configured[dev] = true;
-    }
+    if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    if (configured.get(dev, [&] {
+            return cudaFuncSetAttribute(gemm_ts_kernel<FMT, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(smem)) == cudaSuccess ? 1 : 0;
+        }) <= 0)
+        return LOWBIT_ERR_CUDA;
     const int64_t tiles = ((N + BW - 1) / BW) * ((M + nt - 1) / nt);
     const int64_t sms = device_sm_count();
     const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
@@ -709,27 +708,27 @@ lowbit_status launch_pair_t(const CUtensorMap &mq, const CUtensorMap &mp, const 
 {
     constexpr size_t smem = smem_bytes_pair<FMT, OUT>();
     static_assert(smem <= 232448, "shared memory budget");
-    static int max_pairs[64] = {};
+    static PerDevice max_pairs;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LOWBIT_ERR_CUDA;
-    cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    if (max_pairs[dev] == 0) {
+    if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    // Pairs that can be resident at once (the GPCs decide how many SM pairs
+    // exist), found with the shared-memory attribute set on the first launch
+    // on each device; the persistent grid never exceeds it.
+    const int resident = max_pairs.get(dev, [&] {
         if (cudaFuncSetAttribute(gemm_ts_pair_kernel<FMT, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem)) != cudaSuccess)
-            return LOWBIT_ERR_CUDA;
-        // Pairs that can be resident at once (the GPCs decide how many SM
-        // pairs exist); the persistent grid never exceeds it.
+            return 0;
+        cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * static_cast<unsigned>(device_sm_count() / 2));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, gemm_ts_pair_kernel<FMT, OUT>, &cfg) != cudaSuccess || n <= 0)
-            return LOWBIT_ERR_CUDA;
-        max_pairs[dev] = n;
-    }
+        return cudaOccupancyMaxActiveClusters(&n, gemm_ts_pair_kernel<FMT, OUT>, &cfg) == cudaSuccess ? n : 0;
+    });
+    if (resident <= 0) return LOWBIT_ERR_CUDA;
     const int64_t tiles = ((N + 2 * BW - 1) / (2 * BW)) * ((M + nt - 1) / nt);
-    const int64_t pairs = tiles < max_pairs[dev] ? tiles : max_pairs[dev];
+    const int64_t pairs = tiles < resident ? tiles : resident;
     return launch_pdl(gemm_ts_pair_kernel<FMT, OUT>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kThreads), smem,
                       st, 0, mq, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, nt, status);
 }

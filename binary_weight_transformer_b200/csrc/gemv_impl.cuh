@@ -293,20 +293,19 @@ lowbit_status launch_smem(const int8_t *q, int64_t ldq, const float *s_x, int M,
                           int64_t ldp, int64_t nchunks, const float *s_w, int64_t N, void *y, lowbit_dtype ydt,
                           int64_t ldy, size_t smem, int prefetch, cudaStream_t st)
 {
-    static bool configured[64] = {};
+    static PerDevice configured;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LOWBIT_ERR_CUDA;
-    if (!configured[dev]) {
-        const int lim = static_cast<int>(kGemvSmemMax);
-        if (cudaFuncSetAttribute(gemv_smem_kernel<FMT, MT, U, R, LOWBIT_F32>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, lim) != cudaSuccess ||
-            cudaFuncSetAttribute(gemv_smem_kernel<FMT, MT, U, R, LOWBIT_BF16>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, lim) != cudaSuccess ||
-            cudaFuncSetAttribute(gemv_smem_kernel<FMT, MT, U, R, LOWBIT_I32>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, lim) != cudaSuccess)
-            return LOWBIT_ERR_CUDA;
-        configured[dev] = true;
-    }
+    if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    if (configured.get(dev, [&] {
+            const int lim = static_cast<int>(kGemvSmemMax);
+            return (cudaFuncSetAttribute(gemv_smem_kernel<FMT, MT, U, R, LOWBIT_F32>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, lim) == cudaSuccess &&
+                    cudaFuncSetAttribute(gemv_smem_kernel<FMT, MT, U, R, LOWBIT_BF16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, lim) == cudaSuccess &&
+                    cudaFuncSetAttribute(gemv_smem_kernel<FMT, MT, U, R, LOWBIT_I32>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, lim) == cudaSuccess) ? 1 : 0;
+        }) <= 0)
+        return LOWBIT_ERR_CUDA;
     const int64_t blocks = (N + kWarps * R - 1) / (kWarps * R);
     const dim3 g(static_cast<unsigned>(blocks)), b(kWarps * 32);
     if (ydt == LOWBIT_F32)

@@ -16,6 +16,7 @@
 #include <cuda_bf16.h>
 
 #include "lowbit.h"
+#include "host_once.h"
 
 namespace lowbit {
 

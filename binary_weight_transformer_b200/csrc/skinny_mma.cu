@@ -385,17 +385,16 @@ lowbit_status launch_stream(const CUtensorMap &mp, const int8_t *q, int64_t ldq,
                             int32_t *status, cudaStream_t st)
 {
     constexpr size_t smem = 1024 + static_cast<size_t>(kSStages) * kSStageBytes;
-    static bool configured[64] = {};
+    static PerDevice configured;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LOWBIT_ERR_CUDA;
-    if (!configured[dev]) {
-        if (cudaFuncSetAttribute(stream_mma_kernel<FMT, OUT, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem)) != cudaSuccess ||
-            cudaFuncSetAttribute(stream_mma_kernel<FMT, OUT, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem)) != cudaSuccess)
-            return LOWBIT_ERR_CUDA;
-        configured[dev] = true;
-    }
+    if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    if (configured.get(dev, [&] {
+            return (cudaFuncSetAttribute(stream_mma_kernel<FMT, OUT, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem)) == cudaSuccess &&
+                    cudaFuncSetAttribute(stream_mma_kernel<FMT, OUT, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem)) == cudaSuccess) ? 1 : 0;
+        }) <= 0)
+        return LOWBIT_ERR_CUDA;
     const dim3 grid(static_cast<unsigned>((N + kSRows - 1) / kSRows)), block((kSConsumers + 1) * 32);
     if (M <= 8)
         return launch_pdl(stream_mma_kernel<FMT, OUT, 1>, grid, block, smem, st, 0, mp, q, ldq, s_x, M, K, s_w, N, y,
