@@ -368,8 +368,7 @@ def run_gpu_arm(args, wl):
         "vs_baseline": None,
         "dtype": "int8 x ternary -> int32 (bf16 in/out)" if wl.fmt == wls.TERNARY2 else "int8 x low-bit -> int32",
         "data": "synthetic (seeded N(0,1) activations with outliers, N(0,0.02) weights)",
-        "config": {"workload": f"{wl.name}: " + ", ".join(f"{m.K}->{m.N}" for m in wl.matrices)
-                   + f" x M in {sorted(set(pt.M for pt in points), reverse=True)}",
+        "config": {"workload": workload_name(wl, [pt.M for pt in points]),
                    "timing": "each timed step is a CUDA graph replay; per-kernel times from graphs of back-to-back "
                              "launches of one kernel (rotating weights), events around the replay",
                    "parallelism": f"replicas x{world} (token batches, no collective)",
@@ -461,6 +460,12 @@ def run_e2e(args, wl, points, pool, qs, sxs, ys, torch, bwt, stream, ydt):
 # ---------------------------------------------------------------------------
 # the oracle on the host cores
 # ---------------------------------------------------------------------------
+def workload_name(wl, Ms):
+    """The workload as both arms report it: matrices and token counts."""
+    return (f"{wl.name}: " + ", ".join(f"{m.K}->{m.N}" for m in wl.matrices)
+            + f" x M in {sorted(set(Ms), reverse=True)}")
+
+
 def oracle_sample_step(wl, rows_per_point, nthreads, cache):
     """One bounded step of the oracle: act quant -> add/sub/skip dot ->
     rescale for every point of the sweep, on the first `rows_per_point`
@@ -536,7 +541,10 @@ def run_reference_arm(args, wl):
         "value": round(value, 6), "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt / args.steps * 1e3, 2), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int64 (oracle)", "data": "synthetic",
-        "config": {"workload": f"{wl.name} (bounded sample)"},
+        "config": {"workload": workload_name(wl, wl.Ms),
+                   "timing": f"host wall clock; each step a bounded sample (the first {rows} token rows of "
+                             "every point)",
+                   "parallelism": f"oracle on {nthreads} host threads"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": nthreads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
