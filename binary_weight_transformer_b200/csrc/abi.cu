@@ -210,6 +210,7 @@ lowbit_status lowbit_pack(const float *w, int64_t N, int64_t K, int64_t ldw, low
     if (need > 0 && !aligned(workspace, 8)) return LOWBIT_ERR_ALIGNMENT;
     const lowbit_status d = check_device();
     if (d != LOWBIT_OK) return d;
+    const TraceRange trace("lowbit_pack");
     return pack_launch(w, N, K, ldw, f, eps, packed, ldp, s_w, workspace, status_dev,
                        static_cast<cudaStream_t>(stream));
 }
@@ -223,6 +224,7 @@ lowbit_status lowbit_unpack(const uint8_t *packed, int64_t ldp, int64_t N, int64
     if (ldp % 16 != 0 || !aligned(packed, 16)) return LOWBIT_ERR_ALIGNMENT;
     const lowbit_status d = check_device();
     if (d != LOWBIT_OK) return d;
+    const TraceRange trace("lowbit_unpack");
     return unpack_launch(packed, ldp, N, K, f, codes, ldc, status_dev, static_cast<cudaStream_t>(stream));
 }
 
@@ -238,6 +240,7 @@ lowbit_status lowbit_act_quant(const void *x, lowbit_dtype xdt, int64_t M, int64
         return LOWBIT_ERR_ALIGNMENT;
     const lowbit_status d = check_device();
     if (d != LOWBIT_OK) return d;
+    const TraceRange trace("lowbit_act_quant");
     return act_quant_launch(x, xdt, M, K, ldx, eps, q, ldq, s_x, status_dev, static_cast<cudaStream_t>(stream));
 }
 
@@ -266,6 +269,7 @@ lowbit_status lowbit_linear_ex(const int8_t *q, int64_t ldq, const float *s_x, i
     const lowbit_status d = check_device();
     if (d != LOWBIT_OK) return d;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const TraceRange trace("lowbit_linear");
     switch (choose_kernel(M, N, K, f, rb, path, device_sm_count())) {
     case LOWBIT_KERNEL_GEMV:
         return gemv_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, st);

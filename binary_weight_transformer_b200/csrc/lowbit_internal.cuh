@@ -14,11 +14,22 @@
 #include <utility>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "lowbit.h"
 #include "host_once.h"
 
 namespace lowbit {
+
+// A named range on the NVTX timeline (Nsight Systems, ncu's NVTX filters)
+// around the launches of one ABI call.  With no tool attached the push and
+// the pop return at once.
+struct TraceRange {
+    explicit TraceRange(const char *name) { nvtxRangePushA(name); }
+    ~TraceRange() { nvtxRangePop(); }
+    TraceRange(const TraceRange &) = delete;
+    TraceRange &operator=(const TraceRange &) = delete;
+};
 
 constexpr int kT2 = LOWBIT_TERNARY2;
 constexpr int kB1 = LOWBIT_BINARY1;

@@ -303,6 +303,7 @@ extern "C" lowbit_status lowbit_pack_ternary_noalloc(const float *w, int64_t N, 
     // Every row sum the call reads (rows 0..N-1) is written earlier in the
     // same call, so nothing left by a previous call is ever read and the
     // array needs no clearing.
+    const TraceRange trace("lowbit_pack_ternary_noalloc");
     return pack_launch(w, N, K, ldw, LOWBIT_TERNARY2, eps, packed, ldp, s_w, rows, status_dev,
                        static_cast<cudaStream_t>(stream));
 }
