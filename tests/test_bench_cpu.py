@@ -36,3 +36,32 @@ def test_reference_arm_is_silent_on_other_ranks():
     r = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert not [l for l in r.stdout.splitlines() if l.startswith("{")]
+
+
+def test_profiled_traffic_needs_the_captured_source(tmp_path, monkeypatch):
+    # The roofline's DRAM traffic comes from a committed ncu summary and is
+    # reported only while the kernel source still has the hash recorded there.
+    import hashlib
+    sys.path.insert(0, ROOT)
+    import bench
+    src_dir = tmp_path / "binary_weight_transformer_b200" / "csrc"
+    src_dir.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    src = src_dir / "kernel.cu"
+    src.write_bytes(b"// kernel v1\n")
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    (tmp_path / "profiles" / "k.md").write_text(
+        f"source: binary_weight_transformer_b200/csrc/kernel.cu sha256 prefix {sha}\n\n"
+        "| traffic_bytes_per_launch: 140271360 |\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("k.md", "kernel.cu") == 140271360
+    src.write_bytes(b"// kernel v2\n")
+    assert bench.profiled_traffic("k.md", "kernel.cu") is None
+    assert bench.profiled_traffic("missing.md", "kernel.cu") is None
+
+
+def test_committed_roofline_profile_matches_its_source():
+    # The summary the bench's roofline uses must describe the committed kernel.
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.profiled_traffic("gemm_pair_kernel_ternary_4b_M8192.md", "gemm_sm100.cu") == 140271360
