@@ -256,7 +256,9 @@ typedef enum {
 /* The kernel lowbit_linear_path(..., path, ...) launches for an M x K by
  * K -> N problem in format f, on a GPU with sm_count SMs (sm_count <= 0: the
  * current device, which must be a B200).  Host only: no launch and no device
- * memory, so with sm_count > 0 it needs no GPU.  Writes *kernel and returns
+ * memory, so with sm_count > 0 it needs no GPU.  `kernel` is a HOST pointer
+ * (the one exception to the device-pointer convention above).  Writes *kernel
+ * and returns
  * LOWBIT_OK; returns the status lowbit_linear_path would return for the
  * shape (LOWBIT_ERR_INVALID_ARG for M, N or K <= 0, a path outside 0..6, path
  * 5 with M > 16 or a null kernel; LOWBIT_ERR_OVERFLOW_BOUND for K above
