@@ -232,6 +232,34 @@ def test_int4_matches_float64_pipeline_away_from_ties():
 # packing invariants
 # --------------------------------------------------------------------------
 
+@pytest.mark.parametrize("fmt", [oracle.TERNARY2, oracle.INT4])
+def test_codes_are_odd_in_the_weights(fmt):
+    # Every step of the ternary and 4-bit quantisers is odd or even in w:
+    # mean|W| and max|3 tanh(w/3)| do not see the sign, tanh is odd, and
+    # rounding half to even and the clip are symmetric about 0.  So negating
+    # the weights negates the codes and keeps the scales, bit for bit.  A
+    # floor-style rounding or a one-sided clip breaks this.
+    w = wls.normal_weights(120 + fmt, 33, 257)
+    w[0, :8] = [0.0, -0.0, 1e-30, -1e-30, 0.02, -0.02, 0.5, -0.5]
+    c1, s1 = oracle.quantize(w, fmt)
+    c2, s2 = oracle.quantize(-w, fmt)
+    assert np.array_equal(c2, -c1)
+    assert np.array_equal(np.asarray(s1).view(np.uint32), np.asarray(s2).view(np.uint32))
+
+
+def test_binary_codes_flip_with_the_weights_except_at_zero():
+    # The binary rule is +1 for w >= 0: negation flips every code except at
+    # a zero weight (both signed zeros stay +1); the row scales do not change.
+    w = wls.normal_weights(125, 17, 129)
+    w[0, :4] = [0.0, -0.0, 1e-30, -1e-30]
+    c1, s1 = oracle.quantize(w, oracle.BINARY1)
+    c2, s2 = oracle.quantize(-w, oracle.BINARY1)
+    zero = (w == 0)
+    assert np.array_equal(c2[~zero], -c1[~zero])
+    assert np.all(c1[zero] == 1) and np.all(c2[zero] == 1)
+    assert np.array_equal(s1.view(np.uint32), s2.view(np.uint32))
+
+
 @pytest.mark.parametrize("fmt,alphabet", [(oracle.TERNARY2, [-1, 0, 1]), (oracle.INT4, list(range(-7, 8))),
                                           (oracle.BINARY1, [-1, 1])])
 @pytest.mark.parametrize("K", [1, 3, 4, 5, 31, 32, 33, 255])
