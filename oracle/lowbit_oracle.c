@@ -230,7 +230,7 @@ int orc_int4_codes(const float *w, long N, long K, long ldw, int8_t *codes, floa
  *             means -1 [M8.8 §0x06E]; a row takes ceil(K/8) bytes.
  *   TERNARY2: four codes per byte [Atomic], as 2-bit two's-complement fields
  *             00 = 0, 01 = +1, 11 = -1, 10 reserved.  The pages do not fix the
- *             order of codes inside a byte; this build stores them plane by
+ *             order of codes inside a byte; the layout here stores them plane by
  *             plane within each little-endian 32-bit word of 16 codes: code k
  *             lives in word k/16, byte (k%16)%4, field (k%16)/4, i.e. bits
  *             8*((k%16)%4) + 2*((k%16)/4) and the bit above.  A row takes
