@@ -74,6 +74,9 @@ def _load():
             "orc_rescale_f32": [P, L, L, P, L, P, P, L],
             "orc_rescale_bf16": [P, L, L, P, L, P, P, L],
             "orc_max_threads": [],
+            "orc_binary_centred_codes": [P, L, L, L, P, P, P],
+            "orc_act_prologue_f32": [P, L, L, L, P, I, F, L, P, L, P],
+            "orc_act_prologue_bf16": [P, L, L, L, P, I, F, L, P, L, P],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)
@@ -85,6 +88,8 @@ def _load():
         lib.orc_row_bytes.restype = L
         lib.orc_f32_to_bf16.argtypes = [F]
         lib.orc_f32_to_bf16.restype = ctypes.c_uint16
+        lib.orc_fwht32.argtypes = [P, L]
+        lib.orc_fwht32.restype = None
         _lib = lib
     return _lib
 
@@ -146,6 +151,58 @@ def int4_codes(w: np.ndarray):
     s_w = np.empty(N, np.float32)
     _check(_load().orc_int4_codes(_p(w), N, K, K, _p(codes), _p(s_w)), "int4_codes")
     return codes, s_w
+
+
+def binary_centred_codes(w: np.ndarray):
+    """BitNet v1 centred sign codes (+1 where w > mean(W), else -1) and the
+    per-tensor scale beta = mean|W| (M8.8 §0x02B, §0x02E).  Returns
+    (codes, beta[1], alpha[1])."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    N, K = w.shape
+    codes = np.empty((N, K), np.int8)
+    alpha = np.zeros(1, np.float32)
+    beta = np.zeros(1, np.float32)
+    _check(_load().orc_binary_centred_codes(_p(w), N, K, K, _p(codes), _p(alpha), _p(beta)),
+           "binary_centred_codes")
+    return codes, beta, alpha
+
+
+def fwht32(v: np.ndarray) -> np.ndarray:
+    """Unnormalised fast Walsh-Hadamard transform of each row of v (fp32,
+    row length a power of two), radix-2, stages h = 1, 2, ... (M8.8 §0x07C)."""
+    v = np.array(v, dtype=np.float32, order="C", copy=True)
+    n = v.shape[-1]
+    assert n > 0 and n & (n - 1) == 0
+    flat = v.reshape(-1, n)
+    for r in range(flat.shape[0]):
+        row = flat[r]
+        _load().orc_fwht32(row.ctypes.data_as(ctypes.c_void_p), n)
+    return v
+
+
+def act_prologue(x: np.ndarray, g: np.ndarray | None = None, norm: bool = False, eps_norm: float = 1e-5,
+                 hadamard: int = 0, bf16_bits: bool = False):
+    """RMSNorm (norm=True) with gain g, optional block Hadamard rotation of
+    block size `hadamard`, then per-token absmax int8 codes; returns (q, s_x).
+    The codes come from FWHT(x*g) and the row factors 1/rms and
+    1/sqrt(hadamard) enter the scale only (see lowbit_oracle.c)."""
+    if bf16_bits:
+        x = np.ascontiguousarray(x, dtype=np.uint16)
+        fn = _load().orc_act_prologue_bf16
+    else:
+        x = np.ascontiguousarray(x, dtype=np.float32)
+        fn = _load().orc_act_prologue_f32
+    M, K = x.shape
+    gp = None
+    if g is not None:
+        g = np.ascontiguousarray(g, dtype=np.float32)
+        assert g.shape == (K,)
+        gp = _p(g)
+    q = np.empty((M, K), np.int8)
+    s_x = np.empty(M, np.float32)
+    _check(fn(_p(x), M, K, K, gp, 1 if norm else 0, ctypes.c_float(eps_norm), hadamard, _p(q), K, _p(s_x)),
+           "act_prologue")
+    return q, s_x
 
 
 def quantize(w: np.ndarray, fmt: int, eps: float = 1e-5):

@@ -23,7 +23,8 @@
  *
  * Parity status of each function (the pins live in tests/test_oracle_pins.py):
  *   orc_ternary_codes, orc_binary_codes, orc_int4_codes, orc_tanh,
- *   orc_act_quant_*, orc_int_dot, orc_rescale_*, orc_pack/unpack (binary):
+ *   orc_act_quant_*, orc_int_dot, orc_rescale_*, orc_pack/unpack (binary),
+ *   orc_binary_centred_codes, orc_fwht32, orc_act_prologue_*:
  *     pinned (closed forms, worked cases, library routines, brute force).
  *   orc_pack/orc_unpack for TERNARY2 and INT4: the pages fix "four codes per
  *     byte" and "two's complement" but not the order of codes inside a byte, so
@@ -184,6 +185,40 @@ int orc_binary_codes(const float *w, long N, long K, long ldw, int8_t *codes, fl
         }
         s_w[n] = (float)(r / (double)K);
     }
+    return ORC_OK;
+}
+
+/* BitNet v1 centred binary codes [M8.8 §0x02B, §0x02E]: alpha = mean(W) over
+ * the whole tensor, codes +1 where w - alpha > 0 and -1 otherwise (a weight
+ * equal to the mean takes -1, the tie of the page's trace), and one scale per
+ * tensor beta = mean|W|.  Both sums are fp64 in the ternary scale's fixed
+ * order (k ascending within a row, then rows ascending), divided by N*K in
+ * fp64 and rounded once to fp32.  The difference w - alpha of two fp32 values
+ * is positive exactly when w > alpha, so the code is that comparison.
+ * Writes alpha_out[0] and beta_out[0]. */
+int orc_binary_centred_codes(const float *w, long N, long K, long ldw, int8_t *codes,
+                             float *alpha_out, float *beta_out)
+{
+    if (N <= 0 || K <= 0 || ldw < K) return ORC_EINVAL;
+    double S = 0.0, A = 0.0;
+    for (long n = 0; n < N; ++n) {
+        double r = 0.0, ra = 0.0;
+        for (long k = 0; k < K; ++k) {
+            float v = w[n * ldw + k];
+            if (!finite_f32(v)) return ORC_ENONFINITE;
+            r += (double)v;
+            ra += fabs((double)v);
+        }
+        S += r;
+        A += ra;
+    }
+    float alpha = (float)(S / (double)(N * K));
+    float beta = (float)(A / (double)(N * K));
+    for (long n = 0; n < N; ++n)
+        for (long k = 0; k < K; ++k)
+            codes[n * K + k] = (int8_t)(w[n * ldw + k] > alpha ? 1 : -1);
+    *alpha_out = alpha;
+    *beta_out = beta;
     return ORC_OK;
 }
 
@@ -374,6 +409,119 @@ int orc_act_quant_bf16(const uint16_t *x, long M, long K, long ldx, float eps,
         if (st != ORC_OK) status = st;
     }
     free(row);
+    return status;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Activation prologue: RMSNorm, gain, Hadamard rotation, per-token codes     */
+/* ------------------------------------------------------------------------ */
+/* Fast Walsh-Hadamard transform of one block of n = 2^p fp32 values, in place,
+ * unnormalised: the radix-2 algorithm with stages h = 1, 2, 4, ..., n/2, each
+ * replacing the pair (v[j], v[j+h]) of every 2h-block by (v[j] + v[j+h],
+ * v[j] - v[j+h]) as two fp32 operations.  This is the O(n log n) transform the
+ * BitNet v2 H-BitLinear applies online [M8.8 §0x07C]; its result is the
+ * Sylvester-ordered Hadamard matrix H (H[i][j] = (-1)^popcount(i & j)) times
+ * v, rounded by these fp32 steps. */
+void orc_fwht32(float *v, long n)
+{
+    for (long h = 1; h < n; h *= 2)
+        for (long i = 0; i < n; i += 2 * h)
+            for (long j = i; j < i + h; ++j) {
+                float a = v[j], b = v[j + h];
+                v[j] = a + b;
+                v[j + h] = a - b;
+            }
+}
+
+/* The activation side of a BitLinear layer, row by row:
+ *   1. RMSNorm with gain [M8.8 §0x02C-§0x02E and §0x03: normalise, then take the
+ *      absmax codes; b1.58 and T4NT use RMSNorm]:  y = x * g / rms(x),
+ *      rms(x) = sqrt(mean_k x_k^2 + eps_norm);  norm = 0 skips the division,
+ *      so only the gain (the OneBit input value vector of §0x06A) applies;
+ *   2. optionally the block Hadamard rotation of H-BitLinear [§0x07C]: blocks
+ *      of hb consecutive features (hb a power of two dividing K), each
+ *      multiplied by the normalised Walsh-Hadamard matrix H/sqrt(hb);
+ *   3. per-token absmax int8 codes of the result [§0x05C], eps = 0.
+ * The row factors 1/rms and 1/sqrt(hb) are positive and common to the whole
+ * row, so they cancel in absmax codes: the codes are computed from
+ *   u = FWHT(RN32(x_k * g_k)) (the fp32 transform above, or no transform),
+ * by the per-token rule of act_quant_row, and the factors enter only the
+ * scale, s_x = max|u| / sqrt(hb) / rms / 127, evaluated in fp64 (the sum of
+ * squares k ascending) and rounded once to fp32.  g may be NULL (all ones).
+ * A non-finite x or g, or a non-finite product or transform, returns
+ * ORC_ENONFINITE. */
+static int prologue_row(const float *xf, long K, const float *g, int norm, float eps_norm, long hb,
+                        float *u, int8_t *q, float *s_x)
+{
+    for (long k = 0; k < K; ++k) {
+        if (!finite_f32(xf[k]) || (g && !finite_f32(g[k]))) return ORC_ENONFINITE;
+        u[k] = g ? xf[k] * g[k] : xf[k];
+        if (!finite_f32(u[k])) return ORC_ENONFINITE;
+    }
+    if (hb > 0) {
+        for (long b = 0; b < K; b += hb) orc_fwht32(u + b, hb);
+        for (long k = 0; k < K; ++k)
+            if (!finite_f32(u[k])) return ORC_ENONFINITE;
+    }
+    float s_unused;
+    int st = act_quant_row(u, K, 0.0f, q, &s_unused);
+    if (st != ORC_OK) return st;
+    float gmax = 0.0f;
+    for (long k = 0; k < K; ++k)
+        if (fabsf(u[k]) > gmax) gmax = fabsf(u[k]);
+    if (gmax == 0.0f) {
+        *s_x = 0.0f;
+        return ORC_OK;
+    }
+    double s = (double)gmax;
+    if (hb > 0) s = s / sqrt((double)hb);
+    if (norm) {
+        double ss = 0.0;
+        for (long k = 0; k < K; ++k) ss += (double)xf[k] * (double)xf[k];
+        s = s / sqrt(ss / (double)K + (double)eps_norm);
+    }
+    *s_x = (float)(s / 127.0);
+    return ORC_OK;
+}
+
+static int prologue_args_ok(long M, long K, long ldx, long ldq, int norm, float eps_norm, long hb)
+{
+    if (M <= 0 || K <= 0 || ldx < K || ldq < K || (norm != 0 && norm != 1)) return 0;
+    if (!(eps_norm >= 0.0f) || !finite_f32(eps_norm)) return 0;
+    if (hb < 0 || (hb > 0 && ((hb & (hb - 1)) != 0 || hb > K || K % hb != 0))) return 0;
+    return 1;
+}
+
+int orc_act_prologue_f32(const float *x, long M, long K, long ldx, const float *g, int norm, float eps_norm,
+                         long hb, int8_t *q, long ldq, float *s_x)
+{
+    if (!prologue_args_ok(M, K, ldx, ldq, norm, eps_norm, hb)) return ORC_EINVAL;
+    float *u = (float *)malloc(sizeof(float) * (size_t)K);
+    if (!u) return ORC_EINVAL;
+    int status = ORC_OK;
+    for (long t = 0; t < M; ++t) {
+        int st = prologue_row(x + t * ldx, K, g, norm, eps_norm, hb, u, q + t * ldq, s_x + t);
+        if (st != ORC_OK) status = st;
+    }
+    free(u);
+    return status;
+}
+
+int orc_act_prologue_bf16(const uint16_t *x, long M, long K, long ldx, const float *g, int norm,
+                          float eps_norm, long hb, int8_t *q, long ldq, float *s_x)
+{
+    if (!prologue_args_ok(M, K, ldx, ldq, norm, eps_norm, hb)) return ORC_EINVAL;
+    float *row = (float *)malloc(sizeof(float) * (size_t)K);
+    float *u = (float *)malloc(sizeof(float) * (size_t)K);
+    if (!row || !u) { free(row); free(u); return ORC_EINVAL; }
+    int status = ORC_OK;
+    for (long t = 0; t < M; ++t) {
+        for (long k = 0; k < K; ++k) row[k] = orc_bf16_to_f32(x[t * ldx + k]);
+        int st = prologue_row(row, K, g, norm, eps_norm, hb, u, q + t * ldq, s_x + t);
+        if (st != ORC_OK) status = st;
+    }
+    free(row);
+    free(u);
     return status;
 }
 

@@ -347,6 +347,16 @@ def test_act_quant_worked_rows(golden_dir):
     assert s_x.tolist() == g["s_x"]
 
 
+def test_act_quant_eps_scale_leaves_eps_out(golden_dir):
+    # With eps > 0 the codes divide by gamma + eps, but the reconstruction
+    # scale stays gamma/127: a slip to (gamma + eps)/127 fails here.
+    g = _golden(golden_dir, "act_quant_eps_row.json")
+    q, s_x = oracle.act_quant(np.array(g["x"], np.float32), g["eps"])
+    assert q.tolist() == g["q"]
+    want = (np.array(g["s_x_numerator"], np.float32) / np.float32(127)).astype(np.float32)
+    assert np.array_equal(s_x.view(np.uint32), want.view(np.uint32))
+
+
 def test_act_quant_invariants():
     x = wls.normal_activations(51, 97, 1000)
     q, s_x = oracle.act_quant(x)
