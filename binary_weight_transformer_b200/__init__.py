@@ -12,7 +12,9 @@ Functions carry the ABI's names::
     packed, s_w = lowbit_pack(w, fmt, eps=1e-5)
     codes       = lowbit_unpack(packed, K, fmt)
     q, s_x      = lowbit_act_quant(x, eps=0.0)
+    q, s_x      = lowbit_act_quant_ex(x, g=None, norm=NORM_RMS, eps_norm=1e-5, hadamard=0)
     y           = lowbit_linear(q, s_x, packed, s_w, fmt, N, out_dtype)
+    y           = lowbit_bitlinear(x, packed, s_w, fmt, N, out_dtype, g=None, norm=NORM_RMS)
 """
 from __future__ import annotations
 
@@ -20,6 +22,9 @@ import ctypes
 import os
 
 TERNARY2, BINARY1, INT4 = 0, 1, 2
+NORM_NONE, NORM_RMS = 0, 1
+QUANT_DEFAULT, QUANT_BINARY_CENTRED = 0, 1
+FUSED_MAX_MK = 98304  # LOWBIT_FUSED_MAX_MK
 F32, BF16, I32 = 0, 1, 2
 WEIGHTS_STABLE = 1  # LOWBIT_LINEAR_WEIGHTS_STABLE
 
@@ -51,8 +56,18 @@ ABI = {
     "lowbit_linear_ex": (_I32, [_P, _I64, _P, _I64, _I64, _P, _I64, _P, _I32, _I64, _P, _I32, _I64, _I32,
                                 ctypes.c_uint, _P, _P]),
     "lowbit_linear_kernel": (_I32, [_I64, _I64, _I64, _I32, _I32, _I32, _P]),
+    "lowbit_pack_ex_workspace_bytes": (_SZ, [_I32, _I32, _I64]),
+    "lowbit_pack_ex": (_I32, [_P, _I64, _I64, _I64, _I32, _I32, _F, _P, _I64, _P, _P, _SZ, _P, _P]),
+    "lowbit_act_row_stats": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _I32, _P, _P, _P, _P]),
+    "lowbit_act_quant_given_max": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _I32, _P, _P, _I64, _P, _P]),
+    "lowbit_act_scales": (_I32, [_P, _P, _I64, _I64, _I32, _F, _I32, _P, _P, _P]),
+    "lowbit_rescale": (_I32, [_P, _I64, _I64, _I64, _P, _P, _I32, _P, _I32, _I64, _P, _P]),
+    "lowbit_act_quant_ex": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _I32, _F, _I32, _P, _I64, _P, _P, _P]),
+    "lowbit_bitlinear": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _I32, _F, _I32, _P, _I64, _P, _I32, _I64, _P, _I32,
+                                _I64, _P, _I64, _P, _I32, ctypes.c_uint, _P, _P]),
     "lowbit_kernel_name": (ctypes.c_char_p, [_I32]),
     "lowbit_status_string": (ctypes.c_char_p, [_I32]),
+    "lowbit_set_wait_limit": (_I32, [_I64]),
     "lowbit_version": (_I32, []),
 }
 
@@ -148,6 +163,26 @@ def lowbit_pack(w, fmt: int, eps: float = 1e-5, packed=None, s_w=None, ldp: int 
     return packed, s_w
 
 
+def lowbit_pack_ex(w, fmt: int, quantizer: int = QUANT_DEFAULT, eps: float = 1e-5, packed=None, s_w=None,
+                   ldp: int | None = None, status=None, stream=None):
+    """lowbit_pack with a choice of quantiser (QUANT_BINARY_CENTRED: BitNet v1
+    centred sign codes, one scale mean|W| written to every row's entry)."""
+    import torch
+    N, K = w.shape
+    if ldp is None:
+        ldp = packed_ld(fmt, K)
+    if packed is None:
+        packed = torch.empty((N, ldp), dtype=torch.uint8, device=w.device)
+    if s_w is None:
+        s_w = torch.empty(scale_count(fmt, N), dtype=torch.float32, device=w.device)
+    need = int(lib().lowbit_pack_ex_workspace_bytes(fmt, quantizer, N))
+    workspace = torch.empty(need, dtype=torch.uint8, device=w.device) if need else None
+    st = lib().lowbit_pack_ex(_ptr(w), N, K, w.stride(0), fmt, quantizer, eps, _ptr(packed), packed.stride(0),
+                              _ptr(s_w), _ptr(workspace), need, _ptr(status), _stream(stream))
+    _check(st, "lowbit_pack_ex")
+    return packed, s_w
+
+
 def lowbit_pack_ternary_noalloc(w, eps: float = 1e-5, packed=None, s_w=None, ldp: int | None = None,
                                 status=None, stream=None):
     """Ternary pack that allocates nothing in the library (see lowbit.h);
@@ -216,3 +251,109 @@ def lowbit_linear(q, s_x, packed, s_w, fmt: int, N: int, out_dtype: int = F32, K
                                 WEIGHTS_STABLE if weights_stable else 0, _ptr(status), _stream(stream))
     _check(st, "lowbit_linear")
     return y
+
+
+def _xdt(x):
+    import torch
+    return {torch.float32: F32, torch.bfloat16: BF16}[x.dtype]
+
+
+def lowbit_act_quant_ex(x, g=None, norm: int = NORM_NONE, eps_norm: float = 1e-5, hadamard: int = 0, q=None,
+                        s_x=None, status=None, stream=None):
+    """Activation prologue of a BitLinear layer (see lowbit.h): gain g,
+    RMSNorm, block Hadamard rotation, then per-token int8 codes."""
+    import torch
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, (K + 15) // 16 * 16), dtype=torch.int8, device=x.device)
+    if s_x is None:
+        s_x = torch.empty(M, dtype=torch.float32, device=x.device)
+    st = lib().lowbit_act_quant_ex(_ptr(x), _xdt(x), M, K, x.stride(0), _ptr(g), norm, eps_norm, hadamard,
+                                   _ptr(q), q.stride(0), _ptr(s_x), _ptr(status), _stream(stream))
+    _check(st, "lowbit_act_quant_ex")
+    return q, s_x
+
+
+def bitlinear_fuses(M: int, K: int, hadamard: int = 0, path: int = 0) -> bool:
+    """True when lowbit_bitlinear runs as one fused decode kernel."""
+    return M <= 4 and hadamard == 0 and path in (0, 1) and M * ((K + 127) // 128 * 128) <= FUSED_MAX_MK
+
+
+def lowbit_bitlinear(x, packed, s_w, fmt: int, N: int, out_dtype: int = F32, g=None, norm: int = NORM_NONE,
+                     eps_norm: float = 1e-5, hadamard: int = 0, y=None, q=None, s_x=None, want_codes: bool = False,
+                     status=None, stream=None, path: int = 0, weights_stable: bool = False):
+    """The whole BitLinear forward from activations x[M, K] (fp32 or bf16).
+
+    q and s_x are allocated as workspace when the call is not fused (or when
+    ``want_codes``); returns y, or (y, q, s_x) with ``want_codes``."""
+    import torch
+    M, K = x.shape
+    if y is None:
+        dt = {F32: torch.float32, BF16: torch.bfloat16, I32: torch.int32}[out_dtype]
+        y = torch.empty((M, N), dtype=dt, device=x.device)
+    need = want_codes or not bitlinear_fuses(M, K, hadamard, path)
+    if q is None and need:
+        q = torch.empty((M, (K + 15) // 16 * 16), dtype=torch.int8, device=x.device)
+    if s_x is None and need:
+        s_x = torch.empty(M, dtype=torch.float32, device=x.device)
+    st = lib().lowbit_bitlinear(_ptr(x), _xdt(x), M, K, x.stride(0), _ptr(g), norm, eps_norm, hadamard,
+                                _ptr(packed), packed.stride(0), _ptr(s_w), fmt, N, _ptr(y), out_dtype, y.stride(0),
+                                _ptr(q), q.stride(0) if q is not None else 0, _ptr(s_x), path,
+                                WEIGHTS_STABLE if weights_stable else 0, _ptr(status), _stream(stream))
+    _check(st, "lowbit_bitlinear")
+    return (y, q, s_x) if want_codes else y
+
+
+def lowbit_act_row_stats(x, g=None, hadamard: int = 0, with_ss: bool = False, status=None, stream=None):
+    """Per-row max|x*g| (fp32 [M]) and, with ``with_ss``, the fp64 sum of
+    squares of a row slice (see lowbit.h, row-parallel layers)."""
+    import torch
+    M, K = x.shape
+    row_max = torch.empty(M, dtype=torch.float32, device=x.device)
+    row_ss = torch.empty(M, dtype=torch.float64, device=x.device) if with_ss else None
+    st = lib().lowbit_act_row_stats(_ptr(x), _xdt(x), M, K, x.stride(0), _ptr(g), hadamard, _ptr(row_max),
+                                    _ptr(row_ss), _ptr(status), _stream(stream))
+    _check(st, "lowbit_act_row_stats")
+    return row_max, row_ss
+
+
+def lowbit_act_quant_given_max(x, row_max, g=None, hadamard: int = 0, q=None, status=None, stream=None):
+    import torch
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, (K + 15) // 16 * 16), dtype=torch.int8, device=x.device)
+    st = lib().lowbit_act_quant_given_max(_ptr(x), _xdt(x), M, K, x.stride(0), _ptr(g), hadamard, _ptr(row_max),
+                                          _ptr(q), q.stride(0), _ptr(status), _stream(stream))
+    _check(st, "lowbit_act_quant_given_max")
+    return q
+
+
+def lowbit_act_scales(row_max, row_ss, K_total: int, norm: int = NORM_NONE, eps_norm: float = 1e-5,
+                      hadamard: int = 0, s_x=None, status=None, stream=None):
+    import torch
+    M = row_max.shape[0]
+    if s_x is None:
+        s_x = torch.empty(M, dtype=torch.float32, device=row_max.device)
+    st = lib().lowbit_act_scales(_ptr(row_max), _ptr(row_ss), M, K_total, norm, eps_norm, hadamard, _ptr(s_x),
+                                 _ptr(status), _stream(stream))
+    _check(st, "lowbit_act_scales")
+    return s_x
+
+
+def lowbit_rescale(acc, s_x, s_w, fmt: int, out_dtype: int = F32, y=None, status=None, stream=None):
+    """y = float(acc) * (s_w * s_x) from int32 accumulators acc[M, N]."""
+    import torch
+    M, N = acc.shape
+    if y is None:
+        dt = {F32: torch.float32, BF16: torch.bfloat16, I32: torch.int32}[out_dtype]
+        y = torch.empty((M, N), dtype=dt, device=acc.device)
+    st = lib().lowbit_rescale(_ptr(acc), acc.stride(0), M, N, _ptr(s_x), _ptr(s_w), fmt, _ptr(y), out_dtype,
+                              y.stride(0), _ptr(status), _stream(stream))
+    _check(st, "lowbit_rescale")
+    return y
+
+
+def set_wait_limit(cycles: int = 0):
+    """Bound of the tensor-core kernels' pipeline waits on the current device
+    (SM cycles; 0 restores the default).  See lowbit_set_wait_limit."""
+    _check(lib().lowbit_set_wait_limit(cycles), "lowbit_set_wait_limit")

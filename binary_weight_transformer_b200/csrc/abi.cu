@@ -14,6 +14,8 @@ lowbit_status act_quant_launch(const void *x, lowbit_dtype xdt, int64_t M, int64
 lowbit_status pack_launch(const float *w, int64_t N, int64_t K, int64_t ldw, lowbit_format f, float eps,
                           uint8_t *packed, int64_t ldp, float *s_w, void *workspace, int32_t *status,
                           cudaStream_t st);
+lowbit_status pack_centred_launch(const float *w, int64_t N, int64_t K, int64_t ldw, uint8_t *packed, int64_t ldp,
+                                  float *s_w, void *workspace, int32_t *status, cudaStream_t st);
 lowbit_status unpack_launch(const uint8_t *packed, int64_t ldp, int64_t N, int64_t K, lowbit_format f,
                             int8_t *codes, int64_t ldc, int32_t *status, cudaStream_t st);
 lowbit_status gemv_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
@@ -48,6 +50,30 @@ lowbit_status gemm_ts_pair_launch(const int8_t *q, int64_t ldq, const float *s_x
                                   const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
                                   lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy,
                                   int32_t *status, cudaStream_t st);
+
+lowbit_status act_prologue_launch(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                  const float *g, int norm, float eps_norm, int hb, int8_t *q, int64_t ldq,
+                                  float *s_x, int32_t *status, cudaStream_t st);
+lowbit_status gemv_fused_launch(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx, const float *g,
+                                int norm, float eps_norm, const uint8_t *packed, int64_t ldp, int64_t row_bytes,
+                                const float *s_w, lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy,
+                                int8_t *q_out, int64_t ldq, float *s_x_out, int prefetch, int32_t *status,
+                                cudaStream_t st);
+
+lowbit_status act_row_stats_launch(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                   const float *g, int hb, float *row_max, double *row_ss, int32_t *status,
+                                   cudaStream_t st);
+lowbit_status act_codes_given_max_launch(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                         const float *g, int hb, const float *row_max, int8_t *q, int64_t ldq,
+                                         int32_t *status, cudaStream_t st);
+lowbit_status act_scales_launch(const float *row_max, const double *row_ss, int64_t M, int64_t K_total, int norm,
+                                float eps_norm, int hb, float *s_x, int32_t *status, cudaStream_t st);
+lowbit_status rescale_launch(const int32_t *acc, int64_t ldacc, int64_t M, int64_t N, const float *s_x,
+                             const float *s_w, int per_row, void *y, lowbit_dtype ydt, int64_t ldy, cudaStream_t st);
+
+lowbit_status set_wait_limit_gemm(long long cycles);
+lowbit_status set_wait_limit_gemm_ts(long long cycles);
+lowbit_status set_wait_limit_skinny(long long cycles);
 
 lowbit_status launch_status()
 {
@@ -84,15 +110,6 @@ DeviceInfo device_info()
     d.major = (packed >> 24) & 0x7f;
     d.ok = true;
     return d;
-}
-
-// The kernels are built for sm_100a only.
-lowbit_status check_device()
-{
-    const DeviceInfo d = device_info();
-    if (!d.ok) return LOWBIT_ERR_CUDA;
-    if (d.major != 10 || d.minor != 0) return LOWBIT_ERR_UNSUPPORTED;
-    return LOWBIT_OK;
 }
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -142,6 +159,15 @@ lowbit_status check_linear_shape(int64_t M, int64_t N, int64_t K, lowbit_format 
 }
 
 }  // namespace
+
+// The kernels are built for sm_100a only.
+lowbit_status check_device()
+{
+    const DeviceInfo d = device_info();
+    if (!d.ok) return LOWBIT_ERR_CUDA;
+    if (d.major != 10 || d.minor != 0) return LOWBIT_ERR_UNSUPPORTED;
+    return LOWBIT_OK;
+}
 
 int device_sm_count()
 {
@@ -215,6 +241,36 @@ lowbit_status lowbit_pack(const float *w, int64_t N, int64_t K, int64_t ldw, low
                        static_cast<cudaStream_t>(stream));
 }
 
+size_t lowbit_pack_ex_workspace_bytes(lowbit_format f, int quantizer, int64_t N)
+{
+    if (N <= 0 || !valid_format(f)) return 0;
+    if (quantizer == LOWBIT_QUANT_DEFAULT) return lowbit_pack_workspace_bytes(f, N);
+    if (quantizer == LOWBIT_QUANT_BINARY_CENTRED && f == LOWBIT_BINARY1)
+        return (static_cast<size_t>(N) * 16 + 16 + 255) / 256 * 256;
+    return 0;
+}
+
+lowbit_status lowbit_pack_ex(const float *w, int64_t N, int64_t K, int64_t ldw, lowbit_format f, int quantizer,
+                             float eps, uint8_t *packed, int64_t ldp, float *s_w, void *workspace,
+                             size_t workspace_bytes, int32_t *status_dev, void *stream)
+{
+    if (quantizer == LOWBIT_QUANT_DEFAULT)
+        return lowbit_pack(w, N, K, ldw, f, eps, packed, ldp, s_w, workspace, workspace_bytes, status_dev, stream);
+    if (quantizer != LOWBIT_QUANT_BINARY_CENTRED || f != LOWBIT_BINARY1) return LOWBIT_ERR_INVALID_ARG;
+    if (w == nullptr || packed == nullptr || s_w == nullptr) return LOWBIT_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0 || ldw < K || N > INT32_MAX || K > INT32_MAX) return LOWBIT_ERR_INVALID_ARG;
+    if (ldp < static_cast<int64_t>(lowbit_packed_row_bytes(f, K))) return LOWBIT_ERR_INVALID_ARG;
+    if (ldp % 16 != 0 || !aligned(packed, 16) || !aligned(w, 4) || !aligned(s_w, 4)) return LOWBIT_ERR_ALIGNMENT;
+    const size_t need = lowbit_pack_ex_workspace_bytes(f, quantizer, N);
+    if (workspace == nullptr || workspace_bytes < need) return LOWBIT_ERR_INVALID_ARG;
+    if (!aligned(workspace, 8)) return LOWBIT_ERR_ALIGNMENT;
+    const lowbit_status d = check_device();
+    if (d != LOWBIT_OK) return d;
+    const TraceRange trace("lowbit_pack_ex");
+    return pack_centred_launch(w, N, K, ldw, packed, ldp, s_w, workspace, status_dev,
+                               static_cast<cudaStream_t>(stream));
+}
+
 lowbit_status lowbit_unpack(const uint8_t *packed, int64_t ldp, int64_t N, int64_t K, lowbit_format f,
                             int8_t *codes, int64_t ldc, int32_t *status_dev, void *stream)
 {
@@ -242,6 +298,167 @@ lowbit_status lowbit_act_quant(const void *x, lowbit_dtype xdt, int64_t M, int64
     if (d != LOWBIT_OK) return d;
     const TraceRange trace("lowbit_act_quant");
     return act_quant_launch(x, xdt, M, K, ldx, eps, q, ldq, s_x, status_dev, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+namespace {
+
+// Checks of the activation-side arguments shared by lowbit_act_quant_ex and
+// lowbit_bitlinear (q and s_x checked by the caller, who may allow NULL).
+lowbit_status check_prologue_args(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                  const float *g, int norm, float eps_norm, int hadamard)
+{
+    if (x == nullptr || (xdt != LOWBIT_F32 && xdt != LOWBIT_BF16)) return LOWBIT_ERR_INVALID_ARG;
+    if (M <= 0 || K <= 0 || ldx < K || M > INT32_MAX) return LOWBIT_ERR_INVALID_ARG;
+    if (norm != LOWBIT_NORM_NONE && norm != LOWBIT_NORM_RMS) return LOWBIT_ERR_INVALID_ARG;
+    if (!(eps_norm >= 0.0f) || eps_norm > 3.0e38f) return LOWBIT_ERR_INVALID_ARG;
+    if (hadamard < 0 || hadamard == 1 || (hadamard > 0 && ((hadamard & (hadamard - 1)) != 0 ||
+                                                             hadamard > K || K % hadamard != 0)))
+        return LOWBIT_ERR_INVALID_ARG;
+    const int64_t esz = xdt == LOWBIT_F32 ? 4 : 2;
+    if (!aligned(x, static_cast<uintptr_t>(esz)) || (g != nullptr && !aligned(g, 4))) return LOWBIT_ERR_ALIGNMENT;
+    const bool options = g != nullptr || norm != LOWBIT_NORM_NONE || hadamard > 0;
+    if (options && K > LOWBIT_PROLOGUE_MAX_K) return LOWBIT_ERR_UNSUPPORTED;
+    return LOWBIT_OK;
+}
+
+bool fused_decode(int64_t M, int64_t K, int hadamard, int path)
+{
+    return M <= 4 && hadamard == 0 && (path == 0 || path == 1) && M * ((K + 127) / 128 * 128) <= LOWBIT_FUSED_MAX_MK;
+}
+
+}  // namespace
+
+extern "C" {
+
+lowbit_status lowbit_act_quant_ex(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                  const float *g, int norm, float eps_norm, int hadamard,
+                                  int8_t *q, int64_t ldq, float *s_x, int32_t *status_dev, void *stream)
+{
+    const lowbit_status a = check_prologue_args(x, xdt, M, K, ldx, g, norm, eps_norm, hadamard);
+    if (a != LOWBIT_OK) return a;
+    if (q == nullptr || s_x == nullptr || ldq < K) return LOWBIT_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || ldq % 16 != 0 || !aligned(s_x, 4)) return LOWBIT_ERR_ALIGNMENT;
+    const lowbit_status d = check_device();
+    if (d != LOWBIT_OK) return d;
+    const TraceRange trace("lowbit_act_quant_ex");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (g == nullptr && norm == LOWBIT_NORM_NONE && hadamard == 0)
+        return act_quant_launch(x, xdt, M, K, ldx, 0.0f, q, ldq, s_x, status_dev, st);
+    return act_prologue_launch(x, xdt, M, K, ldx, g, norm, eps_norm, hadamard, q, ldq, s_x, status_dev, st);
+}
+
+lowbit_status lowbit_bitlinear(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                               const float *g, int norm, float eps_norm, int hadamard,
+                               const uint8_t *packed, int64_t ldp, const float *s_w, lowbit_format f, int64_t N,
+                               void *y, lowbit_dtype ydt, int64_t ldy,
+                               int8_t *q, int64_t ldq, float *s_x,
+                               int path, unsigned flags, int32_t *status_dev, void *stream)
+{
+    const lowbit_status a = check_prologue_args(x, xdt, M, K, ldx, g, norm, eps_norm, hadamard);
+    if (a != LOWBIT_OK) return a;
+    if ((flags & ~static_cast<unsigned>(LOWBIT_LINEAR_WEIGHTS_STABLE)) != 0) return LOWBIT_ERR_INVALID_ARG;
+    if (!valid_format(f) || packed == nullptr || s_w == nullptr || y == nullptr) return LOWBIT_ERR_INVALID_ARG;
+    if (ydt != LOWBIT_F32 && ydt != LOWBIT_BF16 && ydt != LOWBIT_I32) return LOWBIT_ERR_INVALID_ARG;
+    if (N <= 0 || ldy < N) return LOWBIT_ERR_INVALID_ARG;
+    const lowbit_status shape = check_linear_shape(M, N, K, f, path);
+    if (shape != LOWBIT_OK) return shape;
+    const int64_t rb = static_cast<int64_t>(lowbit_packed_row_bytes(f, K));
+    if (ldp < rb) return LOWBIT_ERR_INVALID_ARG;
+    const int64_t esz = ydt == LOWBIT_BF16 ? 2 : 4;
+    if (!aligned(packed, 16) || ldp % 16 != 0 || !aligned(s_w, 4) || !aligned(y, static_cast<uintptr_t>(esz)))
+        return LOWBIT_ERR_ALIGNMENT;
+    const bool fused = fused_decode(M, K, hadamard, path);
+    if (!fused && (q == nullptr || s_x == nullptr)) return LOWBIT_ERR_INVALID_ARG;
+    if (q != nullptr) {
+        if (ldq < K) return LOWBIT_ERR_INVALID_ARG;
+        if (!aligned(q, 16) || ldq % 16 != 0) return LOWBIT_ERR_ALIGNMENT;
+    }
+    if (s_x != nullptr && !aligned(s_x, 4)) return LOWBIT_ERR_ALIGNMENT;
+    const lowbit_status d = check_device();
+    if (d != LOWBIT_OK) return d;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int prefetch = (flags & LOWBIT_LINEAR_WEIGHTS_STABLE) != 0 ? 1 : 0;
+    if (fused) {
+        const TraceRange trace("lowbit_bitlinear");
+        return gemv_fused_launch(x, xdt, M, K, ldx, g, norm, eps_norm, packed, ldp, rb, s_w, f, N, y, ydt, ldy, q,
+                                 ldq, s_x, prefetch, status_dev, st);
+    }
+    const lowbit_status s1 = lowbit_act_quant_ex(x, xdt, M, K, ldx, g, norm, eps_norm, hadamard, q, ldq, s_x,
+                                                 status_dev, stream);
+    if (s1 != LOWBIT_OK) return s1;
+    // the prologue kernel just before writes q and s_x, never the weights
+    return lowbit_linear_ex(q, ldq, s_x, M, K, packed, ldp, s_w, f, N, y, ydt, ldy, path, flags, status_dev, stream);
+}
+
+lowbit_status lowbit_act_row_stats(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                   const float *g, int hadamard, float *row_max, double *row_ss,
+                                   int32_t *status_dev, void *stream)
+{
+    const lowbit_status a = check_prologue_args(x, xdt, M, K, ldx, g, LOWBIT_NORM_NONE, 0.0f, hadamard);
+    if (a != LOWBIT_OK) return a;
+    if (row_max == nullptr) return LOWBIT_ERR_INVALID_ARG;
+    if (K > LOWBIT_PROLOGUE_MAX_K) return LOWBIT_ERR_UNSUPPORTED;
+    if (!aligned(row_max, 4) || (row_ss != nullptr && !aligned(row_ss, 8))) return LOWBIT_ERR_ALIGNMENT;
+    const lowbit_status d = check_device();
+    if (d != LOWBIT_OK) return d;
+    const TraceRange trace("lowbit_act_row_stats");
+    return act_row_stats_launch(x, xdt, M, K, ldx, g, hadamard, row_max, row_ss, status_dev,
+                                static_cast<cudaStream_t>(stream));
+}
+
+lowbit_status lowbit_act_quant_given_max(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                         const float *g, int hadamard, const float *row_max,
+                                         int8_t *q, int64_t ldq, int32_t *status_dev, void *stream)
+{
+    const lowbit_status a = check_prologue_args(x, xdt, M, K, ldx, g, LOWBIT_NORM_NONE, 0.0f, hadamard);
+    if (a != LOWBIT_OK) return a;
+    if (row_max == nullptr || q == nullptr || ldq < K) return LOWBIT_ERR_INVALID_ARG;
+    if (K > LOWBIT_PROLOGUE_MAX_K) return LOWBIT_ERR_UNSUPPORTED;
+    if (!aligned(row_max, 4) || !aligned(q, 16) || ldq % 16 != 0) return LOWBIT_ERR_ALIGNMENT;
+    const lowbit_status d = check_device();
+    if (d != LOWBIT_OK) return d;
+    const TraceRange trace("lowbit_act_quant_given_max");
+    return act_codes_given_max_launch(x, xdt, M, K, ldx, g, hadamard, row_max, q, ldq, status_dev,
+                                      static_cast<cudaStream_t>(stream));
+}
+
+lowbit_status lowbit_act_scales(const float *row_max, const double *row_ss, int64_t M, int64_t K_total, int norm,
+                                float eps_norm, int hadamard, float *s_x, int32_t *status_dev, void *stream)
+{
+    if (row_max == nullptr || s_x == nullptr || M <= 0 || K_total <= 0 || M > INT32_MAX) return LOWBIT_ERR_INVALID_ARG;
+    if (norm != LOWBIT_NORM_NONE && norm != LOWBIT_NORM_RMS) return LOWBIT_ERR_INVALID_ARG;
+    if (norm == LOWBIT_NORM_RMS && row_ss == nullptr) return LOWBIT_ERR_INVALID_ARG;
+    if (!(eps_norm >= 0.0f) || eps_norm > 3.0e38f) return LOWBIT_ERR_INVALID_ARG;
+    if (hadamard < 0 || hadamard == 1 || (hadamard > 0 && ((hadamard & (hadamard - 1)) != 0 || hadamard > K_total)))
+        return LOWBIT_ERR_INVALID_ARG;
+    if (!aligned(row_max, 4) || !aligned(s_x, 4) || (row_ss != nullptr && !aligned(row_ss, 8)))
+        return LOWBIT_ERR_ALIGNMENT;
+    const lowbit_status d = check_device();
+    if (d != LOWBIT_OK) return d;
+    const TraceRange trace("lowbit_act_scales");
+    return act_scales_launch(row_max, row_ss, M, K_total, norm, eps_norm, hadamard, s_x, status_dev,
+                             static_cast<cudaStream_t>(stream));
+}
+
+lowbit_status lowbit_rescale(const int32_t *acc, int64_t ldacc, int64_t M, int64_t N, const float *s_x,
+                             const float *s_w, lowbit_format f, void *y, lowbit_dtype ydt, int64_t ldy,
+                             int32_t *status_dev, void *stream)
+{
+    (void)status_dev;
+    if (acc == nullptr || s_x == nullptr || s_w == nullptr || y == nullptr || !valid_format(f))
+        return LOWBIT_ERR_INVALID_ARG;
+    if (ydt != LOWBIT_F32 && ydt != LOWBIT_BF16 && ydt != LOWBIT_I32) return LOWBIT_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || ldacc < N || ldy < N || M > INT32_MAX || N > INT32_MAX) return LOWBIT_ERR_INVALID_ARG;
+    const int64_t esz = ydt == LOWBIT_BF16 ? 2 : 4;
+    if (!aligned(acc, 4) || !aligned(s_x, 4) || !aligned(s_w, 4) || !aligned(y, static_cast<uintptr_t>(esz)))
+        return LOWBIT_ERR_ALIGNMENT;
+    const lowbit_status d = check_device();
+    if (d != LOWBIT_OK) return d;
+    const TraceRange trace("lowbit_rescale");
+    return rescale_launch(acc, ldacc, M, N, s_x, s_w, f == LOWBIT_TERNARY2 ? 0 : 1, y, ydt, ldy,
+                          static_cast<cudaStream_t>(stream));
 }
 
 lowbit_status lowbit_linear_ex(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
@@ -329,6 +546,17 @@ lowbit_status lowbit_linear(const int8_t *q, int64_t ldq, const float *s_x, int6
                             void *y, lowbit_dtype ydt, int64_t ldy, int32_t *status_dev, void *stream)
 {
     return lowbit_linear_path(q, ldq, s_x, M, K, packed, ldp, s_w, f, N, y, ydt, ldy, 0, status_dev, stream);
+}
+
+lowbit_status lowbit_set_wait_limit(int64_t cycles)
+{
+    const lowbit_status d = check_device();
+    if (d != LOWBIT_OK) return d;
+    const long long c = cycles > 0 ? static_cast<long long>(cycles) : 0;
+    lowbit_status s = set_wait_limit_gemm(c);
+    if (s == LOWBIT_OK) s = set_wait_limit_gemm_ts(c);
+    if (s == LOWBIT_OK) s = set_wait_limit_skinny(c);
+    return s;
 }
 
 const char *lowbit_status_string(lowbit_status s)

@@ -1,4 +1,5 @@
-// act_quant.cu -- per-token absmax int8 activation codes.
+// act_quant.cu -- per-token absmax int8 activation codes, with the optional
+// activation prologue of a BitLinear layer in the same pass.
 //
 // "M8.8 - Native Binary and Ternary Transformers", section 0x05C (signed
 // per-token A8: gamma_t = max|x_t|, reconstruction scale gamma_t/127, an
@@ -6,6 +7,19 @@
 // to nearest, ties to even).  Per element: q = clip(rint((x*127) /
 // (gamma_t + eps)), -128, 127) with one fp32 multiply and one IEEE fp32
 // divide.
+//
+// Prologue options (the same page, 0x02E and 0x03: the activation is
+// normalised before its codes are taken; 0x06A: OneBit's input value vector;
+// 0x07C: H-BitLinear's online Hadamard transform):
+//   gain g      u_k = RN32(x_k * g_k) replaces x_k;
+//   RMSNorm     the row factor 1/sqrt(mean_k x_k^2 + eps_norm);
+//   Hadamard    an unnormalised fp32 fast Walsh-Hadamard transform of every
+//               block of hb consecutive features (radix 2, stages h = 1, 2,
+//               4, ...), with the factor 1/sqrt(hb).
+// Both row factors are positive, so they cancel in absmax codes: the codes
+// are taken from u by the rule above (eps = 0) and the factors multiply only
+// the scale, s_x = max|u| / sqrt(hb) / rms / 127, evaluated in fp64 (the
+// sum of squares in fp64) and rounded once to fp32.
 //
 // One HBM pass: a group of TPR threads owns a row, loads it into registers
 // with 16-byte non-allocating loads, reduces the row's absmax with warp
@@ -22,85 +36,14 @@
 // registers), which spreads a row over more threads when rows are few.
 // Measured for bf16 rows on B200: 8192 x 9728 in 49 us deep, 58 us wide, 64 us
 // with the compiler's own register choice; 1024 x 2560 in 4.1 us wide, 4.8 us
-// deep.
-#include "lowbit_internal.cuh"
+// deep.  The Hadamard rotation needs whole blocks of a row at once and runs
+// in a separate kernel that stages the row in shared memory.
+#include "quant_rule.cuh"
 
 namespace lowbit {
 namespace {
 
-template <typename T> struct In;
-template <> struct In<float> {
-    static constexpr int kPerVec = 4;
-    __device__ static float get(const uint4 &v, int i) { return __uint_as_float((&v.x)[i]); }
-    __device__ static float scalar(const void *p, int64_t i) { return static_cast<const float *>(p)[i]; }
-    // max of |x| bits over one vector (a non-finite value sorts above all finite ones)
-    __device__ static uint32_t absmax_bits(const uint4 &v)
-    {
-        return max(max(v.x & 0x7fffffffu, v.y & 0x7fffffffu), max(v.z & 0x7fffffffu, v.w & 0x7fffffffu));
-    }
-};
-template <> struct In<__nv_bfloat16> {
-    static constexpr int kPerVec = 8;
-    __device__ static float get(const uint4 &v, int i)
-    {
-        const uint32_t w = (&v.x)[i >> 1];
-        return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
-    }
-    __device__ static float scalar(const void *p, int64_t i)
-    {
-        const uint16_t h = static_cast<const uint16_t *>(p)[i];
-        return __uint_as_float(static_cast<uint32_t>(h) << 16);
-    }
-    // 16-bit lane-wise max of the |x| bit patterns, then the larger half
-    __device__ static uint32_t absmax_bits(const uint4 &v)
-    {
-        const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7fff7fffu, v.y & 0x7fff7fffu),
-                                    __vmaxu2(v.z & 0x7fff7fffu, v.w & 0x7fff7fffu));
-        return max(m << 16, m & 0xffff0000u);
-    }
-};
-
-__device__ __forceinline__ int8_t quant_one(float x, float d)
-{
-    float t = rintf(__fdiv_rn(__fmul_rn(x, 127.0f), d));
-    t = fminf(fmaxf(t, -128.0f), 127.0f);
-    return static_cast<int8_t>(static_cast<int>(t));
-}
-
-// Codes for four values without a divide or a conversion instruction each.
-// The exact code is rint(z), z = RN(t/d), t = RN(127x).  With c = RN(127 *
-// RN(1/d)) and u = RN(x*c), |u - t/d| <= (127|x|/d) * 4 * 2^-24 < 3.1e-5 and
-// |z - t/d| <= 2^-18 < 3.9e-6 (|z| < 128), so |u - z| < 3.5e-5: u and z round
-// to the same integer unless u lies within that distance of a midpoint
-// k + 1/2.  Rounding uses the IEEE nearest-even addition v = u + 1.5*2^23,
-// exact to the unit for |u| < 2^22: v - 1.5*2^23 is rint(u) and the low byte
-// of v's bit pattern is the code in two's complement.  A value within 1e-4
-// of a midpoint (about 2 in 10^4) sets `near`; the caller then redoes the
-// four values with the IEEE divide.  |u| <= 127.0001, so no clamp is needed.
-// The relative bounds need RN(1/d) and c normal and finite, i.e. d in
-// [2^-121, 2^126); outside it the caller takes the divide for every value.
-__device__ __forceinline__ uint32_t quant4(float x0, float x1, float x2, float x3, float c, bool &near)
-{
-    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-    const float u0 = __fmul_rn(x0, c), u1 = __fmul_rn(x1, c), u2 = __fmul_rn(x2, c), u3 = __fmul_rn(x3, c);
-    const float v0 = __fadd_rn(u0, kMagic), v1 = __fadd_rn(u1, kMagic);
-    const float v2 = __fadd_rn(u2, kMagic), v3 = __fadd_rn(u3, kMagic);
-    near |= fabsf(__fsub_rn(u0, __fsub_rn(v0, kMagic))) > 0.4999f;
-    near |= fabsf(__fsub_rn(u1, __fsub_rn(v1, kMagic))) > 0.4999f;
-    near |= fabsf(__fsub_rn(u2, __fsub_rn(v2, kMagic))) > 0.4999f;
-    near |= fabsf(__fsub_rn(u3, __fsub_rn(v3, kMagic))) > 0.4999f;
-    const uint32_t lo = __byte_perm(__float_as_uint(v0), __float_as_uint(v1), 0x0040);
-    const uint32_t hi = __byte_perm(__float_as_uint(v2), __float_as_uint(v3), 0x0040);
-    return __byte_perm(lo, hi, 0x5410);
-}
-
-__device__ __forceinline__ uint32_t quant4_exact(float x0, float x1, float x2, float x3, float d)
-{
-    return static_cast<uint32_t>(static_cast<uint8_t>(quant_one(x0, d))) |
-           (static_cast<uint32_t>(static_cast<uint8_t>(quant_one(x1, d))) << 8) |
-           (static_cast<uint32_t>(static_cast<uint8_t>(quant_one(x2, d))) << 16) |
-           (static_cast<uint32_t>(static_cast<uint8_t>(quant_one(x3, d))) << 24);
-}
+using namespace qrule;
 
 // Max of a uint32 over the TPR threads that own one row.
 template <int TPR>
@@ -123,22 +66,90 @@ __device__ __forceinline__ uint32_t row_max(uint32_t v, uint32_t *red)
     return v;
 }
 
+// Sum of a double over the TPR threads that own one row (fixed tree order).
+template <int TPR>
+__device__ __forceinline__ double row_sum(double v, double *red)
+{
+#pragma unroll
+    for (int o = (TPR < 32 ? TPR : 32) / 2; o > 0; o >>= 1)
+        v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if constexpr (TPR > 32) {
+        constexpr int kWarps = TPR / 32;
+        const int lane = threadIdx.x & 31;
+        const int warp_in_row = (threadIdx.x % TPR) / 32;
+        const int row_slot = threadIdx.x / TPR;
+        if (lane == 0) red[row_slot * kWarps + warp_in_row] = v;
+        __syncthreads();
+        v = red[row_slot * kWarps];
+#pragma unroll
+        for (int i = 1; i < kWarps; ++i) v = __dadd_rn(v, red[row_slot * kWarps + i]);
+    }
+    return v;
+}
+
 __host__ __device__ constexpr int block_threads(int tpr) { return tpr > 256 ? tpr : 256; }
 
 // The two builds: vectors per thread and resident threads per SM.
 constexpr int kWideVPT = 3, kWideThreads = 2048;
 constexpr int kDeepVPT = 5, kDeepThreads = 1536;
 
+// Option bits of the register kernel.
+constexpr int kOptGain = 1;
+constexpr int kOptNorm = 2;
+
+// Element i of a 16-byte vector of x, times the gain when GAIN.
+template <typename T, bool GAIN>
+__device__ __forceinline__ float elem(const uint4 &b, const float *gv, int i)
+{
+    const float v = In<T>::get(b, i);
+    if constexpr (GAIN) return __fmul_rn(v, gv[i]);
+    else return v;
+}
+
+// The E gains of vector v (E = 4 or 8 floats, one or two 16-byte loads).
+template <int E>
+__device__ __forceinline__ void load_gain(const float *g, int64_t v, float (&gv)[8])
+{
+    const uint4 a = ld_act_u4(g + v * E);
+    gv[0] = __uint_as_float(a.x); gv[1] = __uint_as_float(a.y);
+    gv[2] = __uint_as_float(a.z); gv[3] = __uint_as_float(a.w);
+    if constexpr (E == 8) {
+        const uint4 b = ld_act_u4(g + v * E + 4);
+        gv[4] = __uint_as_float(b.x); gv[5] = __uint_as_float(b.y);
+        gv[6] = __uint_as_float(b.z); gv[7] = __uint_as_float(b.w);
+    }
+}
+
+// s_x of a row from max|u| (nonzero): gamma/127 in fp32 with neither the
+// norm nor the rotation (equal to the fp64 quotient rounded once), else
+// gamma / sqrt(hb) / rms / 127 in fp64, rounded once to fp32.
+__device__ __forceinline__ float row_scale(float gmax, bool norm, double ss, int64_t K, float eps_norm, int hb)
+{
+    if (!norm && hb <= 1) return __fdiv_rn(gmax, 127.0f);
+    double s = static_cast<double>(gmax);
+    if (hb > 1) s = __ddiv_rn(s, __dsqrt_rn(static_cast<double>(hb)));
+    if (norm)
+        s = __ddiv_rn(s, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, static_cast<double>(K)), static_cast<double>(eps_norm))));
+    return __double2float_rn(__ddiv_rn(s, 127.0));
+}
+
 // Rows whose 16-byte vectors fit TPR*VPT registers: one global read.
-template <typename T, int TPR, int VPT, int SM_THREADS>
+// OPT = 0 is the plain per-token quantiser; kOptGain multiplies x by g
+// (g 16-byte aligned), kOptNorm applies the RMSNorm factor to the scale
+// (eps must be 0 with options).
+template <typename T, int TPR, int VPT, int SM_THREADS, int OPT>
 __global__ void __launch_bounds__(block_threads(TPR), SM_THREADS / block_threads(TPR))
 act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, float eps,
-               int8_t *__restrict__ q, int64_t ldq, float *__restrict__ s_x, int32_t *status)
+               int8_t *__restrict__ q, int64_t ldq, float *__restrict__ s_x, int32_t *status,
+               const float *__restrict__ g, float eps_norm)
 {
+    constexpr bool GAIN = (OPT & kOptGain) != 0;
+    constexpr bool NORM = (OPT & kOptNorm) != 0;
     constexpr int kThreads = block_threads(TPR);
     constexpr int kRows = kThreads / TPR;
     constexpr int E = In<T>::kPerVec;
     __shared__ uint32_t red[kThreads / 32];
+    __shared__ double red_ss[NORM ? kThreads / 32 : 1];
     pdl_wait();
     pdl_trigger();
 
@@ -150,12 +161,26 @@ act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
 
     uint4 buf[VPT];
     uint32_t amax = 0;
+    double ss = 0.0;
+    float gv[8];
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
         const int64_t v = r + static_cast<int64_t>(i) * TPR;
         if (live && v < nvec) {
-            buf[i] = ld_stream_u4(xrow + v * 16);
-            amax = max(amax, In<T>::absmax_bits(buf[i]));
+            buf[i] = ld_act_u4(xrow + v * 16);
+            if constexpr (GAIN || NORM) {
+                if constexpr (GAIN) load_gain<E>(g, v, gv);
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    amax = max(amax, __float_as_uint(elem<T, GAIN>(buf[i], gv, e)) & 0x7fffffffu);
+                    if constexpr (NORM) {
+                        const double xd = static_cast<double>(In<T>::get(buf[i], e));
+                        ss = __fma_rn(xd, xd, ss);
+                    }
+                }
+            } else {
+                amax = max(amax, In<T>::absmax_bits(buf[i]));
+            }
         }
     }
     // Tail elements past the last whole vector, one per thread.
@@ -164,15 +189,18 @@ act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
     const bool has_tail = live && (tail0 + r < K) && r < E;
     if (has_tail) {
         tail_x = In<T>::scalar(xrow, tail0 + r);
+        if constexpr (NORM) ss = __fma_rn(static_cast<double>(tail_x), static_cast<double>(tail_x), ss);
+        if constexpr (GAIN) tail_x = __fmul_rn(tail_x, g[tail0 + r]);
         amax = max(amax, __float_as_uint(tail_x) & 0x7fffffffu);
     }
     amax = row_max<TPR>(amax, red);
+    if constexpr (NORM) ss = row_sum<TPR>(ss, red_ss);
     if (!live) return;
 
-    const float g = __uint_as_float(amax);
-    const bool bad = !finite_bits(amax) || !finite_bits(__float_as_uint(__fmul_rn(g, 127.0f)));
+    const float gm = __uint_as_float(amax);
+    const bool bad = !finite_bits(amax) || !finite_bits(__float_as_uint(__fmul_rn(gm, 127.0f)));
     if (bad && r == 0) report(status, LOWBIT_ERR_NONFINITE);
-    const float d = __fadd_rn(g, eps);
+    const float d = __fadd_rn(gm, eps);
     const float c = __fmul_rn(127.0f, __frcp_rn(d));
     // Rows with max|x| below about 3.7e-37, or an eps near the fp32 maximum.
     const bool slow = !(d >= 0x1p-121f && d < 0x1p126f);
@@ -183,19 +211,26 @@ act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
         const int64_t v = r + static_cast<int64_t>(i) * TPR;
         if (v < nvec) {
             const uint4 &b = buf[i];
+            if constexpr (GAIN) load_gain<E>(g, v, gv);
             if constexpr (E == 4) {
                 bool near = slow;
-                uint32_t out = quant4(In<T>::get(b, 0), In<T>::get(b, 1), In<T>::get(b, 2), In<T>::get(b, 3), c, near);
-                if (near) out = quant4_exact(In<T>::get(b, 0), In<T>::get(b, 1), In<T>::get(b, 2), In<T>::get(b, 3), d);
+                const float u0 = elem<T, GAIN>(b, gv, 0), u1 = elem<T, GAIN>(b, gv, 1);
+                const float u2 = elem<T, GAIN>(b, gv, 2), u3 = elem<T, GAIN>(b, gv, 3);
+                uint32_t out = quant4(u0, u1, u2, u3, c, near);
+                if (near) out = quant4_exact(u0, u1, u2, u3, d);
                 if (amax == 0) out = 0;
                 *reinterpret_cast<uint32_t *>(qrow + v * 4) = out;
             } else {
                 bool near = slow;
-                uint32_t lo = quant4(In<T>::get(b, 0), In<T>::get(b, 1), In<T>::get(b, 2), In<T>::get(b, 3), c, near);
-                uint32_t hi = quant4(In<T>::get(b, 4), In<T>::get(b, 5), In<T>::get(b, 6), In<T>::get(b, 7), c, near);
+                uint32_t lo = quant4(elem<T, GAIN>(b, gv, 0), elem<T, GAIN>(b, gv, 1), elem<T, GAIN>(b, gv, 2),
+                                     elem<T, GAIN>(b, gv, 3), c, near);
+                uint32_t hi = quant4(elem<T, GAIN>(b, gv, 4), elem<T, GAIN>(b, gv, 5), elem<T, GAIN>(b, gv, 6),
+                                     elem<T, GAIN>(b, gv, 7), c, near);
                 if (near) {
-                    lo = quant4_exact(In<T>::get(b, 0), In<T>::get(b, 1), In<T>::get(b, 2), In<T>::get(b, 3), d);
-                    hi = quant4_exact(In<T>::get(b, 4), In<T>::get(b, 5), In<T>::get(b, 6), In<T>::get(b, 7), d);
+                    lo = quant4_exact(elem<T, GAIN>(b, gv, 0), elem<T, GAIN>(b, gv, 1), elem<T, GAIN>(b, gv, 2),
+                                      elem<T, GAIN>(b, gv, 3), d);
+                    hi = quant4_exact(elem<T, GAIN>(b, gv, 4), elem<T, GAIN>(b, gv, 5), elem<T, GAIN>(b, gv, 6),
+                                      elem<T, GAIN>(b, gv, 7), d);
                 }
                 if (amax == 0) lo = hi = 0;
                 *reinterpret_cast<uint2 *>(qrow + v * 8) = make_uint2(lo, hi);
@@ -203,7 +238,10 @@ act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
         }
     }
     if (has_tail) qrow[tail0 + r] = amax != 0 ? quant_one(tail_x, d) : 0;
-    if (r == 0) s_x[row] = amax != 0 ? __fdiv_rn(g, 127.0f) : 0.0f;
+    if (r == 0) {
+        if constexpr (OPT == 0) s_x[row] = amax != 0 ? __fdiv_rn(gm, 127.0f) : 0.0f;
+        else s_x[row] = amax != 0 ? row_scale(gm, NORM, ss, K, eps_norm, 0) : 0.0f;
+    }
 }
 
 // Rows too long for registers, or rows without 16-byte alignment: a max
@@ -233,16 +271,146 @@ act_quant_long(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
     if (threadIdx.x == 0) s_x[row] = amax != 0 ? __fdiv_rn(g, 127.0f) : 0.0f;
 }
 
+// The prologue with the row staged in shared memory as fp32: gain, sum of
+// squares, block Hadamard transform (one __syncthreads per stage), absmax,
+// codes.  Any alignment; K * 4 bytes of dynamic shared memory.  One block of
+// 256 threads per row.
+constexpr int kStagedThreads = 256;
+
+//
+// Modes for a row split over ranks (the input dimension of a row-parallel
+// layer), where the per-token statistics are reduced across ranks before the
+// codes are taken: kStagedFull computes codes and scale from this slice
+// alone; kStagedStats writes only the slice's max|u| (stat_max) and sum of
+// squares (stat_ss, when not NULL); kStagedCodes takes the codes with the
+// given row maximum stat_max[t] (the maximum over the whole row).
+constexpr int kStagedFull = 0;
+constexpr int kStagedStats = 1;
+constexpr int kStagedCodes = 2;
+
+template <typename T>
+__global__ void __launch_bounds__(kStagedThreads)
+act_prologue_staged(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx,
+                    const float *__restrict__ g, int norm, float eps_norm, int hb,
+                    int8_t *__restrict__ q, int64_t ldq, float *__restrict__ s_x, int32_t *status,
+                    int mode = kStagedFull, float *__restrict__ stat_max = nullptr,
+                    double *__restrict__ stat_ss = nullptr)
+{
+    extern __shared__ float su[];
+    __shared__ uint32_t red[kStagedThreads / 32];
+    __shared__ double red_ss[kStagedThreads / 32];
+    pdl_wait();
+    pdl_trigger();
+    const int64_t row = blockIdx.x;
+    const char *xrow = static_cast<const char *>(x) + row * ldx * sizeof(T);
+    double ss = 0.0;
+    for (int64_t k = threadIdx.x; k < K; k += kStagedThreads) {
+        const float v = In<T>::scalar(xrow, k);
+        if (norm) ss = __fma_rn(static_cast<double>(v), static_cast<double>(v), ss);
+        su[k] = g != nullptr ? __fmul_rn(v, g[k]) : v;
+    }
+    // the block's sum of squares (fixed tree order)
+    if (norm) {
+        ss = row_sum<kStagedThreads>(ss, red_ss);
+    }
+    __syncthreads();
+    if (hb > 1) {
+        const int64_t half = K / 2;
+        for (int h = 1; h < hb; h <<= 1) {
+            for (int64_t p = threadIdx.x; p < half; p += kStagedThreads) {
+                const int64_t j = (p / h) * 2 * h + (p % h);
+                const float a = su[j], b = su[j + h];
+                su[j] = __fadd_rn(a, b);
+                su[j + h] = __fsub_rn(a, b);
+            }
+            __syncthreads();
+        }
+    }
+    uint32_t amax = 0;
+    for (int64_t k = threadIdx.x; k < K; k += kStagedThreads)
+        amax = max(amax, __float_as_uint(su[k]) & 0x7fffffffu);
+    amax = row_max<kStagedThreads>(amax, red);
+    if (mode == kStagedStats) {
+        if (!finite_bits(amax) && threadIdx.x == 0) report(status, LOWBIT_ERR_NONFINITE);
+        if (threadIdx.x == 0) {
+            stat_max[row] = __uint_as_float(amax);
+            if (stat_ss != nullptr) stat_ss[row] = ss;
+        }
+        return;
+    }
+    if (mode == kStagedCodes) {
+        // this slice's values may not exceed the row maximum it was given
+        const uint32_t given = ld_act_u32(stat_max + row) & 0x7fffffffu;
+        if (amax > given && threadIdx.x == 0) report(status, LOWBIT_ERR_INVALID_ARG);
+        amax = given;
+    }
+    const float gm = __uint_as_float(amax);
+    const bool bad = !finite_bits(amax) || !finite_bits(__float_as_uint(__fmul_rn(gm, 127.0f)));
+    if (bad && threadIdx.x == 0) report(status, LOWBIT_ERR_NONFINITE);
+    int8_t *qrow = q + row * ldq;
+    for (int64_t k = threadIdx.x; k < K; k += kStagedThreads)
+        qrow[k] = amax != 0 ? quant_one(su[k], gm) : 0;
+    if (threadIdx.x == 0 && mode == kStagedFull)
+        s_x[row] = amax != 0 ? row_scale(gm, norm != 0, ss, K, eps_norm, hb) : 0.0f;
+}
+
+// s_x of rows whose statistics were reduced over a split row: max|u| over
+// the whole row, the sum of squares over the whole row (norm), K_total
+// features.
+__global__ void row_scales_from_stats(const float *__restrict__ row_max, const double *__restrict__ row_ss, int64_t M,
+                                      int64_t K_total, int norm, float eps_norm, int hb, float *__restrict__ s_x,
+                                      int32_t *status)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (t >= M) return;
+    const float gm = ld_act_f32(row_max + t);
+    const uint32_t bits = __float_as_uint(gm) & 0x7fffffffu;
+    if (!finite_bits(bits) || !finite_bits(__float_as_uint(__fmul_rn(gm, 127.0f)))) report(status, LOWBIT_ERR_NONFINITE);
+    s_x[t] = bits != 0 ? row_scale(__uint_as_float(bits), norm != 0, norm ? ld_act_f64(row_ss + t) : 0.0, K_total, eps_norm, hb)
+                       : 0.0f;
+}
+
+// Largest row the staged prologue kernel holds in shared memory.
+constexpr int64_t kMaxStagedK = 48 * 1024;
+
+template <typename T>
+lowbit_status launch_staged(const void *x, int64_t M, int64_t K, int64_t ldx, const float *g, int norm,
+                            float eps_norm, int hb, int8_t *q, int64_t ldq, float *s_x, int32_t *status,
+                            cudaStream_t st, int mode = kStagedFull, float *row_max = nullptr,
+                            double *row_ss = nullptr)
+{
+    static PerDevice configured;  // the shared-memory limit is raised once per device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    if (configured.get(dev, [&] {
+            return cudaFuncSetAttribute(act_prologue_staged<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(kMaxStagedK * 4)) == cudaSuccess ? 1 : 0;
+        }) <= 0)
+        return LOWBIT_ERR_CUDA;
+    return launch_pdl(act_prologue_staged<T>, dim3(static_cast<unsigned>(M)), dim3(kStagedThreads),
+                      static_cast<size_t>(K) * 4, st, 0, x, M, K, ldx, g, norm, eps_norm, hb, q, ldq, s_x, status,
+                      mode, row_max, row_ss);
+}
+
 template <typename T>
 lowbit_status launch(const void *x, int64_t M, int64_t K, int64_t ldx, float eps, int8_t *q,
-                     int64_t ldq, float *s_x, int32_t *status, cudaStream_t st)
+                     int64_t ldq, float *s_x, int32_t *status, cudaStream_t st, const float *g, int opt,
+                     float eps_norm)
 {
     constexpr int E = In<T>::kPerVec;
     const int64_t nvec = K / E;
-    // 16-byte vector loads need a 16-byte aligned base and row stride; any
-    // other layout takes the scalar-load kernel.
-    const bool vec_ok = (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (ldx * static_cast<int64_t>(sizeof(T))) % 16 == 0;
+    // 16-byte vector loads need a 16-byte aligned base and row stride (and a
+    // 16-byte aligned gain); any other layout takes a scalar-load kernel.
+    const bool vec_ok = (reinterpret_cast<uintptr_t>(x) & 15u) == 0 &&
+                        (ldx * static_cast<int64_t>(sizeof(T))) % 16 == 0 &&
+                        (g == nullptr || (reinterpret_cast<uintptr_t>(g) & 15u) == 0);
+    auto staged = [&]() {
+        return launch_staged<T>(x, M, K, ldx, g, (opt & kOptNorm) ? 1 : 0, eps_norm, 0, q, ldq, s_x, status, st);
+    };
     if (!vec_ok) {
+        if (opt != 0) return staged();
         return launch_pdl(act_quant_long<T>, dim3(static_cast<unsigned>(M)), dim3(256), 0, st, 0, x, M, K, ldx, eps,
                           q, ldq, s_x, status);
     }
@@ -259,18 +427,28 @@ lowbit_status launch(const void *x, int64_t M, int64_t K, int64_t ldx, float eps
                       (tpr_wide == 0 || (tpr_deep < tpr_wide &&
                                          M * tpr_deep >= 2 * static_cast<int64_t>(device_sm_count()) * kDeepThreads));
     const int tpr = deep ? tpr_deep : tpr_wide;
-    if (tpr == 0)  // longer than either register build holds
+    if (tpr == 0) {  // longer than either register build holds
+        if (opt != 0) return staged();
         return launch_pdl(act_quant_long<T>, dim3(static_cast<unsigned>(M)), dim3(256), 0, st, 0, x, M, K, ldx, eps,
                           q, ldq, s_x, status);
+    }
     const int rows_per_block = block_threads(tpr) / tpr;
     const unsigned grid = static_cast<unsigned>((M + rows_per_block - 1) / rows_per_block);
-#define LOWBIT_AQ(TPR)                                                                                          \
-    if (tpr == TPR) {                                                                                           \
-        if (deep)                                                                                               \
-            return launch_pdl(act_quant_regs<T, TPR, kDeepVPT, kDeepThreads>, dim3(grid), dim3(block_threads(TPR)), \
-                              0, st, 0, x, M, K, ldx, eps, q, ldq, s_x, status);                                \
-        return launch_pdl(act_quant_regs<T, TPR, kWideVPT, kWideThreads>, dim3(grid), dim3(block_threads(TPR)),    \
-                          0, st, 0, x, M, K, ldx, eps, q, ldq, s_x, status);                                    \
+#define LOWBIT_AQ_OPT(TPR, OPT)                                                                                  \
+    if (opt == OPT) {                                                                                            \
+        if (deep)                                                                                                \
+            return launch_pdl(act_quant_regs<T, TPR, kDeepVPT, kDeepThreads, OPT>, dim3(grid),                   \
+                              dim3(block_threads(TPR)), 0, st, 0, x, M, K, ldx, eps, q, ldq, s_x, status, g,     \
+                              eps_norm);                                                                         \
+        return launch_pdl(act_quant_regs<T, TPR, kWideVPT, kWideThreads, OPT>, dim3(grid), dim3(block_threads(TPR)), \
+                          0, st, 0, x, M, K, ldx, eps, q, ldq, s_x, status, g, eps_norm);                        \
+    }
+#define LOWBIT_AQ(TPR)                                                                                           \
+    if (tpr == TPR) {                                                                                            \
+        LOWBIT_AQ_OPT(TPR, 0)                                                                                    \
+        LOWBIT_AQ_OPT(TPR, kOptGain)                                                                             \
+        LOWBIT_AQ_OPT(TPR, kOptNorm)                                                                             \
+        LOWBIT_AQ_OPT(TPR, kOptGain | kOptNorm)                                                                  \
     }
     LOWBIT_AQ(8)
     LOWBIT_AQ(32)
@@ -280,8 +458,8 @@ lowbit_status launch(const void *x, int64_t M, int64_t K, int64_t ldx, float eps
     LOWBIT_AQ(512)
     LOWBIT_AQ(1024)
 #undef LOWBIT_AQ
-    return launch_pdl(act_quant_long<T>, dim3(static_cast<unsigned>(M)), dim3(256), 0, st, 0, x, M, K, ldx, eps, q,
-                      ldq, s_x, status);
+#undef LOWBIT_AQ_OPT
+    return LOWBIT_ERR_INVALID_ARG;
 }
 
 }  // namespace
@@ -290,8 +468,58 @@ lowbit_status act_quant_launch(const void *x, lowbit_dtype xdt, int64_t M, int64
                                float eps, int8_t *q, int64_t ldq, float *s_x, int32_t *status,
                                cudaStream_t st)
 {
-    if (xdt == LOWBIT_F32) return launch<float>(x, M, K, ldx, eps, q, ldq, s_x, status, st);
-    return launch<__nv_bfloat16>(x, M, K, ldx, eps, q, ldq, s_x, status, st);
+    if (xdt == LOWBIT_F32) return launch<float>(x, M, K, ldx, eps, q, ldq, s_x, status, st, nullptr, 0, 0.0f);
+    return launch<__nv_bfloat16>(x, M, K, ldx, eps, q, ldq, s_x, status, st, nullptr, 0, 0.0f);
+}
+
+int64_t act_prologue_max_staged_k() { return kMaxStagedK; }
+
+lowbit_status act_prologue_launch(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                  const float *g, int norm, float eps_norm, int hb, int8_t *q, int64_t ldq,
+                                  float *s_x, int32_t *status, cudaStream_t st)
+{
+    if (hb > 1) {
+        if (xdt == LOWBIT_F32)
+            return launch_staged<float>(x, M, K, ldx, g, norm, eps_norm, hb, q, ldq, s_x, status, st);
+        return launch_staged<__nv_bfloat16>(x, M, K, ldx, g, norm, eps_norm, hb, q, ldq, s_x, status, st);
+    }
+    const int opt = (g != nullptr ? kOptGain : 0) | (norm ? kOptNorm : 0);
+    if (xdt == LOWBIT_F32) return launch<float>(x, M, K, ldx, 0.0f, q, ldq, s_x, status, st, g, opt, eps_norm);
+    return launch<__nv_bfloat16>(x, M, K, ldx, 0.0f, q, ldq, s_x, status, st, g, opt, eps_norm);
+}
+
+// Per-token statistics of a row slice (split-row mode): max|u| after the
+// gain and rotation, and the fp64 sum of squares of x when row_ss is given.
+lowbit_status act_row_stats_launch(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                   const float *g, int hb, float *row_max, double *row_ss, int32_t *status,
+                                   cudaStream_t st)
+{
+    const int norm = row_ss != nullptr ? 1 : 0;
+    if (xdt == LOWBIT_F32)
+        return launch_staged<float>(x, M, K, ldx, g, norm, 0.0f, hb, nullptr, 0, nullptr, status, st, kStagedStats,
+                                    row_max, row_ss);
+    return launch_staged<__nv_bfloat16>(x, M, K, ldx, g, norm, 0.0f, hb, nullptr, 0, nullptr, status, st,
+                                        kStagedStats, row_max, row_ss);
+}
+
+// Codes of a row slice with the given whole-row maximum (split-row mode).
+lowbit_status act_codes_given_max_launch(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                         const float *g, int hb, const float *row_max, int8_t *q, int64_t ldq,
+                                         int32_t *status, cudaStream_t st)
+{
+    float *rm = const_cast<float *>(row_max);  // read only in this mode
+    if (xdt == LOWBIT_F32)
+        return launch_staged<float>(x, M, K, ldx, g, 0, 0.0f, hb, q, ldq, nullptr, status, st, kStagedCodes, rm,
+                                    nullptr);
+    return launch_staged<__nv_bfloat16>(x, M, K, ldx, g, 0, 0.0f, hb, q, ldq, nullptr, status, st, kStagedCodes, rm,
+                                        nullptr);
+}
+
+lowbit_status act_scales_launch(const float *row_max, const double *row_ss, int64_t M, int64_t K_total, int norm,
+                                float eps_norm, int hb, float *s_x, int32_t *status, cudaStream_t st)
+{
+    return launch_pdl(row_scales_from_stats, dim3(static_cast<unsigned>((M + 255) / 256)), dim3(256), 0, st, 0,
+                      row_max, row_ss, M, K_total, norm, eps_norm, hb, s_x, status);
 }
 
 }  // namespace lowbit

@@ -311,7 +311,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
                 // Let copies already issued land before the CTA leaves.
                 for (uint32_t i = 0; i < ST && i < g; ++i) {
                     const uint32_t gi = g - 1 - i;
-                    wait_bar(&full_tma[gi % ST], (gi / ST) & 1u, abort_flag, nullptr, 200000000ll);
+                    drain_bar(&full_tma[gi % ST], (gi / ST) & 1u);
                 }
             }
         }
@@ -346,7 +346,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
             }
             // All MMAs this thread issued are complete once `drain` flips.
             tc_commit(drain);
-            wait_bar(drain, 0, abort_flag, nullptr, 200000000ll);
+            drain_bar(drain, 0);
         }
     } else if (warp < 6) {
         // ---------------- expanders ----------------
@@ -391,7 +391,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
             const int64_t m0 = (tile % num_m) * BM;
             const int64_t n0 = (tile / num_m) * BN;
             const int64_t row0 = m0 + quarter * 32;
-            const float sx = (row0 + lane < M) ? s_x[row0 + lane] : 0.0f;
+            const float sx = (row0 + lane < M) ? ld_act_f32(s_x + row0 + lane) : 0.0f;
 #pragma unroll 1
             for (int cc = 0; cc < BN / 32; ++cc) {
                 const int64_t nc = n0 + cc * 32;
@@ -534,7 +534,7 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
             if (!ok) {
                 for (uint32_t i = 0; i < ST && i < g; ++i) {
                     const uint32_t gi = g - 1 - i;
-                    wait_bar(&full_tma[gi % ST], (gi / ST) & 1u, abort_flag, nullptr, 200000000ll);
+                    drain_bar(&full_tma[gi % ST], (gi / ST) & 1u);
                 }
             }
         }
@@ -556,7 +556,7 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
             }
             if (ok) tc_commit(&acc_full[0]);
             tc_commit(drain);
-            wait_bar(drain, 0, abort_flag, nullptr, 200000000ll);
+            drain_bar(drain, 0);
         }
     } else if (warp < 6) {
         const int et = threadIdx.x - 64;
@@ -622,7 +622,7 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
     cluster_sync_all();
     if (warp >= 6) {
         const uint32_t stage = smem_u32(sStage) + static_cast<uint32_t>((warp - 6) * stage_warp_bytes<OUT>());
-        const float sx = row < M ? s_x[row] : 0.0f;
+        const float sx = row < M ? ld_act_f32(s_x + row) : 0.0f;
         const float sw_tensor = (FMT == kT2) ? s_w[0] : 0.0f;
         for (int cc = 0; cc < W / 32; ++cc) {
             uint32_t v[32];
@@ -823,7 +823,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             if (!ok) {
                 for (uint32_t i = 0; i < ST && i < g; ++i) {
                     const uint32_t gi = g - 1 - i;
-                    wait_bar(&full_tma[gi % ST], (gi / ST) & 1u, abort_flag, nullptr, 200000000ll);
+                    drain_bar(&full_tma[gi % ST], (gi / ST) & 1u);
                 }
             }
         }
@@ -854,7 +854,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 tc_commit_pair_both(&acc_full[b]);
             }
             tc_commit_pair_self(drain);
-            wait_bar(drain, 0, abort_flag, nullptr, 200000000ll);
+            drain_bar(drain, 0);
         }
     } else if (warp < 6) {
         // ---------------- expanders: own 128 features ----------------
@@ -897,7 +897,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             const int64_t m0 = (tile % num_m) * 2 * PBM + rank * PBM;
             const int64_t n0 = (tile / num_m) * 2 * PBN;
             const int64_t row0 = m0 + quarter * 32;
-            const float sx = (row0 + lane < M) ? s_x[row0 + lane] : 0.0f;
+            const float sx = (row0 + lane < M) ? ld_act_f32(s_x + row0 + lane) : 0.0f;
 #pragma unroll 1
             for (int cc = 0; cc < 2 * PBN / 32; ++cc) {
                 const int64_t nc = n0 + cc * 32;
@@ -1078,4 +1078,9 @@ lowbit_status gemm_pair_launch(const int8_t *q, int64_t ldq, const float *s_x, i
         return launch_pair_fmt<kB1>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, st);
     return launch_pair_fmt<kI4>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, st);
 }
+}  // namespace lowbit
+
+namespace lowbit {
+// This file's copy of the pipeline wait bound (see lowbit_set_wait_limit).
+lowbit_status set_wait_limit_gemm(long long cycles) { return tc::set_wait_limit_here(cycles); }
 }  // namespace lowbit

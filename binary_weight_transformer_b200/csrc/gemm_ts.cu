@@ -138,7 +138,7 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&v)[32], float sw, c
             if constexpr (OUT == LOWBIT_I32) {
                 asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
             } else {
-                const float sx = (t0 + i < M) ? __ldg(s_x + t0 + i) : 0.0f;
+                const float sx = (t0 + i < M) ? ld_act_f32(s_x + t0 + i) : 0.0f;
                 const float f = rescale(a, sw, sx);
                 if constexpr (OUT == LOWBIT_F32) {
                     asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(__float_as_uint(f)) : "memory");
@@ -172,9 +172,9 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&v)[32], float sw, c
                 if constexpr (OUT == LOWBIT_I32) {
                     static_cast<int32_t *>(y)[idx] = a;
                 } else if constexpr (OUT == LOWBIT_F32) {
-                    static_cast<float *>(y)[idx] = rescale(a, sw, s_x[t0 + i]);
+                    static_cast<float *>(y)[idx] = rescale(a, sw, ld_act_f32(s_x + t0 + i));
                 } else {
-                    static_cast<__nv_bfloat16 *>(y)[idx] = __float2bfloat16_rn(rescale(a, sw, s_x[t0 + i]));
+                    static_cast<__nv_bfloat16 *>(y)[idx] = __float2bfloat16_rn(rescale(a, sw, ld_act_f32(s_x + t0 + i)));
                 }
             }
         }
@@ -290,7 +290,7 @@ gemm_ts_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             if (!ok) {
                 for (uint32_t i = 0; i < kStages && i < g; ++i) {
                     const uint32_t gi = g - 1 - i;
-                    wait_bar(&full_tma[gi % kStages], (gi / kStages) & 1u, abort_flag, nullptr, 200000000ll);
+                    drain_bar(&full_tma[gi % kStages], (gi / kStages) & 1u);
                 }
             }
         }
@@ -325,7 +325,7 @@ gemm_ts_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 tc_commit(&acc_full[b]);
             }
             tc_commit(drain);
-            wait_bar(drain, 0, abort_flag, nullptr, 200000000ll);
+            drain_bar(drain, 0);
         }
     } else if (warp < 6) {
         // ---------------- expanders: packed -> TMEM ----------------
@@ -590,7 +590,7 @@ gemm_ts_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
             if (!ok) {
                 for (uint32_t i = 0; i < static_cast<uint32_t>(S) && i < g; ++i) {
                     const uint32_t gi = g - 1 - i;
-                    wait_bar(&full_tma[gi % S], (gi / S) & 1u, abort_flag, nullptr, 200000000ll);
+                    drain_bar(&full_tma[gi % S], (gi / S) & 1u);
                 }
             }
         }
@@ -624,7 +624,7 @@ gemm_ts_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
                 tc_commit_pair_both(&acc_full[b]);
             }
             tc_commit_pair_self(drain);
-            wait_bar(drain, 0, abort_flag, nullptr, 200000000ll);
+            drain_bar(drain, 0);
         }
     } else if (warp < 6) {
         // ---------------- expanders: packed -> own TMEM ----------------
@@ -802,4 +802,9 @@ lowbit_status gemm_ts_pair_launch(const int8_t *q, int64_t ldq, const float *s_x
         return launch_pair_fmt<kB1>(mq, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, nt, status, st);
     return launch_pair_fmt<kI4>(mq, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, nt, status, st);
 }
+}  // namespace lowbit
+
+namespace lowbit {
+// This file's copy of the pipeline wait bound (see lowbit_set_wait_limit).
+lowbit_status set_wait_limit_gemm_ts(long long cycles) { return tc::set_wait_limit_here(cycles); }
 }  // namespace lowbit

@@ -85,13 +85,55 @@ __device__ __forceinline__ void report(int32_t *status, int code)
 __device__ __forceinline__ bool finite_bits(uint32_t u) { return (u & 0x7f800000u) != 0x7f800000u; }
 
 // 16-byte streaming load that does not allocate in L1 (weights are read once
-// per launch).
+// per launch).  It takes the non-coherent read-only path, so it is only for
+// data that no kernel writes while the reader is resident: the packed
+// weights (see LOWBIT_LINEAR_WEIGHTS_STABLE).
 __device__ __forceinline__ uint4 ld_stream_u4(const void *p)
 {
     uint4 v;
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
+    return v;
+}
+
+// Loads of activation-side data (x, codes, scales).  The kernels are
+// launched with programmatic stream serialization, so a kernel can be
+// resident while the kernel before it still writes these arrays; after
+// griddepcontrol.wait the writes are visible to coherent loads, but the
+// read-only (.nc) path is defined only for data constant over the reader's
+// lifetime.  These loads are cached in L2 only (.cg), which is coherent and
+// does not allocate in L1.
+__device__ __forceinline__ uint4 ld_act_u4(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ld_act_u32(const void *p)
+{
+    uint32_t v;
+    asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint16_t ld_act_u16(const void *p)
+{
+    uint16_t v;
+    asm volatile("ld.global.cg.u16 %0, [%1];" : "=h"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ float ld_act_f32(const float *p) { return __uint_as_float(ld_act_u32(p)); }
+
+__device__ __forceinline__ double ld_act_f64(const double *p)
+{
+    double v;
+    asm volatile("ld.global.cg.f64 %0, [%1];" : "=d"(v) : "l"(p) : "memory");
     return v;
 }
 
@@ -119,6 +161,9 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 // Host-side launch helpers (defined in abi.cu and pack.cu).
 namespace lowbit {
 lowbit_status launch_status();
+// LOWBIT_OK on a B200 (sm_100); LOWBIT_ERR_UNSUPPORTED on another device,
+// LOWBIT_ERR_CUDA when the device cannot be queried.  Cached per device.
+lowbit_status check_device();
 int device_sm_count();
 
 // Launch with programmatic stream serialization (see pdl_wait); cluster_x > 0

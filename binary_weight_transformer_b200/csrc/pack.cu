@@ -75,6 +75,8 @@ __device__ __forceinline__ float clip_tanh(float w)
 // mode 0: ternary, write the fp64 row sum of |w| to rows[n].
 // mode 1: binary, write s_w[n] = fp32(sum / K).
 // mode 2: 4-bit, write s_w[n] = max_k |clip_tanh(w)| / 7.
+// mode 3: centred binary, write the fp64 row sums of w to rows[n] and of |w|
+//         to rows[N + n].
 __global__ void row_reduce(const float *__restrict__ w, int64_t N, int64_t K, int64_t ldw, int mode,
                            double *__restrict__ rows, float *__restrict__ s_w, int32_t *status)
 {
@@ -90,6 +92,16 @@ __global__ void row_reduce(const float *__restrict__ w, int64_t N, int64_t K, in
             m = fmaxf(m, fabsf(clip_tanh(v)));
         }
         s_w[n] = __fdiv_rn(m, 7.0f);
+    } else if (mode == 3) {
+        double r = 0.0, ra = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            const float v = wr[k];
+            bad |= !finite_bits(__float_as_uint(v));
+            r = __dadd_rn(r, static_cast<double>(v));
+            ra = __dadd_rn(ra, fabs(static_cast<double>(v)));
+        }
+        rows[n] = r;
+        rows[N + n] = ra;
     } else {
         double r = 0.0;
         for (int64_t k = 0; k < K; ++k) {
@@ -110,6 +122,48 @@ __global__ void ternary_gamma(const double *__restrict__ rows, int64_t N, int64_
     double S = 0.0;
     for (int64_t n = 0; n < N; ++n) S = __dadd_rn(S, rows[n]);
     s_w[0] = __double2float_rn(__ddiv_rn(S, static_cast<double>(N) * static_cast<double>(K)));
+}
+
+// Centred binary scalars: one thread sums the row sums in order n = 0..N-1;
+// alpha = mean(W) and beta = mean|W|, each the fp64 mean rounded once to fp32,
+// stored as two floats after the 2N row sums.
+__global__ void centred_scalars(double *__restrict__ rows, int64_t N, int64_t K)
+{
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    double S = 0.0, A = 0.0;
+    for (int64_t n = 0; n < N; ++n) {
+        S = __dadd_rn(S, rows[n]);
+        A = __dadd_rn(A, rows[N + n]);
+    }
+    const double nk = static_cast<double>(N) * static_cast<double>(K);
+    float *out = reinterpret_cast<float *>(rows + 2 * N);
+    out[0] = __double2float_rn(__ddiv_rn(S, nk));
+    out[1] = __double2float_rn(__ddiv_rn(A, nk));
+}
+
+// BitNet v1 centred codes in the binary layout: bit 0 (+1) where w > alpha,
+// bit 1 (-1) otherwise (a weight equal to the mean takes -1); the thread of
+// word 0 of each row also writes that row's scale s_w[n] = beta.
+__global__ void pack_centred_words(const float *__restrict__ w, int64_t N, int64_t K, int64_t ldw,
+                                   const float *__restrict__ ab, uint8_t *__restrict__ packed, int64_t ldp,
+                                   float *__restrict__ s_w)
+{
+    const int64_t words_per_row = ldp / 4;
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= N * words_per_row) return;
+    const int64_t n = idx / words_per_row;
+    const int64_t wi = idx % words_per_row;
+    const float alpha = ab[0];
+    const float *wr = w + n * ldw;
+    uint32_t word = 0;
+    const int64_t k0 = wi * 32;
+    for (int kk = 0; kk < 32; ++kk) {
+        const int64_t k = k0 + kk;
+        if (k >= K) break;
+        word |= (wr[k] > alpha ? 0u : 1u) << kk;
+    }
+    reinterpret_cast<uint32_t *>(packed + n * ldp)[wi] = word;
+    if (wi == 0) s_w[n] = ab[1];
 }
 
 // ---------------------------------------------------------------------------
@@ -231,6 +285,18 @@ lowbit_status pack_launch(const float *w, int64_t N, int64_t K, int64_t ldw, low
     return launch_status();
 }
 
+lowbit_status pack_centred_launch(const float *w, int64_t N, int64_t K, int64_t ldw, uint8_t *packed, int64_t ldp,
+                                  float *s_w, void *workspace, int32_t *status, cudaStream_t st)
+{
+    double *rows = static_cast<double *>(workspace);
+    const int64_t nwords = N * (ldp / 4);
+    row_reduce<<<blocks_for(N, 128), 128, 0, st>>>(w, N, K, ldw, 3, rows, s_w, status);
+    centred_scalars<<<1, 32, 0, st>>>(rows, N, K);
+    pack_centred_words<<<blocks_for(nwords, 256), 256, 0, st>>>(w, N, K, ldw, reinterpret_cast<const float *>(rows + 2 * N),
+                                                                 packed, ldp, s_w);
+    return launch_status();
+}
+
 lowbit_status unpack_launch(const uint8_t *packed, int64_t ldp, int64_t N, int64_t K, lowbit_format f,
                             int8_t *codes, int64_t ldc, int32_t *status, cudaStream_t st)
 {
@@ -293,11 +359,11 @@ extern "C" lowbit_status lowbit_pack_ternary_noalloc(const float *w, int64_t N, 
     if (ldp % 16 != 0 || (reinterpret_cast<uintptr_t>(packed) & 15u) != 0 ||
         (reinterpret_cast<uintptr_t>(w) & 3u) != 0 || (reinterpret_cast<uintptr_t>(s_w) & 3u) != 0)
         return LOWBIT_ERR_ALIGNMENT;
+    // The device check reads a per-device cache filled on the first call.
+    const lowbit_status d = check_device();
+    if (d != LOWBIT_OK) return d;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LOWBIT_ERR_CUDA;
-    cudaDeviceProp prop;
-    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
-    if (prop.major != 10 || prop.minor != 0) return LOWBIT_ERR_UNSUPPORTED;
     double *rows = noalloc_scratch(dev);
     if (rows == nullptr) return LOWBIT_ERR_CUDA;
     // Every row sum the call reads (rows 0..N-1) is written earlier in the

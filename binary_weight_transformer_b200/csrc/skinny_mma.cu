@@ -51,7 +51,10 @@ __device__ __forceinline__ uint32_t q_word(const int8_t *__restrict__ q, int64_t
                                            int64_t K)
 {
     if (token >= M || k >= K) return 0u;
-    uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(q + token * ldq + k));
+    // L1-cached: every warp of every block reads the same few KB of codes.
+    // The asm keeps the load after griddepcontrol.wait (see ld_act_u4).
+    uint32_t v;
+    asm volatile("ld.global.ca.u32 %0, [%1];" : "=r"(v) : "l"(q + token * ldq + k) : "memory");
     const int64_t valid = K - k;
     if (valid < 4) v &= (1u << (8 * valid)) - 1u;
     return v;
@@ -215,7 +218,7 @@ skinny_mma_kernel(const int8_t *__restrict__ q, int64_t ldq, const float *__rest
             if constexpr (OUT == LOWBIT_I32) {
                 static_cast<int32_t *>(y)[idy] = a;
             } else {
-                const float f = rescale(a, s_w[FMT == kT2 ? 0 : n], s_x[token]);
+                const float f = rescale(a, s_w[FMT == kT2 ? 0 : n], ld_act_f32(s_x + token));
                 if constexpr (OUT == LOWBIT_F32) static_cast<float *>(y)[idy] = f;
                 else static_cast<__nv_bfloat16 *>(y)[idy] = __float2bfloat16_rn(f);
             }
@@ -281,6 +284,7 @@ stream_mma_kernel(const __grid_constant__ CUtensorMap map_p, const int8_t *__res
 
     if (producer) {
         if (lane == 0) {
+            int issued = 0;
             for (int st = 0; st < nstages; ++st) {
                 const int s = st % kSStages;
                 // the first kSStages waits cannot block or time out; the wait for
@@ -290,6 +294,14 @@ stream_mma_kernel(const __grid_constant__ CUtensorMap map_p, const int8_t *__res
                 if (!tc::wait_bar(&empty[s], ((st / kSStages) & 1u) ^ 1u, abort_flag, status)) break;
                 tc::mbar_arrive_expect_tx(&full[s], kSStageBytes);
                 tc::tma_load_2d(ring + s * kSStageBytes, &map_p, &full[s], st * kSBox, static_cast<int>(n0));
+                issued = st + 1;
+            }
+            // Every copy issued lands before the block leaves, also when the
+            // consumers gave up on a wait (the last kSStages stages; earlier
+            // ones were consumed before their slot was reissued).
+            for (int i = 0; i < kSStages && i < issued; ++i) {
+                const int st = issued - 1 - i;
+                tc::drain_bar(&full[st % kSStages], (st / kSStages) & 1u);
             }
         }
         // every lane of this warp takes part in the epilogue below
@@ -371,7 +383,7 @@ stream_mma_kernel(const __grid_constant__ CUtensorMap map_p, const int8_t *__res
             if constexpr (OUT == LOWBIT_I32) {
                 static_cast<int32_t *>(y)[idy] = a;
             } else {
-                const float f = rescale(a, s_w[FMT == kT2 ? 0 : n], s_x[token]);
+                const float f = rescale(a, s_w[FMT == kT2 ? 0 : n], ld_act_f32(s_x + token));
                 if constexpr (OUT == LOWBIT_F32) static_cast<float *>(y)[idy] = f;
                 else static_cast<__nv_bfloat16 *>(y)[idy] = __float2bfloat16_rn(f);
             }
@@ -459,4 +471,9 @@ lowbit_status skinny_launch(const int8_t *q, int64_t ldq, const float *s_x, int6
     return skinny::launch_fmt<kI4>(q, ldq, s_x, m, K, packed, ldp, row_bytes, s_w, N, y, ydt, ldy, prefetch, status, st);
 }
 
+}  // namespace lowbit
+
+namespace lowbit {
+// This file's copy of the pipeline wait bound (see lowbit_set_wait_limit).
+lowbit_status set_wait_limit_skinny(long long cycles) { return tc::set_wait_limit_here(cycles); }
 }  // namespace lowbit

@@ -14,6 +14,15 @@ namespace tc {
 constexpr int UMMA_K = 32;  // K of one tcgen05.mma kind::i8
 // Wait bound in SM clock cycles: 4e9 cycles is about 2 s at the B200's clocks.
 constexpr long long kWaitCycles = 4000000000ll;
+// Bound of the drain waits after an abort (copies and MMAs already issued
+// always complete; this only keeps a broken pipeline from holding the SM).
+constexpr long long kDrainCycles = 200000000ll;
+
+// The bound the pipeline waits use, per device (one copy per translation
+// unit that includes this header; lowbit_set_wait_limit writes all of them).
+// Failure-detection tests lower it to make a wait run out.  In constant
+// memory, so reading it on a wait's slow path costs a constant-cache hit.
+static __constant__ long long g_wait_limit_cycles = kWaitCycles;
 
 // ---------------------------------------------------------------------------
 // PTX wrappers
@@ -67,22 +76,40 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr)
 }
 
 // Bounded wait: true once the phase with `parity` has completed; false if the
-// CTA aborted or `limit` SM cycles passed (then the timeout is recorded).
+// CTA aborted or the bound passed (then the timeout is recorded and the CTA
+// aborts).  limit < 0 takes the device's bound (g_wait_limit_cycles).
 __device__ inline bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int32_t *status,
-                                long long limit = kWaitCycles)
+                                long long limit = -1)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
+    const long long lim = limit < 0 ? g_wait_limit_cycles : limit;
+    // the clock is read every 64 polls, or on every poll under a very short
+    // bound (a failure-detection test), so that such a bound takes effect at
+    // the first poll that fails
+    const uint32_t every = lim < 4096 ? 0u : 63u;
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0) {
+        if ((i & every) == 0) {
             if (*abort_flag) return false;
-            if (clock64() - t0 > limit) {
+            if (clock64() - t0 > lim) {
                 *abort_flag = 1;
                 report(status, LOWBIT_ERR_TIMEOUT);
                 return false;
             }
         }
+    }
+}
+
+// Wait of the drain after an abort: the copies and MMAs this thread issued
+// complete on their own, so it waits for them whatever the abort flag says,
+// bounded by kDrainCycles.
+__device__ inline bool drain_bar(uint64_t *bar, uint32_t parity)
+{
+    const long long t0 = clock64();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 0 && clock64() - t0 > kDrainCycles) return false;
     }
 }
 
@@ -216,6 +243,14 @@ inline bool make_map_2d(CUtensorMap *map, const void *ptr, uint64_t inner, uint6
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims, strides, box, estride,
               CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Host: this translation unit's copy of g_wait_limit_cycles on the current
+// device (cycles <= 0 restores kWaitCycles).
+static inline lowbit_status set_wait_limit_here(long long cycles)
+{
+    const long long v = cycles > 0 ? cycles : kWaitCycles;
+    return cudaMemcpyToSymbol(g_wait_limit_cycles, &v, sizeof(v)) == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
 }
 
 }  // namespace tc

@@ -29,6 +29,26 @@ Workloads (page and section the shapes come from):
 * ``ternary_4b`` -- 2560->9728 and 9728->2560, ternary, bf16 activations with
   0.5% x10 outliers, M in {1, 16, 128, 1024, 8192}, bf16 out (4B-class
   ternary shapes from the "Low-Precision Formats" topic list).
+
+Workloads of the prologue and binary variants (same page sources for the
+shapes; "M8.8 - Native Binary and Ternary Transformers" for the variants):
+
+* ``ternary_4b_rmsnorm`` -- ``ternary_4b`` behind an RMSNorm with a gain
+  vector (0x02E, 0x03; b1.58 and T4NT use RMSNorm).
+* ``bitnet_v1_binary`` -- the Impeto stack shapes with BitNet v1 centred
+  binary codes and one scale per tensor (0x02B, 0x02E).
+* ``onebit_4096`` -- 4096->4096 sign codes with OneBit's input and output
+  value vectors (0x06A; d = 4096 is the page's ledger example of 0x06C),
+  M in {1, 16, 4096}.
+* ``h_bitlinear_4b`` -- the 4B-class FFN down projection 9728->2560 and an
+  attention output 2560->2560 as H-BitLinear (0x07C): RMSNorm with gain, then
+  a Hadamard rotation in blocks of 512 before the codes, M in {1, 16, 1024,
+  8192}.
+
+Gain vectors are 1 + 0.1 N(0,1); OneBit value vectors are exp(0.3 N(0,1))
+(input side) and 0.02 exp(0.3 N(0,1)) (output side), all fp32.  Their seeds
+add 2 (gain or input vector) and 3 (output vector) to the matrix's weight
+seed.
 """
 from __future__ import annotations
 
@@ -61,6 +81,12 @@ class Workload:
     outlier_factor: float = 8.0
     notes: str = ""
     extra: dict = field(default_factory=dict)
+    # activation prologue: RMSNorm (with a gain vector), Hadamard block size
+    norm: bool = False
+    hadamard: int = 0
+    # weight quantiser variant: "default", "centred" (BitNet v1) or "onebit"
+    # (sign codes with value vectors)
+    quantizer: str = "default"
 
 
 def _atomic_stack():
@@ -96,6 +122,22 @@ WORKLOADS = {
                            (1, 16, 128, 1024, 8192), BF16, BF16,
                            outlier_p=0.005, outlier_factor=10.0),
 }
+
+
+WORKLOADS.update({
+    "ternary_4b_rmsnorm": Workload("ternary_4b_rmsnorm", 6, TERNARY2,
+                                   (Matrix("ffn_up", 2560, 9728), Matrix("ffn_down", 9728, 2560)),
+                                   (1, 16, 128, 1024, 8192), BF16, BF16, outlier_p=0.005, outlier_factor=10.0,
+                                   norm=True),
+    "bitnet_v1_binary": Workload("bitnet_v1_binary", 7, BINARY1, _impeto_binary(), (16384,), F32, F32,
+                                 quantizer="centred"),
+    "onebit_4096": Workload("onebit_4096", 8, BINARY1, (Matrix("proj", 4096, 4096),), (1, 16, 4096), F32, BF16,
+                            quantizer="onebit"),
+    "h_bitlinear_4b": Workload("h_bitlinear_4b", 9, TERNARY2,
+                               (Matrix("ffn_down", 9728, 2560), Matrix("attn_out", 2560, 2560)),
+                               (1, 16, 1024, 8192), BF16, BF16, outlier_p=0.005, outlier_factor=10.0,
+                               norm=True, hadamard=512),
+})
 
 
 def weight_seed(wl: Workload, matrix_index: int) -> int:
@@ -148,3 +190,33 @@ def workload_activations(wl: Workload, matrix_index: int, M: int):
     if wl.x_dtype == BF16:
         return to_bf16_bits(x)
     return x
+
+
+def gain_vector(seed: int, K: int) -> np.ndarray:
+    """fp32 [K] gains 1 + 0.1 N(0,1) (an RMSNorm gain)."""
+    rng = np.random.default_rng(seed)
+    return (1.0 + 0.1 * rng.standard_normal(K)).astype(np.float32)
+
+
+def value_vector(seed: int, n: int, scale: float) -> np.ndarray:
+    """fp32 [n] positive values scale * exp(0.3 N(0,1)) (a OneBit value vector)."""
+    rng = np.random.default_rng(seed)
+    return (scale * np.exp(0.3 * rng.standard_normal(n))).astype(np.float32)
+
+
+def workload_gain(wl: Workload, matrix_index: int):
+    """The activation-side vector of a matrix: the RMSNorm gain, OneBit's
+    input value vector, or None."""
+    m = wl.matrices[matrix_index]
+    if wl.quantizer == "onebit":
+        return value_vector(weight_seed(wl, matrix_index) + 2, m.K, 1.0)
+    if wl.norm:
+        return gain_vector(weight_seed(wl, matrix_index) + 2, m.K)
+    return None
+
+
+def workload_output_vector(wl: Workload, matrix_index: int):
+    """OneBit's output value vector of a matrix (its per-row weight scale), or None."""
+    if wl.quantizer != "onebit":
+        return None
+    return value_vector(weight_seed(wl, matrix_index) + 3, wl.matrices[matrix_index].N, 0.02)

@@ -123,6 +123,34 @@ lowbit_status lowbit_pack(const float *w, int64_t N, int64_t K, int64_t ldw,
                           void *workspace, size_t workspace_bytes,
                           int32_t *status_dev, void *stream);
 
+/* Weight quantisers of lowbit_pack_ex. */
+#define LOWBIT_QUANT_DEFAULT 0          /* the format's quantiser of lowbit_pack */
+#define LOWBIT_QUANT_BINARY_CENTRED 1   /* BitNet v1 centred sign, LOWBIT_BINARY1 only */
+
+/* Device workspace lowbit_pack_ex needs: lowbit_pack_workspace_bytes for
+ * LOWBIT_QUANT_DEFAULT; 16*N + 16 bytes (rounded up to 256) for
+ * LOWBIT_QUANT_BINARY_CENTRED.  0 for bad arguments. */
+size_t lowbit_pack_ex_workspace_bytes(lowbit_format f, int quantizer, int64_t N);
+
+/* lowbit_pack_ex -- lowbit_pack with a choice of quantiser.
+ *   LOWBIT_QUANT_DEFAULT: exactly lowbit_pack.
+ *   LOWBIT_QUANT_BINARY_CENTRED (f must be LOWBIT_BINARY1), the original
+ *     BitNet's binarisation (M8.8 0x02B, 0x02E): alpha = mean(W) and
+ *     beta = mean|W| over the whole tensor, each an fp64 sum in the ternary
+ *     scale's fixed order (k ascending within a row, then rows ascending)
+ *     divided by N*K and rounded once to fp32; c = +1 where w > alpha and -1
+ *     otherwise (a weight equal to the mean takes -1, the page's tie), packed
+ *     in the LOWBIT_BINARY1 layout.  The scale is one per tensor; it is written
+ *     to all N entries of s_w so that lowbit_linear with LOWBIT_BINARY1 (one
+ *     scale per row) applies it unchanged.  eps is ignored.
+ * Other arguments, outputs and errors as lowbit_pack; `workspace` must hold
+ * lowbit_pack_ex_workspace_bytes(f, quantizer, N) bytes (8-byte aligned). */
+lowbit_status lowbit_pack_ex(const float *w, int64_t N, int64_t K, int64_t ldw,
+                             lowbit_format f, int quantizer, float eps,
+                             uint8_t *packed, int64_t ldp, float *s_w,
+                             void *workspace, size_t workspace_bytes,
+                             int32_t *status_dev, void *stream);
+
 /* Largest N lowbit_pack_ternary_noalloc accepts. */
 #define LOWBIT_NOALLOC_MAX_ROWS 65536
 
@@ -172,6 +200,44 @@ lowbit_status lowbit_unpack(const uint8_t *packed, int64_t ldp, int64_t N, int64
 lowbit_status lowbit_act_quant(const void *x, lowbit_dtype xdt, int64_t M, int64_t K,
                                int64_t ldx, float eps, int8_t *q, int64_t ldq, float *s_x,
                                int32_t *status_dev, void *stream);
+
+/* Activation prologue options of lowbit_act_quant_ex and lowbit_bitlinear. */
+#define LOWBIT_NORM_NONE 0 /* no normalisation */
+#define LOWBIT_NORM_RMS 1  /* RMSNorm: the row factor 1/sqrt(mean_k x_k^2 + eps_norm) */
+
+/* Largest K the prologue accepts with a gain, RMSNorm or Hadamard option. */
+#define LOWBIT_PROLOGUE_MAX_K 49152
+
+/* lowbit_act_quant_ex -- the activation side of a BitLinear layer in one pass
+ * over x: an optional RMSNorm with gain (M8.8 0x02E and 0x03: the activation
+ * is normalised before its codes are taken; b1.58 and the T4NT model card use
+ * RMSNorm), an optional input value vector (the gain alone, OneBit's x * g of
+ * M8.8 0x06A), an optional block Hadamard rotation (H-BitLinear, M8.8 0x07C),
+ * then the per-token absmax int8 codes of lowbit_act_quant with eps = 0:
+ *   u_k   = x_k * g_k                        (fp32 product; g NULL: u = x)
+ *   u     = FWHT_hb(u) on every block of `hadamard` consecutive features:
+ *           the unnormalised radix-2 fast Walsh-Hadamard transform in fp32,
+ *           stages h = 1, 2, 4, ..., each pair (a, b) -> (a + b, a - b)
+ *   q     = clip(rint((u * 127) / max_k |u_k|), -128, 127)   (lowbit_act_quant)
+ *   s_x   = max|u| / sqrt(hadamard) / rms / 127, rms = sqrt(mean_k x_k^2 +
+ *           eps_norm) with LOWBIT_NORM_RMS (1 otherwise), evaluated in fp64
+ *           (the sum of squares in fp64) and rounded once to fp32.
+ * The RMSNorm output is x * g / rms and the normalised rotation is H/sqrt(hb);
+ * both row factors are positive, so they cancel in absmax codes and only the
+ * scale carries them: y = q * s_x reconstructs the normalised, rotated row.
+ * An all-zero u gives zero codes and s_x = 0.
+ * Arguments: x, xdt, M, K, ldx, q, ldq, s_x as lowbit_act_quant.  g: NULL or
+ * a device array of K fp32 gains (4-byte aligned; 16-byte aligned for the
+ * one-pass vector kernel).  norm: LOWBIT_NORM_NONE or LOWBIT_NORM_RMS.
+ * eps_norm >= 0 and finite (ignored without the norm).  hadamard: 0 (none)
+ * or a power of two >= 2 that divides K.  With any option K must be at most
+ * LOWBIT_PROLOGUE_MAX_K (else LOWBIT_ERR_UNSUPPORTED).  With g NULL, no norm
+ * and no rotation the call is exactly lowbit_act_quant with eps = 0.  A
+ * non-finite x or g, or a non-finite product or transform, sets
+ * LOWBIT_ERR_NONFINITE; that row is then unspecified. */
+lowbit_status lowbit_act_quant_ex(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                  const float *g, int norm, float eps_norm, int hadamard,
+                                  int8_t *q, int64_t ldq, float *s_x, int32_t *status_dev, void *stream);
 
 /* lowbit_linear -- the low-bit linear layer on int8 activation codes:
  *   acc[t,n] = sum_{k<K} q[t,k] * c[n,k]  (exact int32: add/sub/skip for
@@ -242,6 +308,80 @@ lowbit_status lowbit_linear_ex(const int8_t *q, int64_t ldq, const float *s_x,
                                int path, unsigned flags,
                                int32_t *status_dev, void *stream);
 
+/* Largest M * K (K rounded up to a multiple of 128) that lowbit_bitlinear
+ * runs as one fused decode kernel. */
+#define LOWBIT_FUSED_MAX_MK 98304
+
+/* lowbit_bitlinear -- the whole BitLinear forward of M8.8 0x02E on activations
+ * x: the prologue of lowbit_act_quant_ex (gain, RMSNorm, Hadamard rotation,
+ * per-token codes) followed by lowbit_linear_ex with the given path and
+ * flags.  y is identical to calling those two functions in turn.
+ *   - Decode: with M <= 4, hadamard == 0, path 0 or 1 and M * K (K rounded
+ *     up to a multiple of 128) <= LOWBIT_FUSED_MAX_MK, one fused kernel runs:
+ *     every block computes the codes of the M tokens in shared memory while
+ *     its first weight loads are in flight, then streams the packed weights
+ *     (one launch instead of two, and the codes never go through global
+ *     memory).  q and s_x may then be NULL; when given, they receive the
+ *     codes and scales.
+ *   - Otherwise the prologue kernel writes q [M, ldq] and s_x [M] (both
+ *     required: device workspace owned by the caller, ldq a multiple of 16,
+ *     ldq >= K, q 16-byte aligned), and the linear kernel reads them.
+ * Arguments and errors as lowbit_act_quant_ex and lowbit_linear_ex.  With
+ * LOWBIT_LINEAR_WEIGHTS_STABLE the packed weights and s_w must not be written
+ * by the kernel that precedes this call on the stream. */
+lowbit_status lowbit_bitlinear(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                               const float *g, int norm, float eps_norm, int hadamard,
+                               const uint8_t *packed, int64_t ldp, const float *s_w, lowbit_format f, int64_t N,
+                               void *y, lowbit_dtype ydt, int64_t ldy,
+                               int8_t *q, int64_t ldq, float *s_x,
+                               int path, unsigned flags, int32_t *status_dev, void *stream);
+
+/* Row-parallel layers (M8.8 0x08A-0x08C).  When the input dimension of a
+ * layer is split over ranks, each rank holds a slice x[:, k0:k1] of every
+ * token row and the packed weights of the same K slice.  The per-token
+ * statistics the codes need (max|u| and, with an RMSNorm, the sum of
+ * squares) span the whole row, so they are reduced across ranks first; the
+ * codes of every slice are then taken with the whole row's maximum, the
+ * int32 partial accumulators of the slices are summed (an all-reduce), and
+ * one epilogue rescales the sum.  Every value is then identical to the
+ * unsplit layer.  The three calls below are the per-rank kernels of that
+ * sequence; the collectives in between belong to the caller.  Slice
+ * boundaries must be multiples of 128 features and of the Hadamard block. */
+
+/* lowbit_act_row_stats -- per token row of the slice: row_max[t] = max_k |u|
+ * (u = x * g, rotated in Hadamard blocks when hadamard > 0, as in
+ * lowbit_act_quant_ex) as fp32, and, when row_ss is not NULL, row_ss[t] =
+ * sum_k x_k^2 in fp64 (the RMSNorm's sum of squares).  row_max: device fp32
+ * [M]; row_ss: device fp64 [M] or NULL.  K <= LOWBIT_PROLOGUE_MAX_K.  A
+ * non-finite u sets LOWBIT_ERR_NONFINITE. */
+lowbit_status lowbit_act_row_stats(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                   const float *g, int hadamard, float *row_max, double *row_ss,
+                                   int32_t *status_dev, void *stream);
+
+/* lowbit_act_quant_given_max -- the int8 codes of a row slice with the whole
+ * row's maximum: q = clip(rint((u * 127) / row_max[t]), -128, 127) (fp32
+ * multiply and IEEE divide, nearest even; row_max[t] == 0 gives zero codes).
+ * A slice value above the maximum it was given sets LOWBIT_ERR_INVALID_ARG in
+ * *status_dev. */
+lowbit_status lowbit_act_quant_given_max(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
+                                         const float *g, int hadamard, const float *row_max,
+                                         int8_t *q, int64_t ldq, int32_t *status_dev, void *stream);
+
+/* lowbit_act_scales -- s_x of lowbit_act_quant_ex from whole-row statistics:
+ * s_x[t] = row_max[t] / sqrt(hadamard) / rms / 127 (fp64, rounded once),
+ * rms = sqrt(row_ss[t] / K_total + eps_norm) with LOWBIT_NORM_RMS (row_ss
+ * then required), 1 otherwise; row_max[t] == 0 gives 0. */
+lowbit_status lowbit_act_scales(const float *row_max, const double *row_ss, int64_t M, int64_t K_total, int norm,
+                                float eps_norm, int hadamard, float *s_x, int32_t *status_dev, void *stream);
+
+/* lowbit_rescale -- the epilogue of lowbit_linear on given int32
+ * accumulators acc [M, ldacc]: y = float(acc) * (s_w[n or 0] * s_x[t]) in
+ * fp32, or rounded to bf16, or acc itself (LOWBIT_I32); s_w holds
+ * lowbit_scale_count(f, N) values.  y [M, ldy], ldy >= N. */
+lowbit_status lowbit_rescale(const int32_t *acc, int64_t ldacc, int64_t M, int64_t N, const float *s_x,
+                             const float *s_w, lowbit_format f, void *y, lowbit_dtype ydt, int64_t ldy,
+                             int32_t *status_dev, void *stream);
+
 /* The kernels lowbit_linear_path can launch. */
 typedef enum {
     LOWBIT_KERNEL_GEMV = 1,           /* packed-weight GEMV (dp4a), groups of up to 4 tokens */
@@ -270,6 +410,17 @@ lowbit_status lowbit_linear_kernel(int64_t M, int64_t N, int64_t K, lowbit_forma
 /* Name of the kernel function(s) behind a lowbit_kernel value, as in a
  * profiler's launch list (static string; "unknown" for other values). */
 const char *lowbit_kernel_name(lowbit_kernel k);
+
+/* lowbit_set_wait_limit -- the bound, in SM clock cycles, of every pipeline
+ * wait in the tensor-core kernels on the current device (the default,
+ * restored by cycles <= 0, is 4e9 cycles, about 2 s).  When a wait runs past
+ * it, the kernel sets LOWBIT_ERR_TIMEOUT in *status_dev, lets the copies and
+ * tensor-core operations it already issued complete, frees its tensor
+ * memory and returns; that launch's output is unspecified and the context
+ * stays usable.  Failure-detection tests lower the bound to make a wait run
+ * out.  Synchronous (a copy to device memory); call it with no kernel of this
+ * library in flight on the device. */
+lowbit_status lowbit_set_wait_limit(int64_t cycles);
 
 /* Human-readable name of a status value (static string). */
 const char *lowbit_status_string(lowbit_status s);
