@@ -4,8 +4,10 @@ One step = one pass of the hot path over a workload's points (every matrix
 at every token count M): the BitLinear call lowbit_bitlinear -- the
 activation prologue (the workload's RMSNorm, gain or Hadamard rotation, if
 any), per-token int8 quantisation, then the low-bit linear layer with the
-workload's output dtype.  Up to 4 tokens the call is one fused kernel; above,
-a prologue kernel and the linear kernel.  The
+workload's output dtype.  Up to 4 tokens the call is one fused kernel, and
+all matrices at the same token count run as one grouped launch
+(lowbit_bitlinear_group; --no-group: one call each); above, a prologue
+kernel and the linear kernel.  The
 default workload is the 4B-class ternary sweep (2560->9728 and 9728->2560,
 M in {8192, 1024, 128, 16, 1}, bf16 in and out).  Weights are packed once,
 off the timed path, into a pool of copies larger than L2 that the launches
@@ -196,11 +198,11 @@ class Point:
     launch: ops = 2*M*N*K; bytes = packed weights + int8 codes and s_x read,
     weight scales read, y written)."""
 
-    def __init__(self, wl, mi, m, M, rows, sm_count=148):
+    def __init__(self, wl, mi, m, M, rows, sm_count=148, fused=True):
         import binary_weight_transformer_b200 as bwt
         self.mi, self.m, self.M, self.rows = mi, m, M, rows
         self.kernel = bwt.linear_kernel(rows, m.N, m.K, wl.fmt, 0, sm_count)
-        self.fused = bwt.bitlinear_fuses(rows, m.K, wl.hadamard, 0)
+        self.fused = bwt.bitlinear_fuses(rows, m.K, wl.hadamard, 0) and fused
         if self.fused:
             self.kernel = "gemv_smem_kernel (fused prologue)"
         self.ops = 2 * rows * m.N * m.K
@@ -215,7 +217,7 @@ class Point:
         return "tensor" if self.ops / self.bytes > ridge else "hbm"
 
 
-def select_points(wl, only_M=None, sm_count=148, rank=0, world=1, shard=False):
+def select_points(wl, only_M=None, sm_count=148, rank=0, world=1, shard=False, fused=True):
     points = []
     for mi, m in enumerate(wl.matrices):
         for M in sorted(wl.Ms, reverse=True):
@@ -225,7 +227,7 @@ def select_points(wl, only_M=None, sm_count=148, rank=0, world=1, shard=False):
                     a, b = shard_range(M, rank, world)
                     rows = b - a
                 if rows > 0:
-                    points.append(Point(wl, mi, m, M, rows, sm_count))
+                    points.append(Point(wl, mi, m, M, rows, sm_count, fused))
     return points
 
 
@@ -317,7 +319,7 @@ def run_gpu_arm(args, wl):
     only_M = set(int(v) for v in args.points.split(",")) if args.points else None
     sms = torch.cuda.get_device_properties(device).multi_processor_count
     shard = args.shard == "m"
-    points = select_points(wl, only_M, sms, rank, world, shard)
+    points = select_points(wl, only_M, sms, rank, world, shard, not args.unfused)
     offset = (lambda M: shard_range(M, rank, world)[0]) if shard else None
     pool, xs, qs, sxs, ys, gains = build_state(wl, points, device, 3 * L2_BYTES, torch, bwt, args.pool_copies,
                                                offset)
@@ -329,10 +331,47 @@ def run_gpu_arm(args, wl):
         """The point's whole BitLinear call; the codes stay in the fused
         kernel's shared memory, else they go through q and s_x."""
         key = (pt.mi, pt.M)
+        if not pt.fused and bwt.bitlinear_fuses(pt.rows, pt.m.K, wl.hadamard, 0):
+            # --unfused: the prologue kernel and the linear kernel, as above 4 tokens
+            bwt.lowbit_act_quant_ex(xs[key] if x is None else x, gains[pt.mi], norm, 1e-5, wl.hadamard, q=qs[key],
+                                    s_x=sxs[key], stream=stream_)
+            bwt.lowbit_linear(qs[key], sxs[key], packed, s_w, wl.fmt, pt.m.N, ydt, K=pt.m.K, y=ys[key],
+                              stream=stream_, weights_stable=True)
+            return 2
         bwt.lowbit_bitlinear(xs[key] if x is None else x, packed, s_w, wl.fmt, pt.m.N, ydt, gains[pt.mi], norm,
                              1e-5, wl.hadamard, y=ys[key], q=None if pt.fused else qs[key],
                              s_x=None if pt.fused else sxs[key], stream=stream_, weights_stable=True)
         return 1 if pt.fused else 2
+
+    # Token counts whose points are all fused decode calls run as grouped
+    # launches (lowbit_bitlinear_group, up to GROUP_MAX layers per launch)
+    # unless --no-group; `calls` lists the points of each API call of a step.
+    group_ms = set()
+    if not args.no_group:
+        for M in sorted({pt.M for pt in points}):
+            at = [pt for pt in points if pt.M == M]
+            if len(at) > 1 and all(pt.fused for pt in at):
+                group_ms.add(M)
+    calls = []
+    for M in sorted(group_ms):
+        at = [(i, pt) for i, pt in enumerate(points) if pt.M == M]
+        calls += [at[c:c + bwt.GROUP_MAX] for c in range(0, len(at), bwt.GROUP_MAX)]
+    calls += [[(i, pt)] for i, pt in enumerate(points) if pt.M not in group_ms]
+
+    def run_call(call, weights, x=None, stream_=None):
+        """One API call of a step: a single point's bitlinear, or a grouped
+        launch; weights(i, pt) gives the (packed, s_w) copy to read."""
+        if call[0][1].M not in group_ms:
+            i, pt = call[0]
+            key = (pt.mi, pt.M)
+            return bitlinear(pt, *weights(i, pt), x=None if x is None else x[key], stream_=stream_)
+        keys = [(pt.mi, pt.M) for _, pt in call]
+        ws = [weights(i, pt) for i, pt in call]
+        bwt.lowbit_bitlinear_group([(xs if x is None else x)[k] for k in keys], [w[0] for w in ws],
+                                   [w[1] for w in ws], wl.fmt, [pt.m.N for _, pt in call], ydt,
+                                   [gains[pt.mi] for _, pt in call], norm, 1e-5, ys=[ys[k] for k in keys],
+                                   stream=stream_, weights_stable=True)
+        return 1
 
     def prologue(pt):
         key = (pt.mi, pt.M)
@@ -348,9 +387,8 @@ def run_gpu_arm(args, wl):
         """One pass of the hot path; each point of step s reads its own pool
         copy of the weights."""
         launches = 0
-        for i, pt in enumerate(points):
-            packed, s_w = pool[(s * len(points) + i) % n_sets][pt.mi]
-            launches += bitlinear(pt, packed, s_w)
+        for call in calls:
+            launches += run_call(call, lambda i, pt: pool[(s * len(points) + i) % n_sets][pt.mi])
         return launches
 
     # eager warm-up (sets kernel attributes, loads modules), then a few
@@ -409,13 +447,18 @@ def run_gpu_arm(args, wl):
     for M in sorted({pt.M for pt in points}, reverse=True):
         pts = [(i, pt) for i, pt in enumerate(points) if pt.M == M]
 
-        def stack(r, pts=pts):
+        def stack(r, M=M, pts=pts):
+            if M in group_ms:
+                for call in calls:
+                    if call[0][1].M == M:
+                        run_call(call, lambda i, pt: pool[(r * len(points) + i) % n_sets][pt.mi])
+                return
             for i, pt in pts:
                 bitlinear(pt, *pool[(r * len(points) + i) % n_sets][pt.mi])
         stacks[M] = summary(time_graph(torch, stream, stack, 1, max(10, args.kernel_reps // 2)))
 
     # end to end through the public API with host buffers (pinned)
-    e2e = None if args.no_e2e else run_e2e(args, wl, points, pool, bitlinear, ys, torch, stream)
+    e2e = None if args.no_e2e else run_e2e(args, wl, points, calls, pool, run_call, ys, torch, stream)
 
     if world > 1:
         torch.distributed.destroy_process_group()
@@ -519,6 +562,14 @@ def run_gpu_arm(args, wl):
         "int_tops_m_ge_128": round(big_ops / (big_ms * 1e-3) / 1e12, 1) if big_ms else None,
         "gemv_packed_gbs": round(gemv_bytes / (gemv_ms * 1e-3) / 1e9, 1) if gemv_ms else None,
         "stack_us": {str(M): round(v["median"] * 1e3, 2) for M, v in stacks.items()},
+        "decode_groups": [{"M": M, "layers": sum(1 for pt in points if pt.M == M),
+                           "launches": sum(1 for c in calls if c[0][1].M == M),
+                           "us": round(stacks[M]["median"] * 1e3, 2),
+                           "packed_gbs": round(sum(pt.packed_bytes for pt in points if pt.M == M)
+                                               / (stacks[M]["median"] * 1e-3) / 1e9, 1),
+                           "frac_hbm_packed": round(sum(pt.packed_bytes for pt in points if pt.M == M)
+                                                    / (stacks[M]["median"] * 1e-3) / 1e9 / hbm, 3)}
+                          for M in sorted(group_ms)],
         "points": pts_out,
         "roofline": roofline,
         "cpu_baseline": cpu,
@@ -529,12 +580,13 @@ def run_gpu_arm(args, wl):
     return line
 
 
-def run_e2e(args, wl, points, pool, bitlinear, ys, torch, stream):
+def run_e2e(args, wl, points, calls, pool, run_call, ys, torch, stream):
     """Same step through the public API from pinned host buffers: H2D copy of
-    each point's activations, the BitLinear call, D2H copy of its output.  The
-    copies run on their own streams (PCIe is full duplex), so one point's
-    uploads and downloads overlap the kernels of the others; events order each
-    buffer's reuse across steps."""
+    each point's activations, the API calls of the step (one per point, or
+    one per decode group), D2H copy of every output.  The copies run on their
+    own streams (PCIe is full duplex), so one call's uploads and downloads
+    overlap the kernels of the others; events order each buffer's reuse
+    across steps."""
     host_x, dev_x, host_y = {}, {}, {}
     for pt in points:
         key = (pt.mi, pt.M)
@@ -555,27 +607,33 @@ def run_e2e(args, wl, points, pool, bitlinear, ys, torch, stream):
     counter = [0]
 
     def step():
-        for pt in points:
-            key = (pt.mi, pt.M)
-            packed, s_w = pool[counter[0] % len(pool)][pt.mi]
-            counter[0] += 1
-            first = key not in started
-            started.add(key)
+        for call in calls:
+            keys = [(pt.mi, pt.M) for _, pt in call]
+            weights = {}
+            for i, pt in call:
+                weights[i] = pool[counter[0] % len(pool)][pt.mi]
+                counter[0] += 1
+            first = keys[0] not in started
+            started.update(keys)
             with torch.cuda.stream(up):
+                for key in keys:
+                    if not first:
+                        up.wait_event(ev["x_free"][key])      # previous step's call has read dev_x
+                    dev_x[key].copy_(host_x[key], non_blocking=True)
+                    ev["x_ready"][key].record(up)
+            for key in keys:
+                stream.wait_event(ev["x_ready"][key])
                 if not first:
-                    up.wait_event(ev["x_free"][key])      # previous step's call has read dev_x
-                dev_x[key].copy_(host_x[key], non_blocking=True)
-                ev["x_ready"][key].record(up)
-            stream.wait_event(ev["x_ready"][key])
-            if not first:
-                stream.wait_event(ev["y_free"][key])      # previous step's download has read y
-            bitlinear(pt, packed, s_w, x=dev_x[key], stream_=stream)
-            ev["x_free"][key].record(stream)
-            ev["y_ready"][key].record(stream)
+                    stream.wait_event(ev["y_free"][key])      # previous step's download has read y
+            run_call(call, lambda i, pt: weights[i], x=dev_x, stream_=stream)
+            for key in keys:
+                ev["x_free"][key].record(stream)
+                ev["y_ready"][key].record(stream)
             with torch.cuda.stream(down):
-                down.wait_event(ev["y_ready"][key])
-                host_y[key].copy_(ys[key], non_blocking=True)
-                ev["y_free"][key].record(down)
+                for key in keys:
+                    down.wait_event(ev["y_ready"][key])
+                    host_y[key].copy_(ys[key], non_blocking=True)
+                    ev["y_free"][key].record(down)
 
     steps = max(1, min(args.steps, args.e2e_steps))
     for _ in range(2):
@@ -739,6 +797,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--points", default=None, help="comma-separated subset of the sweep's M values")
+    ap.add_argument("--unfused", action="store_true",
+                    help="run the prologue kernel and the linear kernel also where one fused call would run")
+    ap.add_argument("--no-group", action="store_true",
+                    help="one call per fused decode point instead of one grouped launch per token count")
     ap.add_argument("--pool-copies", type=int, default=None,
                     help="number of packed weight copies to rotate over (default: enough to exceed 3x L2)")
     args = ap.parse_args(argv)

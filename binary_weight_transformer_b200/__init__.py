@@ -15,6 +15,7 @@ Functions carry the ABI's names::
     q, s_x      = lowbit_act_quant_ex(x, g=None, norm=NORM_RMS, eps_norm=1e-5, hadamard=0)
     y           = lowbit_linear(q, s_x, packed, s_w, fmt, N, out_dtype)
     y           = lowbit_bitlinear(x, packed, s_w, fmt, N, out_dtype, g=None, norm=NORM_RMS)
+    ys          = lowbit_bitlinear_group(xs, packeds, s_ws, fmt, Ns, out_dtype)
 """
 from __future__ import annotations
 
@@ -24,7 +25,8 @@ import os
 TERNARY2, BINARY1, INT4 = 0, 1, 2
 NORM_NONE, NORM_RMS = 0, 1
 QUANT_DEFAULT, QUANT_BINARY_CENTRED = 0, 1
-FUSED_MAX_MK = 98304  # LOWBIT_FUSED_MAX_MK
+FUSED_MAX_BYTES = 98304  # LOWBIT_FUSED_MAX_BYTES
+GROUP_MAX = 32  # LOWBIT_GROUP_MAX
 F32, BF16, I32 = 0, 1, 2
 WEIGHTS_STABLE = 1  # LOWBIT_LINEAR_WEIGHTS_STABLE
 
@@ -65,6 +67,7 @@ ABI = {
     "lowbit_act_quant_ex": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _I32, _F, _I32, _P, _I64, _P, _P, _P]),
     "lowbit_bitlinear": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _I32, _F, _I32, _P, _I64, _P, _I32, _I64, _P, _I32,
                                 _I64, _P, _I64, _P, _I32, ctypes.c_uint, _P, _P]),
+    "lowbit_bitlinear_group": (_I32, [_P, _I32, _I64, _I32, _I32, _F, _I32, _I32, ctypes.c_uint, _P, _P]),
     "lowbit_kernel_name": (ctypes.c_char_p, [_I32]),
     "lowbit_status_string": (ctypes.c_char_p, [_I32]),
     "lowbit_set_wait_limit": (_I32, [_I64]),
@@ -276,7 +279,7 @@ def lowbit_act_quant_ex(x, g=None, norm: int = NORM_NONE, eps_norm: float = 1e-5
 
 def bitlinear_fuses(M: int, K: int, hadamard: int = 0, path: int = 0) -> bool:
     """True when lowbit_bitlinear runs as one fused decode kernel."""
-    return M <= 4 and hadamard == 0 and path in (0, 1) and M * ((K + 127) // 128 * 128) <= FUSED_MAX_MK
+    return M <= 4 and hadamard == 0 and path in (0, 1) and M * ((K + 127) // 128 * 128) <= FUSED_MAX_BYTES
 
 
 def lowbit_bitlinear(x, packed, s_w, fmt: int, N: int, out_dtype: int = F32, g=None, norm: int = NORM_NONE,
@@ -302,6 +305,49 @@ def lowbit_bitlinear(x, packed, s_w, fmt: int, N: int, out_dtype: int = F32, g=N
                                 WEIGHTS_STABLE if weights_stable else 0, _ptr(status), _stream(stream))
     _check(st, "lowbit_bitlinear")
     return (y, q, s_x) if want_codes else y
+
+
+class BitlinearItem(ctypes.Structure):
+    """lowbit_bitlinear_item: one layer of a grouped decode call."""
+    _fields_ = [("x", _P), ("ldx", _I64), ("g", _P), ("packed", _P), ("ldp", _I64), ("s_w", _P), ("N", _I64),
+                ("K", _I64), ("y", _P), ("ldy", _I64), ("q", _P), ("ldq", _I64), ("s_x", _P)]
+
+
+def lowbit_bitlinear_group(xs, packeds, s_ws, fmt: int, Ns, out_dtype: int = F32, gs=None, norm: int = NORM_NONE,
+                           eps_norm: float = 1e-5, ys=None, want_codes: bool = False, status=None, stream=None,
+                           weights_stable: bool = False):
+    """Several independent decode BitLinear layers (M <= 4 tokens each, the
+    same M, activation dtype, format and output dtype) in one launch.
+
+    xs[i] [M, K_i], packeds[i], s_ws[i], Ns[i]; gs: None or a list of gains
+    (entries may be None).  Returns the list of y, or (ys, qs, s_xs) with
+    ``want_codes``."""
+    import torch
+    n = len(xs)
+    if not (len(packeds) == len(s_ws) == len(Ns) == n) or (gs is not None and len(gs) != n):
+        raise ValueError("every per-layer list must have one entry per layer")
+    M = xs[0].shape[0]
+    dt = {F32: torch.float32, BF16: torch.bfloat16, I32: torch.int32}[out_dtype]
+    if ys is None:
+        ys = [torch.empty((M, N), dtype=dt, device=x.device) for x, N in zip(xs, Ns)]
+    qs = [None] * n
+    s_xs = [None] * n
+    if want_codes:
+        qs = [torch.empty((M, (x.shape[1] + 15) // 16 * 16), dtype=torch.int8, device=x.device) for x in xs]
+        s_xs = [torch.empty(M, dtype=torch.float32, device=x.device) for x in xs]
+    items = (BitlinearItem * n)()
+    for i in range(n):
+        x, p, q, y = xs[i], packeds[i], qs[i], ys[i]
+        if x.shape[0] != M or x.dtype != xs[0].dtype:
+            raise ValueError("all layers take the same number of tokens and activation dtype")
+        items[i] = BitlinearItem(_ptr(x), x.stride(0), _ptr(gs[i] if gs is not None else None), _ptr(p), p.stride(0),
+                                 _ptr(s_ws[i]), Ns[i], x.shape[1], _ptr(y), y.stride(0), _ptr(q),
+                                 q.stride(0) if q is not None else 0, _ptr(s_xs[i]))
+    st = lib().lowbit_bitlinear_group(ctypes.cast(items, ctypes.c_void_p), n, M, _xdt(xs[0]), norm, eps_norm, fmt,
+                                      out_dtype, WEIGHTS_STABLE if weights_stable else 0, _ptr(status),
+                                      _stream(stream))
+    _check(st, "lowbit_bitlinear_group")
+    return (ys, qs, s_xs) if want_codes else ys
 
 
 def lowbit_act_row_stats(x, g=None, hadamard: int = 0, with_ss: bool = False, status=None, stream=None):

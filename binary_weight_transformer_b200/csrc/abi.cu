@@ -29,7 +29,7 @@ lowbit_status gemm_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_
 
 // True when the shared-memory GEMM would split K over a cluster on a GPU
 // with `sms` SMs (few output tiles, deep K).
-bool gemm_splits_k(int64_t M, int64_t N, int64_t K, int64_t sms);
+bool gemm_splits_k(lowbit_format f, int64_t M, int64_t N, int64_t K, int64_t sms);
 
 lowbit_status gemm_ts_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
                              const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
@@ -54,10 +54,8 @@ lowbit_status gemm_ts_pair_launch(const int8_t *q, int64_t ldq, const float *s_x
 lowbit_status act_prologue_launch(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
                                   const float *g, int norm, float eps_norm, int hb, int8_t *q, int64_t ldq,
                                   float *s_x, int32_t *status, cudaStream_t st);
-lowbit_status gemv_fused_launch(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx, const float *g,
-                                int norm, float eps_norm, const uint8_t *packed, int64_t ldp, int64_t row_bytes,
-                                const float *s_w, lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy,
-                                int8_t *q_out, int64_t ldq, float *s_x_out, int prefetch, int32_t *status,
+lowbit_status gemv_group_launch(const lowbit_bitlinear_item *items, int n, int64_t M, lowbit_dtype xdt, int norm,
+                                float eps_norm, lowbit_format f, lowbit_dtype ydt, int prefetch, int32_t *status,
                                 cudaStream_t st);
 
 lowbit_status act_row_stats_launch(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,
@@ -140,7 +138,7 @@ lowbit_kernel choose_kernel(int64_t M, int64_t N, int64_t K, lowbit_format f, in
     // the pair kernel is ahead, 9.2 us vs 9.6 us).  4-bit and binary weights
     // take the tensor-memory variant from 512 tokens (the split-K kernel
     // measured faster for some of their shapes and slower for others).
-    const bool splits = gemm_splits_k(M, N, K, sms);
+    const bool splits = gemm_splits_k(f, M, N, K, sms);
     if (path == 0 && M >= 512 && f == LOWBIT_TERNARY2)
         return (K >= 2048 && splits) ? LOWBIT_KERNEL_GEMM_SPLITK : LOWBIT_KERNEL_GEMM_PAIR;
     if (path == 3 || (path == 0 && M >= 512)) return LOWBIT_KERNEL_GEMM_TMEM;
@@ -325,7 +323,7 @@ lowbit_status check_prologue_args(const void *x, lowbit_dtype xdt, int64_t M, in
 
 bool fused_decode(int64_t M, int64_t K, int hadamard, int path)
 {
-    return M <= 4 && hadamard == 0 && (path == 0 || path == 1) && M * ((K + 127) / 128 * 128) <= LOWBIT_FUSED_MAX_MK;
+    return M <= 4 && hadamard == 0 && (path == 0 || path == 1) && M * ((K + 127) / 128 * 128) <= LOWBIT_FUSED_MAX_BYTES;
 }
 
 }  // namespace
@@ -382,14 +380,51 @@ lowbit_status lowbit_bitlinear(const void *x, lowbit_dtype xdt, int64_t M, int64
     const int prefetch = (flags & LOWBIT_LINEAR_WEIGHTS_STABLE) != 0 ? 1 : 0;
     if (fused) {
         const TraceRange trace("lowbit_bitlinear");
-        return gemv_fused_launch(x, xdt, M, K, ldx, g, norm, eps_norm, packed, ldp, rb, s_w, f, N, y, ydt, ldy, q,
-                                 ldq, s_x, prefetch, status_dev, st);
+        const lowbit_bitlinear_item item = {x, ldx, g, packed, ldp, s_w, N, K, y, ldy, q, ldq, s_x};
+        return gemv_group_launch(&item, 1, M, xdt, norm, eps_norm, f, ydt, prefetch, status_dev, st);
     }
     const lowbit_status s1 = lowbit_act_quant_ex(x, xdt, M, K, ldx, g, norm, eps_norm, hadamard, q, ldq, s_x,
                                                  status_dev, stream);
     if (s1 != LOWBIT_OK) return s1;
     // the prologue kernel just before writes q and s_x, never the weights
     return lowbit_linear_ex(q, ldq, s_x, M, K, packed, ldp, s_w, f, N, y, ydt, ldy, path, flags, status_dev, stream);
+}
+
+lowbit_status lowbit_bitlinear_group(const lowbit_bitlinear_item *items, int n_items, int64_t M,
+                                     lowbit_dtype xdt, int norm, float eps_norm, lowbit_format f,
+                                     lowbit_dtype ydt, unsigned flags, int32_t *status_dev, void *stream)
+{
+    if (items == nullptr || n_items < 1 || n_items > LOWBIT_GROUP_MAX || M < 1 || M > 4)
+        return LOWBIT_ERR_INVALID_ARG;
+    if ((flags & ~static_cast<unsigned>(LOWBIT_LINEAR_WEIGHTS_STABLE)) != 0) return LOWBIT_ERR_INVALID_ARG;
+    if (!valid_format(f) || (ydt != LOWBIT_F32 && ydt != LOWBIT_BF16 && ydt != LOWBIT_I32))
+        return LOWBIT_ERR_INVALID_ARG;
+    const int64_t esz = ydt == LOWBIT_BF16 ? 2 : 4;
+    for (int i = 0; i < n_items; ++i) {
+        const lowbit_bitlinear_item &it = items[i];
+        const lowbit_status a = check_prologue_args(it.x, xdt, M, it.K, it.ldx, it.g, norm, eps_norm, 0);
+        if (a != LOWBIT_OK) return a;
+        if (it.packed == nullptr || it.s_w == nullptr || it.y == nullptr) return LOWBIT_ERR_INVALID_ARG;
+        if (it.N <= 0 || it.ldy < it.N) return LOWBIT_ERR_INVALID_ARG;
+        const lowbit_status shape = check_linear_shape(M, it.N, it.K, f, 0);
+        if (shape != LOWBIT_OK) return shape;
+        if (!fused_decode(M, it.K, 0, 0)) return LOWBIT_ERR_UNSUPPORTED;
+        if (it.ldp < static_cast<int64_t>(lowbit_packed_row_bytes(f, it.K))) return LOWBIT_ERR_INVALID_ARG;
+        if (!aligned(it.packed, 16) || it.ldp % 16 != 0 || !aligned(it.s_w, 4) ||
+            !aligned(it.y, static_cast<uintptr_t>(esz)))
+            return LOWBIT_ERR_ALIGNMENT;
+        if (it.q != nullptr) {
+            if (it.ldq < it.K) return LOWBIT_ERR_INVALID_ARG;
+            if (!aligned(it.q, 16) || it.ldq % 16 != 0) return LOWBIT_ERR_ALIGNMENT;
+        }
+        if (it.s_x != nullptr && !aligned(it.s_x, 4)) return LOWBIT_ERR_ALIGNMENT;
+    }
+    const lowbit_status d = check_device();
+    if (d != LOWBIT_OK) return d;
+    const TraceRange trace("lowbit_bitlinear_group");
+    const int prefetch = (flags & LOWBIT_LINEAR_WEIGHTS_STABLE) != 0 ? 1 : 0;
+    return gemv_group_launch(items, n_items, M, xdt, norm, eps_norm, f, ydt, prefetch, status_dev,
+                             static_cast<cudaStream_t>(stream));
 }
 
 lowbit_status lowbit_act_row_stats(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,

@@ -38,18 +38,46 @@ constexpr uint32_t kTmemCols = 512;
 
 template <int FMT> __host__ __device__ constexpr int packed_bytes_per_kblock() { return BK * Fmt<FMT>::kBits / 8; }
 
-// Split K over a cluster when the tiles leave most SMs idle: the largest C in
-// {2, 4, 8} that keeps every split at least 2 k-blocks deep and the whole grid
-// within one wave; 1 when no split applies.
-inline int splitk_clusters(int64_t M, int64_t N, int64_t K, int64_t sms)
+// How the shared-memory GEMM covers a problem whose 128 x 256 output tiles
+// leave most SMs idle: K split over a cluster of c CTAs (1..8) and output
+// tiles tbn = 256 or 128 features wide.
+struct SplitPlan {
+    int tbn;
+    int c;
+};
+
+// Pipeline buffers of the split-K kernel (TMA and expansion rings), which
+// hold the partial slices during the reduction: c * ceil(tbn/32 / c) slots
+// of 16 KB must fit.
+inline int64_t splitk_region_bytes(int stages, int tbn, int packed_bytes_per_kb)
 {
-    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-    const int64_t nkb = (K + BK - 1) / BK;
-    int C = 1;
-    for (int c = 2; c <= 8; c *= 2)
-        if (tiles * c <= sms && nkb >= 2 * c) C = c;
-    return C;
+    return static_cast<int64_t>(stages) * (BM * BK + tbn * packed_bytes_per_kb) + 2LL * tbn * BK;
 }
+
+// The split: 256-feature tiles and the largest cluster c in {2, 4, 8} with
+// tiles * c <= SMs and at least 2 K blocks per split, considered when a
+// factor 2 fits the SMs; otherwise {256, 1}, the unsplit kernel.  (The kernel
+// template also takes 128-feature tiles and any c up to 8, whose reduction
+// divides the columns unevenly; on the decode shapes those measured slower
+// than this rule: 9728 -> 2560 at 128 tokens took 25.9 us as 20 tiles x 7 against
+// 18 us as 10 x 8, and 2560 -> 9728 took 14.9 us as 38 x 3 against 14.2 us as
+// 38 x 2, so the planner keeps to the even splits.)
+inline SplitPlan splitk_plan(int64_t M, int64_t N, int64_t K, int64_t sms, int stages, int pb)
+{
+    const int64_t m_tiles = (M + BM - 1) / BM;
+    const int64_t nkb = (K + BK - 1) / BK;
+    const int64_t tiles = m_tiles * ((N + BN - 1) / BN);
+    SplitPlan best{BN, 1};
+    if (tiles * 2 > sms || nkb < 4) return best;
+    for (int c : {2, 4, 8}) {
+        if (tiles * c > sms || nkb < 2 * c) continue;
+        if (static_cast<int64_t>(c) * ((BN / 32 + c - 1) / c) * 16 * 1024 > splitk_region_bytes(stages, BN, pb))
+            continue;
+        best = SplitPlan{BN, c};
+    }
+    return best;
+}
+
 // Ring depths: TMA stages (activation tile + packed tile) and expanded-tile
 // stages, chosen to fit 227 KB of shared memory with the epilogue staging.
 template <int FMT> __host__ __device__ constexpr int tma_stages() { return FMT == kI4 ? 4 : (FMT == kT2 ? 5 : 6); }
@@ -63,9 +91,13 @@ static_assert(kExpStages < 4, "fewer expansion stages than TMA stages (4 to 6)")
 template <int OUT> __host__ __device__ constexpr int stage_row_bytes() { return OUT == LOWBIT_BF16 ? 80 : 144; }
 template <int OUT> __host__ __device__ constexpr int stage_warp_bytes() { return 32 * stage_row_bytes<OUT>(); }
 
-// Instruction descriptor: s32 accumulate, s8 x s8, both K-major, M=128, N=256.
-constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
-                            (static_cast<uint32_t>(BM >> 4) << 24);
+// Instruction descriptor: s32 accumulate, s8 x s8, both K-major, M=128, N=n.
+__host__ __device__ constexpr uint32_t idesc_m128(int n)
+{
+    return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(BM >> 4) << 24);
+}
+constexpr uint32_t kIdesc = idesc_m128(BN);
 
 // ---------------------------------------------------------------------------
 // Expansion of one stage: ROWS (256, or 128 per CTA of a pair) rows x 128 codes.  Each thread loads 16 bytes of
@@ -191,6 +223,14 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&v)[32], const fl
             }
         }
     }
+}
+
+template <int FMT, int OUT, int TBN>
+__host__ __device__ constexpr size_t splitk_smem_bytes()
+{
+    return 1024 + static_cast<size_t>(tma_stages<FMT>()) * (A_BYTES + TBN * packed_bytes_per_kblock<FMT>()) +
+           static_cast<size_t>(kExpStages) * TBN * BK + 4 * stage_warp_bytes<OUT>() +
+           8 * (2 * tma_stages<FMT>() + 2 * kExpStages + 8);
 }
 
 template <int FMT, int OUT>
@@ -425,15 +465,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
 
 // ---------------------------------------------------------------------------
 // Split-K over a thread-block cluster, for problems with fewer output tiles
-// than SMs (few tokens, or few output features).  The C CTAs of a cluster
-// share one output tile; CTA s accumulates k-blocks [s*nkb/C, (s+1)*nkb/C)
-// into tensor memory.  The partial tiles are then reduce-scattered through
-// distributed shared memory: CTA s receives every peer's partial sums for
-// columns [s*W, (s+1)*W), W = 256/C, adds them (int32 addition is exact, so
-// the result equals the unsplit accumulation bit for bit) and runs the
-// epilogue for those columns.  No global scratch memory is used.
+// than SMs (few tokens, or few output features).  Tiles are 128 tokens x TBN
+// features (256 or 128).  The C CTAs of a cluster (1..8) share one output
+// tile; CTA s accumulates k-blocks [s*nkb/C, (s+1)*nkb/C) into tensor memory.
+// The partial tiles are then reduce-scattered through distributed shared
+// memory: the tile's 32-column chunks are divided among the CTAs (CTA j owns
+// chunks [j*NCH/C, (j+1)*NCH/C), NCH = TBN/32), every CTA sends each owner
+// its partial sums of the owner's chunks, and each owner adds them (int32
+// addition is exact, so the result equals the unsplit accumulation bit for
+// bit) and runs the epilogue for its chunks.  No global scratch memory is used.
 // ---------------------------------------------------------------------------
-template <int FMT, int OUT>
+template <int FMT, int OUT, int TBN = BN>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_p,
                    const float *__restrict__ s_x, const float *__restrict__ s_w, int64_t M, int64_t N, int64_t K,
@@ -442,14 +484,16 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
     constexpr int ST = tma_stages<FMT>();
     constexpr int SE = kExpStages;
     constexpr int PB = packed_bytes_per_kblock<FMT>();
-    constexpr int P_BYTES = BN * PB;
+    constexpr int P_BYTES = TBN * PB;
+    constexpr int TE_BYTES = TBN * BK;
     constexpr int kShift = Fmt<FMT>::kShift;
+    constexpr uint32_t kTileIdesc = idesc_m128(TBN);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = base;
     uint8_t *sE = sA + ST * A_BYTES;
-    uint8_t *sP = sE + SE * E_BYTES;
+    uint8_t *sP = sE + SE * TE_BYTES;
     uint8_t *sStage = sP + ST * P_BYTES;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sStage + 4 * stage_warp_bytes<OUT>());
     uint64_t *full_tma = bars;
@@ -501,7 +545,7 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
     const int64_t num_m = (M + BM - 1) / BM;
     const int64_t tile = blockIdx.x / C;
     const int m0 = static_cast<int>((tile % num_m) * BM);
-    const int n0 = static_cast<int>((tile / num_m) * BN);
+    const int n0 = static_cast<int>((tile / num_m) * TBN);
     const int nkb = static_cast<int>((K + BK - 1) / BK);
     const int kb_begin = static_cast<int>((static_cast<int64_t>(srank) * nkb) / C);
     const int kb_end = static_cast<int>((static_cast<int64_t>(srank + 1) * nkb) / C);
@@ -547,11 +591,11 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
                 if (!wait_bar(&full_exp[s2], (g / SE) & 1u, abort_flag, status)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t a_addr = smem_u32(sA + s1 * A_BYTES);
-                const uint32_t e_addr = smem_u32(sE + s2 * E_BYTES);
+                const uint32_t e_addr = smem_u32(sE + s2 * TE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < BK / UMMA_K; ++kk)
-                    tc_mma_i8(tmem_base, sw128_desc(a_addr + kk * UMMA_K), sw128_desc(e_addr + kk * UMMA_K), kIdesc,
-                              (g | kk) != 0 ? 1u : 0u);
+                    tc_mma_i8(tmem_base, sw128_desc(a_addr + kk * UMMA_K), sw128_desc(e_addr + kk * UMMA_K),
+                              kTileIdesc, (g | kk) != 0 ? 1u : 0u);
                 tc_commit(&mma_done[s1]);
             }
             if (ok) tc_commit(&acc_full[0]);
@@ -570,7 +614,7 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
                 const uint32_t gp = g - SE;
                 if (!wait_bar(&mma_done[gp % ST], (gp / ST) & 1u, abort_flag, status)) break;
             }
-            expand_stage<FMT>(p_base + s1 * P_BYTES, e_base + s2 * E_BYTES, et);
+            expand_stage<FMT, TBN>(p_base + s1 * P_BYTES, e_base + s2 * TE_BYTES, et);
             fence_proxy_async_smem();
             mbar_arrive(&full_exp[s2]);
         }
@@ -586,11 +630,12 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
 
     // Every CTA of the cluster is done with its pipeline buffers: from here
     // they hold the received partial tiles, piece-major: 16-byte piece p
-    // (4 columns) of 32-column chunk cc of row r from source rank s sits at
-    // ((s * NC + cc) * 8 + p) * BM + r, so that the 32 lanes (rows) of one
+    // (4 columns) of the owner's lc-th chunk from source rank s sits at
+    // ((s * MAXC + lc) * 8 + p) * BM + r, so that the 32 lanes (rows) of one
     // remote store instruction write 512 contiguous bytes.
-    const int W = BN / C;                       // columns each CTA finishes
-    const int NC = W / 32;                      // 32-column chunks per slice
+    constexpr int NCH = TBN / 32;               // 32-column chunks of a tile
+    const int MAXC = (NCH + C - 1) / C;         // most chunks one CTA owns
+    auto chunk_begin = [&](int j) { return j * NCH / C; };
     const uint32_t recv = smem_u32(sA);
     cluster_sync_all();
     const int quarter = warp & 3;
@@ -598,18 +643,19 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
     const int64_t row = m0 + row_in_tile;
     if (warp >= 6) {
         for (int j = 0; j < C; ++j) {
-            for (int cc = 0; cc < W / 32; ++cc) {
+            for (int cc = chunk_begin(j); cc < chunk_begin(j + 1); ++cc) {
                 uint32_t v[32];
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                       static_cast<uint32_t>(j * W + cc * 32);
+                                       static_cast<uint32_t>(cc * 32);
                 tmem_ld_32cols(taddr, v);
                 if (!ready) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] = 0;
                 }
                 if (row < M) {
+                    const int lc = cc - chunk_begin(j);
                     const uint32_t dst = map_to_peer(
-                        recv + static_cast<uint32_t>(((static_cast<int>(srank) * NC + cc) * 8 * BM + row_in_tile) * 16),
+                        recv + static_cast<uint32_t>(((static_cast<int>(srank) * MAXC + lc) * 8 * BM + row_in_tile) * 16),
                         static_cast<uint32_t>(j));
 #pragma unroll
                     for (int p = 0; p < 8; ++p)
@@ -624,13 +670,15 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
         const uint32_t stage = smem_u32(sStage) + static_cast<uint32_t>((warp - 6) * stage_warp_bytes<OUT>());
         const float sx = row < M ? ld_act_f32(s_x + row) : 0.0f;
         const float sw_tensor = (FMT == kT2) ? s_w[0] : 0.0f;
-        for (int cc = 0; cc < W / 32; ++cc) {
+        const int own0 = chunk_begin(static_cast<int>(srank));
+        const int own = chunk_begin(static_cast<int>(srank) + 1) - own0;
+        for (int lc = 0; lc < own; ++lc) {
             uint32_t v[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0;
             if (row < M) {
                 for (int s = 0; s < C; ++s) {
-                    const uint32_t src = recv + static_cast<uint32_t>(((s * NC + cc) * 8 * BM + row_in_tile) * 16);
+                    const uint32_t src = recv + static_cast<uint32_t>(((s * MAXC + lc) * 8 * BM + row_in_tile) * 16);
 #pragma unroll
                     for (int p = 0; p < 8; ++p) {
                         const uint4 a = lds128(src + static_cast<uint32_t>(p * BM * 16));
@@ -641,7 +689,7 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
                     }
                 }
             }
-            const int64_t nc = n0 + static_cast<int64_t>(srank) * W + cc * 32;
+            const int64_t nc = n0 + static_cast<int64_t>(own0 + lc) * 32;
             if (nc < N) {
                 float sw[32];
 #pragma unroll
@@ -974,11 +1022,33 @@ lowbit_status launch_pair_fmt(const CUtensorMap &ma, const CUtensorMap &mp, cons
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
+template <int FMT, int OUT, int TBN>
+lowbit_status launch_splitk(const CUtensorMap &ma, const CUtensorMap &mp, const float *s_x, const float *s_w,
+                            int64_t M, int64_t N, int64_t K, void *y, int64_t ldy, int vec_ok, int C, int prefetch,
+                            int32_t *status, cudaStream_t st)
+{
+    constexpr size_t smem = splitk_smem_bytes<FMT, OUT, TBN>();
+    static_assert(smem <= 232448, "shared memory budget");
+    static PerDevice configured;  // the attribute is set once per device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    if (configured.get(dev, [&] {
+            return cudaFuncSetAttribute(gemm_splitk_kernel<FMT, OUT, TBN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(smem)) == cudaSuccess ? 1 : 0;
+        }) <= 0)
+        return LOWBIT_ERR_CUDA;
+    const int64_t tiles = ((M + BM - 1) / BM) * ((N + TBN - 1) / TBN);
+    return launch_pdl(gemm_splitk_kernel<FMT, OUT, TBN>, dim3(static_cast<unsigned>(tiles * C)), dim3(kThreads), smem,
+                      st, static_cast<unsigned>(C), ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, C, prefetch, status);
+}
+
 template <int FMT, int OUT>
 lowbit_status launch_t(const CUtensorMap &ma, const CUtensorMap &mp, const float *s_x, const float *s_w,
                        int64_t M, int64_t N, int64_t K, void *y, int64_t ldy, int vec_ok, int prefetch,
-                       int32_t *status, cudaStream_t st)
+                       int32_t *status, SplitPlan plan, cudaStream_t st)
 {
+    if (plan.c > 1)
+        return launch_splitk<FMT, OUT, 256>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, plan.c, prefetch, status, st);
     constexpr size_t smem = smem_bytes<FMT, OUT>();
     static_assert(smem <= 232448, "shared memory budget");
     static PerDevice configured;  // the attribute is set once per device
@@ -991,18 +1061,6 @@ lowbit_status launch_t(const CUtensorMap &ma, const CUtensorMap &mp, const float
         return LOWBIT_ERR_CUDA;
     const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int64_t sms = device_sm_count();
-    const int C = splitk_clusters(M, N, K, sms);
-    if (C > 1) {
-        static PerDevice configured_split;
-        if (configured_split.get(dev, [&] {
-                return cudaFuncSetAttribute(gemm_splitk_kernel<FMT, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            static_cast<int>(smem)) == cudaSuccess ? 1 : 0;
-            }) <= 0)
-            return LOWBIT_ERR_CUDA;
-        return launch_pdl(gemm_splitk_kernel<FMT, OUT>, dim3(static_cast<unsigned>(tiles * C)), dim3(kThreads), smem,
-                          st, static_cast<unsigned>(C), ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, C, prefetch,
-                          status);
-    }
     const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
     return launch_pdl(gemm_kernel<FMT, OUT>, dim3(grid), dim3(kThreads), smem, st, 0, ma, mp, s_x, s_w, M, N, K, y,
                       ldy, vec_ok, prefetch, status);
@@ -1011,20 +1069,29 @@ lowbit_status launch_t(const CUtensorMap &ma, const CUtensorMap &mp, const float
 template <int FMT>
 lowbit_status launch_fmt(const CUtensorMap &ma, const CUtensorMap &mp, const float *s_x, const float *s_w,
                          int64_t M, int64_t N, int64_t K, void *y, lowbit_dtype ydt, int64_t ldy, int vec_ok,
-                         int prefetch, int32_t *status, cudaStream_t st)
+                         int prefetch, int32_t *status, SplitPlan plan, cudaStream_t st)
 {
     if (ydt == LOWBIT_F32)
-        return launch_t<FMT, LOWBIT_F32>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, st);
+        return launch_t<FMT, LOWBIT_F32>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, plan, st);
     if (ydt == LOWBIT_BF16)
-        return launch_t<FMT, LOWBIT_BF16>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, st);
-    return launch_t<FMT, LOWBIT_I32>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, st);
+        return launch_t<FMT, LOWBIT_BF16>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, plan, st);
+    return launch_t<FMT, LOWBIT_I32>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, plan, st);
+}
+
+// The split plan of a format: its TMA ring depth and packed bytes per K block.
+inline SplitPlan plan_for(lowbit_format f, int64_t M, int64_t N, int64_t K, int64_t sms)
+{
+    if (f == LOWBIT_TERNARY2) return splitk_plan(M, N, K, sms, tma_stages<kT2>(), packed_bytes_per_kblock<kT2>());
+    if (f == LOWBIT_BINARY1) return splitk_plan(M, N, K, sms, tma_stages<kB1>(), packed_bytes_per_kblock<kB1>());
+    return splitk_plan(M, N, K, sms, tma_stages<kI4>(), packed_bytes_per_kblock<kI4>());
 }
 
 }  // namespace tc
 
-bool gemm_splits_k(int64_t M, int64_t N, int64_t K, int64_t sms)
+bool gemm_splits_k(lowbit_format f, int64_t M, int64_t N, int64_t K, int64_t sms)
 {
-    return tc::splitk_clusters(M, N, K, sms) > 1;
+    const tc::SplitPlan p = tc::plan_for(f, M, N, K, sms);
+    return p.c > 1 || p.tbn != tc::BN;
 }
 
 lowbit_status gemm_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
@@ -1040,14 +1107,17 @@ lowbit_status gemm_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_
     const uint32_t pb = f == LOWBIT_TERNARY2 ? packed_bytes_per_kblock<kT2>()
                         : f == LOWBIT_BINARY1 ? packed_bytes_per_kblock<kB1>()
                                               : packed_bytes_per_kblock<kI4>();
+    const SplitPlan plan = plan_for(f, M, N, K, device_sm_count());
     if (!make_map_2d(&mp, packed, static_cast<uint64_t>(row_bytes), static_cast<uint64_t>(N),
-                     static_cast<uint64_t>(ldp), pb, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+                     static_cast<uint64_t>(ldp), pb, static_cast<uint32_t>(plan.tbn), CU_TENSOR_MAP_SWIZZLE_NONE))
         return LOWBIT_ERR_CUDA;
     const int64_t esz = ydt == LOWBIT_BF16 ? 2 : 4;
     const int vec_ok = ((reinterpret_cast<uintptr_t>(y) & 15u) == 0 && (ldy * esz) % 16 == 0) ? 1 : 0;
-    if (f == LOWBIT_TERNARY2) return launch_fmt<kT2>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, st);
-    if (f == LOWBIT_BINARY1) return launch_fmt<kB1>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, st);
-    return launch_fmt<kI4>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, st);
+    if (f == LOWBIT_TERNARY2)
+        return launch_fmt<kT2>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, plan, st);
+    if (f == LOWBIT_BINARY1)
+        return launch_fmt<kB1>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, plan, st);
+    return launch_fmt<kI4>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, plan, st);
 }
 
 }  // namespace lowbit

@@ -308,21 +308,23 @@ lowbit_status lowbit_linear_ex(const int8_t *q, int64_t ldq, const float *s_x,
                                int path, unsigned flags,
                                int32_t *status_dev, void *stream);
 
-/* Largest M * K (K rounded up to a multiple of 128) that lowbit_bitlinear
- * runs as one fused decode kernel. */
-#define LOWBIT_FUSED_MAX_MK 98304
+/* lowbit_bitlinear runs one fused decode kernel when M * K_r <=
+ * LOWBIT_FUSED_MAX_BYTES, K_r = K rounded up to a multiple of 128 (the codes
+ * of the M tokens are held in shared memory). */
+#define LOWBIT_FUSED_MAX_BYTES 98304
 
 /* lowbit_bitlinear -- the whole BitLinear forward of M8.8 0x02E on activations
  * x: the prologue of lowbit_act_quant_ex (gain, RMSNorm, Hadamard rotation,
  * per-token codes) followed by lowbit_linear_ex with the given path and
  * flags.  y is identical to calling those two functions in turn.
- *   - Decode: with M <= 4, hadamard == 0, path 0 or 1 and M * K (K rounded
- *     up to a multiple of 128) <= LOWBIT_FUSED_MAX_MK, one fused kernel runs:
- *     every block computes the codes of the M tokens in shared memory while
- *     its first weight loads are in flight, then streams the packed weights
- *     (one launch instead of two, and the codes never go through global
- *     memory).  q and s_x may then be NULL; when given, they receive the
- *     codes and scales.
+ *   - Decode: with M <= 4, hadamard == 0, path 0 or 1 and the bound of
+ *     LOWBIT_FUSED_MAX_BYTES, one fused kernel runs in clusters of up to 8
+ *     blocks: while their first weight loads are in flight, the blocks of a
+ *     cluster each quantise a share of the M token rows and exchange the
+ *     row statistics and the codes through distributed shared memory, then
+ *     every block streams its packed weight rows (one launch instead of two,
+ *     and the codes never go through global memory).  q and s_x may then be
+ *     NULL; when given, they receive the codes and scales.
  *   - Otherwise the prologue kernel writes q [M, ldq] and s_x [M] (both
  *     required: device workspace owned by the caller, ldq a multiple of 16,
  *     ldq >= K, q 16-byte aligned), and the linear kernel reads them.
@@ -335,6 +337,63 @@ lowbit_status lowbit_bitlinear(const void *x, lowbit_dtype xdt, int64_t M, int64
                                void *y, lowbit_dtype ydt, int64_t ldy,
                                int8_t *q, int64_t ldq, float *s_x,
                                int path, unsigned flags, int32_t *status_dev, void *stream);
+
+/* One layer of a grouped decode call (lowbit_bitlinear_group).  Device
+ * pointers, all owned by the caller:
+ *   x       [M, ldx] token rows of the call's xdt (aligned to its size)
+ *   g       [K] fp32 gain or NULL (4-byte aligned)
+ *   packed  [N, ldp] packed weights of the call's format (16-byte aligned,
+ *           ldp a multiple of 16, ldp >= lowbit_packed_row_bytes(f, K))
+ *   s_w     weight scales (lowbit_scale_count(f, N) fp32)
+ *   y       [M, ldy] output of the call's ydt, ldy >= N
+ *   q, s_x  NULL, or [M, ldq] codes (ldq >= K, multiple of 16, 16-byte
+ *           aligned) and [M] fp32 scales that receive the layer's codes. */
+typedef struct lowbit_bitlinear_item {
+    const void *x;
+    int64_t ldx;
+    const float *g;
+    const uint8_t *packed;
+    int64_t ldp;
+    const float *s_w;
+    int64_t N;
+    int64_t K;
+    void *y;
+    int64_t ldy;
+    int8_t *q;
+    int64_t ldq;
+    float *s_x;
+} lowbit_bitlinear_item;
+
+/* Most layers in one lowbit_bitlinear_group call. */
+#define LOWBIT_GROUP_MAX 32
+
+/* lowbit_bitlinear_group -- several independent decode BitLinear layers in
+ * one launch (M8.8 0x09B: decode streams whole weight matrices for a few
+ * tokens, so the cost of a layer is its packed bytes plus a fixed launch and
+ * dependency latency; several layers that read the same or different token
+ * rows -- the q, k, v projections, or gate and up, of one block -- share that
+ * fixed cost when they run as one kernel).  Each item is computed exactly as
+ * lowbit_bitlinear with hadamard = 0 on that item's arguments: the result is
+ * bit-identical to n_items separate calls.  The kernel is persistent: the
+ * layers' rows are cut into units of up to 8 blocks (a thread-block cluster)
+ * and each resident cluster takes a contiguous range of units of about equal
+ * packed bytes; when a cluster enters a layer, its blocks compute that
+ * layer's codes and scales together while the first weight loads of the
+ * layer are in flight.
+ * items: HOST array of n_items descriptors (read during the call only),
+ * 1 <= n_items <= LOWBIT_GROUP_MAX.  M: tokens, 1..4, the same for all items.
+ * xdt, norm, eps_norm, f, ydt, flags: shared by all items, with the meanings
+ * of lowbit_bitlinear.  Every item needs M * K_r <= LOWBIT_FUSED_MAX_BYTES
+ * (K_r = K rounded up to 128) and K <= LOWBIT_PROLOGUE_MAX_K when it has a
+ * gain or the norm is on.  The items must be independent: no item's y, q or
+ * s_x may overlap another item's inputs or outputs (they are written
+ * concurrently).  Errors: invalid or misaligned arguments of any item are
+ * reported before anything runs (LOWBIT_ERR_INVALID_ARG,
+ * LOWBIT_ERR_ALIGNMENT, LOWBIT_ERR_UNSUPPORTED); device-side conditions
+ * (non-finite activations) set bits in *status_dev as lowbit_bitlinear. */
+lowbit_status lowbit_bitlinear_group(const lowbit_bitlinear_item *items, int n_items, int64_t M,
+                                     lowbit_dtype xdt, int norm, float eps_norm, lowbit_format f,
+                                     lowbit_dtype ydt, unsigned flags, int32_t *status_dev, void *stream);
 
 /* Row-parallel layers (M8.8 0x08A-0x08C).  When the input dimension of a
  * layer is split over ranks, each rank holds a slice x[:, k0:k1] of every

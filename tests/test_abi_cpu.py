@@ -70,21 +70,23 @@ def _linear(lib, **kw):
 # dispatch rules (tiles of 128 tokens x 256 features, K blocks of 128):
 # GEMV up to 4 tokens; warp MMAs up to 16 when a packed row is <= 512 bytes
 # or N >= 3200; the shared-memory GEMM below 512 tokens, split over a cluster
-# of C in {2, 4, 8} when tiles * C fits the SMs and every split keeps 2 K
-# blocks; from 512, SM pairs for ternary weights (split-K kept when K >= 2048
-# and the GEMM splits) and the tensor-memory GEMM for the other formats.
+# of C in {2, 4, 8} CTAs (the largest with tiles * C <= SMs and 2 K blocks per
+# split) when twice its 128 x 256 tiles fit the SMs and K has at least 4
+# blocks; from 512, SM pairs for ternary weights (split-K kept
+# when K >= 2048 and the GEMM splits) and the tensor-memory GEMM for the other
+# formats.
 DISPATCH = [
     ((1, 9728, 2560, bwt.TERNARY2, 0, 148), "gemv_smem_kernel/gemv_kernel"),
     ((4, 9728, 2560, bwt.TERNARY2, 0, 148), "gemv_smem_kernel/gemv_kernel"),
     ((16, 9728, 2560, bwt.TERNARY2, 0, 148), "skinny_mma_kernel/stream_mma_kernel"),  # N >= 3200
     ((8, 192, 768, bwt.BINARY1, 0, 148), "skinny_mma_kernel/stream_mma_kernel"),      # 96-byte rows
-    ((16, 2560, 9728, bwt.TERNARY2, 0, 148), "gemm_splitk_kernel"),  # 2432-byte rows, 10 tiles, C = 8
-    ((128, 9728, 2560, bwt.TERNARY2, 0, 148), "gemm_splitk_kernel"),  # 38 tiles, C = 2
+    ((16, 2560, 9728, bwt.TERNARY2, 0, 148), "gemm_splitk_kernel"),  # 2432-byte rows, 10 tiles x 8
+    ((128, 9728, 2560, bwt.TERNARY2, 0, 148), "gemm_splitk_kernel"),  # 38 tiles x 2
     ((256, 768, 192, bwt.TERNARY2, 0, 148), "gemm_kernel"),  # 2 K blocks: no split
     ((300, 9728, 2560, bwt.TERNARY2, 0, 148), "gemm_kernel"),  # 114 tiles: no split
     ((8192, 9728, 2560, bwt.TERNARY2, 0, 148), "gemm_pair_kernel"),
     ((1024, 2560, 9728, bwt.TERNARY2, 0, 148), "gemm_pair_kernel"),  # 80 tiles: no split
-    ((512, 2560, 9728, bwt.TERNARY2, 0, 148), "gemm_splitk_kernel"),  # 40 tiles, C = 2, deep K
+    ((512, 2560, 9728, bwt.TERNARY2, 0, 148), "gemm_splitk_kernel"),  # 40 tiles x 2, deep K
     ((512, 2560, 9728, bwt.TERNARY2, 0, 64), "gemm_pair_kernel"),    # 40 x 2 > 64 SMs: no split
     ((1024, 256, 1024, bwt.TERNARY2, 0, 148), "gemm_pair_kernel"),   # splits, but K < 2048
     ((8192, 1280, 3584, bwt.INT4, 0, 148), "gemm_ts_kernel"),
@@ -151,6 +153,47 @@ def test_linear_ex_rejects_unknown_flags(lib):
     bad = list(args)
     bad[0] = None                                   # q = NULL with a valid flag
     assert f(*bad, bwt.WEIGHTS_STABLE, None, None) == bwt.ERR_INVALID_ARG
+
+
+def _group(lib, n=2, M=1, fmt=bwt.TERNARY2, ydt=bwt.BF16, flags=0, **item):
+    """lowbit_bitlinear_group on fake device pointers (checks run before any
+    device work, so nothing is dereferenced); item overrides apply to the
+    last layer."""
+    items = (bwt.BitlinearItem * max(n, 1))()
+    for i in range(max(n, 1)):
+        f = dict(x=FAKE, ldx=2560, g=None, packed=FAKE, ldp=640, s_w=FAKE, N=9728, K=2560, y=FAKE, ldy=9728,
+                 q=None, ldq=0, s_x=None)
+        if i == max(n, 1) - 1:
+            f.update(item)
+        items[i] = bwt.BitlinearItem(**f)
+    return lib.lowbit_bitlinear_group(ctypes.cast(items, ctypes.c_void_p), n, M, bwt.BF16, bwt.NORM_NONE, 1e-5, fmt,
+                                      ydt, flags, None, None)
+
+
+def test_bitlinear_group_rejects_bad_arguments(lib):
+    assert lib.lowbit_bitlinear_group(None, 1, 1, bwt.BF16, 0, 1e-5, bwt.TERNARY2, bwt.BF16, 0, None,
+                                      None) == bwt.ERR_INVALID_ARG
+    assert _group(lib, n=0) == bwt.ERR_INVALID_ARG
+    assert _group(lib, n=bwt.GROUP_MAX + 1) == bwt.ERR_INVALID_ARG
+    assert _group(lib, M=0) == bwt.ERR_INVALID_ARG
+    assert _group(lib, M=5) == bwt.ERR_INVALID_ARG                  # decode only: M <= 4
+    assert _group(lib, flags=2) == bwt.ERR_INVALID_ARG
+    assert _group(lib, fmt=3) == bwt.ERR_INVALID_ARG
+    assert _group(lib, ydt=7) == bwt.ERR_INVALID_ARG
+    assert _group(lib, x=None) == bwt.ERR_INVALID_ARG
+    assert _group(lib, y=None) == bwt.ERR_INVALID_ARG
+    assert _group(lib, ldy=100) == bwt.ERR_INVALID_ARG              # ldy < N
+    assert _group(lib, ldp=624) == bwt.ERR_INVALID_ARG              # ldp < row bytes
+    assert _group(lib, ldx=2000) == bwt.ERR_INVALID_ARG             # ldx < K
+    assert _group(lib, packed=FAKE + 8) == bwt.ERR_ALIGNMENT
+    assert _group(lib, y=FAKE + 1) == bwt.ERR_ALIGNMENT
+    assert _group(lib, q=FAKE, ldq=2560 + 8) == bwt.ERR_ALIGNMENT
+    assert _group(lib, q=FAKE, ldq=16) == bwt.ERR_INVALID_ARG       # ldq < K
+    # the codes of a layer must fit the kernel's staging: M * K_r <= 98304
+    k = bwt.FUSED_MAX_BYTES + 128
+    assert _group(lib, K=k, ldx=k, ldp=bwt.packed_ld(bwt.TERNARY2, k)) == bwt.ERR_UNSUPPORTED
+    assert _group(lib, M=4, K=24576 + 128, ldx=24704,
+                  ldp=bwt.packed_ld(bwt.TERNARY2, 24704)) == bwt.ERR_UNSUPPORTED
 
 
 def test_act_quant_rejects_bad_arguments(lib):

@@ -324,6 +324,22 @@ def test_linear_bf16_within_one_ulp(path, fmt, M, N, K):
     assert np.array_equal(got, ref)
 
 
+# Split plans of the shared-memory GEMM (path 2): K split over clusters of
+# 2, 4 and 8 CTAs, with one or two token tiles and ragged N, K and M.
+#   (17, 9728, 2560): 38 tiles x 2        (24, 7168, 2560): 28 tiles x 4
+#   (40, 2560, 9728): 10 tiles x 8        (9, 640, 1024): 3 tiles x 4 (8 K blocks)
+#   (130, 1000, 2000): 2 x 4 tiles x 8    (64, 500, 4096), (3, 2560, 9728): x 8
+SPLIT_SHAPES = [(17, 9728, 2560), (24, 7168, 2560), (40, 2560, 9728), (9, 640, 1024), (130, 1000, 2000),
+                (64, 500, 4096), (3, 2560, 9728)]
+
+
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
+@pytest.mark.parametrize("M,N,K", SPLIT_SHAPES, ids=str)
+def test_split_plans_int32_bit_exact(fmt, M, N, K):
+    y, acc, _, _ = run_case(fmt, M, N, K, 2, bwt.I32, 950 + M + N + K)
+    assert np.array_equal(y.cpu().numpy().astype(np.int64), acc)
+
+
 # LOWBIT_LINEAR_WEIGHTS_STABLE: weight reads start before the wait for the
 # preceding kernel (here the act quant that produced q, launched just before
 # on the same stream); the results must not change.  Shapes cover the GEMV
