@@ -121,12 +121,14 @@ lowbit_kernel choose_kernel(int64_t M, int64_t N, int64_t K, lowbit_format f, in
     // Up to 4 tokens the dp4a GEMV streams weights fastest; from 5 on its
     // int8 MACs outgrow the CUDA cores and tensor-core MMAs win.
     if (path == 1 || (path == 0 && M <= 4)) return LOWBIT_KERNEL_GEMV;
-    // 5 to 16 tokens: warp-level tensor-core MMAs on register fragments
-    // where they were measured faster than the split-K GEMM: rows of at most
-    // 512 packed bytes (one round of register loads), or at least 100 blocks
-    // of 32 output rows.  Longer rows with fewer blocks stay on the GEMM.
-    const bool skinny_wins = rb <= 512 || N >= 3200;
-    if (path == 5 || (path == 0 && M <= 16 && skinny_wins)) return LOWBIT_KERNEL_WARP_MMA;
+    // 5 to 16 tokens: warp-level tensor-core MMAs, with long rows streamed
+    // (weights and token codes) through a TMA ring and K split over a
+    // cluster when the output rows are few; measured faster than the split-K
+    // GEMM on every decode shape of the workloads (e.g. 9728->2560 at M = 16:
+    // 11.0 vs 12.4 us before the cluster split; 3584->1280 at M = 8: 6.7 vs
+    // 10.0 us).
+    (void)rb;
+    if (path == 5 || (path == 0 && M <= 16)) return LOWBIT_KERNEL_WARP_MMA;
     if (path == 6) return LOWBIT_KERNEL_GEMM_PAIR;
     if (path == 4) return LOWBIT_KERNEL_GEMM_TMEM_PAIR;
     // Below 512 tokens the shared-memory variant, which splits K over a

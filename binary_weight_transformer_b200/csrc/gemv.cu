@@ -9,9 +9,9 @@ lowbit_status gemv_launch_b1(const int8_t *, int64_t, const float *, int64_t, in
 lowbit_status gemv_launch_i4(const int8_t *, int64_t, const float *, int64_t, int64_t, const uint8_t *, int64_t,
                              int64_t, const float *, int64_t, void *, lowbit_dtype, int64_t, int, cudaStream_t);
 
-lowbit_status gemv_group_launch_t2(gemv_detail::GroupArgs &, lowbit_dtype, cudaStream_t);
-lowbit_status gemv_group_launch_b1(gemv_detail::GroupArgs &, lowbit_dtype, cudaStream_t);
-lowbit_status gemv_group_launch_i4(gemv_detail::GroupArgs &, lowbit_dtype, cudaStream_t);
+lowbit_status gemv_group_launch_t2(const gemv_detail::GroupArgs &, lowbit_dtype, cudaStream_t);
+lowbit_status gemv_group_launch_b1(const gemv_detail::GroupArgs &, lowbit_dtype, cudaStream_t);
+lowbit_status gemv_group_launch_i4(const gemv_detail::GroupArgs &, lowbit_dtype, cudaStream_t);
 
 // The grouped fused decode call of lowbit_bitlinear_group (and of
 // lowbit_bitlinear with one item): x -> codes in the kernel -> GEMV, for

@@ -10,7 +10,7 @@ lowbit_status gemv_launch_b1(const int8_t *q, int64_t ldq, const float *s_x, int
     return gemv_detail::gemv_launch_fmt<kB1>(q, ldq, s_x, M, K, packed, ldp, row_bytes, s_w, N, y, ydt, ldy, prefetch, st);
 }
 
-lowbit_status gemv_group_launch_b1(gemv_detail::GroupArgs &a, lowbit_dtype ydt, cudaStream_t st)
+lowbit_status gemv_group_launch_b1(const gemv_detail::GroupArgs &a, lowbit_dtype ydt, cudaStream_t st)
 {
     return gemv_detail::gemv_group_launch_fmt<kB1>(a, ydt, st);
 }

@@ -209,291 +209,6 @@ __device__ __forceinline__ int32_t chunk_dot_regs(const uint4 &wv, const uint4 *
     return acc;
 }
 
-// Activation side of one layer of a fused decode call (lowbit_bitlinear,
-// lowbit_bitlinear_group): the token rows x [M, ldx] (fp32 or bf16) with an
-// optional gain g and RMSNorm, from which the blocks of a cluster compute the
-// int8 codes and scales themselves (the per-token rule of quant_rule.cuh; the
-// RMSNorm factor enters only the scale), and to which one cluster also writes
-// the codes and scales (q_out / s_x_out) when they are given.
-struct Prologue {
-    const void *x;
-    int64_t ldx;
-    const float *g;
-    int8_t *q_out;
-    int64_t ldq_out;
-    float *s_x_out;
-    int32_t *status;
-    float eps_norm;
-    int xbf16;
-    int norm;
-};
-
-// Thread-block cluster helpers of the fused decode GEMV.
-__device__ __forceinline__ uint32_t cl_rank()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ uint32_t cl_size()
-{
-    uint32_t n;
-    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
-    return n;
-}
-__device__ __forceinline__ void cl_sync()
-{
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// shared::cluster address of `local` in block `rank` of the cluster
-__device__ __forceinline__ uint32_t cl_map(const void *local, uint32_t rank)
-{
-    uint32_t a;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
-                 : "=r"(a)
-                 : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(local))), "r"(rank));
-    return a;
-}
-__device__ __forceinline__ void cl_st128(uint32_t addr, const uint4 &v)
-{
-    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                 : "memory");
-}
-__device__ __forceinline__ uint32_t cl_ld32(uint32_t addr)
-{
-    uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
-}
-__device__ __forceinline__ double cl_ld64(uint32_t addr)
-{
-    double v;
-    asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(addr) : "memory");
-    return v;
-}
-
-// The 16 values of piece j (features 16j..16j+15) of token row xr, 0 past K.
-__device__ __forceinline__ void piece_values(const Prologue &p, const char *xr, int64_t j, int64_t K, float (&u)[16])
-{
-    const int64_t k0 = 16 * j;
-    const bool vec = k0 + 16 <= K && (reinterpret_cast<uintptr_t>(xr) & 15u) == 0;
-    if (vec && p.xbf16) {
-        const uint4 a = ld_act_u4(xr + k0 * 2);
-        const uint4 b = ld_act_u4(xr + k0 * 2 + 16);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            u[e] = qrule::In<__nv_bfloat16>::get(a, e);
-            u[8 + e] = qrule::In<__nv_bfloat16>::get(b, e);
-        }
-    } else if (vec) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint4 a = ld_act_u4(xr + k0 * 4 + 16 * i);
-            u[4 * i] = __uint_as_float(a.x);
-            u[4 * i + 1] = __uint_as_float(a.y);
-            u[4 * i + 2] = __uint_as_float(a.z);
-            u[4 * i + 3] = __uint_as_float(a.w);
-        }
-    } else {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const int64_t k = k0 + e;
-            u[e] = k >= K ? 0.0f
-                          : (p.xbf16 ? qrule::In<__nv_bfloat16>::scalar(xr, k) : qrule::In<float>::scalar(xr, k));
-        }
-    }
-}
-
-// Codes and scales of the M <= MT token rows, staged into qs (piece-major, as
-// the q staging of gemv_smem_kernel) and sx_s[M] of every block of the
-// cluster.  The blocks of a cluster share the work: block r of C takes code
-// pieces [r P / C, (r + 1) P / C) of every token.  Each block reduces its
-// share's max |x*g| and sum of squares, the C partials are read over
-// distributed shared memory and combined in rank order (so every block gets
-// the same row maximum and scale), then each block quantises its share and
-// writes each 16-code piece into the code buffer of every block of the
-// cluster.  The blocks of one cluster per layer (`writer`) also store the
-// codes and scales to q_out / s_x_out and report non-finite rows.  Called by
-// every thread of every block of the cluster.
-template <int QP, int MT, bool KEEP>
-__device__ void stage_codes_from_x(const Prologue &p, int M, int64_t K, int64_t nchunks, uint4 *qs, float *sx_s,
-                                   bool writer)
-{
-    __shared__ uint32_t red_max[kWarps][MT];
-    __shared__ double red_ss[kWarps][MT];
-    __shared__ uint32_t part_max[MT];
-    __shared__ double part_ss[MT];
-    const uint32_t C = cl_size(), rank = cl_rank();
-    const int64_t qpieces = nchunks * QP;
-    const int64_t j0 = static_cast<int64_t>(rank) * qpieces / C, j1 = static_cast<int64_t>(rank + 1) * qpieces / C;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t xsz = p.xbf16 ? 2 : 4;
-
-    // pass 1: this block's share, max |x*g| and sum of x^2 per token.  With
-    // KEEP (one token) and a share of at most one piece per thread, the piece
-    // stays in registers for the code pass.
-    constexpr bool kKeep = KEEP && MT == 1;
-    const bool keep = kKeep && (j1 - j0) <= static_cast<int64_t>(blockDim.x);
-    float held[16];
-    uint32_t amax[MT];
-    double ss[MT];
-#pragma unroll
-    for (int t = 0; t < MT; ++t) {
-        amax[t] = 0;
-        ss[t] = 0.0;
-    }
-    for (int64_t j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
-        if (16 * j >= K) continue;
-#pragma unroll
-        for (int t = 0; t < MT; ++t) {
-            if (t < M) {
-                float u[16];
-                piece_values(p, static_cast<const char *>(p.x) + t * p.ldx * xsz, j, K, u);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    if (p.norm) ss[t] = __fma_rn(static_cast<double>(u[e]), static_cast<double>(u[e]), ss[t]);
-                    if (p.g != nullptr && 16 * j + e < K) u[e] = __fmul_rn(u[e], p.g[16 * j + e]);
-                    amax[t] = max(amax[t], __float_as_uint(u[e]) & 0x7fffffffu);
-                }
-                if constexpr (kKeep) {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) held[e] = u[e];
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int t = 0; t < MT; ++t) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            amax[t] = max(amax[t], __shfl_xor_sync(0xffffffffu, amax[t], o));
-            ss[t] = __dadd_rn(ss[t], __shfl_xor_sync(0xffffffffu, ss[t], o));
-        }
-        if (lane == 0) {
-            red_max[warp][t] = amax[t];
-            red_ss[warp][t] = ss[t];
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x < MT) {
-        const int t = threadIdx.x;
-        uint32_t a = red_max[0][t];
-        double q2 = red_ss[0][t];
-#pragma unroll
-        for (int w = 1; w < kWarps; ++w) {
-            a = max(a, red_max[w][t]);
-            q2 = __dadd_rn(q2, red_ss[w][t]);
-        }
-        part_max[t] = a;
-        part_ss[t] = q2;
-    }
-    cl_sync();  // every block's partials are visible in the cluster
-    // one thread per (peer, token) fetches that partial into this block
-    __shared__ uint32_t all_max[8][MT];
-    __shared__ double all_ss[8][MT];
-    if (threadIdx.x < C * MT) {
-        const uint32_t s = threadIdx.x / MT, t = threadIdx.x % MT;
-        all_max[s][t] = cl_ld32(cl_map(&part_max[t], s));
-        all_ss[s][t] = cl_ld64(cl_map(&part_ss[t], s));
-    }
-    __syncthreads();
-
-    // the whole rows' statistics, combined in rank order
-    float gm[MT], c[MT];
-    bool slow[MT];
-#pragma unroll
-    for (int t = 0; t < MT; ++t) {
-        uint32_t a = 0;
-        double q2 = 0.0;
-        for (uint32_t s = 0; s < C; ++s) {
-            a = max(a, all_max[s][t]);
-            q2 = __dadd_rn(q2, all_ss[s][t]);
-        }
-        amax[t] = a;
-        gm[t] = __uint_as_float(a);
-        c[t] = __fmul_rn(127.0f, __frcp_rn(gm[t]));
-        slow[t] = !(gm[t] >= 0x1p-121f && gm[t] < 0x1p126f);
-        if (threadIdx.x == 0 && t < M) {
-            float sx = 0.0f;
-            if (a != 0) {
-                if (p.norm) {
-                    double sc = __ddiv_rn(static_cast<double>(gm[t]),
-                                          __dsqrt_rn(__dadd_rn(__ddiv_rn(q2, static_cast<double>(K)),
-                                                               static_cast<double>(p.eps_norm))));
-                    sx = __double2float_rn(__ddiv_rn(sc, 127.0));
-                } else {
-                    sx = __fdiv_rn(gm[t], 127.0f);
-                }
-            }
-            sx_s[t] = sx;
-            const bool bad = !finite_bits(a) || !finite_bits(__float_as_uint(__fmul_rn(gm[t], 127.0f)));
-            if (writer && rank == 0) {
-                if (bad) report(p.status, LOWBIT_ERR_NONFINITE);
-                if (p.s_x_out != nullptr) p.s_x_out[t] = sx;
-            }
-        }
-    }
-    // pass 2: codes of this block's share (pieces past K are zero codes),
-    // written to every block of the cluster
-    for (int64_t j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
-#pragma unroll
-        for (int t = 0; t < MT; ++t) {
-            if (t < M) {
-                uint4 out = make_uint4(0, 0, 0, 0);
-                if (16 * j < K && amax[t] != 0) {
-                    float u[16];
-                    if (keep) {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) u[e] = held[e];
-                    } else {
-                        piece_values(p, static_cast<const char *>(p.x) + t * p.ldx * xsz, j, K, u);
-                        if (p.g != nullptr) {
-#pragma unroll
-                            for (int e = 0; e < 16; ++e)
-                                if (16 * j + e < K) u[e] = __fmul_rn(u[e], p.g[16 * j + e]);
-                        }
-                    }
-                    bool near = slow[t];
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        w[e] = qrule::quant4(u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3], c[t], near);
-                    if (near) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            w[e] = qrule::quant4_exact(u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3], gm[t]);
-                    }
-                    const int64_t valid = K - 16 * j;
-                    if (valid < 16) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int lo = 4 * e;
-                            uint32_t m;
-                            if (valid >= lo + 4) m = 0xffffffffu;
-                            else if (valid <= lo) m = 0u;
-                            else m = (1u << (8 * (valid - lo))) - 1u;
-                            w[e] &= m;
-                        }
-                    }
-                    out = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-                const uint4 *slot = &qs[t * qpieces + (j % QP) * nchunks + j / QP];
-                for (uint32_t s = 0; s < C; ++s) cl_st128(cl_map(slot, s), out);
-                if (writer && p.q_out != nullptr && 16 * j < K) {
-                    int8_t *dst = p.q_out + t * p.ldq_out + 16 * j;
-                    if (16 * j + 16 <= K) {
-                        *reinterpret_cast<uint4 *>(dst) = out;
-                    } else {
-                        const uint8_t *bytes = reinterpret_cast<const uint8_t *>(&out);
-                        for (int64_t e = 0; 16 * j + e < K; ++e) dst[e] = static_cast<int8_t>(bytes[e]);
-                    }
-                }
-            }
-        }
-    }
-    cl_sync();  // every code piece has reached every block
-}
-
 // The R rows of one warp starting at row0, U 16-byte chunks per lane per
 // step, against activation codes staged in shared memory as qs[M][QP][nchunks]
 // (piece-major, so the lanes read consecutive pieces).  stage() runs once,
@@ -632,14 +347,16 @@ lowbit_status launch_smem(const int8_t *q, int64_t ldq, const float *s_x, int M,
 // Grouped fused decode: one launch computes up to kGroupMax BitLinear layers
 // on M <= 4 token rows each, with the activation prologue in the kernel.
 //
-// The work is cut into units of C blocks x 8 warps x R rows of one layer;
-// cluster c of the grid (C blocks, C <= 8) takes a contiguous range of units
-// whose packed bytes are about 1/clusters of the group's (persistent: the
-// grid holds at most as many clusters as are resident at once).  Whenever a
-// cluster reaches a unit of the next layer, its blocks compute that layer's
-// codes together (stage_codes_from_x) while the unit's first weight loads
-// are in flight.  The layers are independent: no layer may read what another
-// writes.
+// The rows of every layer are cut into units of one block (8 warps x R
+// rows); block b of the grid takes a contiguous range of units whose packed
+// bytes are about 1/blocks of the group's (persistent: the grid holds at
+// most as many blocks as are resident at once).  A block first issues the
+// weight loads of its first unit and L2 prefetches for its other units,
+// then computes the codes and scales of the layers of its range itself
+// (every block repeats the prologue of the layers it touches: a few thousand
+// features of arithmetic, cheaper than the barriers and round trips of
+// sharing it), then streams its units against the staged codes.  The layers
+// are independent: no layer may read what another writes.
 struct GroupItem {
     const void *x;         // [M, ldx] token rows
     const float *g;        // [K] gain or nullptr
@@ -654,12 +371,15 @@ struct GroupItem {
     int32_t unit0, units;  // this layer's units: [unit0, unit0 + units)
 };
 constexpr int kGroupMax = 32;
+// Largest staging of one layer's token rows in shared memory.
+constexpr int64_t kXStageMax = 40 * 1024;
 struct GroupArgs {
     GroupItem item[kGroupMax];
     int64_t cost_total;
     int32_t *status;
     float eps_norm;
     int n_items, units, M, xbf16, norm, prefetch;
+    int xstage;  // bytes of shared memory after the codes for one layer's token rows (0: read x from global)
 };
 static_assert(sizeof(GroupArgs) <= 4000, "the group must fit the 4 KB kernel parameter space");
 
@@ -675,64 +395,366 @@ __device__ __forceinline__ int first_unit_at(const GroupArgs &a, int64_t target)
     return a.units;
 }
 
+// The layer that unit u belongs to, searching up from layer i.
+__device__ __forceinline__ int item_of(const GroupArgs &a, int u, int i)
+{
+    while (i + 1 < a.n_items && a.item[i + 1].unit0 <= u) ++i;
+    return i;
+}
+
+// Prefetch `bytes` (a multiple of 16) at a 16-byte aligned address into L2.
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// L1-allocating loads of activation-side data, issued after the wait for
+// the previous kernel (asm volatile keeps them there): the prologue reads
+// every row twice, for the statistics and for the codes.
+__device__ __forceinline__ uint2 ld_ca_u2(const void *p)
+{
+    uint2 v;
+    asm volatile("ld.global.ca.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint4 ld_ca_u4(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.ca.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p)
+                 : "memory");
+    return v;
+}
+
+// Features k0..k0+3 of token row xr (bf16 when xbf16, else fp32), 0 past K.
+__device__ __forceinline__ void quad_x(int xbf16, const char *xr, int64_t k0, int64_t K, float (&f)[4])
+{
+    const bool full = k0 + 4 <= K;
+    if (xbf16) {
+        const char *p = xr + 2 * k0;
+        if (full && (reinterpret_cast<uintptr_t>(p) & 7u) == 0) {
+            const uint2 w = ld_ca_u2(p);
+            f[0] = __uint_as_float(w.x << 16);
+            f[1] = __uint_as_float(w.x & 0xffff0000u);
+            f[2] = __uint_as_float(w.y << 16);
+            f[3] = __uint_as_float(w.y & 0xffff0000u);
+            return;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) f[e] = k0 + e < K ? qrule::In<__nv_bfloat16>::scalar(xr, k0 + e) : 0.0f;
+    } else {
+        const char *p = xr + 4 * k0;
+        if (full && (reinterpret_cast<uintptr_t>(p) & 15u) == 0) {
+            const uint4 w = ld_ca_u4(p);
+            f[0] = __uint_as_float(w.x);
+            f[1] = __uint_as_float(w.y);
+            f[2] = __uint_as_float(w.z);
+            f[3] = __uint_as_float(w.w);
+            return;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) f[e] = k0 + e < K ? qrule::In<float>::scalar(xr, k0 + e) : 0.0f;
+    }
+}
+
+// f *= g[k0..k0+3] (features past K keep their zero).
+__device__ __forceinline__ void quad_gain(const float *g, int64_t k0, int64_t K, float (&f)[4])
+{
+    if (k0 + 4 <= K && (reinterpret_cast<uintptr_t>(g + k0) & 15u) == 0) {
+        const uint4 w = ld_ca_u4(g + k0);
+        f[0] = __fmul_rn(f[0], __uint_as_float(w.x));
+        f[1] = __fmul_rn(f[1], __uint_as_float(w.y));
+        f[2] = __fmul_rn(f[2], __uint_as_float(w.z));
+        f[3] = __fmul_rn(f[3], __uint_as_float(w.w));
+        return;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        if (k0 + e < K) f[e] = __fmul_rn(f[e], ld_act_f32(g + k0 + e));
+}
+
+// Features k0..k0+3 of a token row staged in shared memory at xs (the
+// row's first `staged` bytes; the rest is read from global memory).
+__device__ __forceinline__ void quad_x_staged(int xbf16, const char *xr, uint32_t xs, int64_t staged, int64_t k0,
+                                              int64_t K, float (&f)[4])
+{
+    if (xbf16 && 2 * (k0 + 4) <= staged) {
+        uint32_t lo, hi;
+        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo), "=r"(hi) : "r"(xs + static_cast<uint32_t>(2 * k0)));
+        f[0] = __uint_as_float(lo << 16);
+        f[1] = __uint_as_float(lo & 0xffff0000u);
+        f[2] = __uint_as_float(hi << 16);
+        f[3] = __uint_as_float(hi & 0xffff0000u);
+        return;
+    }
+    if (!xbf16 && 4 * (k0 + 4) <= staged) {
+        uint4 w;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
+                     : "r"(xs + static_cast<uint32_t>(4 * k0)));
+        f[0] = __uint_as_float(w.x);
+        f[1] = __uint_as_float(w.y);
+        f[2] = __uint_as_float(w.z);
+        f[3] = __uint_as_float(w.w);
+        return;
+    }
+    quad_x(xbf16, xr, k0, K, f);
+}
+
+// Copies the whole 16-byte pieces of the M token rows of layer I into
+// shared memory at xs (row t at t * row_bytes rounded up to 16) with
+// cp.async (all copies in flight at once, L2 only), and waits for them.
+// Called by every thread of the block; the buffer is reused layer by layer.
+// Returns the bytes of each row that are staged.
+__device__ __forceinline__ int64_t stage_rows(const GroupItem &I, int M, int64_t xsz, uint32_t xs)
+{
+    const int64_t row = static_cast<int64_t>(I.K) * xsz;
+    const int64_t n16 = row / 16;
+    const int64_t pitch = (row + 15) / 16 * 16;
+    __syncthreads();  // every thread is done with the previous layer's rows
+    for (int64_t c = threadIdx.x; c < M * n16; c += blockDim.x) {
+        const int64_t t = c / n16, j = c % n16;
+        const char *src = static_cast<const char *>(I.x) + t * I.ldx * xsz + 16 * j;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(xs + static_cast<uint32_t>(t * pitch + 16 * j)),
+                     "l"(src)
+                     : "memory");
+    }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    return 16 * n16;
+}
+
+// The codes and scales of layers i0..i1 of the group in this block: codes
+// into qs (layer i at qoff[i - i0], [M][QP][nchunks] piece-major as the GEMV
+// reads them, zero past K) and scales into sx_s[(i - i0) * MT + t].  Per
+// layer: pass 1 reduces max |x*g| and, with the norm, the fp64 sum of x^2
+// over the row in a fixed order (thread tid takes 16-feature pieces tid,
+// tid + 256, ... in turn, then a shuffle tree and the 8 warps in order), so
+// every block -- and every grid -- gets the same row maximum and scale; pass
+// 2 reads the row again (L1) and writes the codes.  The block whose range
+// holds the layer's first unit (`writer`) also stores the codes and scales
+// to q_out / s_x_out and reports non-finite rows.  Called by every thread of
+// the block.
+template <int QP, int MT>
+__device__ void stage_block(const GroupArgs &a, int i0, int i1, int u_begin, int u_end, const int32_t *qoff,
+                            uint4 *qs, float *sx_s, uint32_t xs)
+{
+    __shared__ uint32_t red_max[kWarps][MT];
+    __shared__ double red_ss[kWarps][MT];
+    __shared__ uint32_t gm_s[MT];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool norm = a.norm != 0;
+    const int64_t xsz = a.xbf16 ? 2 : 4;
+    for (int i = i0; i <= i1; ++i) {
+        const GroupItem &I = a.item[i];
+        const bool writer = u_begin <= I.unit0 && I.unit0 < u_end;
+        const int64_t qp = static_cast<int64_t>(I.nchunks) * QP;  // code pieces per token row
+        const int64_t np = (static_cast<int64_t>(I.K) + 15) / 16;  // pieces holding features
+        // with xstage the rows are first copied to shared memory (one round trip)
+        const int64_t staged = a.xstage > 0 ? stage_rows(I, a.M, xsz, xs) : 0;
+        const int64_t pitch = (static_cast<int64_t>(I.K) * xsz + 15) / 16 * 16;
+
+        // pass 1
+        uint32_t amax[MT];
+        double ss[MT];
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+            amax[t] = 0;
+            ss[t] = 0.0;
+        }
+        for (int64_t p = threadIdx.x; p < np; p += blockDim.x) {
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+                if (t >= a.M) continue;
+                const char *xr = static_cast<const char *>(I.x) + t * I.ldx * xsz;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float f[4];
+                    quad_x_staged(a.xbf16, xr, xs + static_cast<uint32_t>(t * pitch), staged, 16 * p + 4 * e, I.K, f);
+                    if (norm) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            ss[t] = __fma_rn(static_cast<double>(f[v]), static_cast<double>(f[v]), ss[t]);
+                    }
+                    if (I.g != nullptr) quad_gain(I.g, 16 * p + 4 * e, I.K, f);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) amax[t] = max(amax[t], __float_as_uint(f[v]) & 0x7fffffffu);
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                amax[t] = max(amax[t], __shfl_xor_sync(0xffffffffu, amax[t], o));
+                ss[t] = __dadd_rn(ss[t], __shfl_xor_sync(0xffffffffu, ss[t], o));
+            }
+            if (lane == 0) {
+                red_max[warp][t] = amax[t];
+                red_ss[warp][t] = ss[t];
+            }
+        }
+        __syncthreads();
+        if (threadIdx.x < a.M) {
+            const int t = threadIdx.x;
+            uint32_t m = red_max[0][t];
+            double q2 = red_ss[0][t];
+#pragma unroll
+            for (int w = 1; w < kWarps; ++w) {
+                m = max(m, red_max[w][t]);
+                q2 = __dadd_rn(q2, red_ss[w][t]);
+            }
+            const float gm = __uint_as_float(m);
+            float sx = 0.0f;
+            if (m != 0) {
+                if (norm) {
+                    const double sc = __ddiv_rn(static_cast<double>(gm),
+                                                __dsqrt_rn(__dadd_rn(__ddiv_rn(q2, static_cast<double>(I.K)),
+                                                                     static_cast<double>(a.eps_norm))));
+                    sx = __double2float_rn(__ddiv_rn(sc, 127.0));
+                } else {
+                    sx = __fdiv_rn(gm, 127.0f);
+                }
+            }
+            gm_s[t] = m;
+            sx_s[(i - i0) * MT + t] = sx;
+            if (writer) {
+                if (!finite_bits(m) || !finite_bits(__float_as_uint(__fmul_rn(gm, 127.0f))))
+                    report(a.status, LOWBIT_ERR_NONFINITE);
+                if (I.s_x_out != nullptr) I.s_x_out[t] = sx;
+            }
+        }
+        __syncthreads();
+
+        // pass 2: codes of every piece of the staging (zero past K)
+        uint4 *qi = qs + qoff[i - i0];
+        for (int64_t p = threadIdx.x; p < qp; p += blockDim.x) {
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+                if (t >= a.M) continue;
+                const uint32_t m = gm_s[t];
+                uint32_t w[4] = {0u, 0u, 0u, 0u};
+                if (p < np && m != 0) {
+                    const char *xr = static_cast<const char *>(I.x) + t * I.ldx * xsz;
+                    const float gm = __uint_as_float(m);
+                    const float c = __fmul_rn(127.0f, __frcp_rn(gm));
+                    const bool slow = !(gm >= 0x1p-121f && gm < 0x1p126f);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float f[4];
+                        quad_x_staged(a.xbf16, xr, xs + static_cast<uint32_t>(t * pitch), staged, 16 * p + 4 * e,
+                                      I.K, f);
+                        if (I.g != nullptr) quad_gain(I.g, 16 * p + 4 * e, I.K, f);
+                        bool near = slow;
+                        w[e] = qrule::quant4(f[0], f[1], f[2], f[3], c, near);
+                        if (near) w[e] = qrule::quant4_exact(f[0], f[1], f[2], f[3], gm);
+                    }
+                    const int64_t valid = static_cast<int64_t>(I.K) - 16 * p;
+                    if (valid < 16) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int lo = 4 * e;
+                            uint32_t mk;
+                            if (valid >= lo + 4) mk = 0xffffffffu;
+                            else if (valid <= lo) mk = 0u;
+                            else mk = (1u << (8 * (valid - lo))) - 1u;
+                            w[e] &= mk;
+                        }
+                    }
+                }
+                const uint4 out = make_uint4(w[0], w[1], w[2], w[3]);
+                qi[t * qp + (p % QP) * I.nchunks + p / QP] = out;
+                if (writer && I.q_out != nullptr && p < np) {
+                    int8_t *dst = I.q_out + t * I.ldq_out + 16 * p;
+                    if (16 * p + 16 <= I.K) {
+                        *reinterpret_cast<uint4 *>(dst) = out;
+                    } else {
+                        const uint8_t *bytes = reinterpret_cast<const uint8_t *>(&out);
+                        for (int64_t e = 0; 16 * p + e < I.K; ++e) dst[e] = static_cast<int8_t>(bytes[e]);
+                    }
+                }
+            }
+        }
+    }
+    __syncthreads();
+}
+
 // Held to three blocks per SM (at most 85 registers a thread).
 template <int FMT, int MT, int U, int R, int OUT>
 __global__ void __launch_bounds__(kWarps * 32, 3) gemv_group_kernel(const __grid_constant__ GroupArgs a)
 {
     constexpr int QP = QPieces<FMT>::value;
     extern __shared__ uint4 qs[];
-    __shared__ float sx_s[MT];
-    const int warp = threadIdx.x >> 5;
-    const uint32_t C = cl_size(), rank = cl_rank();
-    const int64_t clusters = gridDim.x / C, cl = blockIdx.x / C;
-    const int u_begin = first_unit_at(a, cl * a.cost_total / clusters);
-    const int u_end = first_unit_at(a, (cl + 1) * a.cost_total / clusters);
-    // With prefetch the first weight loads are issued before the wait for the
-    // previous kernel (the caller vouches that it does not write the weights).
+    __shared__ float sx_s[kGroupMax * MT];
+    __shared__ int32_t qoff_s[kGroupMax];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t blocks = gridDim.x;
+    const int u_begin = first_unit_at(a, static_cast<int64_t>(blockIdx.x) * a.cost_total / blocks);
+    const int u_end = first_unit_at(a, (static_cast<int64_t>(blockIdx.x) + 1) * a.cost_total / blocks);
+    const int i0 = item_of(a, u_begin, 0);
+    const int i1 = u_end > u_begin ? item_of(a, u_end - 1, i0) : i0;
+    auto row_of = [&](const GroupItem &I, int u) {
+        return (static_cast<int64_t>(u - I.unit0) * kWarps + warp) * R;
+    };
+    // With prefetch the weight loads and prefetches are issued before the
+    // wait for the previous kernel (the caller vouches that it does not
+    // write the weights).
     bool waited = a.prefetch == 0;
     if (waited) pdl_wait();
     pdl_trigger();
-    int it = 0, cur = -1;
+    // L2 prefetch of the rows of this warp's units (the first unit's first
+    // chunks are also loaded into registers right away; its later chunks and
+    // the later units then come from L2)
+    for (int u = u_begin, it = i0; u < u_end; ++u) {
+        it = item_of(a, u, it);
+        const GroupItem &I = a.item[it];
+        const int64_t row = row_of(I, u) + lane;
+        if (lane < R && row < I.N) prefetch_l2(I.packed + row * I.ldp, static_cast<uint32_t>(I.nchunks) * 16u);
+    }
+    if (threadIdx.x == 0) {
+        int32_t off = 0;
+        for (int i = i0; i <= i1; ++i) {
+            qoff_s[i - i0] = off;
+            off += a.M * a.item[i].nchunks * QP;
+        }
+    }
+    // the x staging follows the codes of every layer of the launch
+    int64_t xs_off = 0;
+    for (int i = 0; i < a.n_items; ++i) xs_off += static_cast<int64_t>(a.M) * a.item[i].nchunks * QP * 16;
+    __syncthreads();
+
+    int it = i0;
+    bool staged = false;
     float sxr[MT];
     for (int u = u_begin; u < u_end; ++u) {
-        while (it + 1 < a.n_items && a.item[it + 1].unit0 <= u) ++it;
+        it = item_of(a, u, it);
         const GroupItem &I = a.item[it];
-        const int64_t row0 = ((static_cast<int64_t>(u - I.unit0) * C + rank) * kWarps + warp) * R;
+        const int64_t row0 = row_of(I, u);
         int32_t acc[R][MT];
-        rows_dot<FMT, MT, U, R>(I.packed, I.ldp, I.nchunks, I.N, row0, a.M, qs, [&] {
-            if (it == cur) return;  // the same layer's codes are staged already
-            if (!waited) {
-                pdl_wait();
-                waited = true;
+        rows_dot<FMT, MT, U, R>(I.packed, I.ldp, I.nchunks, I.N, row0, a.M, qs + qoff_s[it - i0], [&] {
+            if (!staged) {
+                if (!waited) {
+                    pdl_wait();
+                    waited = true;
+                }
+                stage_block<QP, MT>(a, i0, i1, u_begin, u_end, qoff_s, qs, sx_s,
+                                    static_cast<uint32_t>(__cvta_generic_to_shared(qs)) +
+                                        static_cast<uint32_t>(xs_off));
+                staged = true;
             }
-            if (cur >= 0) cl_sync();  // every block of the cluster is done with the previous codes
-            Prologue p;
-            p.x = I.x;
-            p.ldx = I.ldx;
-            p.g = I.g;
-            p.q_out = I.q_out;
-            p.ldq_out = I.ldq_out;
-            p.s_x_out = I.s_x_out;
-            p.status = a.status;
-            p.eps_norm = a.eps_norm;
-            p.xbf16 = a.xbf16;
-            p.norm = a.norm;
-            stage_codes_from_x<QP, MT, (U * R <= 5)>(p, a.M, I.K, I.nchunks, qs, sx_s, u == I.unit0);
-            __syncthreads();
 #pragma unroll
-            for (int t = 0; t < MT; ++t) sxr[t] = sx_s[t];
-            cur = it;
+            for (int t = 0; t < MT; ++t) sxr[t] = sx_s[(it - i0) * MT + t];
         }, acc);
         rows_store<FMT, MT, R, OUT>(acc, row0, I.N, a.M, I.s_w, I.y, I.ldy, sxr);
     }
+    if (!waited) pdl_wait();
 }
 
-// Resident clusters of C blocks with `smem` bytes of codes each, per device
-// (cached; 0 when the query fails).
+// Resident blocks with `smem` bytes of codes, per device (cached; 0 when the
+// query fails).
 template <int FMT, int MT, int U, int R, int OUT>
-int group_resident_clusters(unsigned C, size_t smem)
+int group_resident_blocks(size_t smem)
 {
-    struct Entry { int dev; unsigned C; size_t smem; int clusters; };
+    struct Entry { int dev; size_t smem; int blocks; };
     static std::mutex mu;
     static Entry cache[64];
     static int used = 0;
@@ -740,35 +762,26 @@ int group_resident_clusters(unsigned C, size_t smem)
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
     std::lock_guard<std::mutex> lock(mu);
     for (int i = 0; i < used; ++i)
-        if (cache[i].dev == dev && cache[i].C == C && cache[i].smem == smem) return cache[i].clusters;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(C);
-    cfg.blockDim = dim3(kWarps * 32);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = C;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, gemv_group_kernel<FMT, MT, U, R, OUT>, &cfg) != cudaSuccess) {
+        if (cache[i].dev == dev && cache[i].smem == smem) return cache[i].blocks;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_group_kernel<FMT, MT, U, R, OUT>, kWarps * 32,
+                                                      smem) != cudaSuccess) {
         (void)cudaGetLastError();
         return 0;
     }
-    if (clusters > 0 && used < 64) cache[used++] = Entry{dev, C, smem, clusters};
-    return clusters;
+    const int blocks = per_sm * device_sm_count();
+    if (blocks > 0 && used < 64) cache[used++] = Entry{dev, smem, blocks};
+    return blocks;
 }
 
 template <int FMT, int MT, int U, int R, int OUT>
-lowbit_status launch_group_out(GroupArgs &a, unsigned C, size_t smem, cudaStream_t st)
+lowbit_status launch_group_out(GroupArgs &a, size_t smem, cudaStream_t st)
 {
-    const int resident = group_resident_clusters<FMT, MT, U, R, OUT>(C, smem);
+    const int resident = group_resident_blocks<FMT, MT, U, R, OUT>(smem);
     if (resident <= 0) return LOWBIT_ERR_CUDA;
-    const int64_t clusters = a.units < resident ? a.units : resident;
-    return launch_pdl(gemv_group_kernel<FMT, MT, U, R, OUT>, dim3(static_cast<unsigned>(clusters * C)),
-                      dim3(kWarps * 32), smem, st, C, a);
+    const int64_t blocks = a.units < resident ? a.units : resident;
+    return launch_pdl(gemv_group_kernel<FMT, MT, U, R, OUT>, dim3(static_cast<unsigned>(blocks)), dim3(kWarps * 32),
+                      smem, st, 0, a);
 }
 
 template <int FMT, int MT, int U, int R>
@@ -778,7 +791,7 @@ lowbit_status launch_group(GroupArgs &a, lowbit_dtype ydt, size_t smem, cudaStre
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
     if (configured.get(dev, [&] {
-            const int lim = static_cast<int>(kGemvSmemMax);
+            const int lim = static_cast<int>(kGemvSmemMax + kXStageMax);
             return (cudaFuncSetAttribute(gemv_group_kernel<FMT, MT, U, R, LOWBIT_F32>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, lim) == cudaSuccess &&
                     cudaFuncSetAttribute(gemv_group_kernel<FMT, MT, U, R, LOWBIT_BF16>,
@@ -787,20 +800,12 @@ lowbit_status launch_group(GroupArgs &a, lowbit_dtype ydt, size_t smem, cudaStre
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, lim) == cudaSuccess) ? 1 : 0;
         }) <= 0)
         return LOWBIT_ERR_CUDA;
-    // units of C blocks; C = 8 unless every layer has fewer row blocks
     const int64_t rows_per_block = kWarps * R;
-    int64_t max_blocks = 1;
-    for (int i = 0; i < a.n_items; ++i) {
-        const int64_t blocks = (a.item[i].N + rows_per_block - 1) / rows_per_block;
-        max_blocks = blocks > max_blocks ? blocks : max_blocks;
-    }
-    const unsigned C = static_cast<unsigned>(max_blocks < 8 ? max_blocks : 8);
     int64_t units = 0, cost = 0;
     for (int i = 0; i < a.n_items; ++i) {
         GroupItem &I = a.item[i];
-        const int64_t blocks = (I.N + rows_per_block - 1) / rows_per_block;
         I.unit0 = static_cast<int32_t>(units);
-        I.units = static_cast<int32_t>((blocks + C - 1) / C);
+        I.units = static_cast<int32_t>((I.N + rows_per_block - 1) / rows_per_block);
         I.cost0 = cost;
         units += I.units;
         cost += static_cast<int64_t>(I.units) * I.nchunks;
@@ -808,9 +813,9 @@ lowbit_status launch_group(GroupArgs &a, lowbit_dtype ydt, size_t smem, cudaStre
     if (units > INT32_MAX) return LOWBIT_ERR_INVALID_ARG;
     a.units = static_cast<int>(units);
     a.cost_total = cost;
-    if (ydt == LOWBIT_F32) return launch_group_out<FMT, MT, U, R, LOWBIT_F32>(a, C, smem, st);
-    if (ydt == LOWBIT_BF16) return launch_group_out<FMT, MT, U, R, LOWBIT_BF16>(a, C, smem, st);
-    return launch_group_out<FMT, MT, U, R, LOWBIT_I32>(a, C, smem, st);
+    if (ydt == LOWBIT_F32) return launch_group_out<FMT, MT, U, R, LOWBIT_F32>(a, smem, st);
+    if (ydt == LOWBIT_BF16) return launch_group_out<FMT, MT, U, R, LOWBIT_BF16>(a, smem, st);
+    return launch_group_out<FMT, MT, U, R, LOWBIT_I32>(a, smem, st);
 }
 
 // Long rows whose activations do not fit the shared-memory staging: the
@@ -864,22 +869,24 @@ lowbit_status launch_tokens(const int8_t *q, int64_t ldq, const float *s_x, int 
     return launch_smem<FMT, MT, 8, 1>(q, ldq, s_x, M, K, packed, ldp, nchunks, s_w, N, y, ydt, ldy, smem, prefetch, st);
 }
 
-// The same choice of U and R for a group, from its longest rows and its
-// total rows (the persistent grid spreads the rows over the resident blocks).
+// U and R for a group: R (rows per warp) so that the units about fill the
+// resident blocks (three per SM) once, with U = 2 chunks per lane; a group
+// of few rows takes R = 1 and U from its longest rows, as the plain GEMV.
 template <int FMT, int MT>
 lowbit_status launch_group_tokens(GroupArgs &a, int64_t max_nchunks, int64_t rows, lowbit_dtype ydt, size_t smem,
                                   cudaStream_t st)
 {
-    const int64_t slots = static_cast<int64_t>(device_sm_count()) * 2 * kWarps;
-    if (max_nchunks <= 64) {
-        if constexpr (MT == 1) {
-            if (rows >= 4 * slots) return launch_group<FMT, MT, 2, 4>(a, ydt, smem, st);
-        }
-        if (rows >= 2 * slots) return launch_group<FMT, MT, 2, 2>(a, ydt, smem, st);
-        return launch_group<FMT, MT, 2, 1>(a, ydt, smem, st);
+    const int64_t warps = static_cast<int64_t>(device_sm_count()) * 3 * kWarps;  // resident warps
+    if constexpr (MT == 1) {
+        if (rows >= 2 * warps) return launch_group<FMT, MT, 2, 4>(a, ydt, smem, st);
     }
-    if (max_nchunks <= 160) return launch_group<FMT, MT, 5, 1>(a, ydt, smem, st);
-    return launch_group<FMT, MT, 8, 1>(a, ydt, smem, st);
+    if (rows >= warps) return launch_group<FMT, MT, 2, 2>(a, ydt, smem, st);
+    if (max_nchunks <= 64) return launch_group<FMT, MT, 2, 1>(a, ydt, smem, st);
+    // (eight chunks per lane do not fit the registers with four tokens)
+    if constexpr (MT == 1) {
+        if (max_nchunks > 160) return launch_group<FMT, MT, 8, 1>(a, ydt, smem, st);
+    }
+    return launch_group<FMT, MT, 5, 1>(a, ydt, smem, st);
 }
 
 // Tokens are processed in groups of up to 4, one launch per group.
@@ -902,20 +909,50 @@ lowbit_status gemv_launch_fmt(const int8_t *q, int64_t ldq, const float *s_x, in
     return LOWBIT_OK;
 }
 
-// The grouped fused decode call (nchunks of every item set by the caller):
-// the codes of all M tokens of the longest layer must fit the staging.
+// The grouped fused decode call (nchunks of every item set by the caller).
+// The codes of all layers of a launch are staged in shared memory at once,
+// so consecutive layers are launched together while their codes fit
+// kGemvSmemMax (every single layer fits: the caller checks it).
 template <int FMT>
-lowbit_status gemv_group_launch_fmt(GroupArgs &a, lowbit_dtype ydt, cudaStream_t st)
+lowbit_status gemv_group_launch_fmt(const GroupArgs &all, lowbit_dtype ydt, cudaStream_t st)
 {
-    int64_t max_nchunks = 0, rows = 0;
-    for (int i = 0; i < a.n_items; ++i) {
-        max_nchunks = a.item[i].nchunks > max_nchunks ? a.item[i].nchunks : max_nchunks;
-        rows += a.item[i].N;
+    constexpr int QP = QPieces<FMT>::value;
+    int first = 0;
+    while (first < all.n_items) {
+        GroupArgs a = all;
+        int64_t bytes = 0, max_nchunks = 0, rows = 0;
+        int n = 0;
+        while (first + n < all.n_items) {
+            const GroupItem &I = all.item[first + n];
+            const int64_t b = static_cast<int64_t>(all.M) * I.nchunks * QP * 16;
+            if (n > 0 && bytes + b > kGemvSmemMax) break;
+            if (b > kGemvSmemMax) return LOWBIT_ERR_INVALID_ARG;
+            a.item[n] = I;
+            bytes += b;
+            max_nchunks = I.nchunks > max_nchunks ? I.nchunks : max_nchunks;
+            rows += I.N;
+            ++n;
+        }
+        a.n_items = n;
+        // stage x in shared memory when every layer's rows are 16-byte
+        // aligned and the largest layer's M rows fit kXStageMax
+        const int64_t xsz = all.xbf16 ? 2 : 4;
+        int64_t xrows = 0;
+        bool aligned = true;
+        for (int i = 0; i < n; ++i) {
+            const GroupItem &I = a.item[i];
+            aligned = aligned && (reinterpret_cast<uintptr_t>(I.x) & 15u) == 0 && (I.ldx * xsz) % 16 == 0;
+            const int64_t r = static_cast<int64_t>(all.M) * ((I.K * xsz + 15) / 16 * 16);
+            xrows = r > xrows ? r : xrows;
+        }
+        a.xstage = (aligned && xrows <= kXStageMax) ? static_cast<int>(xrows) : 0;
+        const size_t smem = static_cast<size_t>(bytes + a.xstage);
+        const lowbit_status s = all.M == 1 ? launch_group_tokens<FMT, 1>(a, max_nchunks, rows, ydt, smem, st)
+                                           : launch_group_tokens<FMT, 4>(a, max_nchunks, rows, ydt, smem, st);
+        if (s != LOWBIT_OK) return s;
+        first += n;
     }
-    const int64_t smem = static_cast<int64_t>(a.M) * max_nchunks * QPieces<FMT>::value * 16;
-    if (smem > kGemvSmemMax) return LOWBIT_ERR_INVALID_ARG;
-    if (a.M == 1) return launch_group_tokens<FMT, 1>(a, max_nchunks, rows, ydt, static_cast<size_t>(smem), st);
-    return launch_group_tokens<FMT, 4>(a, max_nchunks, rows, ydt, static_cast<size_t>(smem), st);
+    return LOWBIT_OK;
 }
 
 }  // namespace gemv_detail

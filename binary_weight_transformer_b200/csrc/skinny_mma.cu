@@ -231,48 +231,98 @@ skinny_mma_kernel(const int8_t *__restrict__ q, int64_t ldq, const float *__rest
 // weight bytes in flight in registers, four lanes per 16-byte word (the
 // fragment layout gives the same word to the four lanes of a group), so a
 // long row needs several dependent load rounds.  Here one thread streams
-// 32-row x 128-byte boxes of the packed artifact into a ring of shared-memory
-// stages with TMA (128-byte swizzle, so the 8 rows one lds.128 reads hit 8
-// different bank groups), and four consumer warps take two 16-byte chunks of
-// every row of a stage each, reading their fragment words with broadcast
-// shared-memory loads.  The activation words come from L1/L2 as before.
+// 32-row x 128-byte boxes of the packed artifact, and the token codes of the
+// same K range (boxes of 128 codes x 8 or 16 tokens), into a ring of
+// shared-memory stages with TMA (128-byte swizzle, so the 8 rows one
+// ld.shared reads hit 8 different bank groups); four consumer warps take two
+// 16-byte chunks of every row of a stage each and read both fragments from
+// shared memory.
 // ---------------------------------------------------------------------------
 constexpr int kSRows = 32;                       // rows per block (two 16-row slabs)
 constexpr int kSBox = 128;                       // bytes of each row per stage
-constexpr int kSStageBytes = kSRows * kSBox;     // 4 KB
-constexpr int kSStages = 12;
+constexpr int kSStageBytes = kSRows * kSBox;     // 4 KB of packed weights per stage
+constexpr int kSStages = 12;                     // deepest ring
+constexpr int kSRingBytes = 200 * 1024;          // ring budget (one block per SM at the deepest)
 constexpr int kSConsumers = 4;                   // consumer warps; warp 4 is the producer
+
+// Codes one stage covers (128 bytes of a packed row), the token-code boxes of
+// 128 codes that hold them, and a stage's bytes with NT 8-token tiles.
+template <int FMT> __host__ __device__ constexpr int stage_codes() { return 8 * chunk_codes<FMT>(); }
+template <int FMT> __host__ __device__ constexpr int q_boxes() { return stage_codes<FMT>() / 128; }
+template <int FMT, int NT> __host__ __device__ constexpr int s_stage_bytes()
+{
+    return kSStageBytes + q_boxes<FMT>() * 8 * NT * 128;
+}
+template <int FMT, int NT> __host__ __device__ constexpr int s_max_stages()
+{
+    return kSRingBytes / s_stage_bytes<FMT, NT>() < kSStages ? kSRingBytes / s_stage_bytes<FMT, NT>() : kSStages;
+}
 
 __device__ __forceinline__ uint32_t swz128(int row, int chunk)
 {
     return static_cast<uint32_t>(row * kSBox + ((chunk ^ (row & 7)) << 4));
 }
 
+__device__ __forceinline__ uint32_t lds32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+// Four token codes of token row n (of 8 * NT) at code offset o of a stage,
+// from its swizzled q boxes at qbase.
+template <int NT>
+__device__ __forceinline__ uint32_t q_frag(uint32_t qbase, int n, int o)
+{
+    const int within = o & 127;
+    return lds32(qbase + static_cast<uint32_t>((o >> 7) * (8 * NT * 128)) + swz128(n, within >> 4) +
+                 static_cast<uint32_t>(within & 15));
+}
+
+// With ksplit > 1 the blocks run in clusters of ksplit that share 32 output
+// rows: CTA r of a cluster takes stages [r S / ksplit, (r + 1) S / ksplit) of
+// the S stages of a row, the CTAs r > 0 store their int32 partial tile into
+// CTA 0's shared memory, and CTA 0 adds them (exact) and writes y.
+constexpr int kSplitMax = 4;
+
 template <int FMT, int OUT, int NT>
 __global__ void __launch_bounds__((kSConsumers + 1) * 32)
-stream_mma_kernel(const __grid_constant__ CUtensorMap map_p, const int8_t *__restrict__ q, int64_t ldq,
+stream_mma_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ CUtensorMap map_q,
                   const float *__restrict__ s_x, int M, int64_t K, const float *__restrict__ s_w, int64_t N,
-                  void *__restrict__ y, int64_t ldy, int nstages, int prefetch, int32_t *status)
+                  void *__restrict__ y, int64_t ldy, int nstages_all, int ksplit, int depth, int prefetch,
+                  int32_t *status)
 {
+    constexpr int SB = s_stage_bytes<FMT, NT>();
+    constexpr int QB = q_boxes<FMT>();
+    constexpr int QBOX = 8 * NT * 128;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t full[kSStages], empty[kSStages];
+    constexpr int kElems = kSlabs * NT * 4 * 32;
     __shared__ int32_t red[kSConsumers][kSlabs * NT * 4][32];
     __shared__ int abort_word;
     volatile int *abort_flag = &abort_word;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kSRows;
+    const int rank = ksplit > 1 ? static_cast<int>(tc::cluster_rank()) : 0;
+    const int64_t n0 = static_cast<int64_t>(blockIdx.x / ksplit) * kSRows;
+    // this CTA's stages [st0, st0 + nstages) of the row
+    const int st0 = static_cast<int>(static_cast<int64_t>(rank) * nstages_all / ksplit);
+    const int nstages = static_cast<int>(static_cast<int64_t>(rank + 1) * nstages_all / ksplit) - st0;
+    // with ksplit > 1: CTA 0's slots for the partial tiles of CTAs 1.. after the ring
+    int32_t (*part)[kElems] = reinterpret_cast<int32_t (*)[kElems]>(ring + depth * SB);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kSStages; ++i) {
+        for (int i = 0; i < depth; ++i) {
             tc::mbar_init(&full[i], 1);
             tc::mbar_init(&empty[i], kSConsumers);
         }
         abort_word = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_p)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_q)) : "memory");
     }
     __syncthreads();
     // Only the producer may touch global memory before the wait, and only the
@@ -284,24 +334,37 @@ stream_mma_kernel(const __grid_constant__ CUtensorMap map_p, const int8_t *__res
 
     if (producer) {
         if (lane == 0) {
-            int issued = 0;
-            for (int st = 0; st < nstages; ++st) {
-                const int s = st % kSStages;
-                // the first kSStages waits cannot block or time out; the wait for
-                // the previous kernel comes before any that can (a timeout writes
-                // the status word)
-                if (st == kSStages && prefetch != 0) pdl_wait();
-                if (!tc::wait_bar(&empty[s], ((st / kSStages) & 1u) ^ 1u, abort_flag, status)) break;
-                tc::mbar_arrive_expect_tx(&full[s], kSStageBytes);
-                tc::tma_load_2d(ring + s * kSStageBytes, &map_p, &full[s], st * kSBox, static_cast<int>(n0));
+            auto load_q = [&](int st, int s) {
+#pragma unroll
+                for (int b = 0; b < QB; ++b)
+                    tc::tma_load_2d(ring + s * SB + kSStageBytes + b * QBOX, &map_q, &full[s],
+                                    (st0 + st) * stage_codes<FMT>() + 128 * b, 0);
+            };
+            // the first `depth` stages need no slot: their weight boxes go
+            // out first (before the wait for the previous kernel with
+            // prefetch), then their token codes
+            const int first = nstages < depth ? nstages : depth;
+            for (int st = 0; st < first; ++st) {
+                tc::mbar_arrive_expect_tx(&full[st], SB);
+                tc::tma_load_2d(ring + st * SB, &map_p, &full[st], (st0 + st) * kSBox, static_cast<int>(n0));
+            }
+            if (prefetch != 0) pdl_wait();
+            for (int st = 0; st < first; ++st) load_q(st, st);
+            int issued = first;
+            for (int st = first; st < nstages; ++st) {
+                const int s = st % depth;
+                if (!tc::wait_bar(&empty[s], ((st / depth) & 1u) ^ 1u, abort_flag, status)) break;
+                tc::mbar_arrive_expect_tx(&full[s], SB);
+                tc::tma_load_2d(ring + s * SB, &map_p, &full[s], (st0 + st) * kSBox, static_cast<int>(n0));
+                load_q(st, s);
                 issued = st + 1;
             }
             // Every copy issued lands before the block leaves, also when the
-            // consumers gave up on a wait (the last kSStages stages; earlier
+            // consumers gave up on a wait (the last `depth` stages; earlier
             // ones were consumed before their slot was reissued).
-            for (int i = 0; i < kSStages && i < issued; ++i) {
+            for (int i = 0; i < depth && i < issued; ++i) {
                 const int st = issued - 1 - i;
-                tc::drain_bar(&full[st % kSStages], (st / kSStages) & 1u);
+                tc::drain_bar(&full[st % depth], (st / depth) & 1u);
             }
         }
         // every lane of this warp takes part in the epilogue below
@@ -316,35 +379,14 @@ stream_mma_kernel(const __grid_constant__ CUtensorMap map_p, const int8_t *__res
 #pragma unroll
                 for (int i = 0; i < 4; ++i) acc[s][nt][i] = 0;
         const uint32_t ring_base = tc::smem_u32(ring);
-        // activation words of this warp's two chunks of a stage, one stage ahead
-        uint32_t bn[2][chunk_steps<FMT>()][NT][2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-            load_b<FMT, NT>(q, ldq, M, K, static_cast<int64_t>(2 * warp + h) * chunk_codes<FMT>(), g, t, bn[h]);
         for (int st = 0; st < nstages; ++st) {
-            const int s = st % kSStages;
-            uint32_t bc[2][chunk_steps<FMT>()][NT][2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-                for (int j = 0; j < chunk_steps<FMT>(); ++j)
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        bc[h][j][nt][0] = bn[h][j][nt][0];
-                        bc[h][j][nt][1] = bn[h][j][nt][1];
-                    }
-            if (st + 1 < nstages) {
-#pragma unroll
-                for (int h = 0; h < 2; ++h)
-                    load_b<FMT, NT>(q, ldq, M, K,
-                                    ((static_cast<int64_t>(st) + 1) * (kSBox / 16) + 2 * warp + h) * chunk_codes<FMT>(),
-                                    g, t, bn[h]);
-            }
+            const int s = st % depth;
             int ok = 0;
-            if (lane == 0) ok = tc::wait_bar(&full[s], (st / kSStages) & 1u, abort_flag, status) ? 1 : 0;
+            if (lane == 0) ok = tc::wait_bar(&full[s], (st / depth) & 1u, abort_flag, status) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
-            const uint32_t stage = ring_base + static_cast<uint32_t>(s * kSStageBytes);
+            const uint32_t stage = ring_base + static_cast<uint32_t>(s * SB);
+            const uint32_t qbase = stage + kSStageBytes;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int chunk = 2 * warp + h;            // 16-byte chunk of each row in this stage
@@ -354,7 +396,16 @@ stream_mma_kernel(const __grid_constant__ CUtensorMap map_p, const int8_t *__res
                     wa[sl] = tc::lds128(stage + swz128(16 * sl + g, chunk));
                     wb[sl] = tc::lds128(stage + swz128(16 * sl + g + 8, chunk));
                 }
-                chunk_mma<FMT, NT>(wa, wb, bc[h], t, acc);
+                uint32_t b[chunk_steps<FMT>()][NT][2];
+#pragma unroll
+                for (int j = 0; j < chunk_steps<FMT>(); ++j)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const int o = chunk * chunk_codes<FMT>() + 32 * j + 4 * t;
+                        b[j][nt][0] = q_frag<NT>(qbase, 8 * nt + g, o);
+                        b[j][nt][1] = q_frag<NT>(qbase, 8 * nt + g, o + 16);
+                    }
+                chunk_mma<FMT, NT>(wa, wb, b, t, acc);
             }
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&empty[s]);
@@ -368,12 +419,47 @@ stream_mma_kernel(const __grid_constant__ CUtensorMap map_p, const int8_t *__res
     }
     __syncthreads();
 
-    constexpr int kElems = kSlabs * NT * 4 * 32;
-    for (int idx = threadIdx.x; idx < kElems; idx += (kSConsumers + 1) * 32) {
-        const int e = idx >> 5, ln = idx & 31;
-        int32_t v = 0;
+    // this CTA's partial tile, element idx = (fragment element e, lane)
+    constexpr int kThreadsS = (kSConsumers + 1) * 32;
+    constexpr int kPer = (kElems + kThreadsS - 1) / kThreadsS;
+    int32_t vsum[kPer];
 #pragma unroll
-        for (int w = 0; w < kSConsumers; ++w) v += red[w][e][ln];
+    for (int r = 0; r < kPer; ++r) {
+        const int idx = threadIdx.x + r * kThreadsS;
+        int32_t v = 0;
+        if (idx < kElems) {
+#pragma unroll
+            for (int w = 0; w < kSConsumers; ++w) v += red[w][idx >> 5][idx & 31];
+        }
+        vsum[r] = v;
+    }
+    if (ksplit > 1) {
+        if (rank != 0) {
+#pragma unroll
+            for (int r = 0; r < kPer; ++r) {
+                const int idx = threadIdx.x + r * kThreadsS;
+                if (idx < kElems) {
+                    const uint32_t dst = tc::map_to_peer(tc::smem_u32(&part[rank - 1][idx]), 0);
+                    asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(dst), "r"(vsum[r]) : "memory");
+                }
+            }
+        }
+        tc::cluster_sync_all();  // the partial tiles are in CTA 0; no CTA reads another after this
+        if (rank != 0) return;
+#pragma unroll
+        for (int r = 0; r < kPer; ++r) {
+            const int idx = threadIdx.x + r * kThreadsS;
+            if (idx < kElems)
+                for (int p = 0; p + 1 < ksplit; ++p) vsum[r] += part[p][idx];
+        }
+    }
+
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) {
+        const int idx = threadIdx.x + r * kThreadsS;
+        if (idx >= kElems) continue;
+        const int e = idx >> 5, ln = idx & 31;
+        const int32_t v = vsum[r];
         const int sl = e / (NT * 4), nt = (e >> 2) % NT, i = e & 3;
         const int64_t n = n0 + 16 * sl + (ln >> 2) + 8 * (i >> 1);
         const int token = 8 * nt + 2 * (ln & 3) + (i & 1);
@@ -391,28 +477,66 @@ stream_mma_kernel(const __grid_constant__ CUtensorMap map_p, const int8_t *__res
     }
 }
 
+template <int FMT, int OUT, int NT>
+lowbit_status launch_stream_nt(const CUtensorMap &mp, const int8_t *q, int64_t ldq, const float *s_x, int M,
+                               int64_t K, const float *s_w, int64_t N, void *y, int64_t ldy, int nstages, int prefetch,
+                               int32_t *status, cudaStream_t st)
+{
+    constexpr int kMax = s_max_stages<FMT, NT>();
+    constexpr size_t kMaxSmem = 1024 + static_cast<size_t>(kMax) * s_stage_bytes<FMT, NT>() +
+                                (kSplitMax - 1) * kSlabs * NT * 4 * 32 * sizeof(int32_t);
+    static PerDevice configured;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    if (configured.get(dev, [&] {
+            return cudaFuncSetAttribute(stream_mma_kernel<FMT, OUT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(kMaxSmem)) == cudaSuccess ? 1 : 0;
+        }) <= 0)
+        return LOWBIT_ERR_CUDA;
+    CUtensorMap mq;
+    if (!tc::make_map_2d(&mq, q, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(ldq), 128,
+                         8 * NT, CU_TENSOR_MAP_SWIZZLE_128B))
+        return LOWBIT_ERR_CUDA;
+    // K split over a cluster of ksplit CTAs: the largest of 4, 2, 1 whose
+    // grid runs in one wave at no more than 3 blocks per SM with a ring of at
+    // least min(its share of the stages, 4), each CTA keeping 2 stages or
+    // more.  The ring is then as deep as the share and the blocks per SM
+    // allow (short rows keep several blocks per SM).
+    constexpr int64_t kSmSmem = 228 * 1024;   // shared memory per SM
+    constexpr int64_t kStatic = 1024 + sizeof(int32_t) * kSConsumers * kSlabs * NT * 4 * 32 + 512;
+    constexpr int kElemsH = kSlabs * NT * 4 * 32;
+    const int64_t tiles = (N + kSRows - 1) / kSRows;
+    const int64_t sms = device_sm_count();
+    int ksplit = 1, depth = 1;
+    for (int ks : {4, 2, 1}) {
+        const int64_t per_sm = (tiles * ks + sms - 1) / sms;
+        const int share = (nstages + ks - 1) / ks;
+        if (ks > 1 && (per_sm > 3 || nstages < 2 * ks)) continue;
+        const int64_t budget = kSmSmem / (per_sm < 1 ? 1 : per_sm) - kStatic - 1024 -
+                               (ks > 1 ? (ks - 1) * kElemsH * 4 : 0);
+        const int fit = static_cast<int>(budget / s_stage_bytes<FMT, NT>());
+        const int want = share < 4 ? share : 4;
+        if (ks > 1 && fit < want) continue;
+        ksplit = ks;
+        depth = share < kMax ? share : kMax;
+        if (fit < depth) depth = fit < 1 ? 1 : fit;
+        break;
+    }
+    const size_t smem = 1024 + static_cast<size_t>(depth) * s_stage_bytes<FMT, NT>() +
+                        (ksplit > 1 ? static_cast<size_t>(ksplit - 1) * kElemsH * 4 : 0);
+    const dim3 grid(static_cast<unsigned>(tiles * ksplit)), block((kSConsumers + 1) * 32);
+    return launch_pdl(stream_mma_kernel<FMT, OUT, NT>, grid, block, smem, st, ksplit > 1 ? ksplit : 0, mp, mq, s_x, M,
+                      K, s_w, N, y, ldy, nstages, ksplit, depth, prefetch, status);
+}
+
 template <int FMT, int OUT>
 lowbit_status launch_stream(const CUtensorMap &mp, const int8_t *q, int64_t ldq, const float *s_x, int M, int64_t K,
                             const float *s_w, int64_t N, void *y, int64_t ldy, int nstages, int prefetch,
                             int32_t *status, cudaStream_t st)
 {
-    constexpr size_t smem = 1024 + static_cast<size_t>(kSStages) * kSStageBytes;
-    static PerDevice configured;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
-    if (configured.get(dev, [&] {
-            return (cudaFuncSetAttribute(stream_mma_kernel<FMT, OUT, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem)) == cudaSuccess &&
-                    cudaFuncSetAttribute(stream_mma_kernel<FMT, OUT, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem)) == cudaSuccess) ? 1 : 0;
-        }) <= 0)
-        return LOWBIT_ERR_CUDA;
-    const dim3 grid(static_cast<unsigned>((N + kSRows - 1) / kSRows)), block((kSConsumers + 1) * 32);
     if (M <= 8)
-        return launch_pdl(stream_mma_kernel<FMT, OUT, 1>, grid, block, smem, st, 0, mp, q, ldq, s_x, M, K, s_w, N, y,
-                          ldy, nstages, prefetch, status);
-    return launch_pdl(stream_mma_kernel<FMT, OUT, 2>, grid, block, smem, st, 0, mp, q, ldq, s_x, M, K, s_w, N, y, ldy,
-                      nstages, prefetch, status);
+        return launch_stream_nt<FMT, OUT, 1>(mp, q, ldq, s_x, M, K, s_w, N, y, ldy, nstages, prefetch, status, st);
+    return launch_stream_nt<FMT, OUT, 2>(mp, q, ldq, s_x, M, K, s_w, N, y, ldy, nstages, prefetch, status, st);
 }
 
 template <int FMT, int OUT>

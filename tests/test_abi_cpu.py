@@ -68,19 +68,19 @@ def _linear(lib, **kw):
 
 # (M, N, K, format, path, SMs) -> kernel, worked out by hand from the
 # dispatch rules (tiles of 128 tokens x 256 features, K blocks of 128):
-# GEMV up to 4 tokens; warp MMAs up to 16 when a packed row is <= 512 bytes
-# or N >= 3200; the shared-memory GEMM below 512 tokens, split over a cluster
-# of C in {2, 4, 8} CTAs (the largest with tiles * C <= SMs and 2 K blocks per
-# split) when twice its 128 x 256 tiles fit the SMs and K has at least 4
-# blocks; from 512, SM pairs for ternary weights (split-K kept
-# when K >= 2048 and the GEMM splits) and the tensor-memory GEMM for the other
-# formats.
+# GEMV up to 4 tokens; warp MMAs up to 16; the shared-memory GEMM below 512
+# tokens, split over a cluster of C in {2, 4, 8} CTAs (the largest with
+# tiles * C <= SMs and 2 K blocks per split) when twice its 128 x 256 tiles
+# fit the SMs and K has at least 4 blocks; from 512, SM pairs for ternary
+# weights (split-K kept when K >= 2048 and the GEMM splits) and the
+# tensor-memory GEMM for the other formats.
 DISPATCH = [
     ((1, 9728, 2560, bwt.TERNARY2, 0, 148), "gemv_smem_kernel/gemv_kernel"),
     ((4, 9728, 2560, bwt.TERNARY2, 0, 148), "gemv_smem_kernel/gemv_kernel"),
-    ((16, 9728, 2560, bwt.TERNARY2, 0, 148), "skinny_mma_kernel/stream_mma_kernel"),  # N >= 3200
+    ((16, 9728, 2560, bwt.TERNARY2, 0, 148), "skinny_mma_kernel/stream_mma_kernel"),
     ((8, 192, 768, bwt.BINARY1, 0, 148), "skinny_mma_kernel/stream_mma_kernel"),      # 96-byte rows
-    ((16, 2560, 9728, bwt.TERNARY2, 0, 148), "gemm_splitk_kernel"),  # 2432-byte rows, 10 tiles x 8
+    ((16, 2560, 9728, bwt.TERNARY2, 0, 148), "skinny_mma_kernel/stream_mma_kernel"),  # 2432-byte rows
+    ((17, 2560, 9728, bwt.TERNARY2, 0, 148), "gemm_splitk_kernel"),  # 10 tiles x 8
     ((128, 9728, 2560, bwt.TERNARY2, 0, 148), "gemm_splitk_kernel"),  # 38 tiles x 2
     ((256, 768, 192, bwt.TERNARY2, 0, 148), "gemm_kernel"),  # 2 K blocks: no split
     ((300, 9728, 2560, bwt.TERNARY2, 0, 148), "gemm_kernel"),  # 114 tiles: no split

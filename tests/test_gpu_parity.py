@@ -340,6 +340,31 @@ def test_split_plans_int32_bit_exact(fmt, M, N, K):
     assert np.array_equal(y.cpu().numpy().astype(np.int64), acc)
 
 
+# The warp-MMA kernel with rows longer than 512 packed bytes streams weights
+# and token codes through a TMA ring (128 bytes of every row per stage) and
+# splits K over a cluster of 2 or 4 CTAs when the 32-row tiles are few.
+#   (16, 2560, 9728): 80 tiles, 19 stages (ternary) -> 2 CTAs per tile
+#   (9, 1000, 4100): 32 tiles, K ragged in the last stage -> 4 (ternary, 4-bit) or 2 (binary)
+#   (5, 300, 3000): 10 tiles, 6 ternary stages -> 2;  (16, 9728, 2560): 304 tiles, no split
+#   (12, 33, 65536): 2 tiles, 128 ternary stages: the 12-stage ring wraps ten times -> 4
+STREAM_SHAPES = [(16, 2560, 9728), (9, 1000, 4100), (5, 300, 3000), (16, 9728, 2560), (12, 33, 65536)]
+
+
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
+@pytest.mark.parametrize("M,N,K", STREAM_SHAPES, ids=str)
+@pytest.mark.parametrize("path", [0, 5], ids=["auto", "skinny"])
+def test_stream_and_split_int32_bit_exact(fmt, M, N, K, path):
+    y, acc, _, _ = run_case(fmt, M, N, K, path, bwt.I32, 970 + M + N + K)
+    assert np.array_equal(y.cpu().numpy().astype(np.int64), acc)
+
+
+@pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
+def test_stream_split_bf16_bit_exact(fmt):
+    M, N, K = 16, 2560, 9728
+    y, acc, s_w, s_x = run_case(fmt, M, N, K, 5, bwt.BF16, 990, x_bf16=True)
+    assert np.array_equal(bf16_bits(y), oracle.rescale(acc, s_w, s_x, "bf16"))
+
+
 # LOWBIT_LINEAR_WEIGHTS_STABLE: weight reads start before the wait for the
 # preceding kernel (here the act quant that produced q, launched just before
 # on the same stream); the results must not change.  Shapes cover the GEMV
