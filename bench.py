@@ -203,8 +203,10 @@ class Point:
         self.mi, self.m, self.M, self.rows = mi, m, M, rows
         self.kernel = bwt.linear_kernel(rows, m.N, m.K, wl.fmt, 0, sm_count)
         self.fused = bwt.bitlinear_fuses(rows, m.K, wl.hadamard, 0) and fused
+        # decode points whose layers can share a grouped launch
+        self.groupable = bwt.decodes_from_x(rows, m.K, wl.hadamard, 0)
         if self.fused:
-            self.kernel = "gemv_smem_kernel (fused prologue)"
+            self.kernel = "gemv_group_kernel (fused prologue)"
         self.ops = 2 * rows * m.N * m.K
         ysz = 2 if wl.y_dtype == wls.BF16 else 4
         self.packed_bytes = m.N * m.K * FMT_BITS[wl.fmt] // 8
@@ -347,10 +349,10 @@ def run_gpu_arm(args, wl):
     # launches (lowbit_bitlinear_group, up to GROUP_MAX layers per launch)
     # unless --no-group; `calls` lists the points of each API call of a step.
     group_ms = set()
-    if not args.no_group:
+    if not args.no_group and not args.unfused:
         for M in sorted({pt.M for pt in points}):
             at = [pt for pt in points if pt.M == M]
-            if len(at) > 1 and all(pt.fused for pt in at):
+            if len(at) > 1 and all(pt.groupable for pt in at):
                 group_ms.add(M)
     calls = []
     for M in sorted(group_ms):
@@ -367,11 +369,15 @@ def run_gpu_arm(args, wl):
             return bitlinear(pt, *weights(i, pt), x=None if x is None else x[key], stream_=stream_)
         keys = [(pt.mi, pt.M) for _, pt in call]
         ws = [weights(i, pt) for i, pt in call]
+        two = any(pt.m.K > bwt.FUSED_MAX_K for _, pt in call)
         bwt.lowbit_bitlinear_group([(xs if x is None else x)[k] for k in keys], [w[0] for w in ws],
                                    [w[1] for w in ws], wl.fmt, [pt.m.N for _, pt in call], ydt,
                                    [gains[pt.mi] for _, pt in call], norm, 1e-5, ys=[ys[k] for k in keys],
+                                   qs=[qs[k] for k in keys] if two else None,
+                                   s_xs=[sxs[k] for k in keys] if two else None,
                                    stream=stream_, weights_stable=True)
-        return 1
+        n_long = sum(1 for _, pt in call if pt.m.K > bwt.FUSED_MAX_K)
+        return (1 if n_long < len(call) else 0) + 2 * n_long
 
     def prologue(pt):
         key = (pt.mi, pt.M)
@@ -563,7 +569,10 @@ def run_gpu_arm(args, wl):
         "gemv_packed_gbs": round(gemv_bytes / (gemv_ms * 1e-3) / 1e9, 1) if gemv_ms else None,
         "stack_us": {str(M): round(v["median"] * 1e3, 2) for M, v in stacks.items()},
         "decode_groups": [{"M": M, "layers": sum(1 for pt in points if pt.M == M),
-                           "launches": sum(1 for c in calls if c[0][1].M == M),
+                           "launches": sum((1 if any(pt.m.K <= bwt.FUSED_MAX_K for _, pt in c) else 0)
+                                           + 2 * sum(1 for _, pt in c if pt.m.K > bwt.FUSED_MAX_K)
+                                           for c in calls if c[0][1].M == M),
+                           "fused_layers": sum(1 for pt in points if pt.M == M and pt.m.K <= bwt.FUSED_MAX_K),
                            "us": round(stacks[M]["median"] * 1e3, 2),
                            "packed_gbs": round(sum(pt.packed_bytes for pt in points if pt.M == M)
                                                / (stacks[M]["median"] * 1e-3) / 1e9, 1),

@@ -26,6 +26,7 @@ TERNARY2, BINARY1, INT4 = 0, 1, 2
 NORM_NONE, NORM_RMS = 0, 1
 QUANT_DEFAULT, QUANT_BINARY_CENTRED = 0, 1
 FUSED_MAX_BYTES = 98304  # LOWBIT_FUSED_MAX_BYTES
+FUSED_MAX_K = 1024  # LOWBIT_FUSED_MAX_K
 GROUP_MAX = 32  # LOWBIT_GROUP_MAX
 F32, BF16, I32 = 0, 1, 2
 WEIGHTS_STABLE = 1  # LOWBIT_LINEAR_WEIGHTS_STABLE
@@ -277,9 +278,14 @@ def lowbit_act_quant_ex(x, g=None, norm: int = NORM_NONE, eps_norm: float = 1e-5
     return q, s_x
 
 
+def decodes_from_x(M: int, K: int, hadamard: int = 0, path: int = 0) -> bool:
+    """True when the decode GEMV can take these token rows (lowbit_bitlinear_group)."""
+    return M <= 4 and hadamard == 0 and path in (0, 1) and M * ((K + 127) // 128 * 128) <= FUSED_MAX_BYTES
+
+
 def bitlinear_fuses(M: int, K: int, hadamard: int = 0, path: int = 0) -> bool:
     """True when lowbit_bitlinear runs as one fused decode kernel."""
-    return M <= 4 and hadamard == 0 and path in (0, 1) and M * ((K + 127) // 128 * 128) <= FUSED_MAX_BYTES
+    return decodes_from_x(M, K, hadamard, path) and K <= FUSED_MAX_K
 
 
 def lowbit_bitlinear(x, packed, s_w, fmt: int, N: int, out_dtype: int = F32, g=None, norm: int = NORM_NONE,
@@ -315,13 +321,16 @@ class BitlinearItem(ctypes.Structure):
 
 def lowbit_bitlinear_group(xs, packeds, s_ws, fmt: int, Ns, out_dtype: int = F32, gs=None, norm: int = NORM_NONE,
                            eps_norm: float = 1e-5, ys=None, want_codes: bool = False, status=None, stream=None,
-                           weights_stable: bool = False):
+                           weights_stable: bool = False, qs=None, s_xs=None):
     """Several independent decode BitLinear layers (M <= 4 tokens each, the
-    same M, activation dtype, format and output dtype) in one launch.
+    same M, activation dtype, format and output dtype): the layers of at
+    most FUSED_MAX_K features in one persistent fused GEMV launch, each
+    longer layer as lowbit_bitlinear runs it (see lowbit.h).
 
     xs[i] [M, K_i], packeds[i], s_ws[i], Ns[i]; gs: None or a list of gains
-    (entries may be None).  Returns the list of y, or (ys, qs, s_xs) with
-    ``want_codes``."""
+    (entries may be None); qs / s_xs: optional per-layer code and scale
+    buffers (allocated when the call needs them and they are not given).
+    Returns the list of y, or (ys, qs, s_xs) with ``want_codes``."""
     import torch
     n = len(xs)
     if not (len(packeds) == len(s_ws) == len(Ns) == n) or (gs is not None and len(gs) != n):
@@ -330,9 +339,11 @@ def lowbit_bitlinear_group(xs, packeds, s_ws, fmt: int, Ns, out_dtype: int = F32
     dt = {F32: torch.float32, BF16: torch.bfloat16, I32: torch.int32}[out_dtype]
     if ys is None:
         ys = [torch.empty((M, N), dtype=dt, device=x.device) for x, N in zip(xs, Ns)]
-    qs = [None] * n
-    s_xs = [None] * n
-    if want_codes:
+    # layers longer than FUSED_MAX_K run the prologue kernel, which writes
+    # their codes: workspace then (allocated here unless given)
+    if qs is None or s_xs is None:
+        qs, s_xs = [None] * n, [None] * n
+    if (want_codes or any(x.shape[1] > FUSED_MAX_K for x in xs)) and any(q is None for q in qs):
         qs = [torch.empty((M, (x.shape[1] + 15) // 16 * 16), dtype=torch.int8, device=x.device) for x in xs]
         s_xs = [torch.empty(M, dtype=torch.float32, device=x.device) for x in xs]
     items = (BitlinearItem * n)()

@@ -323,9 +323,18 @@ lowbit_status check_prologue_args(const void *x, lowbit_dtype xdt, int64_t M, in
     return LOWBIT_OK;
 }
 
-bool fused_decode(int64_t M, int64_t K, int hadamard, int path)
+// Decode shapes the GEMV can take from activations: M <= 4 rows whose codes
+// fit its shared memory.
+bool decode_from_x(int64_t M, int64_t K, int hadamard, int path)
 {
     return M <= 4 && hadamard == 0 && (path == 0 || path == 1) && M * ((K + 127) / 128 * 128) <= LOWBIT_FUSED_MAX_BYTES;
+}
+
+// ... of which the fused kernel (codes computed in every block) takes the
+// short rows.
+bool fused_decode(int64_t M, int64_t K, int hadamard, int path)
+{
+    return decode_from_x(M, K, hadamard, path) && K <= LOWBIT_FUSED_MAX_K;
 }
 
 }  // namespace
@@ -410,7 +419,7 @@ lowbit_status lowbit_bitlinear_group(const lowbit_bitlinear_item *items, int n_i
         if (it.N <= 0 || it.ldy < it.N) return LOWBIT_ERR_INVALID_ARG;
         const lowbit_status shape = check_linear_shape(M, it.N, it.K, f, 0);
         if (shape != LOWBIT_OK) return shape;
-        if (!fused_decode(M, it.K, 0, 0)) return LOWBIT_ERR_UNSUPPORTED;
+        if (!decode_from_x(M, it.K, 0, 0)) return LOWBIT_ERR_UNSUPPORTED;
         if (it.ldp < static_cast<int64_t>(lowbit_packed_row_bytes(f, it.K))) return LOWBIT_ERR_INVALID_ARG;
         if (!aligned(it.packed, 16) || it.ldp % 16 != 0 || !aligned(it.s_w, 4) ||
             !aligned(it.y, static_cast<uintptr_t>(esz)))
@@ -421,12 +430,32 @@ lowbit_status lowbit_bitlinear_group(const lowbit_bitlinear_item *items, int n_i
         }
         if (it.s_x != nullptr && !aligned(it.s_x, 4)) return LOWBIT_ERR_ALIGNMENT;
     }
+    // layers longer than LOWBIT_FUSED_MAX_K run as lowbit_bitlinear does for
+    // them (prologue kernel, then the GEMV): their q and s_x are required
+    lowbit_bitlinear_item short_items[LOWBIT_GROUP_MAX];
+    int n_short = 0;
+    for (int i = 0; i < n_items; ++i) {
+        if (items[i].K <= LOWBIT_FUSED_MAX_K) short_items[n_short++] = items[i];
+        else if (items[i].q == nullptr || items[i].s_x == nullptr) return LOWBIT_ERR_INVALID_ARG;
+    }
     const lowbit_status d = check_device();
     if (d != LOWBIT_OK) return d;
     const TraceRange trace("lowbit_bitlinear_group");
     const int prefetch = (flags & LOWBIT_LINEAR_WEIGHTS_STABLE) != 0 ? 1 : 0;
-    return gemv_group_launch(items, n_items, M, xdt, norm, eps_norm, f, ydt, prefetch, status_dev,
-                             static_cast<cudaStream_t>(stream));
+    if (n_short > 0) {
+        const lowbit_status s = gemv_group_launch(short_items, n_short, M, xdt, norm, eps_norm, f, ydt, prefetch,
+                                                  status_dev, static_cast<cudaStream_t>(stream));
+        if (s != LOWBIT_OK) return s;
+    }
+    for (int i = 0; i < n_items; ++i) {
+        const lowbit_bitlinear_item &it = items[i];
+        if (it.K <= LOWBIT_FUSED_MAX_K) continue;
+        const lowbit_status s = lowbit_bitlinear(it.x, xdt, M, it.K, it.ldx, it.g, norm, eps_norm, 0, it.packed, it.ldp,
+                                                 it.s_w, f, it.N, it.y, ydt, it.ldy, it.q, it.ldq, it.s_x, 0, flags,
+                                                 status_dev, stream);
+        if (s != LOWBIT_OK) return s;
+    }
+    return LOWBIT_OK;
 }
 
 lowbit_status lowbit_act_row_stats(const void *x, lowbit_dtype xdt, int64_t M, int64_t K, int64_t ldx,

@@ -371,15 +371,12 @@ struct GroupItem {
     int32_t unit0, units;  // this layer's units: [unit0, unit0 + units)
 };
 constexpr int kGroupMax = 32;
-// Largest staging of one layer's token rows in shared memory.
-constexpr int64_t kXStageMax = 40 * 1024;
 struct GroupArgs {
     GroupItem item[kGroupMax];
     int64_t cost_total;
     int32_t *status;
     float eps_norm;
     int n_items, units, M, xbf16, norm, prefetch;
-    int xstage;  // bytes of shared memory after the codes for one layer's token rows (0: read x from global)
 };
 static_assert(sizeof(GroupArgs) <= 4000, "the group must fit the 4 KB kernel parameter space");
 
@@ -472,88 +469,146 @@ __device__ __forceinline__ void quad_gain(const float *g, int64_t k0, int64_t K,
         if (k0 + e < K) f[e] = __fmul_rn(f[e], ld_act_f32(g + k0 + e));
 }
 
-// Features k0..k0+3 of a token row staged in shared memory at xs (the
-// row's first `staged` bytes; the rest is read from global memory).
-__device__ __forceinline__ void quad_x_staged(int xbf16, const char *xr, uint32_t xs, int64_t staged, int64_t k0,
-                                              int64_t K, float (&f)[4])
+// Pass 1 of one 16-feature piece p of token t of layer I: max |x * g| bits
+// into amax and, with norm, the fp64 sum of x^2 (before the gain) into ss,
+// value by value in feature order.
+__device__ __forceinline__ void piece_partial(const GroupItem &I, int xbf16, bool norm, int t, int64_t p,
+                                              uint32_t &amax, double &ss)
 {
-    if (xbf16 && 2 * (k0 + 4) <= staged) {
-        uint32_t lo, hi;
-        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo), "=r"(hi) : "r"(xs + static_cast<uint32_t>(2 * k0)));
-        f[0] = __uint_as_float(lo << 16);
-        f[1] = __uint_as_float(lo & 0xffff0000u);
-        f[2] = __uint_as_float(hi << 16);
-        f[3] = __uint_as_float(hi & 0xffff0000u);
-        return;
+    const char *xr = static_cast<const char *>(I.x) + t * I.ldx * (xbf16 ? 2 : 4);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        float f[4];
+        quad_x(xbf16, xr, 16 * p + 4 * e, I.K, f);
+        if (norm) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) ss = __fma_rn(static_cast<double>(f[v]), static_cast<double>(f[v]), ss);
+        }
+        if (I.g != nullptr) quad_gain(I.g, 16 * p + 4 * e, I.K, f);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) amax = max(amax, __float_as_uint(f[v]) & 0x7fffffffu);
     }
-    if (!xbf16 && 4 * (k0 + 4) <= staged) {
-        uint4 w;
-        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
-                     : "r"(xs + static_cast<uint32_t>(4 * k0)));
-        f[0] = __uint_as_float(w.x);
-        f[1] = __uint_as_float(w.y);
-        f[2] = __uint_as_float(w.z);
-        f[3] = __uint_as_float(w.w);
-        return;
-    }
-    quad_x(xbf16, xr, k0, K, f);
 }
 
-// Copies the whole 16-byte pieces of the M token rows of layer I into
-// shared memory at xs (row t at t * row_bytes rounded up to 16) with
-// cp.async (all copies in flight at once, L2 only), and waits for them.
-// Called by every thread of the block; the buffer is reused layer by layer.
-// Returns the bytes of each row that are staged.
-__device__ __forceinline__ int64_t stage_rows(const GroupItem &I, int M, int64_t xsz, uint32_t xs)
+// s_x of a row from max |x * g| bits m and the sum of squares q2.
+__device__ __forceinline__ float row_scale_of(uint32_t m, double q2, bool norm, int64_t K, float eps_norm)
 {
-    const int64_t row = static_cast<int64_t>(I.K) * xsz;
-    const int64_t n16 = row / 16;
-    const int64_t pitch = (row + 15) / 16 * 16;
-    __syncthreads();  // every thread is done with the previous layer's rows
-    for (int64_t c = threadIdx.x; c < M * n16; c += blockDim.x) {
-        const int64_t t = c / n16, j = c % n16;
-        const char *src = static_cast<const char *>(I.x) + t * I.ldx * xsz + 16 * j;
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(xs + static_cast<uint32_t>(t * pitch + 16 * j)),
-                     "l"(src)
-                     : "memory");
+    if (m == 0) return 0.0f;
+    const float gm = __uint_as_float(m);
+    if (!norm) return __fdiv_rn(gm, 127.0f);
+    const double sc = __ddiv_rn(static_cast<double>(gm),
+                                __dsqrt_rn(__dadd_rn(__ddiv_rn(q2, static_cast<double>(K)), static_cast<double>(eps_norm))));
+    return __double2float_rn(__ddiv_rn(sc, 127.0));
+}
+
+// The 16 codes of piece p of token t of layer I for the row maximum bits m
+// (zero past K and for an all-zero row).
+__device__ __forceinline__ uint4 piece_codes(const GroupItem &I, int xbf16, int t, int64_t p, uint32_t m)
+{
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (16 * p < I.K && m != 0) {
+        const char *xr = static_cast<const char *>(I.x) + t * I.ldx * (xbf16 ? 2 : 4);
+        const float gm = __uint_as_float(m);
+        const float c = __fmul_rn(127.0f, __frcp_rn(gm));
+        const bool slow = !(gm >= 0x1p-121f && gm < 0x1p126f);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float f[4];
+            quad_x(xbf16, xr, 16 * p + 4 * e, I.K, f);
+            if (I.g != nullptr) quad_gain(I.g, 16 * p + 4 * e, I.K, f);
+            bool near = slow;
+            w[e] = qrule::quant4(f[0], f[1], f[2], f[3], c, near);
+            if (near) w[e] = qrule::quant4_exact(f[0], f[1], f[2], f[3], gm);
+        }
+        const int64_t valid = static_cast<int64_t>(I.K) - 16 * p;
+        if (valid < 16) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int lo = 4 * e;
+                uint32_t mk;
+                if (valid >= lo + 4) mk = 0xffffffffu;
+                else if (valid <= lo) mk = 0u;
+                else mk = (1u << (8 * (valid - lo))) - 1u;
+                w[e] &= mk;
+            }
+        }
     }
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Stores piece p's codes into row t of q_out (only the bytes below K).
+__device__ __forceinline__ void store_codes(const GroupItem &I, int t, int64_t p, const uint4 &out)
+{
+    int8_t *dst = I.q_out + t * I.ldq_out + 16 * p;
+    if (16 * p + 16 <= I.K) {
+        *reinterpret_cast<uint4 *>(dst) = out;
+    } else {
+        const uint8_t *bytes = reinterpret_cast<const uint8_t *>(&out);
+        for (int64_t e = 0; 16 * p + e < I.K; ++e) dst[e] = static_cast<int8_t>(bytes[e]);
+    }
+}
+
+// The row statistics of every thread's pieces tid, tid + 256, ... reduced in
+// a fixed order -- a shuffle tree, then the 8 warps in order -- so every
+// block that computes a row gets the same maximum and scale.  Partials are
+// exchanged through red_max / red_ss ([kWarps][MT]); the caller reads them
+// after the block barrier this function ends with.
+template <int MT>
+__device__ __forceinline__ void reduce_rows(uint32_t (&amax)[MT], double (&ss)[MT], uint32_t (*red_max)[MT],
+                                            double (*red_ss)[MT])
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            amax[t] = max(amax[t], __shfl_xor_sync(0xffffffffu, amax[t], o));
+            ss[t] = __dadd_rn(ss[t], __shfl_xor_sync(0xffffffffu, ss[t], o));
+        }
+        if (lane == 0) {
+            red_max[warp][t] = amax[t];
+            red_ss[warp][t] = ss[t];
+        }
+    }
     __syncthreads();
-    return 16 * n16;
 }
 
-// The codes and scales of layers i0..i1 of the group in this block: codes
-// into qs (layer i at qoff[i - i0], [M][QP][nchunks] piece-major as the GEMV
-// reads them, zero past K) and scales into sx_s[(i - i0) * MT + t].  Per
-// layer: pass 1 reduces max |x*g| and, with the norm, the fp64 sum of x^2
-// over the row in a fixed order (thread tid takes 16-feature pieces tid,
-// tid + 256, ... in turn, then a shuffle tree and the 8 warps in order), so
-// every block -- and every grid -- gets the same row maximum and scale; pass
-// 2 reads the row again (L1) and writes the codes.  The block whose range
-// holds the layer's first unit (`writer`) also stores the codes and scales
-// to q_out / s_x_out and reports non-finite rows.  Called by every thread of
-// the block.
+template <int MT>
+__device__ __forceinline__ void combine_row(const uint32_t (*red_max)[MT], const double (*red_ss)[MT], int t,
+                                            uint32_t &m, double &q2)
+{
+    m = red_max[0][t];
+    q2 = red_ss[0][t];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) {
+        m = max(m, red_max[w][t]);
+        q2 = __dadd_rn(q2, red_ss[w][t]);
+    }
+}
+
+// The codes and scales of layers i0..i1 of the group, computed in this block
+// from x: codes into qs (layer i at qoff[i - i0], [M][QP][nchunks]
+// piece-major as the GEMV reads them, zero past K) and scales into
+// sx_s[(i - i0) * MT + t].  Pass 1 reduces max |x*g| and, with the norm, the
+// fp64 sum of x^2 over each row (reduce_rows: a fixed order, so every block
+// gets the same scale), pass 2 reads the row again (L1) and writes the
+// codes.  The block whose range holds the layer's first unit (`writer`) also
+// stores them to q_out / s_x_out and reports non-finite rows.  Called by
+// every thread of the block.
 template <int QP, int MT>
 __device__ void stage_block(const GroupArgs &a, int i0, int i1, int u_begin, int u_end, const int32_t *qoff,
-                            uint4 *qs, float *sx_s, uint32_t xs)
+                            uint4 *qs, float *sx_s)
 {
     __shared__ uint32_t red_max[kWarps][MT];
     __shared__ double red_ss[kWarps][MT];
     __shared__ uint32_t gm_s[MT];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool norm = a.norm != 0;
-    const int64_t xsz = a.xbf16 ? 2 : 4;
     for (int i = i0; i <= i1; ++i) {
         const GroupItem &I = a.item[i];
-        const bool writer = u_begin <= I.unit0 && I.unit0 < u_end;
         const int64_t qp = static_cast<int64_t>(I.nchunks) * QP;  // code pieces per token row
         const int64_t np = (static_cast<int64_t>(I.K) + 15) / 16;  // pieces holding features
-        // with xstage the rows are first copied to shared memory (one round trip)
-        const int64_t staged = a.xstage > 0 ? stage_rows(I, a.M, xsz, xs) : 0;
-        const int64_t pitch = (static_cast<int64_t>(I.K) * xsz + 15) / 16 * 16;
-
-        // pass 1
+        uint4 *qi = qs + qoff[i - i0];
+        const bool writer = u_begin <= I.unit0 && I.unit0 < u_end;
         uint32_t amax[MT];
         double ss[MT];
 #pragma unroll
@@ -563,115 +618,32 @@ __device__ void stage_block(const GroupArgs &a, int i0, int i1, int u_begin, int
         }
         for (int64_t p = threadIdx.x; p < np; p += blockDim.x) {
 #pragma unroll
-            for (int t = 0; t < MT; ++t) {
-                if (t >= a.M) continue;
-                const char *xr = static_cast<const char *>(I.x) + t * I.ldx * xsz;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float f[4];
-                    quad_x_staged(a.xbf16, xr, xs + static_cast<uint32_t>(t * pitch), staged, 16 * p + 4 * e, I.K, f);
-                    if (norm) {
-#pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            ss[t] = __fma_rn(static_cast<double>(f[v]), static_cast<double>(f[v]), ss[t]);
-                    }
-                    if (I.g != nullptr) quad_gain(I.g, 16 * p + 4 * e, I.K, f);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) amax[t] = max(amax[t], __float_as_uint(f[v]) & 0x7fffffffu);
-                }
-            }
+            for (int t = 0; t < MT; ++t)
+                if (t < a.M) piece_partial(I, a.xbf16, norm, t, p, amax[t], ss[t]);
         }
-#pragma unroll
-        for (int t = 0; t < MT; ++t) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                amax[t] = max(amax[t], __shfl_xor_sync(0xffffffffu, amax[t], o));
-                ss[t] = __dadd_rn(ss[t], __shfl_xor_sync(0xffffffffu, ss[t], o));
-            }
-            if (lane == 0) {
-                red_max[warp][t] = amax[t];
-                red_ss[warp][t] = ss[t];
-            }
-        }
-        __syncthreads();
+        reduce_rows<MT>(amax, ss, red_max, red_ss);
         if (threadIdx.x < a.M) {
             const int t = threadIdx.x;
-            uint32_t m = red_max[0][t];
-            double q2 = red_ss[0][t];
-#pragma unroll
-            for (int w = 1; w < kWarps; ++w) {
-                m = max(m, red_max[w][t]);
-                q2 = __dadd_rn(q2, red_ss[w][t]);
-            }
-            const float gm = __uint_as_float(m);
-            float sx = 0.0f;
-            if (m != 0) {
-                if (norm) {
-                    const double sc = __ddiv_rn(static_cast<double>(gm),
-                                                __dsqrt_rn(__dadd_rn(__ddiv_rn(q2, static_cast<double>(I.K)),
-                                                                     static_cast<double>(a.eps_norm))));
-                    sx = __double2float_rn(__ddiv_rn(sc, 127.0));
-                } else {
-                    sx = __fdiv_rn(gm, 127.0f);
-                }
-            }
+            uint32_t m;
+            double q2;
+            combine_row<MT>(red_max, red_ss, t, m, q2);
+            const float sx = row_scale_of(m, q2, norm, I.K, a.eps_norm);
             gm_s[t] = m;
             sx_s[(i - i0) * MT + t] = sx;
             if (writer) {
-                if (!finite_bits(m) || !finite_bits(__float_as_uint(__fmul_rn(gm, 127.0f))))
+                if (!finite_bits(m) || !finite_bits(__float_as_uint(__fmul_rn(__uint_as_float(m), 127.0f))))
                     report(a.status, LOWBIT_ERR_NONFINITE);
                 if (I.s_x_out != nullptr) I.s_x_out[t] = sx;
             }
         }
         __syncthreads();
-
-        // pass 2: codes of every piece of the staging (zero past K)
-        uint4 *qi = qs + qoff[i - i0];
         for (int64_t p = threadIdx.x; p < qp; p += blockDim.x) {
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
                 if (t >= a.M) continue;
-                const uint32_t m = gm_s[t];
-                uint32_t w[4] = {0u, 0u, 0u, 0u};
-                if (p < np && m != 0) {
-                    const char *xr = static_cast<const char *>(I.x) + t * I.ldx * xsz;
-                    const float gm = __uint_as_float(m);
-                    const float c = __fmul_rn(127.0f, __frcp_rn(gm));
-                    const bool slow = !(gm >= 0x1p-121f && gm < 0x1p126f);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float f[4];
-                        quad_x_staged(a.xbf16, xr, xs + static_cast<uint32_t>(t * pitch), staged, 16 * p + 4 * e,
-                                      I.K, f);
-                        if (I.g != nullptr) quad_gain(I.g, 16 * p + 4 * e, I.K, f);
-                        bool near = slow;
-                        w[e] = qrule::quant4(f[0], f[1], f[2], f[3], c, near);
-                        if (near) w[e] = qrule::quant4_exact(f[0], f[1], f[2], f[3], gm);
-                    }
-                    const int64_t valid = static_cast<int64_t>(I.K) - 16 * p;
-                    if (valid < 16) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int lo = 4 * e;
-                            uint32_t mk;
-                            if (valid >= lo + 4) mk = 0xffffffffu;
-                            else if (valid <= lo) mk = 0u;
-                            else mk = (1u << (8 * (valid - lo))) - 1u;
-                            w[e] &= mk;
-                        }
-                    }
-                }
-                const uint4 out = make_uint4(w[0], w[1], w[2], w[3]);
+                const uint4 out = piece_codes(I, a.xbf16, t, p, p < np ? gm_s[t] : 0u);
                 qi[t * qp + (p % QP) * I.nchunks + p / QP] = out;
-                if (writer && I.q_out != nullptr && p < np) {
-                    int8_t *dst = I.q_out + t * I.ldq_out + 16 * p;
-                    if (16 * p + 16 <= I.K) {
-                        *reinterpret_cast<uint4 *>(dst) = out;
-                    } else {
-                        const uint8_t *bytes = reinterpret_cast<const uint8_t *>(&out);
-                        for (int64_t e = 0; 16 * p + e < I.K; ++e) dst[e] = static_cast<int8_t>(bytes[e]);
-                    }
-                }
+                if (writer && I.q_out != nullptr && p < np) store_codes(I, t, p, out);
             }
         }
     }
@@ -717,9 +689,6 @@ __global__ void __launch_bounds__(kWarps * 32, 3) gemv_group_kernel(const __grid
             off += a.M * a.item[i].nchunks * QP;
         }
     }
-    // the x staging follows the codes of every layer of the launch
-    int64_t xs_off = 0;
-    for (int i = 0; i < a.n_items; ++i) xs_off += static_cast<int64_t>(a.M) * a.item[i].nchunks * QP * 16;
     __syncthreads();
 
     int it = i0;
@@ -736,9 +705,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3) gemv_group_kernel(const __grid
                     pdl_wait();
                     waited = true;
                 }
-                stage_block<QP, MT>(a, i0, i1, u_begin, u_end, qoff_s, qs, sx_s,
-                                    static_cast<uint32_t>(__cvta_generic_to_shared(qs)) +
-                                        static_cast<uint32_t>(xs_off));
+                stage_block<QP, MT>(a, i0, i1, u_begin, u_end, qoff_s, qs, sx_s);
                 staged = true;
             }
 #pragma unroll
@@ -791,7 +758,7 @@ lowbit_status launch_group(GroupArgs &a, lowbit_dtype ydt, size_t smem, cudaStre
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
     if (configured.get(dev, [&] {
-            const int lim = static_cast<int>(kGemvSmemMax + kXStageMax);
+            const int lim = static_cast<int>(kGemvSmemMax);
             return (cudaFuncSetAttribute(gemv_group_kernel<FMT, MT, U, R, LOWBIT_F32>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, lim) == cudaSuccess &&
                     cudaFuncSetAttribute(gemv_group_kernel<FMT, MT, U, R, LOWBIT_BF16>,
@@ -934,19 +901,7 @@ lowbit_status gemv_group_launch_fmt(const GroupArgs &all, lowbit_dtype ydt, cuda
             ++n;
         }
         a.n_items = n;
-        // stage x in shared memory when every layer's rows are 16-byte
-        // aligned and the largest layer's M rows fit kXStageMax
-        const int64_t xsz = all.xbf16 ? 2 : 4;
-        int64_t xrows = 0;
-        bool aligned = true;
-        for (int i = 0; i < n; ++i) {
-            const GroupItem &I = a.item[i];
-            aligned = aligned && (reinterpret_cast<uintptr_t>(I.x) & 15u) == 0 && (I.ldx * xsz) % 16 == 0;
-            const int64_t r = static_cast<int64_t>(all.M) * ((I.K * xsz + 15) / 16 * 16);
-            xrows = r > xrows ? r : xrows;
-        }
-        a.xstage = (aligned && xrows <= kXStageMax) ? static_cast<int>(xrows) : 0;
-        const size_t smem = static_cast<size_t>(bytes + a.xstage);
+        const size_t smem = static_cast<size_t>(bytes);
         const lowbit_status s = all.M == 1 ? launch_group_tokens<FMT, 1>(a, max_nchunks, rows, ydt, smem, st)
                                            : launch_group_tokens<FMT, 4>(a, max_nchunks, rows, ydt, smem, st);
         if (s != LOWBIT_OK) return s;

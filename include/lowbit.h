@@ -308,23 +308,27 @@ lowbit_status lowbit_linear_ex(const int8_t *q, int64_t ldq, const float *s_x,
                                int path, unsigned flags,
                                int32_t *status_dev, void *stream);
 
-/* lowbit_bitlinear runs one fused decode kernel when M * K_r <=
- * LOWBIT_FUSED_MAX_BYTES, K_r = K rounded up to a multiple of 128 (the codes
- * of the M tokens are held in shared memory). */
+/* lowbit_bitlinear runs one fused decode kernel when K <= LOWBIT_FUSED_MAX_K
+ * and M * K_r <= LOWBIT_FUSED_MAX_BYTES, K_r = K rounded up to a multiple of
+ * 128 (the codes of the M tokens are held in shared memory).  Every block
+ * of the fused kernel computes the codes it needs; for longer rows that
+ * repeated prologue costs more than a separate prologue kernel, measured on
+ * B200 (K = 9728, M = 1: 12.4 us fused against 7.1 us for the prologue
+ * kernel followed by the GEMV). */
+#define LOWBIT_FUSED_MAX_K 1024
 #define LOWBIT_FUSED_MAX_BYTES 98304
 
 /* lowbit_bitlinear -- the whole BitLinear forward of M8.8 0x02E on activations
  * x: the prologue of lowbit_act_quant_ex (gain, RMSNorm, Hadamard rotation,
  * per-token codes) followed by lowbit_linear_ex with the given path and
  * flags.  y is identical to calling those two functions in turn.
- *   - Decode: with M <= 4, hadamard == 0, path 0 or 1 and the bound of
- *     LOWBIT_FUSED_MAX_BYTES, one fused kernel runs in clusters of up to 8
- *     blocks: while their first weight loads are in flight, the blocks of a
- *     cluster each quantise a share of the M token rows and exchange the
- *     row statistics and the codes through distributed shared memory, then
- *     every block streams its packed weight rows (one launch instead of two,
- *     and the codes never go through global memory).  q and s_x may then be
- *     NULL; when given, they receive the codes and scales.
+ *   - Decode: with M <= 4, hadamard == 0, path 0 or 1, K <=
+ *     LOWBIT_FUSED_MAX_K and the bound of LOWBIT_FUSED_MAX_BYTES, one fused
+ *     kernel runs: while its first weight loads are in flight, every block
+ *     computes the codes and scales of the M token rows itself into shared
+ *     memory, then streams its packed weight rows (one launch instead of
+ *     two, and the codes never go through global memory).  q and s_x may
+ *     then be NULL; when given, they receive the codes and scales.
  *   - Otherwise the prologue kernel writes q [M, ldq] and s_x [M] (both
  *     required: device workspace owned by the caller, ldq a multiple of 16,
  *     ldq >= K, q 16-byte aligned), and the linear kernel reads them.
@@ -368,18 +372,22 @@ typedef struct lowbit_bitlinear_item {
 #define LOWBIT_GROUP_MAX 32
 
 /* lowbit_bitlinear_group -- several independent decode BitLinear layers in
- * one launch (M8.8 0x09B: decode streams whole weight matrices for a few
- * tokens, so the cost of a layer is its packed bytes plus a fixed launch and
- * dependency latency; several layers that read the same or different token
- * rows -- the q, k, v projections, or gate and up, of one block -- share that
- * fixed cost when they run as one kernel).  Each item is computed exactly as
- * lowbit_bitlinear with hadamard = 0 on that item's arguments: the result is
- * bit-identical to n_items separate calls.  The kernel is persistent: the
- * layers' rows are cut into units of up to 8 blocks (a thread-block cluster)
- * and each resident cluster takes a contiguous range of units of about equal
- * packed bytes; when a cluster enters a layer, its blocks compute that
- * layer's codes and scales together while the first weight loads of the
- * layer are in flight.
+ * one persistent GEMV launch (M8.8 0x09B: decode streams whole weight
+ * matrices for a few tokens, so the cost of a layer is its packed bytes plus
+ * a fixed launch and dependency latency; several layers that read the same
+ * or different token rows -- the q, k, v projections, or gate and up, of one
+ * block -- share that fixed cost when they run as one kernel).  Each item is
+ * computed exactly as lowbit_bitlinear with hadamard = 0 on that item's
+ * arguments: codes, scales, int32 sums and outputs are identical to separate
+ * calls (the RMSNorm's sum of squares is reduced in the same order).  The
+ * layers with K <= LOWBIT_FUSED_MAX_K run in one persistent fused GEMV
+ * launch: their rows are cut into units of one block, each resident block
+ * takes a contiguous range of units of about equal packed bytes, computes
+ * the codes of the layers it touches and streams its units (consecutive
+ * layers share a launch while their codes fit 96 KB of shared memory, M *
+ * sum of K_r).  Each longer layer runs as lowbit_bitlinear runs it, the
+ * prologue kernel then the GEMV (measured faster on B200 than any grouped
+ * form for such layers); its q and s_x are then required.
  * items: HOST array of n_items descriptors (read during the call only),
  * 1 <= n_items <= LOWBIT_GROUP_MAX.  M: tokens, 1..4, the same for all items.
  * xdt, norm, eps_norm, f, ydt, flags: shared by all items, with the meanings

@@ -189,6 +189,10 @@ def test_bitlinear_group_rejects_bad_arguments(lib):
     assert _group(lib, y=FAKE + 1) == bwt.ERR_ALIGNMENT
     assert _group(lib, q=FAKE, ldq=2560 + 8) == bwt.ERR_ALIGNMENT
     assert _group(lib, q=FAKE, ldq=16) == bwt.ERR_INVALID_ARG       # ldq < K
+    # a layer longer than LOWBIT_FUSED_MAX_K makes the group run its prologue
+    # kernel first, which needs every layer's q and s_x
+    assert _group(lib) == bwt.ERR_INVALID_ARG
+    assert _group(lib, q=FAKE, ldq=2560, s_x=FAKE) == bwt.ERR_INVALID_ARG   # the first layer has none
     # the codes of a layer must fit the kernel's staging: M * K_r <= 98304
     k = bwt.FUSED_MAX_BYTES + 128
     assert _group(lib, K=k, ldx=k, ldp=bwt.packed_ld(bwt.TERNARY2, k)) == bwt.ERR_UNSUPPORTED

@@ -120,6 +120,24 @@ def test_act_quant_bit_exact_deep(K, bf16):
     assert np.array_equal(s_x.cpu().numpy().view(np.uint32), s_o.view(np.uint32))
 
 
+# Many rows of the decode and prefill shapes: ragged M, the largest
+# workload M at K = 2560, the smallest rows (one 16-byte vector), and zero
+# first and last rows.
+@pytest.mark.parametrize("bf16", [False, True], ids=["f32", "bf16"])
+@pytest.mark.parametrize("M,K", [(512, 2560), (1031, 2048), (8192, 2560), (600, 8), (2000, 1000), (513, 1536)])
+@pytest.mark.parametrize("eps", [0.0, 1e-5])
+def test_act_quant_many_rows_bit_exact(M, K, bf16, eps):
+    x = wls.normal_activations(300 + M + K, M, K, 0.01, 8.0)
+    x[0, :] = 0.0
+    x[M - 1, :] = 0.0
+    if bf16:
+        x = wls.to_bf16_bits(x)
+    q, s_x = gpu_act(x, bf16, eps)
+    q_o, s_o = oracle.act_quant(x, eps, bf16_bits=bf16)
+    assert np.array_equal(q.cpu().numpy()[:, :K], q_o)
+    assert np.array_equal(s_x.cpu().numpy().view(np.uint32), s_o.view(np.uint32))
+
+
 def edge_rows(seed, M, K, eps):
     """Rows that stress the codes' rounding: by row index mod 4, ordinary
     N(0,1); tiny (max |x| from 1e-44 to 1e-36, subnormals included, where the
@@ -147,13 +165,16 @@ def edge_rows(seed, M, K, eps):
 
 
 # eps = 0; 5e37 (d just below 2^126: the fast path); 1e38 (d above it: the
-# divide for every value).  Small M takes the wide build, large M the deep one.
+# divide for every value).  Small M takes the wide build, large M the deep one
+# (K = 9728) and, at M = 1024, the wide build with many blocks (K = 2560, 2048).
 @pytest.mark.parametrize("eps", [0.0, 5e37, 1e38])
 @pytest.mark.parametrize("K,bf16,deep", [(2560, True, False), (2560, False, False), (9728, True, True),
-                                         (9728, False, True)])
+                                         (9728, False, True), (2560, True, "many"), (2048, False, "many")])
 def test_act_quant_rounding_edges(K, bf16, deep, eps):
     M = 64
-    if deep:
+    if deep == "many":
+        M = 1024
+    elif deep:
         nvec = K // (8 if bf16 else 4)
         tpr_deep = next(g for g in (8, 32, 64, 128, 256, 512, 1024) if nvec <= 5 * g)
         sms = torch.cuda.get_device_properties(0).multi_processor_count
@@ -167,7 +188,7 @@ def test_act_quant_rounding_edges(K, bf16, deep, eps):
     assert np.array_equal(s_x.cpu().numpy().view(np.uint32), s_o.view(np.uint32))
 
 
-@pytest.mark.parametrize("M", [4, 300], ids=["regs", "ring"])
+@pytest.mark.parametrize("M", [4, 300, 700], ids=["regs", "ring", "many"])
 def test_act_quant_flags_nonfinite(M):
     x = np.ones((M, 64), np.float32)
     x[2, 5] = np.nan

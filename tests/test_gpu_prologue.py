@@ -73,7 +73,7 @@ OPT_IDS = [f"g{int(g)}-norm{n}-h{h}" for g, n, h in OPTIONS]
 
 @pytest.mark.parametrize("bf16", [False, True], ids=["f32", "bf16"])
 @pytest.mark.parametrize("opt", OPTIONS, ids=OPT_IDS)
-@pytest.mark.parametrize("M,K", [(1, 2560), (7, 1024), (300, 9728), (2048, 512), (33, 2560), (5, 40960)])
+@pytest.mark.parametrize("M,K", [(1, 2560), (7, 1024), (300, 9728), (2048, 512), (33, 2560), (5, 40960), (1024, 2560)])
 def test_act_quant_ex_matches_oracle(M, K, opt, bf16):
     use_g, norm, hb = opt
     if hb and K % hb:
@@ -193,13 +193,14 @@ def test_bitlinear_matches_oracle(fmt, opt, M, N, K, bf16):
 
 
 @pytest.mark.parametrize("fmt", FMTS, ids=FMT_IDS.get)
-@pytest.mark.parametrize("M,K", [(1, 9728), (2, 9728), (4, 9728), (3, 4112), (1, 200)])
+@pytest.mark.parametrize("M,K", [(1, 1024), (2, 1000), (4, 1024), (3, 520), (1, 200)])
 def test_fused_decode_equals_two_launches(fmt, M, K):
-    # The fused kernel (codes computed in every block) and the prologue kernel
-    # followed by lowbit_linear give the same codes and accumulators; without
-    # the norm also the same scales and outputs, bit for bit.
+    # The fused kernel (codes computed in every block; rows of at most
+    # FUSED_MAX_K features) and the prologue kernel followed by lowbit_linear
+    # give the same codes and accumulators; without the norm also the same
+    # scales and outputs, bit for bit.
     N = 2560
-    assert bwt.bitlinear_fuses(M, K)
+    assert bwt.bitlinear_fuses(M, K) and not bwt.bitlinear_fuses(M, bwt.FUSED_MAX_K + 1)
     w = wls.normal_weights(4100 + fmt, N, K)
     x = to_dev(wls.to_bf16_bits(wls.normal_activations(4101, M, K, 0.005, 10.0)), True)
     g = torch.from_numpy(gain(K, 4102)).to(DEV)
