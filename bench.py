@@ -338,11 +338,12 @@ def run_gpu_arm(args, wl):
             bwt.lowbit_act_quant_ex(xs[key] if x is None else x, gains[pt.mi], norm, 1e-5, wl.hadamard, q=qs[key],
                                     s_x=sxs[key], stream=stream_)
             bwt.lowbit_linear(qs[key], sxs[key], packed, s_w, wl.fmt, pt.m.N, ydt, K=pt.m.K, y=ys[key],
-                              stream=stream_, weights_stable=True)
+                              stream=stream_, weights_stable=True, exclusive=True)
             return 2
         bwt.lowbit_bitlinear(xs[key] if x is None else x, packed, s_w, wl.fmt, pt.m.N, ydt, gains[pt.mi], norm,
                              1e-5, wl.hadamard, y=ys[key], q=None if pt.fused else qs[key],
-                             s_x=None if pt.fused else sxs[key], stream=stream_, weights_stable=True)
+                             s_x=None if pt.fused else sxs[key], stream=stream_, weights_stable=True,
+                             exclusive=True)
         return 1 if pt.fused else 2
 
     # Token counts whose points are all fused decode calls run as grouped
@@ -375,7 +376,7 @@ def run_gpu_arm(args, wl):
                                    [gains[pt.mi] for _, pt in call], norm, 1e-5, ys=[ys[k] for k in keys],
                                    qs=[qs[k] for k in keys] if two else None,
                                    s_xs=[sxs[k] for k in keys] if two else None,
-                                   stream=stream_, weights_stable=True)
+                                   stream=stream_, weights_stable=True, exclusive=True)
         n_long = sum(1 for _, pt in call if pt.m.K > bwt.FUSED_MAX_K)
         return (1 if n_long < len(call) else 0) + 2 * n_long
 
@@ -387,7 +388,7 @@ def run_gpu_arm(args, wl):
         key = (pt.mi, pt.M)
         # the prologue kernel just before does not write the weights
         bwt.lowbit_linear(qs[key], sxs[key], packed, s_w, wl.fmt, pt.m.N, ydt, K=pt.m.K, y=ys[key],
-                          weights_stable=True)
+                          weights_stable=True, exclusive=True)
 
     def step(s):
         """One pass of the hot path; each point of step s reads its own pool
@@ -561,6 +562,7 @@ def run_gpu_arm(args, wl):
                              f"launching stream around all K ({elapsed_ms:.0f} ms); per-kernel times are the "
                              f"median of {args.kernel_reps} replays of a graph of back-to-back launches of one "
                              "kernel (rotating weights)",
+                   "flags": "weights-stable and exclusive (every kernel on one stream)",
                    "parallelism": (f"token rows sharded over {world} ranks, no collective" if shard
                                    else f"replicas x{world} (token batches, no collective)"),
                    "l2": f"weights rotate over {len(pool)} packed copies ({len(pool) * n_pool / 2**20:.0f} MiB "

@@ -30,6 +30,7 @@ FUSED_MAX_K = 1024  # LOWBIT_FUSED_MAX_K
 GROUP_MAX = 32  # LOWBIT_GROUP_MAX
 F32, BF16, I32 = 0, 1, 2
 WEIGHTS_STABLE = 1  # LOWBIT_LINEAR_WEIGHTS_STABLE
+EXCLUSIVE = 2  # LOWBIT_LINEAR_EXCLUSIVE
 
 STATUS_NAMES = {
     0: "LOWBIT_OK", 1: "LOWBIT_ERR_INVALID_ARG", 2: "LOWBIT_ERR_ALIGNMENT", 3: "LOWBIT_ERR_UNSUPPORTED",
@@ -232,7 +233,8 @@ def lowbit_act_quant(x, eps: float = 0.0, q=None, s_x=None, status=None, stream=
 
 
 def lowbit_linear(q, s_x, packed, s_w, fmt: int, N: int, out_dtype: int = F32, K: int | None = None,
-                  y=None, status=None, stream=None, path: int = 0, weights_stable: bool = False):
+                  y=None, status=None, stream=None, path: int = 0, weights_stable: bool = False,
+                  exclusive: bool = False):
     """y[M, N] from int8 codes q[M, >=K] and a packed artifact (see lowbit.h).
 
     ``path`` 0 picks the kernel by M; 1 forces the GEMV, 2 the tensor-core GEMM
@@ -252,7 +254,7 @@ def lowbit_linear(q, s_x, packed, s_w, fmt: int, N: int, out_dtype: int = F32, K
         y = torch.empty((M, N), dtype=dt, device=q.device)
     st = lib().lowbit_linear_ex(_ptr(q), q.stride(0), _ptr(s_x), M, K, _ptr(packed), packed.stride(0),
                                 _ptr(s_w), fmt, N, _ptr(y), out_dtype, y.stride(0), path,
-                                WEIGHTS_STABLE if weights_stable else 0, _ptr(status), _stream(stream))
+                                (WEIGHTS_STABLE if weights_stable else 0) | (EXCLUSIVE if exclusive else 0), _ptr(status), _stream(stream))
     _check(st, "lowbit_linear")
     return y
 
@@ -290,7 +292,8 @@ def bitlinear_fuses(M: int, K: int, hadamard: int = 0, path: int = 0) -> bool:
 
 def lowbit_bitlinear(x, packed, s_w, fmt: int, N: int, out_dtype: int = F32, g=None, norm: int = NORM_NONE,
                      eps_norm: float = 1e-5, hadamard: int = 0, y=None, q=None, s_x=None, want_codes: bool = False,
-                     status=None, stream=None, path: int = 0, weights_stable: bool = False):
+                     status=None, stream=None, path: int = 0, weights_stable: bool = False,
+                     exclusive: bool = False):
     """The whole BitLinear forward from activations x[M, K] (fp32 or bf16).
 
     q and s_x are allocated as workspace when the call is not fused (or when
@@ -308,7 +311,7 @@ def lowbit_bitlinear(x, packed, s_w, fmt: int, N: int, out_dtype: int = F32, g=N
     st = lib().lowbit_bitlinear(_ptr(x), _xdt(x), M, K, x.stride(0), _ptr(g), norm, eps_norm, hadamard,
                                 _ptr(packed), packed.stride(0), _ptr(s_w), fmt, N, _ptr(y), out_dtype, y.stride(0),
                                 _ptr(q), q.stride(0) if q is not None else 0, _ptr(s_x), path,
-                                WEIGHTS_STABLE if weights_stable else 0, _ptr(status), _stream(stream))
+                                (WEIGHTS_STABLE if weights_stable else 0) | (EXCLUSIVE if exclusive else 0), _ptr(status), _stream(stream))
     _check(st, "lowbit_bitlinear")
     return (y, q, s_x) if want_codes else y
 
@@ -321,7 +324,7 @@ class BitlinearItem(ctypes.Structure):
 
 def lowbit_bitlinear_group(xs, packeds, s_ws, fmt: int, Ns, out_dtype: int = F32, gs=None, norm: int = NORM_NONE,
                            eps_norm: float = 1e-5, ys=None, want_codes: bool = False, status=None, stream=None,
-                           weights_stable: bool = False, qs=None, s_xs=None):
+                           weights_stable: bool = False, qs=None, s_xs=None, exclusive: bool = False):
     """Several independent decode BitLinear layers (M <= 4 tokens each, the
     same M, activation dtype, format and output dtype): the layers of at
     most FUSED_MAX_K features in one persistent fused GEMV launch, each
@@ -355,7 +358,7 @@ def lowbit_bitlinear_group(xs, packeds, s_ws, fmt: int, Ns, out_dtype: int = F32
                                  _ptr(s_ws[i]), Ns[i], x.shape[1], _ptr(y), y.stride(0), _ptr(q),
                                  q.stride(0) if q is not None else 0, _ptr(s_xs[i]))
     st = lib().lowbit_bitlinear_group(ctypes.cast(items, ctypes.c_void_p), n, M, _xdt(xs[0]), norm, eps_norm, fmt,
-                                      out_dtype, WEIGHTS_STABLE if weights_stable else 0, _ptr(status),
+                                      out_dtype, (WEIGHTS_STABLE if weights_stable else 0) | (EXCLUSIVE if exclusive else 0), _ptr(status),
                                       _stream(stream))
     _check(st, "lowbit_bitlinear_group")
     return (ys, qs, s_xs) if want_codes else ys

@@ -44,7 +44,7 @@ lowbit_status skinny_launch(const int8_t *q, int64_t ldq, const float *s_x, int6
 lowbit_status gemm_pair_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
                                const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
                                lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int prefetch,
-                               int32_t *status, cudaStream_t st);
+                               int exclusive, int32_t *status, cudaStream_t st);
 
 lowbit_status gemm_ts_pair_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
                                   const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
@@ -367,7 +367,7 @@ lowbit_status lowbit_bitlinear(const void *x, lowbit_dtype xdt, int64_t M, int64
 {
     const lowbit_status a = check_prologue_args(x, xdt, M, K, ldx, g, norm, eps_norm, hadamard);
     if (a != LOWBIT_OK) return a;
-    if ((flags & ~static_cast<unsigned>(LOWBIT_LINEAR_WEIGHTS_STABLE)) != 0) return LOWBIT_ERR_INVALID_ARG;
+    if ((flags & ~(LOWBIT_LINEAR_WEIGHTS_STABLE | LOWBIT_LINEAR_EXCLUSIVE)) != 0) return LOWBIT_ERR_INVALID_ARG;
     if (!valid_format(f) || packed == nullptr || s_w == nullptr || y == nullptr) return LOWBIT_ERR_INVALID_ARG;
     if (ydt != LOWBIT_F32 && ydt != LOWBIT_BF16 && ydt != LOWBIT_I32) return LOWBIT_ERR_INVALID_ARG;
     if (N <= 0 || ldy < N) return LOWBIT_ERR_INVALID_ARG;
@@ -407,7 +407,7 @@ lowbit_status lowbit_bitlinear_group(const lowbit_bitlinear_item *items, int n_i
 {
     if (items == nullptr || n_items < 1 || n_items > LOWBIT_GROUP_MAX || M < 1 || M > 4)
         return LOWBIT_ERR_INVALID_ARG;
-    if ((flags & ~static_cast<unsigned>(LOWBIT_LINEAR_WEIGHTS_STABLE)) != 0) return LOWBIT_ERR_INVALID_ARG;
+    if ((flags & ~(LOWBIT_LINEAR_WEIGHTS_STABLE | LOWBIT_LINEAR_EXCLUSIVE)) != 0) return LOWBIT_ERR_INVALID_ARG;
     if (!valid_format(f) || (ydt != LOWBIT_F32 && ydt != LOWBIT_BF16 && ydt != LOWBIT_I32))
         return LOWBIT_ERR_INVALID_ARG;
     const int64_t esz = ydt == LOWBIT_BF16 ? 2 : 4;
@@ -532,7 +532,7 @@ lowbit_status lowbit_linear_ex(const int8_t *q, int64_t ldq, const float *s_x, i
                                void *y, lowbit_dtype ydt, int64_t ldy, int path, unsigned flags,
                                int32_t *status_dev, void *stream)
 {
-    if ((flags & ~static_cast<unsigned>(LOWBIT_LINEAR_WEIGHTS_STABLE)) != 0) return LOWBIT_ERR_INVALID_ARG;
+    if ((flags & ~(LOWBIT_LINEAR_WEIGHTS_STABLE | LOWBIT_LINEAR_EXCLUSIVE)) != 0) return LOWBIT_ERR_INVALID_ARG;
     const int prefetch = (flags & LOWBIT_LINEAR_WEIGHTS_STABLE) != 0 ? 1 : 0;
     if (!valid_format(f) || q == nullptr || s_x == nullptr || packed == nullptr || s_w == nullptr || y == nullptr)
         return LOWBIT_ERR_INVALID_ARG;
@@ -559,7 +559,8 @@ lowbit_status lowbit_linear_ex(const int8_t *q, int64_t ldq, const float *s_x, i
     case LOWBIT_KERNEL_WARP_MMA:
         return skinny_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
     case LOWBIT_KERNEL_GEMM_PAIR:
-        return gemm_pair_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch, status_dev, st);
+        return gemm_pair_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, prefetch,
+                                (flags & LOWBIT_LINEAR_EXCLUSIVE) != 0 ? 1 : 0, status_dev, st);
     case LOWBIT_KERNEL_GEMM_TMEM_PAIR:
         return gemm_ts_pair_launch(q, ldq, s_x, M, K, packed, ldp, rb, s_w, f, N, y, ydt, ldy, status_dev, st);
     case LOWBIT_KERNEL_GEMM_TMEM:

@@ -106,15 +106,16 @@ __device__ __forceinline__ float elem(const uint4 &b, const float *gv, int i)
     else return v;
 }
 
-// The E gains of vector v (E = 4 or 8 floats, one or two 16-byte loads).
+// The E gains of vector v (E = 4 or 8 floats, one or two 16-byte loads,
+// through L1: every row of the grid reads the same gains, twice).
 template <int E>
 __device__ __forceinline__ void load_gain(const float *g, int64_t v, float (&gv)[8])
 {
-    const uint4 a = ld_act_u4(g + v * E);
+    const uint4 a = ld_act_ca_u4(g + v * E);
     gv[0] = __uint_as_float(a.x); gv[1] = __uint_as_float(a.y);
     gv[2] = __uint_as_float(a.z); gv[3] = __uint_as_float(a.w);
     if constexpr (E == 8) {
-        const uint4 b = ld_act_u4(g + v * E + 4);
+        const uint4 b = ld_act_ca_u4(g + v * E + 4);
         gv[4] = __uint_as_float(b.x); gv[5] = __uint_as_float(b.y);
         gv[6] = __uint_as_float(b.z); gv[7] = __uint_as_float(b.w);
     }
@@ -354,6 +355,176 @@ act_prologue_staged(const void *__restrict__ x, int64_t M, int64_t K, int64_t ld
         s_x[row] = amax != 0 ? row_scale(gm, norm != 0, ss, K, eps_norm, hb) : 0.0f;
 }
 
+// The Hadamard prologue in registers, for blocks of at most 512 features and
+// rows of at most kFwhtChunks * 8 * 512 features: one block of 8 warps per
+// token row; warp w holds the 512-feature chunks w, w + 8, ... of the row,
+// lane l features 16l..16l+15 of each.  Every hb-feature block lies inside
+// one chunk (512 / hb is whole), so the stages h < 16 of its transform run
+// within a lane and the stages 16 <= h < hb across lanes (partner lane
+// l ^ h/16), with the staged kernel's fp32 additions and subtractions in
+// the same order: bit-identical values, without shared memory or a barrier
+// per stage.  Then the row maximum (and the sum of squares) over the block,
+// the codes from registers (the fast rule of quant_rule.cuh) and the scale;
+// `mode` as act_prologue_staged.
+constexpr int kFwhtChunks = 3;
+constexpr int64_t kFwhtMaxK = static_cast<int64_t>(kFwhtChunks) * 8 * 512;
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+act_prologue_fwht(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, const float *__restrict__ g,
+                  int norm, float eps_norm, int hb, int8_t *__restrict__ q, int64_t ldq, float *__restrict__ s_x,
+                  int32_t *status, int mode, float *__restrict__ stat_max, double *__restrict__ stat_ss)
+{
+    __shared__ uint32_t red[8];
+    __shared__ double red_ss[8];
+    pdl_wait();
+    pdl_trigger();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row = blockIdx.x;
+    const char *xrow = static_cast<const char *>(x) + row * ldx * static_cast<int64_t>(sizeof(T));
+    const bool xvec = (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (ldx * static_cast<int64_t>(sizeof(T))) % 16 == 0;
+    const bool gvec = g == nullptr || (reinterpret_cast<uintptr_t>(g) & 15u) == 0;
+    float u[kFwhtChunks][16];
+    double ss = 0.0;
+    uint32_t amax = 0;
+#pragma unroll
+    for (int c = 0; c < kFwhtChunks; ++c) {
+        const int64_t chunk = warp + 8 * c;
+        if (chunk * 512 >= K) {  // the same for the whole warp
+#pragma unroll
+            for (int e = 0; e < 16; ++e) u[c][e] = 0.0f;
+            continue;
+        }
+        const int64_t k0 = (chunk * 32 + lane) * 16;
+        if (xvec && k0 + 16 <= K) {
+            if constexpr (sizeof(T) == 2) {
+#pragma unroll
+                for (int v = 0; v < 2; ++v) {
+                    const uint4 w = ld_act_u4(xrow + 2 * (k0 + 8 * v));
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) u[c][8 * v + e] = In<T>::get(w, e);
+                }
+            } else {
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const uint4 w = ld_act_u4(xrow + 4 * (k0 + 4 * v));
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) u[c][4 * v + e] = In<T>::get(w, e);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) u[c][e] = k0 + e < K ? In<T>::scalar(xrow, k0 + e) : 0.0f;
+        }
+        if (norm) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ss = __fma_rn(static_cast<double>(u[c][e]), static_cast<double>(u[c][e]), ss);
+        }
+        if (g != nullptr) {
+            if (gvec && k0 + 16 <= K) {
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const uint4 w = ld_act_ca_u4(g + k0 + 4 * v);
+                    u[c][4 * v] = __fmul_rn(u[c][4 * v], __uint_as_float(w.x));
+                    u[c][4 * v + 1] = __fmul_rn(u[c][4 * v + 1], __uint_as_float(w.y));
+                    u[c][4 * v + 2] = __fmul_rn(u[c][4 * v + 2], __uint_as_float(w.z));
+                    u[c][4 * v + 3] = __fmul_rn(u[c][4 * v + 3], __uint_as_float(w.w));
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    if (k0 + e < K) u[c][e] = __fmul_rn(u[c][e], ld_act_f32(g + k0 + e));
+            }
+        }
+        // the transform of every hb-feature block: stages h < 16 in the lane
+#pragma unroll
+        for (int h = 1; h < 16; h <<= 1) {
+            if (h >= hb) break;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                if (e & h) continue;
+                const float a = u[c][e], b = u[c][e + h];
+                u[c][e] = __fadd_rn(a, b);
+                u[c][e + h] = __fsub_rn(a, b);
+            }
+        }
+        // stages 16 <= h < hb across lanes: the lane with bit h/16 clear
+        // holds a, its partner b; (a, b) -> (a + b, a - b)
+        for (int h = 16; h < hb; h <<= 1) {
+            const int lm = h >> 4;
+            const bool upper = (lane & lm) != 0;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const float other = __shfl_xor_sync(0xffffffffu, u[c][e], lm);
+                u[c][e] = upper ? __fsub_rn(other, u[c][e]) : __fadd_rn(u[c][e], other);
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) amax = max(amax, __float_as_uint(u[c][e]) & 0x7fffffffu);
+    }
+    // the row's maximum and sum of squares over the block (fixed tree order)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if (norm) ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
+    }
+    if (lane == 0) {
+        red[warp] = amax;
+        red_ss[warp] = ss;
+    }
+    __syncthreads();
+    amax = red[0];
+    ss = red_ss[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) {
+        amax = max(amax, red[w]);
+        if (norm) ss = __dadd_rn(ss, red_ss[w]);
+    }
+    if (mode == kStagedStats) {
+        if (threadIdx.x == 0) {
+            if (!finite_bits(amax)) report(status, LOWBIT_ERR_NONFINITE);
+            stat_max[row] = __uint_as_float(amax);
+            if (stat_ss != nullptr) stat_ss[row] = ss;
+        }
+        return;
+    }
+    if (mode == kStagedCodes) {
+        // this slice's values may not exceed the row maximum it was given
+        const uint32_t given = ld_act_u32(stat_max + row) & 0x7fffffffu;
+        if (amax > given && threadIdx.x == 0) report(status, LOWBIT_ERR_INVALID_ARG);
+        amax = given;
+    }
+    const float gm = __uint_as_float(amax);
+    const bool bad = !finite_bits(amax) || !finite_bits(__float_as_uint(__fmul_rn(gm, 127.0f)));
+    if (bad && threadIdx.x == 0) report(status, LOWBIT_ERR_NONFINITE);
+    const float c127 = __fmul_rn(127.0f, __frcp_rn(gm));
+    const bool slow = !(gm >= 0x1p-121f && gm < 0x1p126f);
+    int8_t *qrow = q + row * ldq;
+#pragma unroll
+    for (int c = 0; c < kFwhtChunks; ++c) {
+        const int64_t chunk = warp + 8 * c;
+        if (chunk * 512 >= K) continue;
+        const int64_t k0 = (chunk * 32 + lane) * 16;
+        if (k0 >= K) continue;
+        uint32_t wq[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            bool near = slow;
+            wq[e] = quant4(u[c][4 * e], u[c][4 * e + 1], u[c][4 * e + 2], u[c][4 * e + 3], c127, near);
+            if (near) wq[e] = quant4_exact(u[c][4 * e], u[c][4 * e + 1], u[c][4 * e + 2], u[c][4 * e + 3], gm);
+            if (amax == 0) wq[e] = 0;
+        }
+        if (k0 + 16 <= K) {
+            *reinterpret_cast<uint4 *>(qrow + k0) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
+        } else {
+            const uint8_t *bytes = reinterpret_cast<const uint8_t *>(wq);
+            for (int64_t e = 0; k0 + e < K; ++e) qrow[k0 + e] = static_cast<int8_t>(bytes[e]);
+        }
+    }
+    if (threadIdx.x == 0 && mode == kStagedFull)
+        s_x[row] = amax != 0 ? row_scale(gm, norm != 0, ss, K, eps_norm, hb) : 0.0f;
+}
+
 // s_x of rows whose statistics were reduced over a split row: max|u| over
 // the whole row, the sum of squares over the whole row (norm), K_total
 // features.
@@ -381,6 +552,10 @@ lowbit_status launch_staged(const void *x, int64_t M, int64_t K, int64_t ldx, co
                             cudaStream_t st, int mode = kStagedFull, float *row_max = nullptr,
                             double *row_ss = nullptr)
 {
+    // blocks of at most 512 features in rows of at most kFwhtMaxK: registers
+    if (hb >= 2 && hb <= 512 && K <= kFwhtMaxK)
+        return launch_pdl(act_prologue_fwht<T>, dim3(static_cast<unsigned>(M)), dim3(256), 0, st, 0, x, M, K, ldx, g,
+                          norm, eps_norm, hb, q, ldq, s_x, status, mode, row_max, row_ss);
     static PerDevice configured;  // the shared-memory limit is raised once per device
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;

@@ -764,11 +764,109 @@ __device__ __forceinline__ void tc_commit_pair_self(uint64_t *bar)
                  ::"r"(smem_u32(bar)) : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// Last-round split of the SM-pair GEMM.  The tiles run round by round (tile
+// p + r P on pair p of P); when the last round holds T < P tiles, each of them
+// can be split along K into S parts (T S <= P) that run on otherwise idle
+// pairs.  Parts 1..S-1 store their int32 partial tiles in a per-device
+// workspace and publish an epoch flag per epilogue warp (32 token rows); the
+// matching warp of part 0 waits for it (bounded), adds
+// them (integer addition: the sum is the unsplit accumulation bit for bit)
+// and runs the epilogue.  The workspace is shared by all launches on the
+// device, so the split runs only for callers that exclude concurrent SM-pair
+// GEMMs (LOWBIT_LINEAR_EXCLUSIVE).
+// ---------------------------------------------------------------------------
+constexpr int kPairSplitMax = 8;
+constexpr int kPairSplitMinKb = 16;                       // K blocks of 128 per part, at least
+constexpr int kPairWsSlots = 96;                          // partial tiles held at once
+constexpr int kPairWsWords = 2 * PBM * 2 * PBN;  // one 256 x 256 int32 tile (both CTAs)
+__device__ uint4 g_pair_ws[kPairWsSlots][kPairWsWords / 4];
+__device__ uint32_t g_pair_flag[kPairWsSlots][2][4];  // per partial tile, CTA and epilogue warp
+
+// Parts S per last-round tile and pairs P to launch, given the resident
+// pairs: with at least as many tiles as pairs, P = resident and the T tiles
+// of the partial last round split S ways (T S <= P); with fewer tiles, every
+// tile splits and P = tiles * S.  S is also held to kPairSplitMax, to
+// kPairSplitMinKb K blocks per part and to the workspace (T (S - 1) <=
+// kPairWsSlots); S = 1 when the last round is full.  Shorter parts lose more
+// to the partial tiles' 256 KB round trip through L2 than the idle pairs
+// win back (measured: 2560 -> 9728 at M = 8192, 2 parts of 10 K blocks,
+// 149.6 us against 142.2 unsplit; at M = 1024, 8 parts of 2 or 3, 53.5 us
+// against 29.6; 9728 -> 2560 at M = 8192, 3 parts of 25, 141.9 against
+// 147.3).
+inline void pair_split(int64_t tiles, int64_t resident, int64_t nkb, int &S_out, int64_t &P_out)
+{
+    S_out = 1;
+    P_out = tiles < resident ? tiles : resident;
+    if (resident <= 0 || tiles <= 0) return;
+    const int64_t T = tiles >= resident ? tiles % resident : tiles;
+    if (T == 0) return;
+    int64_t S = resident / T;
+    if (S > kPairSplitMax) S = kPairSplitMax;
+    if (S > nkb / kPairSplitMinKb) S = nkb / kPairSplitMinKb;
+    while (S > 1 && T * (S - 1) > kPairWsSlots) --S;
+    if (S <= 1) return;
+    S_out = static_cast<int>(S);
+    if (tiles < resident) P_out = tiles * S;
+}
+
+// One unit of work of a pair: K blocks [kb0, kb1) of `tile`; `tail` is the
+// index of a split last-round tile (-1 when the tile is whole) and `part` the
+// unit's part of it.
+struct PairUnit {
+    int64_t tile, tail;
+    int kb0, kb1, part;
+};
+
+// Unit `it` of pair p (false past the pair's last unit).  With S = 1 this is
+// the plain round-robin order, tile p + it P.
+__device__ __forceinline__ bool pair_unit(int64_t p, int64_t P, int64_t num_tiles, int nkb, int S, int64_t it,
+                                          PairUnit &u)
+{
+    if (S <= 1) {
+        const int64_t tile = p + it * P;
+        if (tile >= num_tiles) return false;
+        u = PairUnit{tile, -1, 0, nkb, 0};
+        return true;
+    }
+    const int64_t full = num_tiles / P;
+    if (it < full) {
+        u = PairUnit{p + it * P, -1, 0, nkb, 0};
+        return true;
+    }
+    const int64_t T = num_tiles - full * P;
+    if (it > full || p >= T * S) return false;
+    const int part = static_cast<int>(p % S);
+    u = PairUnit{full * P + p / S, p / S, part * nkb / S, (part + 1) * nkb / S, part};
+    return true;
+}
+
+// Waits (bounded by the pipeline wait limit) until flag == epoch, with
+// acquire order for the reads that follow.  False on timeout (reported).
+__device__ inline bool wait_flag(const uint32_t *flag, uint32_t epoch, volatile int *abort_flag, int32_t *status)
+{
+    const long long t0 = clock64();
+    for (uint32_t i = 1;; ++i) {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if (v == epoch) return true;
+        if ((i & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (clock64() - t0 > g_wait_limit_cycles) {
+                *abort_flag = 1;
+                report(status, LOWBIT_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
 template <int FMT, int OUT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_p,
                  const float *__restrict__ s_x, const float *__restrict__ s_w, int64_t M, int64_t N, int64_t K,
-                 void *__restrict__ y, int64_t ldy, int vec_ok, int prefetch, int32_t *status)
+                 void *__restrict__ y, int64_t ldy, int vec_ok, int prefetch, int32_t *status, int split,
+                 uint32_t epoch)
 {
     constexpr int ST = pair_tma_stages<FMT>();
     constexpr int SE = kExpStages;
@@ -842,21 +940,23 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             uint32_t g = 0;
             bool ok = true;
             uint32_t npre = 0;
+            PairUnit u;
             if (prefetch != 0) {
-                if (pair < num_tiles) {
-                    const int n0 = static_cast<int>((pair / num_m) * 2 * PBN + rank * PBN);
-                    npre = static_cast<uint32_t>(nkb < ST ? nkb : ST);
+                if (pair_unit(pair, num_pairs, num_tiles, nkb, split, 0, u)) {
+                    const int n0 = static_cast<int>((u.tile / num_m) * 2 * PBN + rank * PBN);
+                    const int nloc = u.kb1 - u.kb0;
+                    npre = static_cast<uint32_t>(nloc < ST ? nloc : ST);
                     for (uint32_t i = 0; i < npre; ++i) {
                         mbar_arrive_expect_tx(&full_tma[i], A_BYTES + P_BYTES);
-                        tma_load_2d(sP + i * P_BYTES, &map_p, &full_tma[i], static_cast<int>(i) * PB, n0);
+                        tma_load_2d(sP + i * P_BYTES, &map_p, &full_tma[i], (u.kb0 + static_cast<int>(i)) * PB, n0);
                     }
                 }
                 pdl_wait();
             }
-            for (int64_t tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-                const int m0 = static_cast<int>((tile % num_m) * 2 * PBM + rank * PBM);
-                const int n0 = static_cast<int>((tile / num_m) * 2 * PBN + rank * PBN);
-                for (int kb = 0; kb < nkb; ++kb, ++g) {
+            for (int64_t it = 0; ok && pair_unit(pair, num_pairs, num_tiles, nkb, split, it, u); ++it) {
+                const int m0 = static_cast<int>((u.tile % num_m) * 2 * PBM + rank * PBM);
+                const int n0 = static_cast<int>((u.tile / num_m) * 2 * PBN + rank * PBN);
+                for (int kb = u.kb0; kb < u.kb1; ++kb, ++g) {
                     const int s = g % ST;
                     if (g < npre) {
                         tma_load_2d(sA + s * A_BYTES, &map_a, &full_tma[s], kb * BK, m0);
@@ -881,12 +981,13 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             uint32_t g = 0;
             uint32_t t = 0;
             bool ok = true;
-            for (int64_t tile = pair; tile < num_tiles && ok; tile += num_pairs, ++t) {
+            PairUnit u;
+            for (int64_t it = 0; ok && pair_unit(pair, num_pairs, num_tiles, nkb, split, it, u); ++it, ++t) {
                 const int b = t & 1;
                 if (!wait_bar(&acc_empty[b], ((t >> 1) & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * 2 * PBN);
-                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                for (int kb = u.kb0; kb < u.kb1; ++kb, ++g) {
                     const int s1 = g % ST, s2 = g % SE;
                     if (!wait_bar(&full_exp[s2], (g / SE) & 1u, abort_flag, status)) { ok = false; break; }
                     tc_fence_after();
@@ -895,7 +996,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 #pragma unroll
                     for (int kk = 0; kk < BK / UMMA_K; ++kk)
                         tc_mma_i8_pair(d_tmem, sw128_desc(a_addr + kk * UMMA_K), sw128_desc(e_addr + kk * UMMA_K),
-                                       kPairIdesc, (kb | kk) != 0 ? 1u : 0u);
+                                       kPairIdesc, (kb != u.kb0 || kk != 0) ? 1u : 0u);
                     tc_commit_pair_both(&mma_done[s1]);
                 }
                 if (!ok) break;
@@ -912,8 +1013,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         const uint32_t full_exp_leader = map_to_peer(smem_u32(full_exp), 0);
         uint32_t g = 0;
         bool ok = true;
-        for (int64_t tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-            for (int kb = 0; kb < nkb; ++kb, ++g) {
+        PairUnit u;
+        for (int64_t it = 0; ok && pair_unit(pair, num_pairs, num_tiles, nkb, split, it, u); ++it) {
+            for (int kb = u.kb0; kb < u.kb1; ++kb, ++g) {
                 const int s1 = g % ST, s2 = g % SE;
                 if (!wait_bar(&full_tma[s1], (g / ST) & 1u, abort_flag, status)) { ok = false; break; }
                 if (g >= static_cast<uint32_t>(SE)) {
@@ -935,23 +1037,67 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         const uint32_t acc_empty_leader = map_to_peer(smem_u32(acc_empty), 0);
         const float sw_tensor = (FMT == kT2) ? s_w[0] : 0.0f;
         uint32_t t = 0;
-        for (int64_t tile = pair; tile < num_tiles; tile += num_pairs, ++t) {
+        PairUnit u;
+        const int row_in = quarter * 32 + lane;  // this thread's token row within the CTA's 128
+        for (int64_t it = 0; pair_unit(pair, num_pairs, num_tiles, nkb, split, it, u); ++it, ++t) {
             const int b = t & 1;
             int ready = 0;
             if (lane == 0) ready = wait_bar(&acc_full[b], (t >> 1) & 1u, abort_flag, status) ? 1 : 0;
             ready = __shfl_sync(0xffffffffu, ready, 0);
             if (!ready) break;
             tc_fence_after();
-            const int64_t m0 = (tile % num_m) * 2 * PBM + rank * PBM;
-            const int64_t n0 = (tile / num_m) * 2 * PBN;
+            const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * 2 * PBN);
+            if (u.tail >= 0 && u.part > 0) {
+                // a later part of a split tile: publish the partial tile.
+                // Workspace layout per CTA: [chunk][4-column group][row], so
+                // the 32 lanes (rows) of one store write 512 contiguous bytes.
+                const int slot = static_cast<int>(u.tail) * (split - 1) + u.part - 1;
+                uint4 *ws = g_pair_ws[slot] + rank * (PBM * 2 * PBN / 4);
+#pragma unroll 1
+                for (int cc = 0; cc < 2 * PBN / 32; ++cc) {
+                    uint32_t v[32];
+                    tmem_ld_32cols(tacc + static_cast<uint32_t>(cc * 32), v);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        ws[(cc * 8 + j) * PBM + row_in] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                }
+                __threadfence();
+                __syncwarp();  // this warp's 32 rows are stored
+                if (lane == 0)
+                    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(&g_pair_flag[slot][rank][quarter]),
+                                 "r"(epoch)
+                                 : "memory");
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(acc_empty_leader + static_cast<uint32_t>(b * 8));
+                continue;
+            }
+            // part 0 of a split tile: the other parts' partial tiles are added
+            const int nsum = u.tail >= 0 ? split - 1 : 0;
+            bool have = true;  // every lane acquires the flags of its warp's rows itself
+            for (int p = 0; p < nsum; ++p)
+                have = have && wait_flag(&g_pair_flag[static_cast<int>(u.tail) * (split - 1) + p][rank][quarter],
+                                         epoch, abort_flag, status);
+            const int64_t m0 = (u.tile % num_m) * 2 * PBM + rank * PBM;
+            const int64_t n0 = (u.tile / num_m) * 2 * PBN;
             const int64_t row0 = m0 + quarter * 32;
             const float sx = (row0 + lane < M) ? ld_act_f32(s_x + row0 + lane) : 0.0f;
 #pragma unroll 1
             for (int cc = 0; cc < 2 * PBN / 32; ++cc) {
                 const int64_t nc = n0 + cc * 32;
                 uint32_t v[32];
-                tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                   static_cast<uint32_t>(b * 2 * PBN + cc * 32), v);
+                tmem_ld_32cols(tacc + static_cast<uint32_t>(cc * 32), v);
+                for (int p = 0; p < nsum && have; ++p) {
+                    const uint4 *ws = g_pair_ws[static_cast<int>(u.tail) * (split - 1) + p] + rank * (PBM * 2 * PBN / 4);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint4 a = ld_act_u4(ws + (cc * 8 + j) * PBM + row_in);
+                        v[4 * j] += a.x;
+                        v[4 * j + 1] += a.y;
+                        v[4 * j + 2] += a.z;
+                        v[4 * j + 3] += a.w;
+                    }
+                }
                 if (nc < N) {
                     float sw[32];
 #pragma unroll
@@ -980,7 +1126,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 template <int FMT, int OUT>
 lowbit_status launch_pair_t(const CUtensorMap &ma, const CUtensorMap &mp, const float *s_x, const float *s_w,
                             int64_t M, int64_t N, int64_t K, void *y, int64_t ldy, int vec_ok, int prefetch,
-                            int32_t *status, cudaStream_t st)
+                            int exclusive, int32_t *status, cudaStream_t st)
 {
     constexpr size_t smem = pair_smem_bytes<FMT, OUT>();
     static_assert(smem <= 232448, "shared memory budget");
@@ -1002,21 +1148,28 @@ lowbit_status launch_pair_t(const CUtensorMap &ma, const CUtensorMap &mp, const 
     });
     if (resident <= 0) return LOWBIT_ERR_CUDA;
     const int64_t tiles = ((M + 2 * PBM - 1) / (2 * PBM)) * ((N + 2 * PBN - 1) / (2 * PBN));
-    const int64_t pairs = tiles < resident ? tiles : resident;
+    int64_t pairs = tiles < resident ? tiles : resident;
+    int split = 1;
+    if (exclusive) pair_split(tiles, resident, (K + BK - 1) / BK, split, pairs);
+    static std::atomic<uint32_t> epochs{0};
+    uint32_t epoch = epochs.fetch_add(1, std::memory_order_relaxed) + 1;
+    if (epoch == 0) epoch = epochs.fetch_add(1, std::memory_order_relaxed) + 1;  // 0 is the flags' initial value
     return launch_pdl(gemm_pair_kernel<FMT, OUT>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kThreads), smem, st,
-                      0, ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status);
+                      0, ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, split, epoch);
 }
 
 template <int FMT>
 lowbit_status launch_pair_fmt(const CUtensorMap &ma, const CUtensorMap &mp, const float *s_x, const float *s_w,
                               int64_t M, int64_t N, int64_t K, void *y, lowbit_dtype ydt, int64_t ldy, int vec_ok,
-                              int prefetch, int32_t *status, cudaStream_t st)
+                              int prefetch, int exclusive, int32_t *status, cudaStream_t st)
 {
     if (ydt == LOWBIT_F32)
-        return launch_pair_t<FMT, LOWBIT_F32>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, st);
+        return launch_pair_t<FMT, LOWBIT_F32>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, exclusive, status,
+                                              st);
     if (ydt == LOWBIT_BF16)
-        return launch_pair_t<FMT, LOWBIT_BF16>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, st);
-    return launch_pair_t<FMT, LOWBIT_I32>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, st);
+        return launch_pair_t<FMT, LOWBIT_BF16>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, exclusive, status,
+                                               st);
+    return launch_pair_t<FMT, LOWBIT_I32>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, exclusive, status, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -1127,7 +1280,7 @@ namespace lowbit {
 lowbit_status gemm_pair_launch(const int8_t *q, int64_t ldq, const float *s_x, int64_t M, int64_t K,
                                const uint8_t *packed, int64_t ldp, int64_t row_bytes, const float *s_w,
                                lowbit_format f, int64_t N, void *y, lowbit_dtype ydt, int64_t ldy, int prefetch,
-                               int32_t *status, cudaStream_t st)
+                               int exclusive, int32_t *status, cudaStream_t st)
 {
     using namespace tc;
     CUtensorMap ma, mp;
@@ -1143,10 +1296,13 @@ lowbit_status gemm_pair_launch(const int8_t *q, int64_t ldq, const float *s_x, i
     const int64_t esz = ydt == LOWBIT_BF16 ? 2 : 4;
     const int vec_ok = ((reinterpret_cast<uintptr_t>(y) & 15u) == 0 && (ldy * esz) % 16 == 0) ? 1 : 0;
     if (f == LOWBIT_TERNARY2)
-        return launch_pair_fmt<kT2>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, st);
+        return launch_pair_fmt<kT2>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, exclusive, status,
+                                     st);
     if (f == LOWBIT_BINARY1)
-        return launch_pair_fmt<kB1>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, st);
-    return launch_pair_fmt<kI4>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, status, st);
+        return launch_pair_fmt<kB1>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, exclusive, status,
+                                     st);
+    return launch_pair_fmt<kI4>(ma, mp, s_x, s_w, M, N, K, y, ydt, ldy, vec_ok, prefetch, exclusive, status,
+                                     st);
 }
 }  // namespace lowbit
 

@@ -114,6 +114,19 @@ __device__ __forceinline__ uint4 ld_act_u4(const void *p)
     return v;
 }
 
+// The same for activation-side data that every row of a kernel re-reads (a
+// gain vector): L1-allocating (.ca), still issued after griddepcontrol.wait
+// by the asm volatile.
+__device__ __forceinline__ uint4 ld_act_ca_u4(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.ca.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+
 __device__ __forceinline__ uint32_t ld_act_u32(const void *p)
 {
     uint32_t v;

@@ -148,8 +148,10 @@ def test_linear_rejects_bad_arguments(lib):
 def test_linear_ex_rejects_unknown_flags(lib):
     f = lib.lowbit_linear_ex
     args = [FAKE, 256, FAKE, 4, 256, FAKE, 64, FAKE, bwt.TERNARY2, 8, FAKE, bwt.F32, 8, 0]
-    for flags in (2, 4, 0x80000000, 0xFFFFFFFF):
+    for flags in (4, 8, 0x80000000, 0xFFFFFFFF):
         assert f(*args, flags, None, None) == bwt.ERR_INVALID_ARG
+    for flags in (bwt.EXCLUSIVE, bwt.WEIGHTS_STABLE | bwt.EXCLUSIVE):  # accepted: the call gets past the checks
+        assert f(*args, flags, None, None) != bwt.ERR_INVALID_ARG
     bad = list(args)
     bad[0] = None                                   # q = NULL with a valid flag
     assert f(*bad, bwt.WEIGHTS_STABLE, None, None) == bwt.ERR_INVALID_ARG

@@ -386,6 +386,44 @@ def test_stream_split_bf16_bit_exact(fmt):
     assert np.array_equal(bf16_bits(y), oracle.rescale(acc, s_w, s_x, "bf16"))
 
 
+# LOWBIT_LINEAR_EXCLUSIVE: the SM-pair GEMM (path 6) splits each tile of a
+# partial last round along K over idle pairs (parts of at least 16 K blocks)
+# and adds the int32 partial tiles through a device workspace.  Shapes: 24
+# last-round tiles of 320 split 3 ways (8192, 2560, 9728); no whole round, 6
+# ragged tiles x 2 parts of 16 K blocks (300, 700, 4096); 8 tiles x 8 parts
+# (512, 1000, 16384); 4 tiles of 152 that stay whole (1024, 9728, 2560: 20 K
+# blocks).  The output must equal the unsplit launch bit for bit, and the
+# oracle on sampled rows (every row of the small shapes).
+PAIR_SPLIT_SHAPES = [(8192, 2560, 9728), (300, 700, 4096), (512, 1000, 16384), (1024, 9728, 2560)]
+
+
+@pytest.mark.parametrize("M,N,K", PAIR_SPLIT_SHAPES, ids=str)
+def test_pair_last_round_split_bit_exact(M, N, K):
+    fmt = bwt.TERNARY2
+    w = wls.normal_weights(1100 + M + K, N, K)
+    x = wls.normal_activations(1101 + M + K, M, K, 0.01, 8.0)
+    packed, s_w = gpu_pack(w, fmt)
+    q, s_x = gpu_act(x, False)
+    st = status_word()
+    ys = {}
+    for exclusive in (False, True, True):  # twice split: the epoch flags must not carry over
+        for out in (bwt.I32, bwt.BF16):
+            ys[(exclusive, out)] = bwt.lowbit_linear(q, s_x, packed, s_w, fmt, N, out, K=K, status=st, path=6,
+                                                     exclusive=exclusive)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    for out in (bwt.I32, bwt.BF16):
+        assert torch.equal(ys[(True, out)], ys[(False, out)])
+    codes, _ = oracle.quantize(w, fmt, 1e-5)
+    q_o, _ = oracle.act_quant(x, 0.0)
+    rows = np.arange(M)
+    if M * N * K > 2e9:  # first and last row of every 256-row tile, and random rows
+        rng = np.random.default_rng(1102)
+        rows = np.unique(np.concatenate([np.arange(0, M, 256), np.arange(255, M, 256), rng.choice(M, 64)]))
+    acc = oracle.int_dot(q_o[rows], codes, fmt, nthreads=oracle.max_threads())
+    assert np.array_equal(ys[(True, bwt.I32)].cpu().numpy()[rows].astype(np.int64), acc)
+
+
 # LOWBIT_LINEAR_WEIGHTS_STABLE: weight reads start before the wait for the
 # preceding kernel (here the act quant that produced q, launched just before
 # on the same stream); the results must not change.  Shapes cover the GEMV
