@@ -384,10 +384,21 @@ def run_gpu_arm(args, wl):
         key = (pt.mi, pt.M)
         bwt.lowbit_act_quant_ex(xs[key], gains[pt.mi], norm, 1e-5, wl.hadamard, q=qs[key], s_x=sxs[key])
 
-    def linear(pt, packed, s_w):
+    # The linear kernel timed alone reads codes that no prologue rewrites in
+    # between, so each point rotates over copies of its codes whose total
+    # exceeds twice L2 (at least two): every launch reads its codes from HBM,
+    # as it does in the step.
+    code_pool = {}
+    for pt in points:
         key = (pt.mi, pt.M)
+        copies = max(2, min(8, int(np.ceil(2 * L2_BYTES / max(1, qs[key].numel())))))
+        code_pool[key] = [(qs[key], sxs[key])] + [(qs[key].clone(), sxs[key].clone()) for _ in range(copies - 1)]
+
+    def linear(pt, packed, s_w, r=0):
+        key = (pt.mi, pt.M)
+        q_r, s_x_r = code_pool[key][r % len(code_pool[key])]
         # the prologue kernel just before does not write the weights
-        bwt.lowbit_linear(qs[key], sxs[key], packed, s_w, wl.fmt, pt.m.N, ydt, K=pt.m.K, y=ys[key],
+        bwt.lowbit_linear(q_r, s_x_r, packed, s_w, wl.fmt, pt.m.N, ydt, K=pt.m.K, y=ys[key],
                           weights_stable=True, exclusive=True)
 
     def step(s):
@@ -443,8 +454,9 @@ def run_gpu_arm(args, wl):
     for i, pt in enumerate(points):
         launches_g = 4 if pt.rows >= 4096 else 20
         per_act.append(summary(time_graph(torch, stream, lambda r: prologue(pt), launches_g, args.kernel_reps)))
+        launches_l = max(launches_g, len(code_pool[(pt.mi, pt.M)]))  # every code copy in each replay
         per_point.append(summary(time_graph(
-            torch, stream, lambda r: linear(pt, *pool[(i + r) % n_sets][pt.mi]), launches_g, args.kernel_reps)))
+            torch, stream, lambda r: linear(pt, *pool[(i + r) % n_sets][pt.mi], r=r), launches_l, args.kernel_reps)))
         per_call.append(summary(time_graph(
             torch, stream, lambda r: bitlinear(pt, *pool[(i + r) % n_sets][pt.mi]), launches_g, args.kernel_reps)))
 
@@ -561,7 +573,8 @@ def run_gpu_arm(args, wl):
                    "timing": f"K timed steps replay {n_graphs} captured step graphs cyclically, events on the "
                              f"launching stream around all K ({elapsed_ms:.0f} ms); per-kernel times are the "
                              f"median of {args.kernel_reps} replays of a graph of back-to-back launches of one "
-                             "kernel (rotating weights)",
+                             "kernel (rotating weights, and rotating activation codes > 2x L2 for the linear "
+                             "kernels)",
                    "flags": "weights-stable and exclusive (every kernel on one stream)",
                    "parallelism": (f"token rows sharded over {world} ranks, no collective" if shard
                                    else f"replicas x{world} (token batches, no collective)"),
