@@ -23,6 +23,7 @@
 // LOWBIT_ERR_TIMEOUT, drains its copies and MMAs, frees tensor memory and
 // returns.
 #include "tc_common.cuh"
+#include <atomic>
 
 namespace lowbit {
 namespace tc {
@@ -728,16 +729,17 @@ gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_const
 constexpr int PBM = 128;                      // tokens per CTA (the pair's MMA has M = 256)
 constexpr int PBN = 128;                      // features expanded per CTA (the pair's N = 256)
 constexpr int PE_BYTES = PBN * BK;
-template <int FMT> __host__ __device__ constexpr int pair_tma_stages() { return FMT == kI4 ? 7 : 8; }
+template <int FMT, int OUT> __host__ __device__ constexpr int pair_tma_stages() { return FMT == kI4 ? 7 : 8; }
+template <int FMT, int OUT> __host__ __device__ constexpr int pair_exp_stages() { return kExpStages; }
 constexpr uint32_t kPairIdesc = (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>((2 * PBN) >> 3) << 17) |
                                 (static_cast<uint32_t>((2 * PBM) >> 4) << 24);
 
 template <int FMT, int OUT>
 __host__ __device__ constexpr size_t pair_smem_bytes()
 {
-    return 1024 + static_cast<size_t>(pair_tma_stages<FMT>()) * (A_BYTES + PBN * packed_bytes_per_kblock<FMT>()) +
-           static_cast<size_t>(kExpStages) * PE_BYTES + 4 * stage_warp_bytes<OUT>() +
-           8 * (2 * pair_tma_stages<FMT>() + kExpStages + 8);
+    return 1024 + static_cast<size_t>(pair_tma_stages<FMT, OUT>()) * (A_BYTES + PBN * packed_bytes_per_kblock<FMT>()) +
+           static_cast<size_t>(pair_exp_stages<FMT, OUT>()) * PE_BYTES + 4 * stage_warp_bytes<OUT>() +
+           8 * (2 * pair_tma_stages<FMT, OUT>() + pair_exp_stages<FMT, OUT>() + 8);
 }
 
 __device__ __forceinline__ void tc_mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
@@ -765,81 +767,129 @@ __device__ __forceinline__ void tc_commit_pair_self(uint64_t *bar)
 }
 
 // ---------------------------------------------------------------------------
-// Last-round split of the SM-pair GEMM.  The tiles run round by round (tile
-// p + r P on pair p of P); when the last round holds T < P tiles, each of them
-// can be split along K into S parts (T S <= P) that run on otherwise idle
-// pairs.  Parts 1..S-1 store their int32 partial tiles in a per-device
-// workspace and publish an epoch flag per epilogue warp (32 token rows); the
-// matching warp of part 0 waits for it (bounded), adds
-// them (integer addition: the sum is the unsplit accumulation bit for bit)
-// and runs the epilogue.  The workspace is shared by all launches on the
-// device, so the split runs only for callers that exclude concurrent SM-pair
-// GEMMs (LOWBIT_LINEAR_EXCLUSIVE).
+// Stream-K tail of the SM-pair GEMM.  The tiles run round by round (tile
+// p + r P on pair p of P) while every pair has a whole tile to take; when the
+// last round would be partial, the K blocks of the tiles left after the
+// whole rounds (the partial round plus one whole round, or every tile when
+// there are fewer tiles than pairs) are shared evenly: pair p takes the
+// blocks [p W / P, (p + 1) W / P) of the W = tiles_left x nkb blocks laid out
+// tile after tile.  A pair's range is one or more pieces of tiles; only the
+// first piece can start inside a tile (kb0 > 0), and only the last can end
+// inside one.  A piece that starts inside a tile stores its int32 partial
+// tile in the workspace slot of its pair and publishes an epoch flag per
+// epilogue warp (32 token rows).  The piece that starts the tile (kb0 = 0)
+// and ends inside it is the pair's last; it waits (bounded) for the flags of
+// the following pairs that hold the rest of the tile, adds their partial
+// tiles (integer addition: the sum is the unsplit accumulation bit for bit)
+// and runs the epilogue.  Those pairs start with their pieces, so the wait is
+// short.  The workspace is shared by all launches on the device, so the
+// split runs only for callers that exclude concurrent SM-pair GEMMs
+// (LOWBIT_LINEAR_EXCLUSIVE).
 // ---------------------------------------------------------------------------
-constexpr int kPairSplitMax = 8;
-constexpr int kPairSplitMinKb = 16;                       // K blocks of 128 per part, at least
-constexpr int kPairWsSlots = 96;                          // partial tiles held at once
+constexpr int kPairSkMinKb = 8;                           // K blocks of 128 per pair's share, at least
+constexpr int kPairSkFixupKb = 12;                       // cost of the tail, in K blocks of MMA time
+constexpr int kPairWsSlots = 96;                          // partial tiles held at once (one per pair)
 constexpr int kPairWsWords = 2 * PBM * 2 * PBN;  // one 256 x 256 int32 tile (both CTAs)
+constexpr int kWsWarpVecs = 32 * 2 * PBN / 4;     // one epilogue warp's 32 rows x 256 int32, in uint4
 __device__ uint4 g_pair_ws[kPairWsSlots][kPairWsWords / 4];
-__device__ uint32_t g_pair_flag[kPairWsSlots][2][4];  // per partial tile, CTA and epilogue warp
+__device__ uint32_t g_pair_flag[kPairWsSlots][2][4];  // per pair (slot), CTA and epilogue warp
+// One epoch per launch, shared by every instantiation of the kernel (they
+// share the flags), so no launch can take another launch's flag for its own.
+static std::atomic<uint32_t> g_pair_epoch{0};
 
-// Parts S per last-round tile and pairs P to launch, given the resident
-// pairs: with at least as many tiles as pairs, P = resident and the T tiles
-// of the partial last round split S ways (T S <= P); with fewer tiles, every
-// tile splits and P = tiles * S.  S is also held to kPairSplitMax, to
-// kPairSplitMinKb K blocks per part and to the workspace (T (S - 1) <=
-// kPairWsSlots); S = 1 when the last round is full.  Shorter parts lose more
-// to the partial tiles' 256 KB round trip through L2 than the idle pairs
-// win back (measured: 2560 -> 9728 at M = 8192, 2 parts of 10 K blocks,
-// 149.6 us against 142.2 unsplit; at M = 1024, 8 parts of 2 or 3, 53.5 us
-// against 29.6; 9728 -> 2560 at M = 8192, 3 parts of 25, 141.9 against
-// 147.3).
-inline void pair_split(int64_t tiles, int64_t resident, int64_t nkb, int &S_out, int64_t &P_out)
+// The schedule of a launch: P pairs, the first dp_tiles tiles in whole
+// rounds (a multiple of P, or every tile), the rest shared by K block.  The
+// shared tail is taken when its estimated time, in K blocks per pair plus
+// kPairSkFixupKb, beats the whole-round schedule (ceil(tiles / P) rounds of
+// nkb).  The fix-up estimate is measured: a partial tile's store, the
+// finisher's staging and its longer epilogue, and the pieces' shorter
+// pipelines cost about 12 K blocks of MMA time (4B-class shapes, 74 pairs,
+// bf16 out: 9728 -> 2560 at M = 8192, 4 rounds + 24 tiles of 76 blocks, 145.8
+// -> 137.6 us; at M = 1024, 40 tiles of 76, 37.3 -> 33.1 us; 2560 -> 9728 at
+// M = 8192, 16 rounds + 32 tiles of 20, 147.0 -> 150.8 us, so that shape keeps
+// whole rounds: 300 + 29 + 12 >= 340).
+inline void pair_plan(int64_t tiles, int64_t resident, int64_t nkb, int64_t &dp_tiles, int64_t &P_out)
 {
-    S_out = 1;
     P_out = tiles < resident ? tiles : resident;
-    if (resident <= 0 || tiles <= 0) return;
-    const int64_t T = tiles >= resident ? tiles % resident : tiles;
-    if (T == 0) return;
-    int64_t S = resident / T;
-    if (S > kPairSplitMax) S = kPairSplitMax;
-    if (S > nkb / kPairSplitMinKb) S = nkb / kPairSplitMinKb;
-    while (S > 1 && T * (S - 1) > kPairWsSlots) --S;
-    if (S <= 1) return;
-    S_out = static_cast<int>(S);
-    if (tiles < resident) P_out = tiles * S;
+    dp_tiles = tiles;
+    if (resident <= 0 || tiles <= 0 || resident > kPairWsSlots || tiles % resident == 0) return;
+    const int64_t whole = (tiles + P_out - 1) / P_out * nkb;
+    const int64_t rounds = tiles / resident;
+    const int64_t dp = rounds > 0 ? (rounds - 1) * resident : 0;
+    const int64_t W = (tiles - dp) * nkb;
+    int64_t P = resident;
+    if (rounds == 0 && W / P < kPairSkMinKb) P = W / kPairSkMinKb;
+    if (P <= 1 || (rounds == 0 && P <= tiles)) return;
+    const int64_t shared = dp / P * nkb + (W + P - 1) / P + kPairSkFixupKb;
+    if (shared >= whole) return;
+    dp_tiles = dp;
+    P_out = P;
 }
 
-// One unit of work of a pair: K blocks [kb0, kb1) of `tile`; `tail` is the
-// index of a split last-round tile (-1 when the tile is whole) and `part` the
-// unit's part of it.
+// 16-byte copy global -> shared by this thread (L2 only), and the wait for
+// all of the thread's copies.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// One unit of work of a pair: K blocks [kb0, kb1) of `tile`.  kb0 > 0: the
+// unit's partial tile goes to the pair's workspace slot.  last >= 0: the
+// unit starts the tile and ends inside it, and the partial tiles of pairs
+// p + 1 .. last are added to it.
 struct PairUnit {
-    int64_t tile, tail;
-    int kb0, kb1, part;
+    int64_t tile;
+    int kb0, kb1, last;
 };
 
-// Unit `it` of pair p (false past the pair's last unit).  With S = 1 this is
-// the plain round-robin order, tile p + it P.
-__device__ __forceinline__ bool pair_unit(int64_t p, int64_t P, int64_t num_tiles, int nkb, int S, int64_t it,
-                                          PairUnit &u)
-{
-    if (S <= 1) {
-        const int64_t tile = p + it * P;
-        if (tile >= num_tiles) return false;
-        u = PairUnit{tile, -1, 0, nkb, 0};
+// The units of pair p in order: the whole rounds (tiles p, p + P, ... below
+// dp_tiles), then the pair's share of the tail.  The divisions run once, when
+// the schedule is made, so a unit boundary costs the MMA issuer no more than a
+// few integer operations.
+struct PairSched {
+    int64_t next_dp, dp_tiles, P, W;
+    int64_t t, left;  // tail: current tile (from dp_tiles on), K blocks left
+    int kb, nkb;      // first K block of the next tail piece
+
+    __device__ __forceinline__ PairSched(int64_t p, int64_t P_, int64_t num_tiles, int nkb_, int64_t dp_tiles_)
+        : next_dp(p), dp_tiles(dp_tiles_), P(P_), W(0), t(0), left(0), kb(0), nkb(nkb_)
+    {
+        if (dp_tiles < num_tiles) {
+            W = (num_tiles - dp_tiles) * nkb;
+            const int64_t s = p * W / P, e = (p + 1) * W / P;
+            t = s / nkb;
+            kb = static_cast<int>(s - t * nkb);
+            left = e - s;
+        }
+    }
+
+    // The next unit (false past the pair's last one).
+    __device__ __forceinline__ bool next(PairUnit &u)
+    {
+        if (next_dp < dp_tiles) {
+            u = PairUnit{next_dp, 0, nkb, -1};
+            next_dp += P;
+            return true;
+        }
+        if (left <= 0) return false;
+        const int n = static_cast<int>(left < nkb - kb ? left : nkb - kb);
+        u.tile = dp_tiles + t;
+        u.kb0 = kb;
+        u.kb1 = kb + n;
+        // a piece that starts its tile and ends inside it: the pair holding
+        // the tile's last K block is the max q with q W / P <= end - 1
+        u.last = (kb == 0 && n < nkb) ? static_cast<int>(((t + 1) * nkb * P - 1) / W) : -1;
+        left -= n;
+        kb = 0;
+        ++t;
         return true;
     }
-    const int64_t full = num_tiles / P;
-    if (it < full) {
-        u = PairUnit{p + it * P, -1, 0, nkb, 0};
-        return true;
-    }
-    const int64_t T = num_tiles - full * P;
-    if (it > full || p >= T * S) return false;
-    const int part = static_cast<int>(p % S);
-    u = PairUnit{full * P + p / S, p / S, part * nkb / S, (part + 1) * nkb / S, part};
-    return true;
-}
+};
 
 // Waits (bounded by the pipeline wait limit) until flag == epoch, with
 // acquire order for the reads that follow.  False on timeout (reported).
@@ -861,19 +911,52 @@ __device__ inline bool wait_flag(const uint32_t *flag, uint32_t epoch, volatile 
     }
 }
 
+// Runs f(v, cc) on the 8 32-column chunks of this warp's accumulator rows
+// in order.  With kOverlap the TMEM load of chunk cc + 1 is in flight while
+// chunk cc is processed; it is used where the registers of both chunks fit
+// without spilling (ternary weights: one weight scale), since a register
+// spilled between a load and its wait would be read before it is written.
+template <bool kOverlap, typename F>
+__device__ __forceinline__ void pair_chunks(uint32_t tacc, F &&f)
+{
+    constexpr int kChunks = 2 * PBN / 32;
+    static_assert(kChunks % 2 == 0, "chunks are processed in pairs");
+    if constexpr (!kOverlap) {
+#pragma unroll 1
+        for (int cc = 0; cc < kChunks; ++cc) {
+            uint32_t v[32];
+            tmem_ld_32cols(tacc + static_cast<uint32_t>(cc * 32), v);
+            f(v, cc);
+        }
+        return;
+    }
+    uint32_t va[32], vb[32];
+    tmem_ld_32cols(tacc, va);
+#pragma unroll 1
+    for (int cc = 0; cc < kChunks; cc += 2) {
+        tmem_ld_32cols_async(tacc + static_cast<uint32_t>((cc + 1) * 32), vb);
+        f(va, cc);
+        tmem_ld_wait(vb);
+        if (cc + 2 < kChunks) tmem_ld_32cols_async(tacc + static_cast<uint32_t>((cc + 2) * 32), va);
+        f(vb, cc + 1);
+        if (cc + 2 < kChunks) tmem_ld_wait(va);
+    }
+}
+
 template <int FMT, int OUT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_p,
                  const float *__restrict__ s_x, const float *__restrict__ s_w, int64_t M, int64_t N, int64_t K,
-                 void *__restrict__ y, int64_t ldy, int vec_ok, int prefetch, int32_t *status, int split,
+                 void *__restrict__ y, int64_t ldy, int vec_ok, int prefetch, int32_t *status, int64_t dp_tiles,
                  uint32_t epoch)
 {
-    constexpr int ST = pair_tma_stages<FMT>();
-    constexpr int SE = kExpStages;
+    constexpr int ST = pair_tma_stages<FMT, OUT>();
+    constexpr int SE = pair_exp_stages<FMT, OUT>();
     constexpr int PB = packed_bytes_per_kblock<FMT>();
     constexpr int P_BYTES = PBN * PB;
     constexpr int kShift = Fmt<FMT>::kShift;
     static_assert(SE < ST, "an expansion stage is freed through the MMA barrier of an older TMA stage");
+    static_assert(ST * A_BYTES + SE * PE_BYTES >= 4 * kWsWarpVecs * 16, "a partial tile is staged in the rings");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -947,8 +1030,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             bool ok = true;
             uint32_t npre = 0;
             PairUnit u;
+            PairSched sched(pair, num_pairs, num_tiles, nkb, dp_tiles);
             if (prefetch != 0) {
-                if (pair_unit(pair, num_pairs, num_tiles, nkb, split, 0, u)) {
+                PairSched first = sched;
+                if (first.next(u)) {
                     const int n0 = static_cast<int>((u.tile % num_n) * 2 * PBN + rank * PBN);
                     const int nloc = u.kb1 - u.kb0;
                     npre = static_cast<uint32_t>(nloc < ST ? nloc : ST);
@@ -959,7 +1044,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 }
                 pdl_wait();
             }
-            for (int64_t it = 0; ok && pair_unit(pair, num_pairs, num_tiles, nkb, split, it, u); ++it) {
+            while (ok && sched.next(u)) {
                 const int m0 = static_cast<int>((u.tile / num_n) * 2 * PBM + rank * PBM);
                 const int n0 = static_cast<int>((u.tile % num_n) * 2 * PBN + rank * PBN);
                 for (int kb = u.kb0; kb < u.kb1; ++kb, ++g) {
@@ -988,7 +1073,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             uint32_t t = 0;
             bool ok = true;
             PairUnit u;
-            for (int64_t it = 0; ok && pair_unit(pair, num_pairs, num_tiles, nkb, split, it, u); ++it, ++t) {
+            PairSched sched(pair, num_pairs, num_tiles, nkb, dp_tiles);
+            for (; ok && sched.next(u); ++t) {
                 const int b = t & 1;
                 if (!wait_bar(&acc_empty[b], ((t >> 1) & 1u) ^ 1u, abort_flag, status)) { ok = false; break; }
                 tc_fence_after();
@@ -1020,7 +1106,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         uint32_t g = 0;
         bool ok = true;
         PairUnit u;
-        for (int64_t it = 0; ok && pair_unit(pair, num_pairs, num_tiles, nkb, split, it, u); ++it) {
+        PairSched sched(pair, num_pairs, num_tiles, nkb, dp_tiles);
+        while (ok && sched.next(u)) {
             for (int kb = u.kb0; kb < u.kb1; ++kb, ++g) {
                 const int s1 = g % ST, s2 = g % SE;
                 if (!wait_bar(&full_tma[s1], (g / ST) & 1u, abort_flag, status)) { ok = false; break; }
@@ -1044,8 +1131,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         const float sw_tensor = (FMT == kT2) ? s_w[0] : 0.0f;
         uint32_t t = 0;
         PairUnit u;
-        const int row_in = quarter * 32 + lane;  // this thread's token row within the CTA's 128
-        for (int64_t it = 0; pair_unit(pair, num_pairs, num_tiles, nkb, split, it, u); ++it, ++t) {
+        PairSched sched(pair, num_pairs, num_tiles, nkb, dp_tiles);
+        for (; sched.next(u); ++t) {
             const int b = t & 1;
             int ready = 0;
             if (lane == 0) ready = wait_bar(&acc_full[b], (t >> 1) & 1u, abort_flag, status) ? 1 : 0;
@@ -1053,24 +1140,22 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             if (!ready) break;
             tc_fence_after();
             const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * 2 * PBN);
-            if (u.tail >= 0 && u.part > 0) {
-                // a later part of a split tile: publish the partial tile.
-                // Workspace layout per CTA: [chunk][4-column group][row], so
-                // the 32 lanes (rows) of one store write 512 contiguous bytes.
-                const int slot = static_cast<int>(u.tail) * (split - 1) + u.part - 1;
-                uint4 *ws = g_pair_ws[slot] + rank * (PBM * 2 * PBN / 4);
-#pragma unroll 1
-                for (int cc = 0; cc < 2 * PBN / 32; ++cc) {
-                    uint32_t v[32];
-                    tmem_ld_32cols(tacc + static_cast<uint32_t>(cc * 32), v);
+            if (u.kb0 > 0) {
+                // a piece that starts inside its tile: publish the partial
+                // tile in this pair's slot.  Workspace layout per CTA:
+                // [epilogue warp][chunk][4-column group][row], so the 32 lanes
+                // (rows) of one store write 512 contiguous bytes and each
+                // warp's rows are one contiguous 32 KB block.
+                uint4 *ws = g_pair_ws[pair] + rank * (PBM * 2 * PBN / 4) + quarter * kWsWarpVecs;
+                pair_chunks<FMT == kT2>(tacc, [=](const uint32_t(&v)[32], int cc) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
-                        ws[(cc * 8 + j) * PBM + row_in] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-                }
+                        ws[(cc * 8 + j) * 32 + lane] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                });
                 __threadfence();
                 __syncwarp();  // this warp's 32 rows are stored
                 if (lane == 0)
-                    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(&g_pair_flag[slot][rank][quarter]),
+                    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(&g_pair_flag[pair][rank][quarter]),
                                  "r"(epoch)
                                  : "memory");
                 tc_fence_before();
@@ -1078,26 +1163,46 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 if (lane == 0) mbar_arrive_remote(acc_empty_leader + static_cast<uint32_t>(b * 8));
                 continue;
             }
-            // part 0 of a split tile: the other parts' partial tiles are added
-            const int nsum = u.tail >= 0 ? split - 1 : 0;
+            // a piece that starts its tile and ends inside it: the partial
+            // tiles of the pairs after this one complete it.  It is the
+            // pair's last unit, so its MMAs are complete and nothing else
+            // uses the TMA and expansion rings: the first partial tile is
+            // staged there with all of a warp's copies in flight at once
+            // (one round trip instead of one per chunk); further ones are
+            // added from global memory chunk by chunk.
+            const int nsum = u.last >= 0 ? u.last - static_cast<int>(pair) : 0;
             bool have = true;  // every lane acquires the flags of its warp's rows itself
-            for (int p = 0; p < nsum; ++p)
-                have = have && wait_flag(&g_pair_flag[static_cast<int>(u.tail) * (split - 1) + p][rank][quarter],
-                                         epoch, abort_flag, status);
+            for (int p = 1; p <= nsum; ++p)
+                have = have && wait_flag(&g_pair_flag[pair + p][rank][quarter], epoch, abort_flag, status);
+            const uint32_t staged = smem_u32(sA) + static_cast<uint32_t>(quarter * kWsWarpVecs * 16);
+            if (nsum > 0 && have) {
+                const uint4 *ws = g_pair_ws[pair + 1] + rank * (PBM * 2 * PBN / 4) + quarter * kWsWarpVecs;
+#pragma unroll 8
+                for (int i = 0; i < kWsWarpVecs / 32; ++i)
+                    cp_async_16(staged + static_cast<uint32_t>((i * 32 + lane) * 16), ws + i * 32 + lane);
+                cp_async_wait_all();
+            }
             const int64_t m0 = (u.tile / num_n) * 2 * PBM + rank * PBM;
             const int64_t n0 = (u.tile % num_n) * 2 * PBN;
             const int64_t row0 = m0 + quarter * 32;
             const float sx = (row0 + lane < M) ? ld_act_f32(s_x + row0 + lane) : 0.0f;
-#pragma unroll 1
-            for (int cc = 0; cc < 2 * PBN / 32; ++cc) {
+            pair_chunks<FMT == kT2>(tacc, [=](uint32_t(&v)[32], int cc) {
                 const int64_t nc = n0 + cc * 32;
-                uint32_t v[32];
-                tmem_ld_32cols(tacc + static_cast<uint32_t>(cc * 32), v);
-                for (int p = 0; p < nsum && have; ++p) {
-                    const uint4 *ws = g_pair_ws[static_cast<int>(u.tail) * (split - 1) + p] + rank * (PBM * 2 * PBN / 4);
+                if (nsum > 0 && have) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        const uint4 a = ld_act_u4(ws + (cc * 8 + j) * PBM + row_in);
+                        const uint4 a = lds128(staged + static_cast<uint32_t>(((cc * 8 + j) * 32 + lane) * 16));
+                        v[4 * j] += a.x;
+                        v[4 * j + 1] += a.y;
+                        v[4 * j + 2] += a.z;
+                        v[4 * j + 3] += a.w;
+                    }
+                }
+                for (int p = 2; p <= nsum && have; ++p) {
+                    const uint4 *ws = g_pair_ws[pair + p] + rank * (PBM * 2 * PBN / 4) + quarter * kWsWarpVecs;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint4 a = ld_act_u4(ws + (cc * 8 + j) * 32 + lane);
                         v[4 * j] += a.x;
                         v[4 * j + 1] += a.y;
                         v[4 * j + 2] += a.z;
@@ -1111,7 +1216,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                         sw[i] = (FMT == kT2) ? sw_tensor : ((nc + i < N) ? __ldg(s_w + nc + i) : 0.0f);
                     epilogue_chunk<OUT>(v, sw, sx, kShift, y, ldy, row0, M, nc, N, vec_ok != 0, stage, lane);
                 }
-            }
+            });
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(acc_empty_leader + static_cast<uint32_t>(b * 8));
@@ -1155,13 +1260,12 @@ lowbit_status launch_pair_t(const CUtensorMap &ma, const CUtensorMap &mp, const 
     if (resident <= 0) return LOWBIT_ERR_CUDA;
     const int64_t tiles = ((M + 2 * PBM - 1) / (2 * PBM)) * ((N + 2 * PBN - 1) / (2 * PBN));
     int64_t pairs = tiles < resident ? tiles : resident;
-    int split = 1;
-    if (exclusive) pair_split(tiles, resident, (K + BK - 1) / BK, split, pairs);
-    static std::atomic<uint32_t> epochs{0};
-    uint32_t epoch = epochs.fetch_add(1, std::memory_order_relaxed) + 1;
-    if (epoch == 0) epoch = epochs.fetch_add(1, std::memory_order_relaxed) + 1;  // 0 is the flags' initial value
+    int64_t dp_tiles = tiles;
+    if (exclusive) pair_plan(tiles, resident, (K + BK - 1) / BK, dp_tiles, pairs);
+    uint32_t epoch = g_pair_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
+    if (epoch == 0) epoch = g_pair_epoch.fetch_add(1, std::memory_order_relaxed) + 1;  // 0 is the flags' initial value
     return launch_pdl(gemm_pair_kernel<FMT, OUT>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kThreads), smem, st,
-                      0, ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, split, epoch);
+                      0, ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, dp_tiles, epoch);
 }
 
 template <int FMT>

@@ -386,42 +386,53 @@ def test_stream_split_bf16_bit_exact(fmt):
     assert np.array_equal(bf16_bits(y), oracle.rescale(acc, s_w, s_x, "bf16"))
 
 
-# LOWBIT_LINEAR_EXCLUSIVE: the SM-pair GEMM (path 6) splits each tile of a
-# partial last round along K over idle pairs (parts of at least 16 K blocks)
-# and adds the int32 partial tiles through a device workspace.  Shapes: 24
-# last-round tiles of 320 split 3 ways (8192, 2560, 9728); no whole round, 6
-# ragged tiles x 2 parts of 16 K blocks (300, 700, 4096); 8 tiles x 8 parts
-# (512, 1000, 16384); 4 tiles of 152 that stay whole (1024, 9728, 2560: 20 K
-# blocks).  The output must equal the unsplit launch bit for bit, and the
-# oracle on sampled rows (every row of the small shapes).
-PAIR_SPLIT_SHAPES = [(8192, 2560, 9728), (300, 700, 4096), (512, 1000, 16384), (1024, 9728, 2560)]
+# LOWBIT_LINEAR_EXCLUSIVE: when the SM-pair GEMM (path 6) would end on a
+# partial round, it shares the K blocks of the remaining tiles evenly over the
+# pairs (stream-K) and adds the int32 partial tiles through a device
+# workspace.  Schedules on 74 pairs: 17 whole rounds, the tail not shared
+# (8192, 9728, 2560: 16 rounds + 32 tiles of 20 K blocks, where sharing does
+# not pay); 3 rounds, then 98 tiles of 76 blocks (8192,
+# 2560, 9728); 40 tiles of 76 blocks, no whole round (1024, 2560, 9728); one
+# round, then 78 tiles of 20 (1024, 9728, 2560); 6 ragged tiles of 32 blocks
+# on 24 pairs, 3 partial tiles added per tile (300, 700, 4096); 8 tiles of 128
+# blocks (512, 1000, 16384); 9 tiles of 6 blocks, no split (768, 768, 768).
+# Each launch gets its own activations and output dtype, so that a partial
+# tile or flag left by an earlier launch cannot pass for this one's; the
+# output must equal the unsplit launch bit for bit, and the oracle on
+# sampled rows (every row of the small shapes).
+PAIR_SPLIT_SHAPES = [(8192, 9728, 2560), (8192, 2560, 9728), (1024, 2560, 9728), (1024, 9728, 2560),
+                     (300, 700, 4096), (512, 1000, 16384), (768, 768, 768)]
 
 
-@pytest.mark.parametrize("M,N,K", PAIR_SPLIT_SHAPES, ids=str)
-def test_pair_last_round_split_bit_exact(M, N, K):
-    fmt = bwt.TERNARY2
+@pytest.mark.parametrize("M,N,K,fmt", [s + (bwt.TERNARY2,) for s in PAIR_SPLIT_SHAPES]
+                         + [(300, 700, 4096, f) for f in (bwt.BINARY1, bwt.INT4)]
+                         + [(1024, 2560, 9728, f) for f in (bwt.BINARY1, bwt.INT4)], ids=str)
+def test_pair_stream_k_bit_exact(M, N, K, fmt):
     w = wls.normal_weights(1100 + M + K, N, K)
-    x = wls.normal_activations(1101 + M + K, M, K, 0.01, 8.0)
     packed, s_w = gpu_pack(w, fmt)
-    q, s_x = gpu_act(x, False)
+    xs = [wls.normal_activations(1101 + M + K + i, M, K, 0.01, 8.0) for i in range(3)]
+    acts = [gpu_act(x, False) for x in xs]
     st = status_word()
+    outs = [bwt.I32, bwt.BF16, bwt.I32]
     ys = {}
     for exclusive in (False, True, True):  # twice split: the epoch flags must not carry over
-        for out in (bwt.I32, bwt.BF16):
-            ys[(exclusive, out)] = bwt.lowbit_linear(q, s_x, packed, s_w, fmt, N, out, K=K, status=st, path=6,
-                                                     exclusive=exclusive)
+        for i, out in enumerate(outs):
+            q, s_x = acts[i]
+            ys[(exclusive, i)] = bwt.lowbit_linear(q, s_x, packed, s_w, fmt, N, out, K=K, status=st, path=6,
+                                                   exclusive=exclusive)
     torch.cuda.synchronize()
     assert st.item() == 0
-    for out in (bwt.I32, bwt.BF16):
-        assert torch.equal(ys[(True, out)], ys[(False, out)])
+    for i in range(len(outs)):
+        assert torch.equal(ys[(True, i)], ys[(False, i)])
     codes, _ = oracle.quantize(w, fmt, 1e-5)
-    q_o, _ = oracle.act_quant(x, 0.0)
     rows = np.arange(M)
     if M * N * K > 2e9:  # first and last row of every 256-row tile, and random rows
         rng = np.random.default_rng(1102)
         rows = np.unique(np.concatenate([np.arange(0, M, 256), np.arange(255, M, 256), rng.choice(M, 64)]))
-    acc = oracle.int_dot(q_o[rows], codes, fmt, nthreads=oracle.max_threads())
-    assert np.array_equal(ys[(True, bwt.I32)].cpu().numpy()[rows].astype(np.int64), acc)
+    for i in (0, 2):
+        q_o, _ = oracle.act_quant(xs[i], 0.0)
+        acc = oracle.int_dot(q_o[rows], codes, fmt, nthreads=oracle.max_threads())
+        assert np.array_equal(ys[(True, i)].cpu().numpy()[rows].astype(np.int64), acc)
 
 
 # LOWBIT_LINEAR_WEIGHTS_STABLE: weight reads start before the wait for the
