@@ -97,6 +97,15 @@ constexpr int kDeepVPT = 5, kDeepThreads = 1536;
 constexpr int kOptGain = 1;
 constexpr int kOptNorm = 2;
 
+// Resident threads of a build.  With the gain, rows keep x g as fp32 between
+// the passes (twice the registers of a 16-bit row), so both builds run 1024
+// threads (64 registers).
+template <typename T, int OPT>
+__host__ __device__ constexpr int build_threads(bool deep)
+{
+    return (OPT & kOptGain) != 0 ? 1024 : (deep ? kDeepThreads : kWideThreads);
+}
+
 // Element i of a 16-byte vector of x, times the gain when GAIN.
 template <typename T, bool GAIN>
 __device__ __forceinline__ float elem(const uint4 &b, const float *gv, int i)
@@ -107,7 +116,7 @@ __device__ __forceinline__ float elem(const uint4 &b, const float *gv, int i)
 }
 
 // The E gains of vector v (E = 4 or 8 floats, one or two 16-byte loads,
-// through L1: every row of the grid reads the same gains, twice).
+// through L1: every row of the grid reads the same gains).
 template <int E>
 __device__ __forceinline__ void load_gain(const float *g, int64_t v, float (&gv)[8])
 {
@@ -161,6 +170,10 @@ act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
     const char *xrow = static_cast<const char *>(x) + (live ? row : 0) * ldx * sizeof(T);
 
     uint4 buf[VPT];
+    // With the gain, u = x g is kept from the first pass for the second, so
+    // the gains are read once (the L1 reads of the gains, twice per element,
+    // bounded the kernel).
+    float uf[GAIN ? VPT : 1][GAIN ? E : 1];
     uint32_t amax = 0;
     double ss = 0.0;
     float gv[8];
@@ -173,7 +186,9 @@ act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
                 if constexpr (GAIN) load_gain<E>(g, v, gv);
 #pragma unroll
                 for (int e = 0; e < E; ++e) {
-                    amax = max(amax, __float_as_uint(elem<T, GAIN>(buf[i], gv, e)) & 0x7fffffffu);
+                    const float u = elem<T, GAIN>(buf[i], gv, e);
+                    if constexpr (GAIN) uf[i][e] = u;
+                    amax = max(amax, __float_as_uint(u) & 0x7fffffffu);
                     if constexpr (NORM) {
                         const double xd = static_cast<double>(In<T>::get(buf[i], e));
                         ss = __fma_rn(xd, xd, ss);
@@ -212,26 +227,26 @@ act_quant_regs(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, fl
         const int64_t v = r + static_cast<int64_t>(i) * TPR;
         if (v < nvec) {
             const uint4 &b = buf[i];
-            if constexpr (GAIN) load_gain<E>(g, v, gv);
+            // u_e: element e of this vector (times its gain)
+            auto ue = [&](int e) {
+                if constexpr (GAIN) return uf[i][e];
+                else return elem<T, false>(b, gv, e);
+            };
             if constexpr (E == 4) {
                 bool near = slow;
-                const float u0 = elem<T, GAIN>(b, gv, 0), u1 = elem<T, GAIN>(b, gv, 1);
-                const float u2 = elem<T, GAIN>(b, gv, 2), u3 = elem<T, GAIN>(b, gv, 3);
+                const float u0 = ue(0), u1 = ue(1);
+                const float u2 = ue(2), u3 = ue(3);
                 uint32_t out = quant4(u0, u1, u2, u3, c, near);
                 if (near) out = quant4_exact(u0, u1, u2, u3, d);
                 if (amax == 0) out = 0;
                 *reinterpret_cast<uint32_t *>(qrow + v * 4) = out;
             } else {
                 bool near = slow;
-                uint32_t lo = quant4(elem<T, GAIN>(b, gv, 0), elem<T, GAIN>(b, gv, 1), elem<T, GAIN>(b, gv, 2),
-                                     elem<T, GAIN>(b, gv, 3), c, near);
-                uint32_t hi = quant4(elem<T, GAIN>(b, gv, 4), elem<T, GAIN>(b, gv, 5), elem<T, GAIN>(b, gv, 6),
-                                     elem<T, GAIN>(b, gv, 7), c, near);
+                uint32_t lo = quant4(ue(0), ue(1), ue(2), ue(3), c, near);
+                uint32_t hi = quant4(ue(4), ue(5), ue(6), ue(7), c, near);
                 if (near) {
-                    lo = quant4_exact(elem<T, GAIN>(b, gv, 0), elem<T, GAIN>(b, gv, 1), elem<T, GAIN>(b, gv, 2),
-                                      elem<T, GAIN>(b, gv, 3), d);
-                    hi = quant4_exact(elem<T, GAIN>(b, gv, 4), elem<T, GAIN>(b, gv, 5), elem<T, GAIN>(b, gv, 6),
-                                      elem<T, GAIN>(b, gv, 7), d);
+                    lo = quant4_exact(ue(0), ue(1), ue(2), ue(3), d);
+                    hi = quant4_exact(ue(4), ue(5), ue(6), ue(7), d);
                 }
                 if (amax == 0) lo = hi = 0;
                 *reinterpret_cast<uint2 *>(qrow + v * 8) = make_uint2(lo, hi);
@@ -612,11 +627,11 @@ lowbit_status launch(const void *x, int64_t M, int64_t K, int64_t ldx, float eps
 #define LOWBIT_AQ_OPT(TPR, OPT)                                                                                  \
     if (opt == OPT) {                                                                                            \
         if (deep)                                                                                                \
-            return launch_pdl(act_quant_regs<T, TPR, kDeepVPT, kDeepThreads, OPT>, dim3(grid),                   \
+            return launch_pdl(act_quant_regs<T, TPR, kDeepVPT, build_threads<T, OPT>(true), OPT>, dim3(grid),    \
                               dim3(block_threads(TPR)), 0, st, 0, x, M, K, ldx, eps, q, ldq, s_x, status, g,     \
                               eps_norm);                                                                         \
-        return launch_pdl(act_quant_regs<T, TPR, kWideVPT, kWideThreads, OPT>, dim3(grid), dim3(block_threads(TPR)), \
-                          0, st, 0, x, M, K, ldx, eps, q, ldq, s_x, status, g, eps_norm);                        \
+        return launch_pdl(act_quant_regs<T, TPR, kWideVPT, build_threads<T, OPT>(false), OPT>, dim3(grid),       \
+                          dim3(block_threads(TPR)), 0, st, 0, x, M, K, ldx, eps, q, ldq, s_x, status, g, eps_norm); \
     }
 #define LOWBIT_AQ(TPR)                                                                                           \
     if (tpr == TPR) {                                                                                            \
