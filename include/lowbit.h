@@ -300,12 +300,14 @@ lowbit_status lowbit_linear_path(const int8_t *q, int64_t ldq, const float *s_x,
 /* Flag for lowbit_linear_ex: the caller guarantees that no other SM-pair GEMM
  * of this library runs on the device while this call's kernels run (for
  * example: all linear layers are issued on one stream).  The SM-pair GEMM
- * (ternary weights from 512 tokens) then splits each tile of its last,
- * partial round of tiles along K over the SM pairs that would otherwise
- * idle: parts 1.. store their int32 partial tiles in a workspace shared by
- * the device (24 MB of static device memory) and the first part adds them
- * (exact) before the epilogue.  Concurrent GEMMs would share that
- * workspace, hence the flag.  Results are identical with and without it. */
+ * (ternary weights from 512 tokens) may then share the K blocks of the
+ * tiles of its last, partial round (plus one whole round) evenly over all
+ * SM pairs (stream-K): a pair whose piece starts inside a tile stores its
+ * int32 partial tile in a workspace shared by the device (24 MB of static
+ * device memory), and the pair holding the tile's first K blocks adds the
+ * partial tiles (exact) before the epilogue.  Concurrent GEMMs would share
+ * that workspace, hence the flag.  Results are identical with and without
+ * it. */
 #define LOWBIT_LINEAR_EXCLUSIVE 2u
 
 /* lowbit_linear_path with launch flags (0 or any of LOWBIT_LINEAR_WEIGHTS_STABLE,
