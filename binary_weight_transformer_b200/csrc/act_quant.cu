@@ -375,23 +375,24 @@ act_prologue_staged(const void *__restrict__ x, int64_t M, int64_t K, int64_t ld
 // token row; warp w holds the 512-feature chunks w, w + 8, ... of the row,
 // lane l features 16l..16l+15 of each.  Every hb-feature block lies inside
 // one chunk (512 / hb is whole), so the stages h < 16 of its transform run
-// within a lane and the stages 16 <= h < hb across lanes (partner lane
-// l ^ h/16), with the staged kernel's fp32 additions and subtractions in
-// the same order: bit-identical values, without shared memory or a barrier
-// per stage.  Then the row maximum (and the sum of squares) over the block,
+// within a lane; for the stages 16 <= h < hb the chunk is transposed through
+// a per-warp shared-memory buffer, leaving one stage across lanes.  The
+// staged kernel's fp32 additions and subtractions run in the same order:
+// bit-identical values, with no barrier per stage.  Then the row maximum (and the sum of squares) over the block,
 // the codes from registers (the fast rule of quant_rule.cuh) and the scale;
 // `mode` as act_prologue_staged.
 constexpr int kFwhtChunks = 3;
 constexpr int64_t kFwhtMaxK = static_cast<int64_t>(kFwhtChunks) * 8 * 512;
 
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 3)
 act_prologue_fwht(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, const float *__restrict__ g,
                   int norm, float eps_norm, int hb, int8_t *__restrict__ q, int64_t ldq, float *__restrict__ s_x,
                   int32_t *status, int mode, float *__restrict__ stat_max, double *__restrict__ stat_ss)
 {
     __shared__ uint32_t red[8];
     __shared__ double red_ss[8];
+    __shared__ float fwht_sm[8 * 512];  // one 512-feature chunk per warp
     pdl_wait();
     pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -463,15 +464,57 @@ act_prologue_fwht(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx,
                 u[c][e + h] = __fsub_rn(a, b);
             }
         }
-        // stages 16 <= h < hb across lanes: the lane with bit h/16 clear
-        // holds a, its partner b; (a, b) -> (a + b, a - b)
-        for (int h = 16; h < hb; h <<= 1) {
-            const int lm = h >> 4;
-            const bool upper = (lane & lm) != 0;
+        // stages 16 <= h < hb: the chunk moves through shared memory so that
+        // lane l holds features 32 j + l (j = 0..15).  Stage 16 then pairs
+        // lane l with lane l ^ 16 (the lane with bit 16 clear holds a, its
+        // partner b; (a, b) -> (a + b, a - b)), and stages 32.. pair t[j]
+        // with t[j ^ h/32] inside the lane; the chunk moves back for the
+        // codes.  Feature f is stored at f ^ (f >> 5), which keeps both the
+        // row-wise writes and the column-wise reads free of bank conflicts.
+        if (hb > 16) {
+            float *sw = fwht_sm + warp * 512;
+            __syncwarp();  // the previous chunk's reads are done
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-                const float other = __shfl_xor_sync(0xffffffffu, u[c][e], lm);
-                u[c][e] = upper ? __fsub_rn(other, u[c][e]) : __fadd_rn(u[c][e], other);
+                const int f = 16 * lane + e;
+                sw[f ^ (f >> 5)] = u[c][e];
+            }
+            __syncwarp();
+            float t[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int f = 32 * j + lane;
+                t[j] = sw[f ^ (f >> 5)];
+            }
+            const bool upper = (lane & 16) != 0;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float other = __shfl_xor_sync(0xffffffffu, t[j], 16);
+                t[j] = upper ? __fsub_rn(other, t[j]) : __fadd_rn(t[j], other);
+            }
+#pragma unroll
+            for (int h = 32; h < 512; h <<= 1) {
+                if (h >= hb) break;
+                const int jm = h >> 5;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    if (j & jm) continue;
+                    const float a = t[j], b = t[j + jm];
+                    t[j] = __fadd_rn(a, b);
+                    t[j + jm] = __fsub_rn(a, b);
+                }
+            }
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int f = 32 * j + lane;
+                sw[f ^ (f >> 5)] = t[j];
+            }
+            __syncwarp();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int f = 16 * lane + e;
+                u[c][e] = sw[f ^ (f >> 5)];
             }
         }
 #pragma unroll

@@ -115,30 +115,48 @@ __global__ void row_reduce(const float *__restrict__ w, int64_t N, int64_t K, in
     if (bad) report(status, LOWBIT_ERR_NONFINITE);
 }
 
-// Ternary gamma: one thread sums the row sums in order n = 0..N-1.
+// Ternary gamma: the row sums added in order n = 0..N-1.  One warp: the
+// lanes load 32 consecutive row sums at a time and every lane adds them in
+// order from shuffles (the same additions in the same order in every lane),
+// so the loads are not serialised behind the additions.
 __global__ void ternary_gamma(const double *__restrict__ rows, int64_t N, int64_t K, float *s_w)
 {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    if (blockIdx.x != 0 || threadIdx.x >= 32) return;
+    const int lane = threadIdx.x;
     double S = 0.0;
-    for (int64_t n = 0; n < N; ++n) S = __dadd_rn(S, rows[n]);
-    s_w[0] = __double2float_rn(__ddiv_rn(S, static_cast<double>(N) * static_cast<double>(K)));
+    for (int64_t n0 = 0; n0 < N; n0 += 32) {
+        const double v = n0 + lane < N ? rows[n0 + lane] : 0.0;
+        const int cnt = N - n0 < 32 ? static_cast<int>(N - n0) : 32;
+        for (int i = 0; i < cnt; ++i) S = __dadd_rn(S, __shfl_sync(0xffffffffu, v, i));
+    }
+    if (lane == 0) s_w[0] = __double2float_rn(__ddiv_rn(S, static_cast<double>(N) * static_cast<double>(K)));
 }
 
-// Centred binary scalars: one thread sums the row sums in order n = 0..N-1;
-// alpha = mean(W) and beta = mean|W|, each the fp64 mean rounded once to fp32,
-// stored as two floats after the 2N row sums.
+// Centred binary scalars: the row sums added in order n = 0..N-1 (one warp,
+// as ternary_gamma); alpha = mean(W) and beta = mean|W|, each the fp64 mean
+// rounded once to fp32, stored as two floats after the 2N row sums.
 __global__ void centred_scalars(double *__restrict__ rows, int64_t N, int64_t K)
 {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    if (blockIdx.x != 0 || threadIdx.x >= 32) return;
+    const int lane = threadIdx.x;
     double S = 0.0, A = 0.0;
-    for (int64_t n = 0; n < N; ++n) {
-        S = __dadd_rn(S, rows[n]);
-        A = __dadd_rn(A, rows[N + n]);
+    for (int64_t n0 = 0; n0 < N; n0 += 32) {
+        const bool in = n0 + lane < N;
+        const double v = in ? rows[n0 + lane] : 0.0;
+        const double a = in ? rows[N + n0 + lane] : 0.0;
+        const int cnt = N - n0 < 32 ? static_cast<int>(N - n0) : 32;
+        for (int i = 0; i < cnt; ++i) {
+            S = __dadd_rn(S, __shfl_sync(0xffffffffu, v, i));
+            A = __dadd_rn(A, __shfl_sync(0xffffffffu, a, i));
+        }
     }
-    const double nk = static_cast<double>(N) * static_cast<double>(K);
-    float *out = reinterpret_cast<float *>(rows + 2 * N);
-    out[0] = __double2float_rn(__ddiv_rn(S, nk));
-    out[1] = __double2float_rn(__ddiv_rn(A, nk));
+    __syncwarp();  // every lane has read its row sums before lane 0 writes after them
+    if (lane == 0) {
+        const double nk = static_cast<double>(N) * static_cast<double>(K);
+        float *out = reinterpret_cast<float *>(rows + 2 * N);
+        out[0] = __double2float_rn(__ddiv_rn(S, nk));
+        out[1] = __double2float_rn(__ddiv_rn(A, nk));
+    }
 }
 
 // BitNet v1 centred codes in the binary layout: bit 0 (+1) where w > alpha,
