@@ -371,85 +371,95 @@ act_prologue_staged(const void *__restrict__ x, int64_t M, int64_t K, int64_t ld
 }
 
 // The Hadamard prologue in registers, for blocks of at most 512 features and
-// rows of at most kFwhtChunks * 8 * 512 features: one block of 8 warps per
-// token row; warp w holds the 512-feature chunks w, w + 8, ... of the row,
-// lane l features 16l..16l+15 of each.  Every hb-feature block lies inside
-// one chunk (512 / hb is whole), so the stages h < 16 of its transform run
+// rows of at most kFwhtMaxK features: one block per token row with one warp
+// per 512-feature chunk (ceil(K / 512) warps); lane l holds features
+// 16l..16l+15 of its warp's chunk.  Every hb-feature block lies inside one
+// chunk (512 / hb is whole), so the stages h < 16 of its transform run
 // within a lane; for the stages 16 <= h < hb the chunk is transposed through
-// a per-warp shared-memory buffer, leaving one stage across lanes.  The
-// staged kernel's fp32 additions and subtractions run in the same order:
-// bit-identical values, with no barrier per stage.  Then the row maximum (and the sum of squares) over the block,
-// the codes from registers (the fast rule of quant_rule.cuh) and the scale;
-// `mode` as act_prologue_staged.
-constexpr int kFwhtChunks = 3;
-constexpr int64_t kFwhtMaxK = static_cast<int64_t>(kFwhtChunks) * 8 * 512;
+// the warp's 2 KB of dynamic shared memory, leaving one stage across lanes.
+// The staged kernel's fp32 additions and subtractions run in the same order:
+// bit-identical values, with no barrier per stage.  Then the row maximum
+// (and the sum of squares) over the block, the codes from registers (the
+// fast rule of quant_rule.cuh) and the scale; `mode` as act_prologue_staged.
+// One chunk per warp keeps the registers low (about 40 warps resident per SM
+// at 4B-class rows; the earlier build with up to three chunks per warp of 8
+// ran 24).
+constexpr int kFwhtMaxWarps = 32;
+constexpr int64_t kFwhtMaxK = static_cast<int64_t>(kFwhtMaxWarps) * 512;
+// Rows of at most 20 chunks take a build bounded to two 640-thread blocks per
+// SM (48 registers): 38 warps resident at K = 9728 instead of 19.
+constexpr int kFwhtWarpsTwo = 20;
+constexpr int kFwhtWarpFloats = 512 + 16;  // a chunk with one float of padding per 32
 
-template <typename T>
-__global__ void __launch_bounds__(256, 3)
+template <typename T, int MAXW>
+__global__ void __launch_bounds__(MAXW * 32, MAXW <= kFwhtWarpsTwo ? 2 : 1)
 act_prologue_fwht(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx, const float *__restrict__ g,
                   int norm, float eps_norm, int hb, int8_t *__restrict__ q, int64_t ldq, float *__restrict__ s_x,
                   int32_t *status, int mode, float *__restrict__ stat_max, double *__restrict__ stat_ss)
 {
-    __shared__ uint32_t red[8];
-    __shared__ double red_ss[8];
-    __shared__ float fwht_sm[8 * 512];  // one 512-feature chunk per warp
+    __shared__ uint32_t red[kFwhtMaxWarps];
+    __shared__ double red_ss[kFwhtMaxWarps];
+    extern __shared__ float fwht_sm[];  // kFwhtWarpFloats per warp
     pdl_wait();
     pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nw = static_cast<int>(blockDim.x >> 5);
     const int64_t row = blockIdx.x;
     const char *xrow = static_cast<const char *>(x) + row * ldx * static_cast<int64_t>(sizeof(T));
     const bool xvec = (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (ldx * static_cast<int64_t>(sizeof(T))) % 16 == 0;
     const bool gvec = g == nullptr || (reinterpret_cast<uintptr_t>(g) & 15u) == 0;
-    float u[kFwhtChunks][16];
+    float u[16];
     double ss = 0.0;
     uint32_t amax = 0;
+    const int64_t chunk = warp;
+    const int64_t k0 = (chunk * 32 + lane) * 16;
+    {
+        // the gains are requested before x, so their round trip overlaps
+        // x's instead of following the first use of x
+        const bool gv = g != nullptr && gvec && k0 + 16 <= K;
+        uint4 gw[4];
+        if (gv) {
 #pragma unroll
-    for (int c = 0; c < kFwhtChunks; ++c) {
-        const int64_t chunk = warp + 8 * c;
-        if (chunk * 512 >= K) {  // the same for the whole warp
-#pragma unroll
-            for (int e = 0; e < 16; ++e) u[c][e] = 0.0f;
-            continue;
+            for (int v = 0; v < 4; ++v) gw[v] = ld_act_ca_u4(g + k0 + 4 * v);
         }
-        const int64_t k0 = (chunk * 32 + lane) * 16;
         if (xvec && k0 + 16 <= K) {
             if constexpr (sizeof(T) == 2) {
 #pragma unroll
                 for (int v = 0; v < 2; ++v) {
                     const uint4 w = ld_act_u4(xrow + 2 * (k0 + 8 * v));
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) u[c][8 * v + e] = In<T>::get(w, e);
+                    for (int e = 0; e < 8; ++e) u[8 * v + e] = In<T>::get(w, e);
                 }
             } else {
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
                     const uint4 w = ld_act_u4(xrow + 4 * (k0 + 4 * v));
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) u[c][4 * v + e] = In<T>::get(w, e);
+                    for (int e = 0; e < 4; ++e) u[4 * v + e] = In<T>::get(w, e);
                 }
             }
         } else {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) u[c][e] = k0 + e < K ? In<T>::scalar(xrow, k0 + e) : 0.0f;
+            for (int e = 0; e < 16; ++e) u[e] = k0 + e < K ? In<T>::scalar(xrow, k0 + e) : 0.0f;
         }
         if (norm) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) ss = __fma_rn(static_cast<double>(u[c][e]), static_cast<double>(u[c][e]), ss);
+            for (int e = 0; e < 16; ++e) ss = __fma_rn(static_cast<double>(u[e]), static_cast<double>(u[e]), ss);
         }
         if (g != nullptr) {
-            if (gvec && k0 + 16 <= K) {
+            if (gv) {
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
-                    const uint4 w = ld_act_ca_u4(g + k0 + 4 * v);
-                    u[c][4 * v] = __fmul_rn(u[c][4 * v], __uint_as_float(w.x));
-                    u[c][4 * v + 1] = __fmul_rn(u[c][4 * v + 1], __uint_as_float(w.y));
-                    u[c][4 * v + 2] = __fmul_rn(u[c][4 * v + 2], __uint_as_float(w.z));
-                    u[c][4 * v + 3] = __fmul_rn(u[c][4 * v + 3], __uint_as_float(w.w));
+                    const uint4 w = gw[v];
+                    u[4 * v] = __fmul_rn(u[4 * v], __uint_as_float(w.x));
+                    u[4 * v + 1] = __fmul_rn(u[4 * v + 1], __uint_as_float(w.y));
+                    u[4 * v + 2] = __fmul_rn(u[4 * v + 2], __uint_as_float(w.z));
+                    u[4 * v + 3] = __fmul_rn(u[4 * v + 3], __uint_as_float(w.w));
                 }
             } else {
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                    if (k0 + e < K) u[c][e] = __fmul_rn(u[c][e], ld_act_f32(g + k0 + e));
+                    if (k0 + e < K) u[e] = __fmul_rn(u[e], ld_act_f32(g + k0 + e));
             }
         }
         // the transform of every hb-feature block: stages h < 16 in the lane
@@ -459,9 +469,9 @@ act_prologue_fwht(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx,
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 if (e & h) continue;
-                const float a = u[c][e], b = u[c][e + h];
-                u[c][e] = __fadd_rn(a, b);
-                u[c][e + h] = __fsub_rn(a, b);
+                const float a = u[e], b = u[e + h];
+                u[e] = __fadd_rn(a, b);
+                u[e + h] = __fsub_rn(a, b);
             }
         }
         // stages 16 <= h < hb: the chunk moves through shared memory so that
@@ -469,28 +479,28 @@ act_prologue_fwht(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx,
         // lane l with lane l ^ 16 (the lane with bit 16 clear holds a, its
         // partner b; (a, b) -> (a + b, a - b)), and stages 32.. pair t[j]
         // with t[j ^ h/32] inside the lane; the chunk moves back for the
-        // codes.  Feature f is stored at f ^ (f >> 5), which keeps both the
-        // row-wise writes and the column-wise reads free of bank conflicts.
+        // codes.  Feature f is stored at f + f / 32 (one float of padding per
+        // 32): the row-wise writes (16 l + e) and the column-wise reads
+        // (32 j + l) are both free of bank conflicts, and both address a
+        // per-lane base plus a constant.
         if (hb > 16) {
-            float *sw = fwht_sm + warp * 512;
+            float *sw = fwht_sm + warp * kFwhtWarpFloats;
+            float *wr = sw + 16 * lane + (lane >> 1);  // feature 16 lane + e at wr[e]
+            float *rd = sw + lane;                     // feature 32 j + lane at rd[33 j]
             __syncwarp();  // the previous chunk's reads are done
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int f = 16 * lane + e;
-                sw[f ^ (f >> 5)] = u[c][e];
-            }
+            for (int e = 0; e < 16; ++e) wr[e] = u[e];
             __syncwarp();
             float t[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int f = 32 * j + lane;
-                t[j] = sw[f ^ (f >> 5)];
-            }
-            const bool upper = (lane & 16) != 0;
+            for (int j = 0; j < 16; ++j) t[j] = rd[33 * j];
+            // a + b in the lower lane, a - b = b * -1 + a in the upper one: one
+            // fused multiply-add by +-1 is exact before its single rounding
+            const float sgn = (lane & 16) != 0 ? -1.0f : 1.0f;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const float other = __shfl_xor_sync(0xffffffffu, t[j], 16);
-                t[j] = upper ? __fsub_rn(other, t[j]) : __fadd_rn(t[j], other);
+                t[j] = __fmaf_rn(sgn, t[j], other);
             }
 #pragma unroll
             for (int h = 32; h < 512; h <<= 1) {
@@ -506,19 +516,13 @@ act_prologue_fwht(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx,
             }
             __syncwarp();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int f = 32 * j + lane;
-                sw[f ^ (f >> 5)] = t[j];
-            }
+            for (int j = 0; j < 16; ++j) rd[33 * j] = t[j];
             __syncwarp();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int f = 16 * lane + e;
-                u[c][e] = sw[f ^ (f >> 5)];
-            }
+            for (int e = 0; e < 16; ++e) u[e] = wr[e];
         }
 #pragma unroll
-        for (int e = 0; e < 16; ++e) amax = max(amax, __float_as_uint(u[c][e]) & 0x7fffffffu);
+        for (int e = 0; e < 16; ++e) amax = max(amax, __float_as_uint(u[e]) & 0x7fffffffu);
     }
     // the row's maximum and sum of squares over the block (fixed tree order)
 #pragma unroll
@@ -531,12 +535,14 @@ act_prologue_fwht(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx,
         red_ss[warp] = ss;
     }
     __syncthreads();
-    amax = red[0];
-    ss = red_ss[0];
+    // every warp reduces the warps' partials with the same shuffle tree (lane
+    // w holds warp w's), so all threads get the same maximum and sum
+    amax = lane < nw ? red[lane] : 0u;
+    ss = lane < nw ? red_ss[lane] : 0.0;
 #pragma unroll
-    for (int w = 1; w < 8; ++w) {
-        amax = max(amax, red[w]);
-        if (norm) ss = __dadd_rn(ss, red_ss[w]);
+    for (int o = 16; o > 0; o >>= 1) {
+        amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if (norm) ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
     }
     if (mode == kStagedStats) {
         if (threadIdx.x == 0) {
@@ -558,18 +564,13 @@ act_prologue_fwht(const void *__restrict__ x, int64_t M, int64_t K, int64_t ldx,
     const float c127 = __fmul_rn(127.0f, __frcp_rn(gm));
     const bool slow = !(gm >= 0x1p-121f && gm < 0x1p126f);
     int8_t *qrow = q + row * ldq;
-#pragma unroll
-    for (int c = 0; c < kFwhtChunks; ++c) {
-        const int64_t chunk = warp + 8 * c;
-        if (chunk * 512 >= K) continue;
-        const int64_t k0 = (chunk * 32 + lane) * 16;
-        if (k0 >= K) continue;
+    if (k0 < K) {
         uint32_t wq[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             bool near = slow;
-            wq[e] = quant4(u[c][4 * e], u[c][4 * e + 1], u[c][4 * e + 2], u[c][4 * e + 3], c127, near);
-            if (near) wq[e] = quant4_exact(u[c][4 * e], u[c][4 * e + 1], u[c][4 * e + 2], u[c][4 * e + 3], gm);
+            wq[e] = quant4(u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3], c127, near);
+            if (near) wq[e] = quant4_exact(u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3], gm);
             if (amax == 0) wq[e] = 0;
         }
         if (k0 + 16 <= K) {
@@ -611,12 +612,26 @@ lowbit_status launch_staged(const void *x, int64_t M, int64_t K, int64_t ldx, co
                             double *row_ss = nullptr)
 {
     // blocks of at most 512 features in rows of at most kFwhtMaxK: registers
-    if (hb >= 2 && hb <= 512 && K <= kFwhtMaxK)
-        return launch_pdl(act_prologue_fwht<T>, dim3(static_cast<unsigned>(M)), dim3(256), 0, st, 0, x, M, K, ldx, g,
-                          norm, eps_norm, hb, q, ldq, s_x, status, mode, row_max, row_ss);
-    static PerDevice configured;  // the shared-memory limit is raised once per device
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    if (hb >= 2 && hb <= 512 && K <= kFwhtMaxK) {
+        const int warps = static_cast<int>((K + 511) / 512);
+        if (warps <= kFwhtWarpsTwo)
+            return launch_pdl(act_prologue_fwht<T, kFwhtWarpsTwo>, dim3(static_cast<unsigned>(M)), dim3(32 * warps),
+                              static_cast<size_t>(warps) * kFwhtWarpFloats * 4, st, 0, x, M, K, ldx, g, norm, eps_norm, hb, q,
+                              ldq, s_x, status, mode, row_max, row_ss);
+        static PerDevice fwht_configured;  // up to 64 KB of dynamic shared memory
+        if (fwht_configured.get(dev, [&] {
+                return cudaFuncSetAttribute(act_prologue_fwht<T, kFwhtMaxWarps>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            kFwhtMaxWarps * kFwhtWarpFloats * 4) == cudaSuccess ? 1 : 0;
+            }) <= 0)
+            return LOWBIT_ERR_CUDA;
+        return launch_pdl(act_prologue_fwht<T, kFwhtMaxWarps>, dim3(static_cast<unsigned>(M)), dim3(32 * warps),
+                          static_cast<size_t>(warps) * kFwhtWarpFloats * 4, st, 0, x, M, K, ldx, g, norm, eps_norm, hb, q, ldq,
+                          s_x, status, mode, row_max, row_ss);
+    }
+    static PerDevice configured;  // the shared-memory limit is raised once per device
     if (configured.get(dev, [&] {
             return cudaFuncSetAttribute(act_prologue_staged<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         static_cast<int>(kMaxStagedK * 4)) == cudaSuccess ? 1 : 0;

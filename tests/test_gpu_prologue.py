@@ -73,7 +73,8 @@ OPT_IDS = [f"g{int(g)}-norm{n}-h{h}" for g, n, h in OPTIONS]
 
 @pytest.mark.parametrize("bf16", [False, True], ids=["f32", "bf16"])
 @pytest.mark.parametrize("opt", OPTIONS, ids=OPT_IDS)
-@pytest.mark.parametrize("M,K", [(1, 2560), (7, 1024), (300, 9728), (2048, 512), (33, 2560), (5, 40960), (1024, 2560)])
+@pytest.mark.parametrize("M,K", [(1, 2560), (7, 1024), (300, 9728), (2048, 512), (33, 2560), (5, 40960), (1024, 2560),
+                                 (3, 16384), (4, 2624)])
 def test_act_quant_ex_matches_oracle(M, K, opt, bf16):
     use_g, norm, hb = opt
     if hb and K % hb:
