@@ -788,6 +788,7 @@ __device__ __forceinline__ void tc_commit_pair_self(uint64_t *bar)
 // ---------------------------------------------------------------------------
 constexpr int kPairSkMinKb = 8;                           // K blocks of 128 per pair's share, at least
 constexpr int kPairSkFixupKb = 12;                       // cost of the tail, in K blocks of MMA time
+constexpr int kPairSkExtraKb = 11;                        // and of each partial tile after the first
 constexpr int kPairWsSlots = 96;                          // partial tiles held at once (one per pair)
 constexpr int kPairWsWords = 2 * PBM * 2 * PBN;  // one 256 x 256 int32 tile (both CTAs)
 constexpr int kWsWarpVecs = 32 * 2 * PBN / 4;     // one epilogue warp's 32 rows x 256 int32, in uint4
@@ -803,7 +804,10 @@ static std::atomic<uint32_t> g_pair_epoch{0};
 // kPairSkFixupKb, beats the whole-round schedule (ceil(tiles / P) rounds of
 // nkb).  The fix-up estimate is measured: a partial tile's store, the
 // finisher's staging and its longer epilogue, and the pieces' shorter
-// pipelines cost about 12 K blocks of MMA time (4B-class shapes, 74 pairs,
+// pipelines cost about 12 K blocks of MMA time, and each further partial
+// tile added from L2 about 11 more (9728 -> 2560 at M = 128, forced onto
+// pairs: 10 K blocks per pair, up to 8 partial tiles per tile, 44 us against
+// 19 on the split-K GEMM) (4B-class shapes, 74 pairs,
 // bf16 out: 9728 -> 2560 at M = 8192, 4 rounds + 24 tiles of 76 blocks, 145.8
 // -> 137.6 us; at M = 1024, 40 tiles of 76, 37.3 -> 33.1 us; 2560 -> 9728 at
 // M = 8192, 16 rounds + 32 tiles of 20, 147.0 -> 150.8 us, so that shape keeps
@@ -820,7 +824,13 @@ inline void pair_plan(int64_t tiles, int64_t resident, int64_t nkb, int64_t &dp_
     int64_t P = resident;
     if (rounds == 0 && W / P < kPairSkMinKb) P = W / kPairSkMinKb;
     if (P <= 1 || (rounds == 0 && P <= tiles)) return;
-    const int64_t shared = dp / P * nkb + (W + P - 1) / P + kPairSkFixupKb;
+    // a tile is shared by up to ceil(nkb / share) + 1 pairs, so its finisher
+    // adds up to ceil(nkb / share) partial tiles; after the first, which is
+    // staged in shared memory, each costs about 8 L2 round trips
+    const int64_t share = W / P > 0 ? W / P : 1;
+    const int64_t partials = (nkb + share - 1) / share;
+    const int64_t shared = dp / P * nkb + (W + P - 1) / P + kPairSkFixupKb +
+                           kPairSkExtraKb * (partials > 1 ? partials - 1 : 0);
     if (shared >= whole) return;
     dp_tiles = dp;
     P_out = P;

@@ -393,19 +393,22 @@ def test_stream_split_bf16_bit_exact(fmt):
 # (8192, 9728, 2560: 16 rounds + 32 tiles of 20 K blocks, where sharing does
 # not pay); 3 rounds, then 98 tiles of 76 blocks (8192,
 # 2560, 9728); 40 tiles of 76 blocks, no whole round (1024, 2560, 9728); one
-# round, then 78 tiles of 20 (1024, 9728, 2560); 6 ragged tiles of 32 blocks
-# on 24 pairs, 3 partial tiles added per tile (300, 700, 4096); 8 tiles of 128
-# blocks (512, 1000, 16384); 9 tiles of 6 blocks, no split (768, 768, 768).
+# round, then 78 tiles of 20 (1024, 9728, 2560); 40 ragged tiles of 76 blocks,
+# up to 2 partial tiles added per tile (1000, 2500, 9728); 6 ragged tiles of 32
+# blocks, kept whole since 4 partial tiles per tile would cost more (300, 700,
+# 4096); 8 tiles of 128 blocks, up to 10 partial tiles per tile (512, 1000,
+# 16384); 9 tiles of 6 blocks, no split (768, 768, 768).
 # Each launch gets its own activations and output dtype, so that a partial
 # tile or flag left by an earlier launch cannot pass for this one's; the
 # output must equal the unsplit launch bit for bit, and the oracle on
 # sampled rows (every row of the small shapes).
 PAIR_SPLIT_SHAPES = [(8192, 9728, 2560), (8192, 2560, 9728), (1024, 2560, 9728), (1024, 9728, 2560),
-                     (300, 700, 4096), (512, 1000, 16384), (768, 768, 768)]
+                     (1000, 2500, 9728), (300, 700, 4096), (512, 1000, 16384), (768, 768, 768)]
 
 
 @pytest.mark.parametrize("M,N,K,fmt", [s + (bwt.TERNARY2,) for s in PAIR_SPLIT_SHAPES]
                          + [(300, 700, 4096, f) for f in (bwt.BINARY1, bwt.INT4)]
+                         + [(1000, 2500, 9728, f) for f in (bwt.BINARY1, bwt.INT4)]
                          + [(1024, 2560, 9728, f) for f in (bwt.BINARY1, bwt.INT4)], ids=str)
 def test_pair_stream_k_bit_exact(M, N, K, fmt):
     w = wls.normal_weights(1100 + M + K, N, K)
