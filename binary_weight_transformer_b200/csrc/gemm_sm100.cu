@@ -731,14 +731,22 @@ constexpr int PBN = 128;                      // features expanded per CTA (the 
 constexpr int PE_BYTES = PBN * BK;
 template <int FMT, int OUT> __host__ __device__ constexpr int pair_tma_stages() { return FMT == kI4 ? 7 : 8; }
 template <int FMT, int OUT> __host__ __device__ constexpr int pair_exp_stages() { return kExpStages; }
+// A pair CTA has EW epilogue warps (warps 6..): one per TMEM lane quarter
+// (EW = 4), or two converting half of the columns each (EW = 8).  A warp's
+// 32-column chunks run as one dependent chain, so EW = 8 halves a tile's
+// epilogue; it pays where that epilogue is exposed (few tiles per pair) and
+// costs where it overlaps the next tile's mainloop (measured, bf16 out, 74
+// pairs: 9728 -> 2560 at M = 1024 34.3 -> 31.1 us, 2560 -> 9728 30.4 -> 28.4;
+// at M = 8192 135.5 -> 139.1 and 143.7 -> 151.6).
+template <int EW> __host__ __device__ constexpr int pair_threads() { return (6 + EW) * 32; }
 constexpr uint32_t kPairIdesc = (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>((2 * PBN) >> 3) << 17) |
                                 (static_cast<uint32_t>((2 * PBM) >> 4) << 24);
 
-template <int FMT, int OUT>
+template <int FMT, int OUT, int EW = 4>
 __host__ __device__ constexpr size_t pair_smem_bytes()
 {
     return 1024 + static_cast<size_t>(pair_tma_stages<FMT, OUT>()) * (A_BYTES + PBN * packed_bytes_per_kblock<FMT>()) +
-           static_cast<size_t>(pair_exp_stages<FMT, OUT>()) * PE_BYTES + 4 * stage_warp_bytes<OUT>() +
+           static_cast<size_t>(pair_exp_stages<FMT, OUT>()) * PE_BYTES + static_cast<size_t>(EW) * stage_warp_bytes<OUT>() +
            8 * (2 * pair_tma_stages<FMT, OUT>() + pair_exp_stages<FMT, OUT>() + 8);
 }
 
@@ -793,7 +801,7 @@ constexpr int kPairWsSlots = 96;                          // partial tiles held 
 constexpr int kPairWsWords = 2 * PBM * 2 * PBN;  // one 256 x 256 int32 tile (both CTAs)
 constexpr int kWsWarpVecs = 32 * 2 * PBN / 4;     // one epilogue warp's 32 rows x 256 int32, in uint4
 __device__ uint4 g_pair_ws[kPairWsSlots][kPairWsWords / 4];
-__device__ uint32_t g_pair_flag[kPairWsSlots][2][4];  // per pair (slot), CTA and epilogue warp
+__device__ uint32_t g_pair_flag[kPairWsSlots][2][8];  // per pair (slot), CTA and epilogue warp
 // One epoch per launch, shared by every instantiation of the kernel (they
 // share the flags), so no launch can take another launch's flag for its own.
 static std::atomic<uint32_t> g_pair_epoch{0};
@@ -921,40 +929,22 @@ __device__ inline bool wait_flag(const uint32_t *flag, uint32_t epoch, volatile 
     }
 }
 
-// Runs f(v, cc) on the 8 32-column chunks of this warp's accumulator rows
-// in order.  With kOverlap the TMEM load of chunk cc + 1 is in flight while
-// chunk cc is processed; it is used where the registers of both chunks fit
-// without spilling (ternary weights: one weight scale), since a register
-// spilled between a load and its wait would be read before it is written.
-template <bool kOverlap, typename F>
-__device__ __forceinline__ void pair_chunks(uint32_t tacc, F &&f)
+// Runs f(v, cc) on the 32-column chunks c0 .. c0 + nch - 1 of this warp's
+// accumulator rows in order.  (Keeping the next chunk's TMEM load in flight
+// while the current one is stored measured no faster.)
+template <typename F>
+__device__ __forceinline__ void pair_chunks(uint32_t tacc, int c0, int nch, F &&f)
 {
-    constexpr int kChunks = 2 * PBN / 32;
-    static_assert(kChunks % 2 == 0, "chunks are processed in pairs");
-    if constexpr (!kOverlap) {
 #pragma unroll 1
-        for (int cc = 0; cc < kChunks; ++cc) {
-            uint32_t v[32];
-            tmem_ld_32cols(tacc + static_cast<uint32_t>(cc * 32), v);
-            f(v, cc);
-        }
-        return;
-    }
-    uint32_t va[32], vb[32];
-    tmem_ld_32cols(tacc, va);
-#pragma unroll 1
-    for (int cc = 0; cc < kChunks; cc += 2) {
-        tmem_ld_32cols_async(tacc + static_cast<uint32_t>((cc + 1) * 32), vb);
-        f(va, cc);
-        tmem_ld_wait(vb);
-        if (cc + 2 < kChunks) tmem_ld_32cols_async(tacc + static_cast<uint32_t>((cc + 2) * 32), va);
-        f(vb, cc + 1);
-        if (cc + 2 < kChunks) tmem_ld_wait(va);
+    for (int cc = c0; cc < c0 + nch; ++cc) {
+        uint32_t v[32];
+        tmem_ld_32cols(tacc + static_cast<uint32_t>(cc * 32), v);
+        f(v, cc);
     }
 }
 
-template <int FMT, int OUT>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+template <int FMT, int OUT, int EW>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<EW>(), 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_p,
                  const float *__restrict__ s_x, const float *__restrict__ s_w, int64_t M, int64_t N, int64_t K,
                  void *__restrict__ y, int64_t ldy, int vec_ok, int prefetch, int32_t *status, int64_t dp_tiles,
@@ -974,7 +964,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     uint8_t *sE = sA + ST * A_BYTES;           // SE x 16 KB, 1024-aligned
     uint8_t *sP = sE + SE * PE_BYTES;          // ST x P_BYTES
     uint8_t *sStage = sP + ST * P_BYTES;       // 4 x epilogue staging
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sStage + 4 * stage_warp_bytes<OUT>());
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sStage + EW * stage_warp_bytes<OUT>());
     uint64_t *full_tma = bars;
     uint64_t *mma_done = bars + ST;
     uint64_t *full_exp = bars + 2 * ST;
@@ -997,7 +987,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         for (int s = 0; s < SE; ++s) mbar_init(&full_exp[s], 8);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 8);
+            mbar_init(&acc_empty[b], 2 * EW);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -1136,6 +1126,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     } else {
         // ---------------- epilogue: own 128 tokens x 256 features ----------------
         const int quarter = warp & 3;
+        constexpr int kChunksPerWarp = 8 * 4 / EW;             // of the 8 32-column chunks
+        const int c0 = ((warp - 6) >> 2) * kChunksPerWarp;     // this warp's first chunk
+        const int flag = quarter * 2 + ((warp - 6) >> 2);      // this warp's flag (rows and columns)
         const uint32_t stage = smem_u32(sStage) + static_cast<uint32_t>((warp - 6) * stage_warp_bytes<OUT>());
         const uint32_t acc_empty_leader = map_to_peer(smem_u32(acc_empty), 0);
         const float sw_tensor = (FMT == kT2) ? s_w[0] : 0.0f;
@@ -1157,15 +1150,15 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 // (rows) of one store write 512 contiguous bytes and each
                 // warp's rows are one contiguous 32 KB block.
                 uint4 *ws = g_pair_ws[pair] + rank * (PBM * 2 * PBN / 4) + quarter * kWsWarpVecs;
-                pair_chunks<FMT == kT2>(tacc, [=](const uint32_t(&v)[32], int cc) {
+                pair_chunks(tacc, c0, kChunksPerWarp, [=](const uint32_t(&v)[32], int cc) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
                         ws[(cc * 8 + j) * 32 + lane] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
                 });
                 __threadfence();
-                __syncwarp();  // this warp's 32 rows are stored
+                __syncwarp();  // this warp's 32 rows and columns are stored
                 if (lane == 0)
-                    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(&g_pair_flag[pair][rank][quarter]),
+                    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(&g_pair_flag[pair][rank][flag]),
                                  "r"(epoch)
                                  : "memory");
                 tc_fence_before();
@@ -1183,12 +1176,12 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             const int nsum = u.last >= 0 ? u.last - static_cast<int>(pair) : 0;
             bool have = true;  // every lane acquires the flags of its warp's rows itself
             for (int p = 1; p <= nsum; ++p)
-                have = have && wait_flag(&g_pair_flag[pair + p][rank][quarter], epoch, abort_flag, status);
+                have = have && wait_flag(&g_pair_flag[pair + p][rank][flag], epoch, abort_flag, status);
             const uint32_t staged = smem_u32(sA) + static_cast<uint32_t>(quarter * kWsWarpVecs * 16);
             if (nsum > 0 && have) {
                 const uint4 *ws = g_pair_ws[pair + 1] + rank * (PBM * 2 * PBN / 4) + quarter * kWsWarpVecs;
 #pragma unroll 8
-                for (int i = 0; i < kWsWarpVecs / 32; ++i)
+                for (int i = c0 * 8; i < (c0 + kChunksPerWarp) * 8; ++i)  // this warp's chunks
                     cp_async_16(staged + static_cast<uint32_t>((i * 32 + lane) * 16), ws + i * 32 + lane);
                 cp_async_wait_all();
             }
@@ -1196,7 +1189,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             const int64_t n0 = (u.tile % num_n) * 2 * PBN;
             const int64_t row0 = m0 + quarter * 32;
             const float sx = (row0 + lane < M) ? ld_act_f32(s_x + row0 + lane) : 0.0f;
-            pair_chunks<FMT == kT2>(tacc, [=](uint32_t(&v)[32], int cc) {
+            pair_chunks(tacc, c0, kChunksPerWarp, [=](uint32_t(&v)[32], int cc) {
                 const int64_t nc = n0 + cc * 32;
                 if (nsum > 0 && have) {
 #pragma unroll
@@ -1244,38 +1237,65 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     }
 }
 
-template <int FMT, int OUT>
-lowbit_status launch_pair_t(const CUtensorMap &ma, const CUtensorMap &mp, const float *s_x, const float *s_w,
-                            int64_t M, int64_t N, int64_t K, void *y, int64_t ldy, int vec_ok, int prefetch,
-                            int exclusive, int32_t *status, cudaStream_t st)
+// Pairs of one instantiation that can be resident at once, found (with the
+// shared-memory attribute set) on the first launch on each device.
+template <int FMT, int OUT, int EW>
+int pair_resident(int dev)
 {
-    constexpr size_t smem = pair_smem_bytes<FMT, OUT>();
+    constexpr size_t smem = pair_smem_bytes<FMT, OUT, EW>();
     static_assert(smem <= 232448, "shared memory budget");
-    // Pairs that can be resident at once, found (with the shared-memory
-    // attribute set) on the first launch on each device.
     static PerDevice max_pairs;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
-    const int resident = max_pairs.get(dev, [&] {
-        if (cudaFuncSetAttribute(gemm_pair_kernel<FMT, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return max_pairs.get(dev, [&] {
+        if (cudaFuncSetAttribute(gemm_pair_kernel<FMT, OUT, EW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem)) != cudaSuccess)
             return 0;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * static_cast<unsigned>(device_sm_count() / 2));
-        cfg.blockDim = dim3(kThreads);
+        cfg.blockDim = dim3(pair_threads<EW>());
         cfg.dynamicSmemBytes = smem;
         int n = 0;
-        return cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<FMT, OUT>, &cfg) == cudaSuccess ? n : 0;
+        return cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<FMT, OUT, EW>, &cfg) == cudaSuccess ? n : 0;
     });
-    if (resident <= 0) return LOWBIT_ERR_CUDA;
+}
+
+template <int FMT, int OUT, int EW>
+lowbit_status launch_pair_ew(const CUtensorMap &ma, const CUtensorMap &mp, const float *s_x, const float *s_w,
+                             int64_t M, int64_t N, int64_t K, void *y, int64_t ldy, int vec_ok, int prefetch,
+                             int exclusive, int32_t *status, int resident, cudaStream_t st)
+{
     const int64_t tiles = ((M + 2 * PBM - 1) / (2 * PBM)) * ((N + 2 * PBN - 1) / (2 * PBN));
     int64_t pairs = tiles < resident ? tiles : resident;
     int64_t dp_tiles = tiles;
     if (exclusive) pair_plan(tiles, resident, (K + BK - 1) / BK, dp_tiles, pairs);
     uint32_t epoch = g_pair_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
     if (epoch == 0) epoch = g_pair_epoch.fetch_add(1, std::memory_order_relaxed) + 1;  // 0 is the flags' initial value
-    return launch_pdl(gemm_pair_kernel<FMT, OUT>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kThreads), smem, st,
-                      0, ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, status, dp_tiles, epoch);
+    return launch_pdl(gemm_pair_kernel<FMT, OUT, EW>, dim3(static_cast<unsigned>(2 * pairs)),
+                      dim3(pair_threads<EW>()), pair_smem_bytes<FMT, OUT, EW>(), st, 0, ma, mp, s_x, s_w, M, N, K,
+                      y, ldy, vec_ok, prefetch, status, dp_tiles, epoch);
+}
+
+// Eight epilogue warps where a tile's epilogue is mostly exposed (at most
+// three tiles per pair) and their staging fits shared memory (bf16 out);
+// four otherwise.
+template <int FMT, int OUT>
+lowbit_status launch_pair_t(const CUtensorMap &ma, const CUtensorMap &mp, const float *s_x, const float *s_w,
+                            int64_t M, int64_t N, int64_t K, void *y, int64_t ldy, int vec_ok, int prefetch,
+                            int exclusive, int32_t *status, cudaStream_t st)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    const int64_t tiles = ((M + 2 * PBM - 1) / (2 * PBM)) * ((N + 2 * PBN - 1) / (2 * PBN));
+    if constexpr (OUT == LOWBIT_BF16) {
+        const int resident = pair_resident<FMT, OUT, 8>(dev);
+        if (resident <= 0) return LOWBIT_ERR_CUDA;
+        if (tiles <= 3 * static_cast<int64_t>(resident))
+            return launch_pair_ew<FMT, OUT, 8>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, exclusive,
+                                                status, resident, st);
+    }
+    const int resident = pair_resident<FMT, OUT, 4>(dev);
+    if (resident <= 0) return LOWBIT_ERR_CUDA;
+    return launch_pair_ew<FMT, OUT, 4>(ma, mp, s_x, s_w, M, N, K, y, ldy, vec_ok, prefetch, exclusive, status,
+                                       resident, st);
 }
 
 template <int FMT>
